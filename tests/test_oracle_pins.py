@@ -1,0 +1,241 @@
+"""Pins for the fp64 CPU oracle, independent of the oracle's own formulas.
+
+Each test ties the oracle to something the linear-attention pages or plain
+mathematics fix, chosen so that a plausible slip (a dropped term, a wrong
+index or sign, a transposed state, an exclusive instead of inclusive prefix,
+the wrong feature-map branch) fails at least one of them:
+
+- the recurrence equals the quadratic, row-normalised form (the
+  associativity identity of "Efficient Transformers Survey", Proposition
+  "Linear Attention via Kernel Decomposition", Intuition and Proof Sketch);
+- the feature map matches torch's library elu / relu;
+- closed forms: D = 1 reduces attention to a phi(k)-weighted mean of v;
+  identical keys reduce it to a plain prefix (or global) mean of v;
+- invariants: V = 1 gives O = 1; N = 1 gives o = v; the first causal output
+  is v_1; causal outputs ignore later tokens; non-causal outputs ignore the
+  order of (k, v) pairs;
+- the token-by-token decode recurrence ("Why It Matters": update S and z
+  incrementally) reproduces the causal forward and its final state;
+- S is D x D and z has D entries (section Exercises, ExerciseCore);
+- the backward matches central finite differences of L = sum(dO * O), and
+  satisfies the homogeneity / linearity identities of the definition.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import PHI_ELU1, PHI_RELU_EPS
+
+
+def rnd(shape, seed, scale=1.0, away_from_zero=False):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal(shape) * scale
+    if away_from_zero:
+        # keep the ReLU map differentiable for finite differences
+        x = np.where(np.abs(x) < 1e-2, np.sign(x + 1e-300) * (1e-2 + np.abs(x)), x)
+    return x
+
+
+SHAPES = [(1, 1, 1, 4), (1, 2, 7, 3), (2, 1, 16, 8), (1, 1, 33, 16)]
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+def test_recurrence_equals_quadratic_form(shape, causal, phi):
+    q, k, v = (rnd(shape, s) for s in (1, 2, 3))
+    o_lin, _, _ = oracle.forward(q, k, v, causal, phi)
+    o_quad = oracle.quadratic(q, k, v, causal, phi)
+    np.testing.assert_allclose(o_lin, o_quad, rtol=1e-12, atol=1e-12)
+
+
+def test_feature_map_matches_library():
+    x = torch.linspace(-6, 6, 1001, dtype=torch.float64)
+    elu1 = torch.nn.functional.elu(x, alpha=1.0) + 1.0
+    relu = torch.relu(x) + 1e-6
+    np.testing.assert_allclose(oracle.phi_map(x, PHI_ELU1), elu1.numpy(), rtol=1e-13, atol=0)
+    np.testing.assert_allclose(oracle.phi_map(x, PHI_RELU_EPS), relu.numpy(), rtol=1e-13, atol=0)
+    # slope of elu+1: 1 for x > 0, exp(x) for x <= 0 (autograd of the library map)
+    xg = x.clone().requires_grad_(True)
+    (torch.nn.functional.elu(xg) + 1.0).sum().backward()
+    np.testing.assert_allclose(oracle.dphi_map(x, PHI_ELU1), xg.grad.numpy(), rtol=1e-13)
+
+
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+@pytest.mark.parametrize("causal", [True, False])
+def test_d1_is_phi_weighted_mean(phi, causal):
+    # D = 1: o_i = sum_j phi(k_j) v_j / sum_j phi(k_j); the query cancels.
+    N = 9
+    q, k, v = (rnd((1, 1, N, 1), s) for s in (4, 5, 6))
+    kt = torch.from_numpy(k[0, 0, :, 0])
+    w = (torch.nn.functional.elu(kt) + 1.0) if phi == PHI_ELU1 else (torch.relu(kt) + 1e-6)
+    w = w.numpy()
+    vv = v[0, 0, :, 0]
+    if causal:
+        expect = np.cumsum(w * vv) / np.cumsum(w)
+    else:
+        expect = np.full(N, (w * vv).sum() / w.sum())
+    o, _, _ = oracle.forward(q, k, v, causal, phi)
+    np.testing.assert_allclose(o[0, 0, :, 0], expect, rtol=1e-13, atol=1e-15)
+    o2 = oracle.quadratic(q, k, v, causal, phi)
+    np.testing.assert_allclose(o2[0, 0, :, 0], expect, rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_identical_keys_give_mean_of_values(causal):
+    B, H, N, D = 1, 2, 11, 5
+    q = rnd((B, H, N, D), 7)
+    v = rnd((B, H, N, D), 8)
+    k = np.broadcast_to(rnd((B, H, 1, D), 9), (B, H, N, D)).copy()
+    o, _, _ = oracle.forward(q, k, v, causal, PHI_ELU1)
+    if causal:
+        expect = np.cumsum(v, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    else:
+        expect = np.broadcast_to(v.mean(axis=2, keepdims=True), v.shape)
+    np.testing.assert_allclose(o, expect, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+def test_unit_values_give_unit_output(causal, phi):
+    shape = (2, 2, 13, 6)
+    q, k = rnd(shape, 10), rnd(shape, 11)
+    v = np.ones(shape)
+    o, _, _ = oracle.forward(q, k, v, causal, phi)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
+
+
+def test_single_token_and_first_causal_output():
+    q, k, v = (rnd((2, 3, 1, 8), s) for s in (12, 13, 14))
+    for causal in (True, False):
+        o, _, _ = oracle.forward(q, k, v, causal, PHI_ELU1)
+        np.testing.assert_allclose(o, v, rtol=1e-14, atol=1e-15)
+    q, k, v = (rnd((1, 2, 10, 8), s) for s in (15, 16, 17))
+    o, _, _ = oracle.forward(q, k, v, True, PHI_ELU1)
+    np.testing.assert_allclose(o[:, :, 0], v[:, :, 0], rtol=1e-14, atol=1e-15)
+
+
+def test_causal_output_ignores_later_tokens():
+    shape = (1, 1, 20, 6)
+    q, k, v = (rnd(shape, s) for s in (18, 19, 20))
+    o, _, _ = oracle.forward(q, k, v, True, PHI_ELU1)
+    cut = 8
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    q2[:, :, cut:] += 3.0
+    k2[:, :, cut:] -= 2.0
+    v2[:, :, cut:] *= -5.0
+    o2, _, _ = oracle.forward(q2, k2, v2, True, PHI_ELU1)
+    np.testing.assert_array_equal(o[:, :, :cut], o2[:, :, :cut])
+    assert np.abs(o[:, :, cut:] - o2[:, :, cut:]).max() > 1e-3
+
+
+def test_noncausal_ignores_key_order():
+    shape = (1, 2, 15, 4)
+    q, k, v = (rnd(shape, s) for s in (21, 22, 23))
+    perm = np.random.default_rng(24).permutation(shape[2])
+    o, _, _ = oracle.forward(q, k, v, False, PHI_ELU1)
+    o2, _, _ = oracle.forward(q, k[:, :, perm], v[:, :, perm], False, PHI_ELU1)
+    np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-14)
+
+
+def test_state_shapes_and_final_state():
+    B, H, N, D = 2, 3, 9, 5
+    q, k, v = (rnd((B, H, N, D), s) for s in (25, 26, 27))
+    for causal in (True, False):
+        _, S, z = oracle.forward(q, k, v, causal, PHI_ELU1)
+        assert S.shape == (B, H, D, D) and z.shape == (B, H, D)
+        # a single extra decode step with v = 1 column: S, z equal the quadratic
+        # row sums on the last query (both modes end with the full prefix)
+        o_last = oracle.quadratic(q, k, v, True, PHI_ELU1)[:, :, -1]
+        a = oracle.phi_map(q[:, :, -1])
+        num = np.einsum("bhf,bhfe->bhe", a, S)
+        den = np.einsum("bhf,bhf->bh", a, z)
+        np.testing.assert_allclose(num / den[..., None], o_last, rtol=1e-12)
+
+
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+def test_decode_recurrence_equals_causal_forward(phi):
+    B, H, T, D = 2, 2, 17, 6
+    q, k, v = (rnd((B, H, T, D), s) for s in (28, 29, 30))
+    o_ref, S_ref, z_ref = oracle.forward(q, k, v, True, phi)
+    S = np.zeros((B, H, D, D))
+    z = np.zeros((B, H, D))
+    for t in range(T):
+        o_t = oracle.decode_step(S, z, q[:, :, t], k[:, :, t], v[:, :, t], phi)
+        np.testing.assert_allclose(o_t, o_ref[:, :, t], rtol=1e-12, atol=1e-14)
+        if t == 0:
+            np.testing.assert_allclose(o_t, v[:, :, 0], rtol=1e-14)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(z, z_ref, rtol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+
+
+def fd_grads(q, k, v, dO, causal, phi, h=1e-6):
+    """Central differences of L = sum(dO * O) with the (pinned) forward."""
+    def loss(qq, kk, vv):
+        o, _, _ = oracle.forward(qq, kk, vv, causal, phi)
+        return float((o * dO).sum())
+
+    out = []
+    for which in range(3):
+        base = [q, k, v]
+        g = np.zeros_like(base[which])
+        it = np.nditer(base[which], flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [x.copy() for x in base]
+            minus = [x.copy() for x in base]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            g[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        out.append(g)
+    return out
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 3), (1, 1, 6, 4), (1, 2, 11, 5)])
+def test_backward_matches_finite_differences(causal, phi, shape):
+    relu = phi == PHI_RELU_EPS
+    q = rnd(shape, 31, away_from_zero=relu)
+    k = rnd(shape, 32, away_from_zero=relu)
+    v = rnd(shape, 33)
+    dO = rnd(shape, 34)
+    dq, dk, dv = oracle.backward(q, k, v, dO, causal, phi)
+    for got, ref in zip((dq, dk, dv), fd_grads(q, k, v, dO, causal, phi)):
+        scale = max(np.abs(ref).max(), 1e-3)
+        assert np.abs(got - ref).max() <= 1e-6 * scale + 1e-9, (np.abs(got - ref).max(), scale)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_backward_identities(causal):
+    shape = (2, 2, 14, 6)
+    q, k, v, dO = (rnd(shape, s) for s in (35, 36, 37, 38))
+    phi = PHI_ELU1
+    dq, dk, dv = oracle.backward(q, k, v, dO, causal, phi)
+    o, _, _ = oracle.forward(q, k, v, causal, phi)
+    # O is linear in V: sum <dV, V> = sum <dO, O>
+    np.testing.assert_allclose((dv * v).sum(), (dO * o).sum(), rtol=1e-11)
+    # o_i is homogeneous of degree 0 in a_i: <dA_i, a_i> = 0 per query
+    A = oracle.phi_map(q)
+    dA = dq / oracle.dphi_map(q)
+    per_i = (dA * A).sum(-1)
+    assert np.abs(per_i).max() < 1e-11 * max(1.0, np.abs(dA * A).max())
+    # scaling every phi(k) by one constant leaves O unchanged: sum_j <dB_j, b_j> = 0
+    Bm = oracle.phi_map(k)
+    dB = dk / oracle.dphi_map(k)
+    per_head = (dB * Bm).sum(axis=(-1, -2))
+    assert np.abs(per_head).max() < 1e-10 * max(1.0, np.abs(dB * Bm).max())
+    # V = 1 makes O = 1 whatever Q and K are: dQ = dK = 0
+    dq1, dk1, _ = oracle.backward(q, k, np.ones(shape), dO, causal, phi)
+    assert np.abs(dq1).max() < 1e-12 and np.abs(dk1).max() < 1e-12
+
+
+def test_backward_d1_has_no_query_gradient():
+    q, k, v, dO = (rnd((1, 1, 10, 1), s) for s in (39, 40, 41, 42))
+    for causal in (True, False):
+        dq, _, _ = oracle.backward(q, k, v, dO, causal, PHI_ELU1)
+        assert np.abs(dq).max() < 1e-13
