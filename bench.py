@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark: causal linear-attention forward + backward tokens/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one training pass of the attention layer on the timed workload
+(causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward followed by
+la_backward through the library's Python binding, inputs resident in HBM.
+The inputs (4 x 128 MiB) are larger than the 126 MB L2, so consecutive steps
+cannot serve each other from cache.  W untimed warm-up steps, then exactly K
+steps between two barrier + synchronize points, timed with CUDA events on the
+launching stream; with several GPUs each rank runs its own replica (there is
+no exchange step in this op) and the max time over ranks is used.
+
+The printed JSON line also carries:
+  roofline      the dominant kernel's algorithmic bytes per launch over its
+                measured launch time (CUDA events recorded by the library on
+                its launch stream during the timed steps) against the measured
+                HBM copy bandwidth;
+  e2e           the same metric with the inputs copied from pinned host
+                memory and the outputs read back inside the timed region;
+  cpu_baseline  the fp64 CPU oracle, as it stands, on a bounded sample;
+  clocks        SM clocks and throttle reasons sampled during the timed steps.
+
+``--impl reference`` times the CPU oracle on the same workload instead (this
+op has no runnable upstream implementation; the oracle is the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from linear_attention_transformers_b200 import inputs  # noqa: E402
+
+WORKLOAD = inputs.WORKLOADS["causal_fwdbwd_b8h16n8192d64_bf16"]
+METRIC = "linear-attn fwd+bwd tokens/s per B200; % of roofline (HBM GB/s, TC util)"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def algorithmic_bytes(kernel: str, w) -> float:
+    """Bytes a launch of `kernel` must move at minimum for workload w.
+
+    Element size e; per head N*D elements per tensor.  forward: read q, k, v,
+    write o (4 tensors); backward: read q, k, v, dO, write dq, dk, dv (7).
+    Kernels that implement part of a pass are charged the tensors they must
+    touch (listed beside each name).
+    """
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    t = w.B * w.H * w.N * w.D * e  # bytes of one [B,H,N,D] tensor
+    table = {
+        "fwd_generic": 4 * t,           # q, k, v -> o
+        "bwd_generic": 7 * t,           # q, k, v, dO -> dq, dk, dv
+    }
+    return float(table.get(kernel, 0.0))
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML on a thread."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80, "sync_boost": 0x10,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mask = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w, heads: int, tokens: int, threads: int):
+    """Time the oracle's forward+backward on `heads` heads x `tokens` tokens
+    of workload w (a bounded sample: the first heads, the first tokens)."""
+    import oracle
+    q, k, v, dO = inputs.make_tensors(1, heads, tokens, w.D, w.dtype, w.seed + 7,
+                                      with_grad_out=True)
+    oracle.build()
+    oracle.set_threads(threads)
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, w.causal, w.phi)
+    oracle.backward(q, k, v, dO, w.causal, w.phi)
+    dt = time.perf_counter() - t0
+    # one workload token covers H heads
+    return (heads * tokens / w.H) / dt, dt
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, target_s: float = 15.0):
+    cores = cpu_cores()
+    # calibrate on a short prefix, then take whole heads (full N) until the
+    # sample is about target_s of work
+    _, dt = oracle_sample(w, cores, 256, cores)
+    t_head = dt / 256 * w.N  # seconds for one full head on one core
+    heads = int(min(w.B * w.H, max(1, round(target_s * cores / max(t_head, 1e-9)))))
+    heads = max(1, (heads // cores) * cores) if heads >= cores else heads
+    value, dt = oracle_sample(w, heads, w.N, cores)
+    return {"value": value, "unit": UNIT, "cores": min(cores, heads), "kind": "oracle",
+            "sample": f"fp64 oracle forward+backward on {heads} of {w.B * w.H} heads x all "
+                      f"{w.N} tokens (same shape and distribution, OpenMP over heads), "
+                      f"{dt:.1f} s; tokens/s = heads*N/H / time"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = WORKLOAD
+    cores = cpu_cores()
+    # each step: the oracle on `cores` heads x `tokens` tokens, sized so the
+    # whole (warmup + steps) run stays near two minutes
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    _, dt = oracle_sample(w, cores, 256, cores)
+    tokens = int(max(64, min(w.N, budget / max(dt / 256, 1e-9))))
+    for _ in range(args.warmup):
+        oracle_sample(w, cores, tokens, cores)
+    total = 0.0
+    for _ in range(args.steps):
+        _, dt = oracle_sample(w, cores, tokens, cores)
+        total += dt
+    value = (args.steps * cores * tokens / w.H) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: fp64 oracle forward+backward on {cores} heads x "
+                                   f"first {tokens} tokens (one thread per head)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(w, gpus):
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
+            "causal": w.causal, "phi": "elu1" if w.phi == 0 else "relu_eps",
+            "global_batch": w.B * gpus, "seq_len": w.N, "parallelism": f"replicas{gpus}",
+            "l2": "inputs larger than L2 (4 x 128 MiB per step)"}
+
+
+# --------------------------------------------------------------------- ours
+def run_ours(args, world, rank, local):
+    from linear_attention_transformers_b200 import api
+    w = WORKLOAD
+    dev = torch.device("cuda", local)
+    api.load_library()
+    q, k, v, dO = (t for t in inputs.make_inputs(w, device=dev))
+    B, H, N, D = q.shape
+    o = torch.empty_like(q)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_f = api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal, w.dtype)
+    ws_b = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, w.causal, w.dtype)
+    ws = torch.empty(max(ws_f, ws_b, 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream)
+        api.la_backward(q, k, v, dO, w.causal, w.phi, dq=dq, dk=dk, dv=dv, workspace=ws,
+                        stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    api.la_get_device_error(stream)
+
+    # ---- timed region
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    api.la_profile_enable(True)
+    api.la_profile_collect()
+    launches0 = api.la_launch_count()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = api.la_launch_count() - launches0
+    prof = api.la_profile_collect()
+    api.la_profile_enable(False)
+    api.la_get_device_error(stream)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world)
+    tokens_per_step = w.B * w.N
+    value = world * tokens_per_step * args.steps / (ms_max / 1e3)
+
+    # ---- dominant kernel roofline
+    peaks, peaks_src = load_peaks()
+    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    roofline = None
+    if dom:
+        name, (n_launch, tot_ms) = dom
+        avg_s = tot_ms / n_launch / 1e3
+        alg = algorithmic_bytes(name, w)
+        achieved = alg / avg_s / 1e9
+        roofline = {"kernel": name, "bound": "hbm", "achieved": achieved,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_s * 1e3,
+                    "peak_source": f"{peaks_src} hbm_gbs",
+                    "share_of_step": tot_ms / max(ms, 1e-9)}
+    kernels = {k: {"launches": n, "total_ms": t, "share": t / max(ms, 1e-9)}
+               for k, (n, t) in prof.items()}
+    step_bytes = algorithmic_bytes("fwd_generic", w) + algorithmic_bytes("bwd_generic", w)
+    step_frac = (step_bytes / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"]
+
+    # ---- end to end: pinned host inputs in, outputs back, every step
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdO = (t.cpu().pin_memory() for t in (q, k, v, dO))
+        ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
+        e2e_steps = max(3, min(args.steps, 10))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            dO.copy_(hdO, non_blocking=True)
+            step()
+            for dst, src in zip(ho, (o, dq, dk, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * tokens_per_step * e2e_steps / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
+               "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w, world),
+            "roofline": roofline,
+            "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
+                              "frac": step_frac, "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+            "kernels": kernels,
+            "gpu_launches": int(launches),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

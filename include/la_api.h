@@ -1,0 +1,184 @@
+/*
+ * la_api.h — C ABI of the B200 kernelized linear-attention library
+ * (liblinattn.so).
+ *
+ * The operation (per batch b and head h; tensors [B, H, N, D], D innermost):
+ *
+ *     a_i = phi(q_i),   b_j = phi(k_j)
+ *     S_i = sum_{j in J(i)} b_j v_j^T   (D x D),   z_i = sum_{j in J(i)} b_j
+ *     o_i = S_i^T a_i / (a_i . z_i)
+ *
+ * J(i) is every key (non-causal) or j <= i (causal).  This is the
+ * kernel-decomposition form of attention in "Efficient Transformers Survey",
+ * section Linear Attention, Proposition "Linear Attention via Kernel
+ * Decomposition" (Statement: S and z are precomputed sums, each output is one
+ * query against them); the causal prefix and the decode step are the
+ * recurrent computation of the same proposition ("Why It Matters": S and z
+ * updated token by token, constant memory per step).  The backward pass
+ * ("Transformer Based Linear Attention with Optimized GPU Kernel
+ * Implementation", Abstract: forward and backward passes of O(N D^2) cost)
+ * returns the gradients of sum(dO * O) with respect to q, k and v.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers, contiguous [B, H, N, D] (or
+ *     [B, H, D] for decode vectors, [B, H, D, D] for states), 16-byte
+ *     aligned.  Element type: `dt` for q, k, v, o, dO, dq, dk, dv; float32
+ *     always for states (S, z) and the workspace.
+ *   - The caller owns all memory.  The library never allocates or frees
+ *     device memory.  Calls that need scratch take a caller-provided
+ *     workspace of at least la_workspace_size() bytes (256-byte aligned).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and never synchronises the host.
+ *   - Arguments are validated before anything is launched.  Invalid input
+ *     returns a status; nothing crosses the ABI as an exception or abort.
+ *   - phi is LA_PHI_ELU1: elu(x)+1 (= x+1 for x > 0, exp(x) otherwise) or
+ *     LA_PHI_RELU_EPS: max(x, 0) + 1e-6.  Both are > 0, so no epsilon is
+ *     added to the denominator.
+ *   - Supported head sizes D: 16, 32, 64, 128.  N, B, H >= 0 (a zero size
+ *     launches nothing and returns LA_OK; a requested final state is then
+ *     zero-filled).  B*H*N*D must stay below 2^62, N below 2^31.
+ *   - Accumulation is float32 throughout; bf16 inputs are read exactly.
+ */
+#ifndef LA_API_H
+#define LA_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LA_API_VERSION 1
+
+#if defined(__GNUC__)
+#define LA_EXPORT __attribute__((visibility("default")))
+#else
+#define LA_EXPORT
+#endif
+
+/* ABI-identical to cudaStream_t; declared here so this header needs no CUDA
+ * headers. */
+typedef struct CUstream_st *la_stream_t;
+
+typedef enum la_status {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, negative size, bad enum */
+    LA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. D = 48) */
+    LA_ERR_CUDA = 3,           /* a CUDA launch or runtime call failed */
+    LA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+    LA_ERR_DEVICE_TIMEOUT = 5  /* a bounded on-device wait gave up (see below) */
+} la_status;
+
+typedef enum la_phi {
+    LA_PHI_ELU1 = 0,      /* elu(x) + 1 */
+    LA_PHI_RELU_EPS = 1   /* max(x, 0) + 1e-6 */
+} la_phi;
+
+typedef enum la_dtype {
+    LA_F32 = 0,   /* float32 tensors */
+    LA_BF16 = 1   /* bfloat16 tensors, float32 accumulation */
+} la_dtype;
+
+typedef enum la_op {
+    LA_OP_FORWARD = 0,
+    LA_OP_BACKWARD = 1
+} la_op;
+
+/*
+ * Bytes of device workspace that la_forward (op = LA_OP_FORWARD) or
+ * la_backward (op = LA_OP_BACKWARD) needs for these sizes; 0 means none.
+ * Returns 0 as well for arguments the calls would reject.  The amount
+ * depends only on the arguments, so one buffer can be sized once and reused
+ * by calls on the same stream.
+ */
+LA_EXPORT size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D,
+                         int causal, la_dtype dt);
+
+/*
+ * Forward pass.  q, k, v (read) and o (written): [B, H, N, D] of dtype `dt`.
+ * causal != 0 selects the prefix sums j <= i.  S_out [B, H, D, D] (row = key
+ * feature f, column = value index) and z_out [B, H, D], float32, may each be
+ * NULL; when given they receive the state after all N tokens (both modes),
+ * which la_decode_step can continue from.  Workspace: see la_workspace_size;
+ * may be NULL when that is 0.
+ * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE,
+ * LA_ERR_CUDA.  On error nothing has been launched except for LA_ERR_CUDA,
+ * where earlier launches of the same call may have run.
+ */
+LA_EXPORT la_status la_forward(const void *q, const void *k, const void *v, void *o,
+                     float *S_out, float *z_out,
+                     int64_t B, int64_t H, int64_t N, int64_t D,
+                     la_dtype dt, int causal, la_phi phi,
+                     void *workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Backward pass of L = sum(dO * O) for the same forward.  q, k, v, dO
+ * (read) and dq, dk, dv (written): [B, H, N, D] of dtype `dt`.  The forward
+ * is recomputed inside (no saved O or state is needed) and no N x D x D
+ * tensor is ever stored: the prefix states are rebuilt chunk by chunk.
+ * dq/dk/dv must not alias the inputs.  Errors as la_forward.
+ */
+LA_EXPORT la_status la_backward(const void *q, const void *k, const void *v, const void *dO,
+                      void *dq, void *dk, void *dv,
+                      int64_t B, int64_t H, int64_t N, int64_t D,
+                      la_dtype dt, int causal, la_phi phi,
+                      void *workspace, size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * One recurrent decode step for every (b, h), in place:
+ *     S += phi(k) v^T,   z += phi(k),   o = S^T phi(q) / (phi(q) . z)
+ * (the update comes first, so the new token attends to itself).  S: float32
+ * [B, H, D, D] read and written; z: float32 [B, H, D] read and written;
+ * q, k, v (read) and o (written): [B, H, D] of dtype `dt`.  A zero state is
+ * a valid start (the first step then returns o = v).  o must not alias S,
+ * z, q, k or v.  Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA.
+ */
+LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void *k,
+                         const void *v, void *o, int64_t B, int64_t H, int64_t D,
+                         la_dtype dt, la_phi phi, la_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+LA_EXPORT const char *la_status_string(la_status status);
+
+/*
+ * Kernels that wait on other thread blocks do so for a bounded number of
+ * iterations; when a wait gives up, the kernel records it in a device-side
+ * error word and finishes without hanging (its outputs are then invalid).
+ * This call synchronises `stream`, reads and clears that word, and returns
+ * LA_ERR_DEVICE_TIMEOUT if it was set, LA_ERR_CUDA if the synchronisation
+ * itself failed, LA_OK otherwise.
+ */
+LA_EXPORT la_status la_get_device_error(la_stream_t stream);
+
+/*
+ * Launch accounting.  la_launch_count() is the number of kernels this
+ * library has launched since it was loaded (counted on the host at launch).
+ *
+ * Launch timing, for benchmarks: after la_profile_enable(1) every kernel the
+ * library launches is bracketed by two CUDA events recorded on its launch
+ * stream.  la_profile_collect() synchronises those events, writes up to
+ * `max_entries` per-kernel aggregates (name, launches, total milliseconds)
+ * to `out`, clears the records and returns the number of distinct kernels
+ * (which may exceed max_entries).  la_profile_enable(0) stops recording.
+ * Event bookkeeping is host-side and not thread-safe across concurrent
+ * callers; it allocates no device memory.
+ */
+typedef struct la_profile_entry {
+    char name[48];
+    int64_t launches;
+    double total_ms;
+} la_profile_entry;
+
+LA_EXPORT uint64_t la_launch_count(void);
+LA_EXPORT void la_profile_enable(int on);
+LA_EXPORT int la_profile_collect(la_profile_entry *out, int max_entries);
+
+/* Library version (LA_API_VERSION at build time). */
+LA_EXPORT int la_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LA_API_H */

@@ -1,0 +1,254 @@
+"""Thin Python binding of liblinattn (the C ABI in include/la_api.h).
+
+Argument marshalling only: every function checks tensor placement, dtype,
+shape and contiguity, allocates the outputs (and the workspace) it is not
+given with torch, and calls the C entry point of the same name on the
+current CUDA stream.  No arithmetic of the method runs here, and there is no
+fallback: if ``liblinattn.so`` is missing or cannot be loaded, every call
+raises ``RuntimeError``.
+
+    la_forward(q, k, v, causal=True, phi="elu1", ...)        -> o [, S, z]
+    la_backward(q, k, v, dO, causal=True, phi="elu1", ...)   -> dq, dk, dv
+    la_decode_step(S, z, q, k, v, phi="elu1", ...)           -> o   (S, z in place)
+    la_workspace_size(op, B, H, N, D, causal, dtype)         -> bytes
+    la_get_device_error(stream=None)                         -> raises on a device timeout
+    LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+LA_OK = 0
+LA_ERR_INVALID_ARG = 1
+LA_ERR_UNSUPPORTED = 2
+LA_ERR_CUDA = 3
+LA_ERR_WORKSPACE = 4
+LA_ERR_DEVICE_TIMEOUT = 5
+
+LA_F32 = 0
+LA_BF16 = 1
+LA_OP_FORWARD = 0
+LA_OP_BACKWARD = 1
+PHI = {"elu1": 0, "relu_eps": 1, 0: 0, 1: 1}
+DTYPE = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblinattn.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class ProfileEntry(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double)]
+
+
+class LinearAttentionError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {la_status_string(status)} (status {status})")
+
+
+def load_library(path: str | None = None):
+    """Load liblinattn.so (built in-tree by ``build.py``); raises if absent."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(
+                f"liblinattn.so not found at {p}; build it with "
+                "`python -m linear_attention_transformers_b200.build` (there is no fallback)")
+        lib = ctypes.CDLL(p)
+        vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        lib.la_workspace_size.argtypes = [ci, i64, i64, i64, i64, ci, ci]
+        lib.la_workspace_size.restype = sz
+        lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp, sz,
+                                   vp]
+        lib.la_forward.restype = ci
+        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
+                                    vp, sz, vp]
+        lib.la_backward.restype = ci
+        lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
+        lib.la_decode_step.restype = ci
+        lib.la_status_string.argtypes = [ci]
+        lib.la_status_string.restype = ctypes.c_char_p
+        lib.la_get_device_error.argtypes = [vp]
+        lib.la_get_device_error.restype = ci
+        lib.la_version.argtypes = []
+        lib.la_version.restype = ci
+        lib.la_launch_count.argtypes = []
+        lib.la_launch_count.restype = ctypes.c_uint64
+        lib.la_profile_enable.argtypes = [ci]
+        lib.la_profile_enable.restype = None
+        lib.la_profile_collect.argtypes = [ctypes.POINTER(ProfileEntry), ci]
+        lib.la_profile_collect.restype = ci
+        _lib = lib
+        return lib
+
+
+def la_status_string(status: int) -> str:
+    return load_library().la_status_string(int(status)).decode()
+
+
+def la_version() -> int:
+    return int(load_library().la_version())
+
+
+def _check(fn: str, status: int) -> None:
+    if status != LA_OK:
+        raise LinearAttentionError(fn, status)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _phi(phi) -> int:
+    if phi not in PHI:
+        raise ValueError(f"phi must be 'elu1' or 'relu_eps', got {phi!r}")
+    return PHI[phi]
+
+
+def _check_qkv(name: str, ref: torch.Tensor, *ts: torch.Tensor) -> None:
+    if not ref.is_cuda:
+        raise ValueError(f"{name}: tensors must be on a CUDA device")
+    if ref.dtype not in DTYPE:
+        raise ValueError(f"{name}: dtype must be float32 or bfloat16, got {ref.dtype}")
+    for t in (ref, *ts):
+        if t.device != ref.device or t.dtype != ref.dtype or t.shape != ref.shape:
+            raise ValueError(f"{name}: all tensors need the same device, dtype and shape")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: tensors must be contiguous")
+
+
+def la_workspace_size(op: int, B: int, H: int, N: int, D: int, causal: bool,
+                      dtype: torch.dtype) -> int:
+    return int(load_library().la_workspace_size(int(op), B, H, N, D, int(bool(causal)),
+                                                DTYPE[dtype]))
+
+
+def _workspace(op, q, causal, workspace):
+    B, H, N, D = q.shape
+    need = la_workspace_size(op, B, H, N, D, causal, q.dtype)
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=False,
+               workspace=None, stream=None):
+    """o = linear attention of q, k, v [B, H, N, D]; optionally the final (S, z)."""
+    lib = load_library()
+    _check_qkv("la_forward", q, k, v)
+    if q.dim() != 4:
+        raise ValueError("la_forward: q, k, v must be [B, H, N, D]")
+    B, H, N, D = q.shape
+    if o is None:
+        o = torch.empty_like(q)
+    else:
+        _check_qkv("la_forward", q, o)
+    S = z = None
+    if return_state:
+        S = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+        z = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    ws, ws_bytes = _workspace(LA_OP_FORWARD, q, causal, workspace)
+    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, H, N, D,
+                        DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
+                        _stream_handle(stream))
+    _check("la_forward", st)
+    return (o, S, z) if return_state else o
+
+
+def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, dv=None,
+                workspace=None, stream=None):
+    """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi)."""
+    lib = load_library()
+    _check_qkv("la_backward", q, k, v, dO)
+    if q.dim() != 4:
+        raise ValueError("la_backward: tensors must be [B, H, N, D]")
+    B, H, N, D = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _check_qkv("la_backward", q, dq, dk, dv)
+    ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
+    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+                         B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
+                         ws_bytes, _stream_handle(stream))
+    _check("la_backward", st)
+    return dq, dk, dv
+
+
+def la_decode_step(S, z, q, k, v, phi="elu1", o=None, stream=None):
+    """One in-place recurrent step: S, z (float32) updated, o [B, H, D] returned."""
+    lib = load_library()
+    _check_qkv("la_decode_step", q, k, v)
+    if q.dim() != 3:
+        raise ValueError("la_decode_step: q, k, v must be [B, H, D]")
+    B, H, D = q.shape
+    for name, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
+                or t.device != q.device:
+            raise ValueError(f"la_decode_step: {name} must be contiguous float32 {shape} "
+                             "on the device of q")
+    if o is None:
+        o = torch.empty_like(q)
+    st = lib.la_decode_step(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, D,
+                            DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
+    _check("la_decode_step", st)
+    return o
+
+
+def la_get_device_error(stream=None) -> None:
+    """Synchronise the stream and raise if a bounded device-side wait gave up."""
+    _check("la_get_device_error", load_library().la_get_device_error(_stream_handle(stream)))
+
+
+def la_launch_count() -> int:
+    """Kernels launched by liblinattn since it was loaded."""
+    return int(load_library().la_launch_count())
+
+
+def la_profile_enable(on: bool = True) -> None:
+    """Bracket every library launch with CUDA events on its stream."""
+    load_library().la_profile_enable(int(bool(on)))
+
+
+def la_profile_collect() -> dict:
+    """{kernel name: (launches, total ms)} since the last collect (synchronises)."""
+    lib = load_library()
+    buf = (ProfileEntry * 64)()
+    n = lib.la_profile_collect(buf, 64)
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms))
+            for i in range(min(n, 64))}
+
+
+class LinearAttention(torch.autograd.Function):
+    """torch autograd wrapper: forward and backward both run in liblinattn."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal=True, phi="elu1"):
+        ctx.save_for_backward(q, k, v)
+        ctx.causal, ctx.phi = causal, phi
+        return la_forward(q.contiguous(), k.contiguous(), v.contiguous(), causal, phi)
+
+    @staticmethod
+    def backward(ctx, dO):
+        q, k, v = ctx.saved_tensors
+        dq, dk, dv = la_backward(q.contiguous(), k.contiguous(), v.contiguous(),
+                                 dO.contiguous(), ctx.causal, ctx.phi)
+        return dq, dk, dv, None, None

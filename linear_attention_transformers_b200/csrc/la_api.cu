@@ -1,0 +1,312 @@
+// la_api.cu — the C ABI of liblinattn (declared in include/la_api.h):
+// argument validation, workspace sizing and kernel dispatch.
+//
+// Every entry point validates all of its arguments before it launches
+// anything, maps CUDA launch failures to LA_ERR_CUDA, never throws and never
+// synchronises (except la_get_device_error, which exists to do so).
+#include "la_api.h"
+
+#include <cuda_runtime.h>
+
+#include "la_common.cuh"
+#include "la_decode.cuh"
+#include "la_generic.cuh"
+#include "la_runtime.cuh"
+
+namespace {
+
+using la::PHI_ELU1;
+using la::PHI_RELU_EPS;
+
+constexpr int64_t kMaxElems = int64_t(1) << 62;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool supported_d(int64_t D) { return D == 16 || D == 32 || D == 64 || D == 128; }
+
+la_status check_sizes(int64_t B, int64_t H, int64_t N, int64_t D) {
+    if (B < 0 || H < 0 || N < 0 || D <= 0) return LA_ERR_INVALID_ARG;
+    if (!supported_d(D)) return LA_ERR_UNSUPPORTED;
+    if (N >= (int64_t(1) << 31) || B * H >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
+    // B*H*N*D < 2^62 without overflowing on the way
+    if (B != 0 && H != 0 && N != 0) {
+        const int64_t bh = B * H;
+        if (bh > kMaxElems / N || bh * N > kMaxElems / D) return LA_ERR_UNSUPPORTED;
+    }
+    return LA_OK;
+}
+
+la_status check_enums(la_dtype dt, la_phi phi) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (phi != LA_PHI_ELU1 && phi != LA_PHI_RELU_EPS) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+la_status check_ptr(const void* p) {
+    if (p == nullptr || !aligned16(p)) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+la_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------ workspace plan
+// Backward: g and dg, float32 [B, H, N] each.
+struct BwdWorkspace {
+    size_t g_off = 0, dg_off = 0, bytes = 0;
+};
+
+BwdWorkspace plan_bwd(int64_t B, int64_t H, int64_t N) {
+    BwdWorkspace w;
+    const size_t tok = size_t(B) * size_t(H) * size_t(N) * sizeof(float);
+    w.g_off = 0;
+    w.dg_off = round_up(tok, 256);
+    w.bytes = w.dg_off + round_up(tok, 256);
+    return w;
+}
+
+// ------------------------------------------------------------ generic path
+template <typename T, int PHI>
+la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
+                          float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
+                          cudaStream_t st) {
+    auto kern = la::fwd_generic_kernel<T, PHI>;
+    const size_t smem = la::generic_smem_bytes(int(D));
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    la::LaunchScope scope("fwd_generic", st);
+    kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+        static_cast<T*>(o), S_out, z_out, int(N), int(D), causal);
+    return launch_status();
+}
+
+template <typename T, int PHI>
+la_status run_bwd_generic(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                          void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
+                          float* gbuf, float* dgbuf, cudaStream_t st) {
+    auto kern = la::bwd_generic_kernel<T, PHI>;
+    const size_t smem = la::generic_smem_bytes(int(D)) + size_t(D) * sizeof(float);
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    la::LaunchScope scope("bwd_generic", st);
+    kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
+        static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+        static_cast<const T*>(dO), static_cast<T*>(dq), static_cast<T*>(dk), static_cast<T*>(dv),
+        gbuf, dgbuf, int(N), int(D), causal);
+    return launch_status();
+}
+
+template <typename T, int PHI>
+la_status run_decode(float* S, float* z, const void* q, const void* k, const void* v, void* o,
+                     int64_t heads, int64_t D, cudaStream_t st) {
+    const T* qq = static_cast<const T*>(q);
+    const T* kk = static_cast<const T*>(k);
+    const T* vv = static_cast<const T*>(v);
+    T* oo = static_cast<T*>(o);
+    const unsigned grid = unsigned(heads);
+    la::LaunchScope scope("decode_step", st);
+    switch (D) {
+        case 16: la::decode_step_kernel<T, PHI, 16><<<grid, 32, 0, st>>>(S, z, qq, kk, vv, oo); break;
+        case 32: la::decode_step_kernel<T, PHI, 32><<<grid, 64, 0, st>>>(S, z, qq, kk, vv, oo); break;
+        case 64: la::decode_step_kernel<T, PHI, 64><<<grid, 128, 0, st>>>(S, z, qq, kk, vv, oo); break;
+        case 128: la::decode_step_kernel<T, PHI, 128><<<grid, 256, 0, st>>>(S, z, qq, kk, vv, oo); break;
+        default: return LA_ERR_UNSUPPORTED;
+    }
+    return launch_status();
+}
+
+// dtype x phi dispatch helper
+template <template <typename, int> class F, typename... Args>
+la_status dispatch(la_dtype dt, la_phi phi, Args... args) {
+    if (dt == LA_F32) {
+        return phi == LA_PHI_ELU1 ? F<float, PHI_ELU1>::run(args...)
+                                  : F<float, PHI_RELU_EPS>::run(args...);
+    }
+    return phi == LA_PHI_ELU1 ? F<__nv_bfloat16, PHI_ELU1>::run(args...)
+                              : F<__nv_bfloat16, PHI_RELU_EPS>::run(args...);
+}
+
+template <typename T, int PHI>
+struct FwdOp {
+    static la_status run(const void* q, const void* k, const void* v, void* o, float* S_out,
+                         float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
+                         cudaStream_t st) {
+        return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, heads, N, D, causal, st);
+    }
+};
+
+template <typename T, int PHI>
+struct BwdOp {
+    static la_status run(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                         void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
+                         float* gbuf, float* dgbuf, cudaStream_t st) {
+        return run_bwd_generic<T, PHI>(q, k, v, dO, dq, dk, dv, heads, N, D, causal, gbuf, dgbuf,
+                                       st);
+    }
+};
+
+template <typename T, int PHI>
+struct DecodeOp {
+    static la_status run(float* S, float* z, const void* q, const void* k, const void* v,
+                         void* o, int64_t heads, int64_t D, cudaStream_t st) {
+        return run_decode<T, PHI>(S, z, q, k, v, o, heads, D, st);
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+int la_version(void) { return LA_API_VERSION; }
+
+const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "ok";
+        case LA_ERR_INVALID_ARG: return "invalid argument";
+        case LA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case LA_ERR_CUDA: return "CUDA error";
+        case LA_ERR_WORKSPACE: return "workspace missing or too small";
+        case LA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                         la_dtype dt) {
+    (void)causal;
+    if (check_sizes(B, H, N, D) != LA_OK) return 0;
+    if (dt != LA_F32 && dt != LA_BF16) return 0;
+    if (B == 0 || H == 0 || N == 0) return 0;
+    if (op == LA_OP_FORWARD) return 0;
+    if (op == LA_OP_BACKWARD) return plan_bwd(B, H, N).bytes;
+    return 0;
+}
+
+la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
+                     float* z_out, int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt,
+                     int causal, la_phi phi, void* workspace, size_t workspace_bytes,
+                     la_stream_t stream) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if ((S_out && !aligned16(S_out)) || (z_out && !aligned16(z_out))) return LA_ERR_INVALID_ARG;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if (N == 0) {
+        // nothing to attend over; a requested final state is all zero
+        if (S_out && cudaMemsetAsync(S_out, 0, size_t(heads * D * D) * 4, st) != cudaSuccess)
+            return LA_ERR_CUDA;
+        if (z_out && cudaMemsetAsync(z_out, 0, size_t(heads * D) * 4, st) != cudaSuccess)
+            return LA_ERR_CUDA;
+        return LA_OK;
+    }
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
+        return s;
+    const size_t need = la_workspace_size(LA_OP_FORWARD, B, H, N, D, causal, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
+    return dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, heads, N, D, causal ? 1 : 0, st);
+}
+
+la_status la_backward(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                      void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
+                      la_dtype dt, int causal, la_phi phi, void* workspace,
+                      size_t workspace_bytes, la_stream_t stream) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
+        (s = check_ptr(dq)) || (s = check_ptr(dk)) || (s = check_ptr(dv)))
+        return s;
+    const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const BwdWorkspace w = plan_bwd(B, H, N);
+    char* ws = static_cast<char*>(workspace);
+    float* gbuf = reinterpret_cast<float*>(ws + w.g_off);
+    float* dgbuf = reinterpret_cast<float*>(ws + w.dg_off);
+    return dispatch<BwdOp>(dt, phi, q, k, v, dO, dq, dk, dv, heads, N, D, causal ? 1 : 0, gbuf,
+                           dgbuf, st);
+}
+
+la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
+                         void* o, int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
+                         la_stream_t stream) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, 1, D)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if ((s = check_ptr(S)) || (s = check_ptr(z)) || (s = check_ptr(q)) || (s = check_ptr(k)) ||
+        (s = check_ptr(v)) || (s = check_ptr(o)))
+        return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return dispatch<DecodeOp>(dt, phi, S, z, q, k, v, o, heads, D, st);
+}
+
+uint64_t la_launch_count(void) { return la::profiler().launches.load(); }
+
+void la_profile_enable(int on) { la::profiler().on.store(on != 0); }
+
+int la_profile_collect(la_profile_entry* out, int max_entries) {
+    la::Profiler& p = la::profiler();
+    std::lock_guard<std::mutex> g(p.mu);
+    struct Agg {
+        const char* name;
+        int64_t n;
+        double ms;
+    };
+    std::vector<Agg> agg;
+    for (auto& r : p.records) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.stop) == cudaSuccess &&
+            cudaEventElapsedTime(&ms, r.start, r.stop) == cudaSuccess) {
+            bool found = false;
+            for (auto& a : agg)
+                if (strcmp(a.name, r.name) == 0) {
+                    a.n += 1;
+                    a.ms += ms;
+                    found = true;
+                    break;
+                }
+            if (!found) agg.push_back({r.name, 1, double(ms)});
+        }
+        p.pool.push_back(r.start);
+        p.pool.push_back(r.stop);
+    }
+    p.records.clear();
+    for (int i = 0; i < int(agg.size()) && i < max_entries && out; ++i) {
+        memset(out[i].name, 0, sizeof(out[i].name));
+        strncpy(out[i].name, agg[i].name, sizeof(out[i].name) - 1);
+        out[i].launches = agg[i].n;
+        out[i].total_ms = agg[i].ms;
+    }
+    return int(agg.size());
+}
+
+la_status la_get_device_error(la_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return LA_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, la::g_device_error, sizeof(word)) != cudaSuccess)
+        return LA_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(la::g_device_error, &zero, sizeof(zero)) != cudaSuccess)
+            return LA_ERR_CUDA;
+        return LA_ERR_DEVICE_TIMEOUT;
+    }
+    return LA_OK;
+}
+
+}  // extern "C"

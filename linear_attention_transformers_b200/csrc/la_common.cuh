@@ -1,0 +1,64 @@
+// la_common.cuh — element types, the feature map and small device helpers
+// shared by the CUDA kernels of liblinattn.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace la {
+
+enum : int { PHI_ELU1 = 0, PHI_RELU_EPS = 1 };
+
+// Error word for bounded waits (set by a kernel that gave up waiting).  The
+// library is one translation unit, so the definition lives here.
+__device__ unsigned int g_device_error = 0;
+
+// ---------------------------------------------------------------- feature map
+// phi is elementwise: elu(x)+1 (x+1 for x > 0, exp(x) otherwise) or
+// max(x,0)+1e-6.  The pages leave phi generic ("Efficient Transformers
+// Survey", Proposition "Linear Attention via Kernel Decomposition": any
+// phi: R^d -> R^m); m = D here.
+
+// Accurate variant (libm expf) for the reference-quality kernels.
+template <int PHI>
+__device__ __forceinline__ float phi_exact(float x) {
+    if (PHI == PHI_ELU1) return x > 0.f ? x + 1.f : expf(x);
+    return fmaxf(x, 0.f) + 1e-6f;
+}
+template <int PHI>
+__device__ __forceinline__ float dphi_exact(float x) {
+    if (PHI == PHI_ELU1) return x > 0.f ? 1.f : expf(x);
+    return x > 0.f ? 1.f : 0.f;
+}
+
+// Fast variant (hardware exp2 approximation) for the streaming kernels.
+template <int PHI>
+__device__ __forceinline__ float phi_fast(float x) {
+    if (PHI == PHI_ELU1) return x > 0.f ? x + 1.f : __expf(x);
+    return fmaxf(x, 0.f) + 1e-6f;
+}
+template <int PHI>
+__device__ __forceinline__ float dphi_fast(float x) {
+    if (PHI == PHI_ELU1) return x > 0.f ? 1.f : __expf(x);
+    return x > 0.f ? 1.f : 0.f;
+}
+
+// ---------------------------------------------------------------- elements
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// ---------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+}  // namespace la

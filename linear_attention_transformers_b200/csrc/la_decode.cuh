@@ -1,0 +1,93 @@
+// la_decode.cuh — one recurrent decode step, in place, for every (b, h):
+//     S += phi(k) v^T,  z += phi(k),  o = S^T phi(q) / (phi(q) . z)
+// ("Efficient Transformers Survey", Proposition "Linear Attention via Kernel
+// Decomposition", "Why It Matters": S and z updated token by token with
+// constant memory per step).
+//
+// The step is a single streaming pass over the float32 state: each S element
+// is read once and written once (8 bytes per element), so the kernel is HBM
+// bound.  One thread block per head; 2*D threads; thread (rg, cg) owns
+// columns 4*cg..4*cg+3 (one 16-byte vector) of rows rg, rg+8, ..., so a warp
+// reads whole 128-byte segments.  All of a thread's loads are issued before
+// any arithmetic so a block keeps D*D*4 bytes in flight; loads and stores
+// use the streaming cache hint because the state is not reused within the
+// step.  The partial numerators of the 8 row groups are summed through
+// shared memory in a fixed order (deterministic).
+#pragma once
+
+#include "la_common.cuh"
+
+namespace la {
+
+template <typename T, int PHI, int D>
+__global__ void __launch_bounds__(2 * D)
+decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
+                   const T* __restrict__ q, const T* __restrict__ k,
+                   const T* __restrict__ v, T* __restrict__ o) {
+    constexpr int CG = D / 4;    // 16-byte column groups
+    constexpr int RG = 8;        // row groups
+    constexpr int RPT = D / RG;  // rows per thread
+    constexpr int NT = 2 * D;
+    static_assert(CG * RG == NT, "thread layout");
+    __shared__ float a_s[D], b_s[D];
+    __shared__ float4 v_s4[CG];
+    __shared__ float4 part[RG][CG];
+    __shared__ float den_part[NT / 32];
+
+    const size_t h = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int cg = tid % CG, rg = tid / CG;
+    float4* Sh = reinterpret_cast<float4*>(S + h * D * D);
+
+    // Issue the state loads first; the vectors arrive while they are in flight.
+    float4 s[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = __ldcs(Sh + (rg + RG * r) * CG + cg);
+
+    float znew = 0.f;
+    if (tid < D) {
+        const float af = phi_fast<PHI>(to_f32(q[h * D + tid]));
+        const float bf = phi_fast<PHI>(to_f32(k[h * D + tid]));
+        a_s[tid] = af;
+        b_s[tid] = bf;
+        reinterpret_cast<float*>(v_s4)[tid] = to_f32(v[h * D + tid]);
+        znew = z[h * D + tid] + bf;
+        z[h * D + tid] = znew;
+        znew *= af;  // this thread's term of phi(q) . z
+    }
+    const float wsum = warp_sum(znew);
+    if ((tid & 31) == 0) den_part[tid >> 5] = wsum;
+    __syncthreads();
+
+    const float4 vv = v_s4[cg];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int f = rg + RG * r;
+        const float bf = b_s[f], af = a_s[f];
+        float4 x = s[r];
+        x.x = fmaf(bf, vv.x, x.x);
+        x.y = fmaf(bf, vv.y, x.y);
+        x.z = fmaf(bf, vv.z, x.z);
+        x.w = fmaf(bf, vv.w, x.w);
+        __stcs(Sh + f * CG + cg, x);
+        acc.x = fmaf(af, x.x, acc.x);
+        acc.y = fmaf(af, x.y, acc.y);
+        acc.z = fmaf(af, x.z, acc.z);
+        acc.w = fmaf(af, x.w, acc.w);
+    }
+    part[rg][cg] = acc;
+    __syncthreads();
+    if (tid < D) {
+        float den = 0.f;
+#pragma unroll
+        for (int w = 0; w < NT / 32; ++w) den += den_part[w];
+        const float* pf = reinterpret_cast<const float*>(&part[0][0]);
+        float num = 0.f;
+#pragma unroll
+        for (int g = 0; g < RG; ++g) num += pf[g * D + tid];
+        o[h * D + tid] = from_f32<T>(num / den);
+    }
+}
+
+}  // namespace la

@@ -1,0 +1,92 @@
+"""Host-side checks of the C ABI: the library loads, exports every entry point
+that include/la_api.h declares, and rejects bad arguments before it launches
+anything.  No test here runs device code (fake pointers are only ever given
+to calls that must refuse them during validation)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_transformers_b200 import api, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "la_api.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return api.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"LA_EXPORT\s+[\w\s\*]+?\b(la_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    for fn in ("la_forward", "la_backward", "la_decode_step", "la_workspace_size",
+               "la_status_string", "la_get_device_error", "la_version"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert lib.la_version() == 1
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert api.la_status_string(code)
+    assert api.la_status_string(99) == "unknown status"
+
+
+FAKE = 0x100000  # aligned, non-null, never dereferenced: every use below must fail validation
+
+
+def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=None, z=None, B=1, H=1, N=8, D=64, dt=1,
+        causal=1, phi=0, ws=None, ws_bytes=0):
+    return lib.la_forward(q, k, v, o, S, z, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
+
+
+def bwd(lib, p=FAKE, B=1, H=1, N=8, D=64, dt=1, causal=1, phi=0, ws=None, ws_bytes=0, dq=FAKE):
+    return lib.la_backward(p, p, p, p, dq, p, p, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
+
+
+def test_rejects_bad_arguments_before_launch(lib):
+    assert fwd(lib, q=None) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, o=FAKE + 4) == api.LA_ERR_INVALID_ARG          # misaligned
+    assert fwd(lib, D=48) == api.LA_ERR_UNSUPPORTED
+    assert fwd(lib, D=0) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, N=-1) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, dt=7) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, phi=9) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, N=1 << 31) == api.LA_ERR_UNSUPPORTED
+    assert fwd(lib, B=1 << 20, H=1 << 20, N=1 << 20) == api.LA_ERR_UNSUPPORTED
+    assert bwd(lib, dq=None) == api.LA_ERR_INVALID_ARG
+    assert bwd(lib, D=96) == api.LA_ERR_UNSUPPORTED
+    p = FAKE
+    assert lib.la_decode_step(p, p, p, p, p, None, 2, 2, 64, 1, 0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step(p, p, p, p, p, p, 2, 2, 40, 1, 0, None) == api.LA_ERR_UNSUPPORTED
+
+
+def test_workspace_is_checked(lib):
+    need = lib.la_workspace_size(api.LA_OP_BACKWARD, 2, 4, 1000, 64, 1, api.LA_BF16)
+    assert need > 0
+    assert bwd(lib, B=2, H=4, N=1000, ws=None, ws_bytes=0) == api.LA_ERR_WORKSPACE
+    assert bwd(lib, B=2, H=4, N=1000, ws=FAKE, ws_bytes=need - 1) == api.LA_ERR_WORKSPACE
+    assert bwd(lib, B=2, H=4, N=1000, ws=FAKE + 8, ws_bytes=need) == api.LA_ERR_INVALID_ARG
+    # sizes that are rejected report no workspace
+    assert lib.la_workspace_size(api.LA_OP_BACKWARD, 1, 1, 100, 48, 1, api.LA_BF16) == 0
+
+
+def test_empty_sizes_launch_nothing(lib):
+    # zero batch / heads / tokens: LA_OK with nothing launched (no final state asked)
+    assert fwd(lib, B=0) == api.LA_OK
+    assert fwd(lib, H=0) == api.LA_OK
+    assert fwd(lib, N=0) == api.LA_OK
+    assert bwd(lib, N=0) == api.LA_OK
+    assert lib.la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 64, 1, 0, None) == api.LA_OK
