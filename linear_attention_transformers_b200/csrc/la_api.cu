@@ -6,12 +6,19 @@
 // synchronises (except la_get_device_error, which exists to do so).
 #include "la_api.h"
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <string.h>
 
+#include <algorithm>
+
+#include "la_chunk_fwd.cuh"
 #include "la_common.cuh"
 #include "la_decode.cuh"
 #include "la_generic.cuh"
 #include "la_runtime.cuh"
+#include "la_sm100.cuh"
+#include "la_state.cuh"
 
 namespace {
 
@@ -66,6 +73,199 @@ BwdWorkspace plan_bwd(int64_t B, int64_t H, int64_t N) {
     w.dg_off = round_up(tok, 256);
     w.bytes = w.dg_off + round_up(tok, 256);
     return w;
+}
+
+
+// ------------------------------------------------------------ tensor maps
+// cuTensorMapEncodeTiled, fetched through the runtime so the library does
+// not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// [heads][N][D] bf16 viewed as a 3-D tensor (D, N, heads); box (64, C, 1),
+// 128-byte swizzle.  Rows past N read as zero and are clipped on store.
+bool make_qkv_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, int64_t D, int C) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(N), cuuint64_t(heads)};
+    cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * cuuint64_t(D) * 2};
+    cuuint32_t box[3] = {64, cuuint32_t(C), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ chunked path
+constexpr int kNumSM = 148;
+
+bool fast_path(la_dtype dt, int64_t D) { return dt == LA_BF16 && (D == 64 || D == 128); }
+int chunk_len(int64_t D) { return D == 64 ? 128 : 64; }
+
+// Segments per head: enough blocks to cover the SMs twice when there are few
+// heads, at least two chunks per segment.
+int pick_nseg(int64_t heads, int64_t nchunks) {
+    if (heads >= 120) return 1;
+    const int64_t want = (2 * kNumSM + heads - 1) / heads;
+    return int(std::max<int64_t>(1, std::min<int64_t>(want, nchunks / 2)));
+}
+
+struct SegSplit {
+    int nseg = 1, seg_len = 0;
+};
+SegSplit split(int64_t N, int C, int nseg) {
+    SegSplit s;
+    const int64_t per = (N + nseg - 1) / nseg;
+    s.seg_len = int((per + C - 1) / C * C);
+    s.nseg = int((N + s.seg_len - 1) / s.seg_len);
+    return s;
+}
+
+struct FwdPlan {
+    bool fast = false;
+    int C = 0;
+    SegSplit seg, qseg;
+    size_t rec_off = 0, tot_off = 0, bytes = 0;
+};
+
+FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
+    FwdPlan p;
+    if (!fast_path(dt, D) || N == 0 || B * H == 0) return p;
+    p.fast = true;
+    p.C = chunk_len(D);
+    const int64_t heads = B * H;
+    const int64_t nch = (N + p.C - 1) / p.C;
+    p.seg = split(N, p.C, pick_nseg(heads, nch));
+    const size_t R = size_t(D) * D + D;
+    if (causal) {
+        p.rec_off = 0;
+        p.bytes = p.seg.nseg > 1 ? size_t(heads) * p.seg.nseg * R * sizeof(float) : 0;
+    } else {
+        const int64_t want = heads >= 2 * kNumSM ? 1 : (2 * kNumSM + heads - 1) / heads;
+        p.qseg = split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
+        p.rec_off = 0;
+        p.tot_off = round_up(size_t(heads) * p.seg.nseg * R * sizeof(float), 256);
+        p.bytes = p.tot_off + round_up(size_t(heads) * R * sizeof(float), 256);
+    }
+    return p;
+}
+
+template <int D, int C, int PHI, int MODE>
+la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st,
+                       const char* name) {
+    auto kern = la::chunk_fwd_kernel<D, C, PHI, MODE>;
+    constexpr int smem = la::ChunkCfg<D, C>::SMEM;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+        return LA_ERR_CUDA;
+    la::LaunchScope scope(name, st);
+    kern<<<unsigned(grid), la::kChunkThreads, smem, st>>>(prm);
+    return launch_status();
+}
+
+la_status launch_state_kernel(int which, float* rec, float* out, float* S, float* z,
+                              int64_t heads, int nseg, int64_t D, cudaStream_t st) {
+    const int R = int(D * D + D);
+    const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
+    const unsigned grid = unsigned(heads * bph);
+    if (which == 0) {
+        la::LaunchScope scope("state_scan", st);
+        la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
+    } else if (which == 1) {
+        la::LaunchScope scope("state_sum", st);
+        la::state_sum_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, out, nseg, R, bph);
+    } else {
+        la::LaunchScope scope("state_unpack", st);
+        la::state_unpack_kernel<<<grid, la::kStateThreads, 0, st>>>(out, S, z, int(D), bph);
+    }
+    return launch_status();
+}
+
+template <int D, int PHI>
+la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, float* S_out,
+                          float* z_out, int64_t heads, int64_t N, int causal, const FwdPlan& p,
+                          char* ws, cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    la::ChunkParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) || !make_qkv_map(&prm.tm_o, o, heads, N, D, C))
+        return LA_ERR_CUDA;
+    prm.N = int(N);
+    const int64_t R = int64_t(D) * D + D;
+    float* rec = reinterpret_cast<float*>(ws + p.rec_off);
+    la_status s;
+    if (causal) {
+        if (p.seg.nseg > 1) {
+            la::ChunkParams r = prm;
+            r.seg_len = p.seg.seg_len;
+            r.nseg = p.seg.nseg;
+            r.S_out = rec;
+            r.z_out = rec + D * D;
+            r.stride_S = r.stride_z = R;
+            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
+                                                             "chunk_reduce")) != LA_OK)
+                return s;
+            if ((s = launch_state_kernel(0, rec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
+                                         st)) != LA_OK)
+                return s;
+            prm.state_in = rec;
+            prm.in_per_head = 0;
+        }
+        prm.seg_len = p.seg.seg_len;
+        prm.nseg = p.seg.nseg;
+        prm.S_out = S_out;
+        prm.z_out = z_out;
+        prm.stride_S = int64_t(D) * D;
+        prm.stride_z = D;
+        return launch_chunk<D, C, PHI, la::MODE_CAUSAL>(prm, heads * p.seg.nseg, st, "chunk_causal");
+    }
+    // non-causal: segment sums -> totals -> query pass
+    float* tot = reinterpret_cast<float*>(ws + p.tot_off);
+    la::ChunkParams r = prm;
+    r.seg_len = p.seg.seg_len;
+    r.nseg = p.seg.nseg;
+    r.S_out = rec;
+    r.z_out = rec + D * D;
+    r.stride_S = r.stride_z = R;
+    if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st, "chunk_reduce")) !=
+        LA_OK)
+        return s;
+    if ((s = launch_state_kernel(1, rec, tot, nullptr, nullptr, heads, p.seg.nseg, D, st)) != LA_OK)
+        return s;
+    if ((S_out || z_out) &&
+        (s = launch_state_kernel(2, nullptr, tot, S_out, z_out, heads, 1, D, st)) != LA_OK)
+        return s;
+    prm.seg_len = p.qseg.seg_len;
+    prm.nseg = p.qseg.nseg;
+    prm.state_in = tot;
+    prm.in_per_head = 1;
+    return launch_chunk<D, C, PHI, la::MODE_QUERY>(prm, heads * p.qseg.nseg, st, "chunk_query");
+}
+
+template <int PHI>
+la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o, float* S_out,
+                            float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
+                            const FwdPlan& p, char* ws, cudaStream_t st) {
+    if (D == 64)
+        return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, heads, N, causal, p, ws, st);
+    return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, heads, N, causal, p, ws, st);
 }
 
 // ------------------------------------------------------------ generic path
@@ -179,11 +379,10 @@ const char* la_status_string(la_status s) {
 
 size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
                          la_dtype dt) {
-    (void)causal;
     if (check_sizes(B, H, N, D) != LA_OK) return 0;
     if (dt != LA_F32 && dt != LA_BF16) return 0;
     if (B == 0 || H == 0 || N == 0) return 0;
-    if (op == LA_OP_FORWARD) return 0;
+    if (op == LA_OP_FORWARD) return plan_fwd(B, H, N, D, causal, dt).bytes;
     if (op == LA_OP_BACKWARD) return plan_bwd(B, H, N).bytes;
     return 0;
 }
@@ -210,8 +409,17 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
     }
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
-    const size_t need = la_workspace_size(LA_OP_FORWARD, B, H, N, D, causal, dt);
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
+    const FwdPlan plan = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
+    if (plan.bytes > 0 && (workspace == nullptr || workspace_bytes < plan.bytes))
+        return LA_ERR_WORKSPACE;
+    if (plan.fast) {
+        char* ws = static_cast<char*>(workspace);
+        return phi == LA_PHI_ELU1
+                   ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, heads, N, D,
+                                                 causal ? 1 : 0, plan, ws, st)
+                   : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, heads, N, D,
+                                                     causal ? 1 : 0, plan, ws, st);
+    }
     return dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, heads, N, D, causal ? 1 : 0, st);
 }
 

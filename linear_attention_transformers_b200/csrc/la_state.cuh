@@ -1,0 +1,62 @@
+// la_state.cuh — small kernels over per-segment states.
+//
+// States are additive: the state after a run of tokens is the sum of the
+// states of its pieces (S and z are sums over tokens, "Efficient
+// Transformers Survey", Proposition "Linear Attention via Kernel
+// Decomposition", Statement).  A record holds S [D][D] (row = key feature)
+// followed by z [D], float32; records are laid out [head][segment][R] with
+// R = D*D + D.  Every sum below runs over segments in a fixed order, so the
+// results are bitwise reproducible.
+#pragma once
+
+#include "la_common.cuh"
+
+namespace la {
+
+constexpr int kStateThreads = 256;
+
+// rec[h][p] <- sum_{p' < p} rec[h][p'] (exclusive prefix, in place).
+__global__ void __launch_bounds__(kStateThreads)
+state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head) {
+    const size_t h = blockIdx.x / blocks_per_head;
+    const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
+    if (e >= R) return;
+    float* base = rec + h * size_t(nseg) * R + e;
+    float run = 0.f;
+    for (int p = 0; p < nseg; ++p) {
+        const float x = base[size_t(p) * R];
+        base[size_t(p) * R] = run;
+        run += x;
+    }
+}
+
+// out[h] <- sum_p rec[h][p]; out record stride R.
+__global__ void __launch_bounds__(kStateThreads)
+state_sum_kernel(const float* __restrict__ rec, float* __restrict__ out, int nseg, int R,
+                 int blocks_per_head) {
+    const size_t h = blockIdx.x / blocks_per_head;
+    const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
+    if (e >= R) return;
+    const float* base = rec + h * size_t(nseg) * R + e;
+    float run = 0.f;
+    for (int p = 0; p < nseg; ++p) run += base[size_t(p) * R];
+    out[h * size_t(R) + e] = run;
+}
+
+// Split records into the caller's S [h][D][D] and z [h][D] arrays.
+__global__ void __launch_bounds__(kStateThreads)
+state_unpack_kernel(const float* __restrict__ rec, float* __restrict__ S, float* __restrict__ z,
+                    int D, int blocks_per_head) {
+    const size_t h = blockIdx.x / blocks_per_head;
+    const int R = D * D + D;
+    const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
+    if (e >= R) return;
+    const float x = rec[h * size_t(R) + e];
+    if (e < D * D) {
+        if (S) S[h * size_t(D) * D + e] = x;
+    } else if (z) {
+        z[h * size_t(D) + (e - D * D)] = x;
+    }
+}
+
+}  // namespace la
