@@ -28,6 +28,7 @@ op has no runnable upstream implementation; the oracle is the reference arm).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -71,9 +72,13 @@ def algorithmic_bytes(kernel: str, w) -> float:
     """
     e = 2 if w.dtype == torch.bfloat16 else 4
     t = w.B * w.H * w.N * w.D * e  # bytes of one [B,H,N,D] tensor
+    n = w.B * w.H * w.N * 4  # one float32 per token (g or dg)
     table = {
         "fwd_generic": 4 * t,           # q, k, v -> o
         "bwd_generic": 7 * t,           # q, k, v, dO -> dq, dk, dv
+        "chunk_causal": 4 * t,          # q, k, v -> o
+        "bwd_dq": 5 * t + 2 * n,        # q, k, v, dO -> dq, g, dg
+        "bwd_dkdv": 6 * t + 2 * n,      # q, k, v, dO, g, dg -> dk, dv
     }
     return float(table.get(kernel, 0.0))
 
@@ -237,6 +242,16 @@ def run_reference(args, world, rank):
     return 0
 
 
+def workload_from_args(args):
+    """The timed workload, or a reshaped copy of it (--shape B,H,N,D) for
+    small profiling runs."""
+    if not args.shape:
+        return WORKLOAD
+    B, H, N, D = (int(x) for x in args.shape.split(","))
+    return dataclasses.replace(WORKLOAD, name=f"causal_fwdbwd_b{B}h{H}n{N}d{D}_bf16", B=B, H=H,
+                               N=N, D=D)
+
+
 def config_dict(w, gpus):
     return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "D": w.D,
             "causal": w.causal, "phi": "elu1" if w.phi == 0 else "relu_eps",
@@ -247,7 +262,7 @@ def config_dict(w, gpus):
 # --------------------------------------------------------------------- ours
 def run_ours(args, world, rank, local):
     from linear_attention_transformers_b200 import api
-    w = WORKLOAD
+    w = workload_from_args(args)
     dev = torch.device("cuda", local)
     api.load_library()
     q, k, v, dO = (t for t in inputs.make_inputs(w, device=dev))
@@ -377,6 +392,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shape", default="", help="B,H,N,D override (profiling runs only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -142,6 +142,13 @@ LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void
 LA_EXPORT const char *la_status_string(la_status status);
 
 /*
+ * Detail of the most recent LA_ERR_CUDA returned on the calling host thread:
+ * the failing step and the CUDA runtime's error name ("" if none).  The
+ * string stays valid until the thread's next failing call.
+ */
+LA_EXPORT const char *la_last_error(void);
+
+/*
  * Kernels that wait on other thread blocks do so for a bounded number of
  * iterations; when a wait gives up, the kernel records it in a device-side
  * error word and finishes without hanging (its outputs are then invalid).

@@ -50,7 +50,10 @@ class ProfileEntry(ctypes.Structure):
 class LinearAttentionError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {la_status_string(status)} (status {status})")
+        msg = f"{fn} failed: {la_status_string(status)} (status {status})"
+        if status == LA_ERR_CUDA:
+            msg += f" [{la_last_error()}]"
+        super().__init__(msg)
 
 
 def load_library(path: str | None = None):
@@ -78,6 +81,8 @@ def load_library(path: str | None = None):
         lib.la_decode_step.restype = ci
         lib.la_status_string.argtypes = [ci]
         lib.la_status_string.restype = ctypes.c_char_p
+        lib.la_last_error.argtypes = []
+        lib.la_last_error.restype = ctypes.c_char_p
         lib.la_get_device_error.argtypes = [vp]
         lib.la_get_device_error.restype = ci
         lib.la_version.argtypes = []
@@ -94,6 +99,11 @@ def load_library(path: str | None = None):
 
 def la_status_string(status: int) -> str:
     return load_library().la_status_string(int(status)).decode()
+
+
+def la_last_error() -> str:
+    """Detail of the last CUDA failure on this thread ("" if none)."""
+    return load_library().la_last_error().decode()
 
 
 def la_version() -> int:

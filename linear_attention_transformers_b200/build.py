@@ -21,9 +21,13 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "liblinattn.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# The CUDA runtime is linked as a shared library so the library follows the
+# caller's current device and shares its runtime state (torch loads the same
+# libcudart.so.12); the rpath finds the toolkit's copy when loaded alone.
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo", "--expt-relaxed-constexpr",
     "-Xcompiler", "-fPIC,-fvisibility=hidden", "-shared",
+    "-cudart", "shared", "-Xlinker", "-rpath,/usr/local/cuda/lib64",
     "-Xptxas", "-warn-spills",
 ]
 

@@ -8,10 +8,12 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <algorithm>
 
+#include "la_chunk_bwd.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_common.cuh"
 #include "la_decode.cuh"
@@ -54,8 +56,26 @@ la_status check_ptr(const void* p) {
     return LA_OK;
 }
 
+thread_local char g_last_error[160] = "";
+
+la_status cuda_fail(const char* where, cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorName(e));
+    return LA_ERR_CUDA;
+}
+
+// Make the calling thread's current device context current at the driver
+// level too: the runtime binds it lazily, and the tensor-map encoder (a
+// driver call) needs it.  The current device is left unchanged.
+la_status bind_context() {
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail("cudaGetDevice", e);
+    if (cudaError_t e = cudaSetDevice(dev)) return cuda_fail("cudaSetDevice", e);
+    return LA_OK;
+}
+
 la_status launch_status() {
-    return cudaGetLastError() == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LA_OK : cuda_fail("kernel launch", e);
 }
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -106,10 +126,15 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, in
     cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(N) * cuuint64_t(D) * 2};
     cuuint32_t box[3] = {64, cuuint32_t(C), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
-               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "cuTensorMapEncodeTiled: CUresult %d (map at %p, base %p)", int(r),
+                 static_cast<void*>(m), base);
+    return r == CUDA_SUCCESS;
 }
 
 // ------------------------------------------------------------ chunked path
@@ -171,9 +196,8 @@ la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st
                        const char* name) {
     auto kern = la::chunk_fwd_kernel<D, C, PHI, MODE>;
     constexpr int smem = la::ChunkCfg<D, C>::SMEM;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-        return LA_ERR_CUDA;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+        return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope(name, st);
     kern<<<unsigned(grid), la::kChunkThreads, smem, st>>>(prm);
     return launch_status();
@@ -187,6 +211,9 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
     if (which == 0) {
         la::LaunchScope scope("state_scan", st);
         la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
+    } else if (which == 3) {
+        la::LaunchScope scope("state_rscan", st);
+        la::state_exclusive_rscan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
     } else if (which == 1) {
         la::LaunchScope scope("state_sum", st);
         la::state_sum_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, out, nseg, R, bph);
@@ -268,6 +295,162 @@ la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o
     return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, heads, N, causal, p, ws, st);
 }
 
+
+// ------------------------------------------------------------ chunked backward
+struct BwdPlan {
+    bool fast = false;
+    int C = 0;
+    SegSplit seg;   // causal: segments of both passes; non-causal: reduce split
+    SegSplit qseg;  // non-causal: split of the two gradient passes
+    size_t g_off = 0, dg_off = 0, srec_off = 0, stot_off = 0, rrec_off = 0, rtot_off = 0;
+    size_t bytes = 0;
+};
+
+BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
+    BwdPlan p;
+    if (!fast_path(dt, D) || N == 0 || B * H == 0) return p;
+    p.fast = true;
+    p.C = chunk_len(D);
+    const int64_t heads = B * H;
+    const int64_t nch = (N + p.C - 1) / p.C;
+    const size_t R = size_t(D) * D + D;
+    const size_t tok = size_t(heads) * size_t(N) * sizeof(float);
+    size_t off = 0;
+    p.g_off = off;
+    off += round_up(tok, 256);
+    p.dg_off = off;
+    off += round_up(tok, 256);
+    p.seg = split(N, p.C, pick_nseg(heads, nch));
+    if (causal) {
+        p.qseg = p.seg;
+        if (p.seg.nseg > 1) {
+            p.srec_off = off;
+            off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
+            p.rrec_off = off;
+            off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
+        }
+    } else {
+        const int64_t want = heads >= 2 * kNumSM ? 1 : (2 * kNumSM + heads - 1) / heads;
+        p.qseg = split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
+        p.srec_off = off;
+        off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
+        p.stot_off = off;
+        off += round_up(size_t(heads) * R * 4, 256);
+        p.rrec_off = off;
+        off += round_up(size_t(heads) * p.qseg.nseg * R * 4, 256);
+        p.rtot_off = off;
+        off += round_up(size_t(heads) * R * 4, 256);
+    }
+    p.bytes = off;
+    return p;
+}
+
+template <typename Kern>
+la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64_t grid,
+                            cudaStream_t st, const char* name) {
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+        return cuda_fail("cudaFuncSetAttribute", e);
+    la::LaunchScope scope(name, st);
+    kern<<<unsigned(grid), 320, smem, st>>>(prm);
+    return launch_status();
+}
+
+template <int D, int PHI>
+la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                          void* dk, void* dv, int64_t heads, int64_t N, int causal,
+                          const BwdPlan& p, char* ws, cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    la::BwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_do, dO, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dq, dq, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dk, dk, heads, N, D, C) || !make_qkv_map(&prm.tm_dv, dv, heads, N, D, C))
+        return LA_ERR_CUDA;
+    prm.N = int(N);
+    prm.gbuf = reinterpret_cast<float*>(ws + p.g_off);
+    prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
+    const int64_t R = int64_t(D) * D + D;
+    float* srec = reinterpret_cast<float*>(ws + p.srec_off);
+    float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
+    constexpr int smem1 = la::Bwd1Cfg<D, C>::SMEM;
+    constexpr int smem2 = la::Bwd2Cfg<D, C>::SMEM;
+    la_status s;
+
+    // (S, z) of earlier segments / the whole sequence
+    la::ChunkParams red;
+    memset(&red, 0, sizeof(red));
+    red.tm_k = prm.tm_k;
+    red.tm_v = prm.tm_v;
+    red.N = int(N);
+    red.seg_len = p.seg.seg_len;
+    red.nseg = p.seg.nseg;
+    red.S_out = srec;
+    red.z_out = srec + D * D;
+    red.stride_S = red.stride_z = R;
+
+    if (causal) {
+        la::BwdParams p1 = prm, p2 = prm;
+        p1.seg_len = p2.seg_len = p.seg.seg_len;
+        p1.nseg = p2.nseg = p.seg.nseg;
+        if (p.seg.nseg > 1) {
+            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
+                                                             "chunk_reduce")) != LA_OK)
+                return s;
+            if ((s = launch_state_kernel(0, srec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
+                                         st)) != LA_OK)
+                return s;
+            p1.state_in = srec;
+            p1.rec_out = rrec;
+        }
+        if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true>, smem1, p1,
+                                   heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
+            return s;
+        if (p.seg.nseg > 1) {
+            if ((s = launch_state_kernel(3, rrec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
+                                         st)) != LA_OK)
+                return s;
+            p2.state_in = rrec;
+        }
+        return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
+                                 heads * p.seg.nseg, st, "bwd_dkdv");
+    }
+    float* stot = reinterpret_cast<float*>(ws + p.stot_off);
+    float* rtot = reinterpret_cast<float*>(ws + p.rtot_off);
+    if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
+                                                     "chunk_reduce")) != LA_OK)
+        return s;
+    if ((s = launch_state_kernel(1, srec, stot, nullptr, nullptr, heads, p.seg.nseg, D, st)) !=
+        LA_OK)
+        return s;
+    la::BwdParams p1 = prm, p2 = prm;
+    p1.seg_len = p2.seg_len = p.qseg.seg_len;
+    p1.nseg = p2.nseg = p.qseg.nseg;
+    p1.state_in = stot;
+    p1.in_per_head = 1;
+    p1.rec_out = rrec;
+    if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false>, smem1, p1,
+                               heads * p.qseg.nseg, st, "bwd_dq")) != LA_OK)
+        return s;
+    if ((s = launch_state_kernel(1, rrec, rtot, nullptr, nullptr, heads, p.qseg.nseg, D, st)) !=
+        LA_OK)
+        return s;
+    p2.state_in = rtot;
+    p2.in_per_head = 1;
+    return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, false>, smem2, p2,
+                             heads * p.qseg.nseg, st, "bwd_dkdv");
+}
+
+template <int PHI>
+la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO, void* dq,
+                            void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
+                            const BwdPlan& p, char* ws, cudaStream_t st) {
+    if (D == 64)
+        return run_bwd_chunked<64, PHI>(q, k, v, dO, dq, dk, dv, heads, N, causal, p, ws, st);
+    return run_bwd_chunked<128, PHI>(q, k, v, dO, dq, dk, dv, heads, N, causal, p, ws, st);
+}
+
 // ------------------------------------------------------------ generic path
 template <typename T, int PHI>
 la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
@@ -275,9 +458,9 @@ la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, 
                           cudaStream_t st) {
     auto kern = la::fwd_generic_kernel<T, PHI>;
     const size_t smem = la::generic_smem_bytes(int(D));
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return LA_ERR_CUDA;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem)))
+        return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope("fwd_generic", st);
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
@@ -291,9 +474,9 @@ la_status run_bwd_generic(const void* q, const void* k, const void* v, const voi
                           float* gbuf, float* dgbuf, cudaStream_t st) {
     auto kern = la::bwd_generic_kernel<T, PHI>;
     const size_t smem = la::generic_smem_bytes(int(D)) + size_t(D) * sizeof(float);
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
-        cudaSuccess)
-        return LA_ERR_CUDA;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem)))
+        return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope("bwd_generic", st);
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
@@ -365,6 +548,8 @@ extern "C" {
 
 int la_version(void) { return LA_API_VERSION; }
 
+const char* la_last_error(void) { return g_last_error; }
+
 const char* la_status_string(la_status s) {
     switch (s) {
         case LA_OK: return "ok";
@@ -383,7 +568,10 @@ size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, i
     if (dt != LA_F32 && dt != LA_BF16) return 0;
     if (B == 0 || H == 0 || N == 0) return 0;
     if (op == LA_OP_FORWARD) return plan_fwd(B, H, N, D, causal, dt).bytes;
-    if (op == LA_OP_BACKWARD) return plan_bwd(B, H, N).bytes;
+    if (op == LA_OP_BACKWARD) {
+        const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal, dt);
+        return bp.fast ? bp.bytes : plan_bwd(B, H, N).bytes;
+    }
     return 0;
 }
 
@@ -412,6 +600,7 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
     const FwdPlan plan = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
     if (plan.bytes > 0 && (workspace == nullptr || workspace_bytes < plan.bytes))
         return LA_ERR_WORKSPACE;
+    if ((s = bind_context()) != LA_OK) return s;
     if (plan.fast) {
         char* ws = static_cast<char*>(workspace);
         return phi == LA_PHI_ELU1
@@ -439,6 +628,16 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt);
+    if ((s = bind_context()) != LA_OK) return s;
+    if (bp.fast) {
+        char* wsp = static_cast<char*>(workspace);
+        return phi == LA_PHI_ELU1
+                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, dq, dk, dv, heads, N, D,
+                                                 causal ? 1 : 0, bp, wsp, st)
+                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, dq, dk, dv, heads, N, D,
+                                                     causal ? 1 : 0, bp, wsp, st);
+    }
     const BwdWorkspace w = plan_bwd(B, H, N);
     char* ws = static_cast<char*>(workspace);
     float* gbuf = reinterpret_cast<float*>(ws + w.g_off);

@@ -1,0 +1,935 @@
+// la_chunk_bwd.cuh — chunked linear-attention backward on sm_100a tensor cores.
+//
+// Gradients of L = sum(dO * O) (the pages print none; derived from the
+// definition in "Efficient Transformers Survey", Proposition "Linear
+// Attention via Kernel Decomposition", Statement).  Per head, with
+// a = phi(q), b = phi(k), g_i = a_i.z_i and o_i = S_i^T a_i / g_i:
+//
+//   du_i = dO_i / g_i,   dg_i = -(dO_i . o_i) / g_i
+//   dA_i = S_i du_i + z_i dg_i              = sum_{j<=i} b_j (v_j.du_i + dg_i)
+//   dB_j = R_j v_j + r_j                    = sum_{i>=j} a_i (v_j.du_i + dg_i)
+//   dV_j = R_j^T b_j                        = sum_{i>=j} (a_i.b_j) du_i
+//   dQ = dA * phi'(q),  dK = dB * phi'(k)
+//
+// with the suffix sums R_j = sum_{i>=j} a_i du_i^T, r_j = sum_{i>=j} a_i dg_i
+// (non-causal: every sum runs over all tokens).  Neither pass stores an
+// N x D x D tensor; the prefix (S, z) and suffix (R, r) states are rebuilt
+// chunk by chunk, in the spirit of the abstract of "Transformer Based Linear
+// Attention with Optimized GPU Kernel Implementation" (an O(N D^2) forward and
+// backward).
+//
+// Pass 1 (token order) per C-token chunk, S/z = state of earlier chunks:
+//   P = A B^T, num = (P.M) V + A S, g = rowsum(P.M) + A z, o = num / g
+//   du, dg;  W' = ((dU V^T) + dg 1^T).M;  dA = W' B + dU S^T + dg z^T
+//   S += B^T V, z += B^T 1;  saves g, dg;  optionally R += A^T dU, r += A^T dg
+// Pass 2 (reverse token order), R/r = state of later chunks:
+//   X1 = (B A^T).M^T,  X2 = (V dU^T + 1 dg^T).M^T
+//   dV = X1 dU + B R,  dB = X2 A + V R^T + 1 r^T;  R += A^T dU, r += A^T dg
+// (M = lower-triangular mask with the diagonal.)  Both passes use the same
+// warp roles as the forward: TMA producer, phi warpgroup, single-thread MMA
+// issuer, epilogue warpgroup; all waits are bounded.
+#pragma once
+
+#include "la_common.cuh"
+#include "la_sm100.cuh"
+
+namespace la {
+
+struct BwdParams {
+    CUtensorMap tm_q, tm_k, tm_v, tm_do, tm_dq, tm_dk, tm_dv;
+    int N, seg_len, nseg;
+    // pass 1: initial (S, z) record; pass 2: initial (R, r) record.  Record =
+    // [D][D] row-major (row = key feature) then [D].  Index = head
+    // (in_per_head) or block; null = zero state.
+    const float* state_in;
+    int in_per_head;
+    float* gbuf;     // [heads][N] g_i (pass 1 writes, pass 2 reads)
+    float* dgbuf;    // [heads][N] dg_i
+    float* rec_out;  // pass 1: (R, r) of the block's tokens, record per block (nullable)
+};
+
+template <int D, int C>
+struct Bwd1Cfg {
+    static constexpr int NSTAGE = 2;
+    static constexpr int TILE = C * D * 2;
+    static constexpr int STAGE = 4 * TILE;  // Q, K, V, dO
+    static constexpr int OFF_SPREV = NSTAGE * STAGE;
+    static constexpr int OFF_ZOP = OFF_SPREV + D * D * 2;
+    static constexpr int OFF_E = OFF_ZOP + 16 * D * 2;
+    static constexpr int OFF_X = OFF_E + 16 * C * 2;
+    static constexpr int OFF_DU = OFF_X + C * C * 2;
+    static constexpr int OFF_DG = OFF_DU + C * D * 2;
+    static constexpr int OFF_STG = OFF_DG + 16 * C * 2;
+    static constexpr int OFF_ZF = OFF_STG + C * D * 2;
+    static constexpr int OFF_BAR = OFF_ZF + ((D * 4 + 15) / 16) * 16;
+    static constexpr int NBAR = 3 * NSTAGE + 9;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static constexpr int T_P = 0, T_O = C, T_OZ = C + D, T_S = C + D + 16, T_Z = C + 2 * D + 16;
+    static constexpr int T_R = C + 2 * D + 32, T_RZ = C + 3 * D + 32;
+    static constexpr int T_COLS = 512;
+    static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+template <int D, int C>
+struct Bwd2Cfg {
+    static constexpr int NSTAGE = 2;
+    static constexpr int TILE = C * D * 2;
+    static constexpr int OFF_DGT = 4 * TILE;           // in-stage: DG operand [16][C]
+    static constexpr int OFF_DGF = 4 * TILE + 16 * C * 2;  // in-stage: dg float [C]
+    static constexpr int STAGE = ((OFF_DGF + C * 4) + 1023) / 1024 * 1024;
+    static constexpr int OFF_RPREV = NSTAGE * STAGE;
+    static constexpr int OFF_RF = OFF_RPREV + D * D * 2;
+    static constexpr int OFF_X1 = OFF_RF + 1024;
+    static constexpr int OFF_X2 = OFF_X1 + C * C * 2;
+    static constexpr bool STG_ALIAS = C >= D;  // dV/dK staging reuses X1/X2
+    static constexpr int OFF_STGV = STG_ALIAS ? OFF_X1 : OFF_X2 + C * C * 2;
+    static constexpr int OFF_STGK = STG_ALIAS ? OFF_X2 : OFF_STGV + C * D * 2;
+    static constexpr int OFF_BAR = STG_ALIAS ? OFF_X2 + C * C * 2 : OFF_STGK + C * D * 2;
+    static constexpr int NBAR = 3 * NSTAGE + 5;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    static constexpr int T_1 = 0, T_2 = C, T_3 = 0, T_4 = D;
+    static constexpr int T_R = (2 * C > 2 * D ? 2 * C : 2 * D), T_RZ = T_R + D;
+    static constexpr int T_COLS = 512;
+    static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// phi'(x) from the bf16 value a = phi(x) that the MMAs read:
+// elu+1: 1 for x > 0 (a > 1), exp(x) = a otherwise -> min(a, 1);
+// relu+eps: 1 where x > 0, i.e. where a exceeds the x <= 0 value bf16(1e-6).
+template <int PHI>
+__device__ __forceinline__ float dphi_from_phi(float a) {
+    if (PHI == PHI_ELU1) return fminf(a, 1.f);
+    const float floor_val = __bfloat162float(__float2bfloat16_rn(1e-6f));
+    return a > floor_val ? 1.f : 0.f;
+}
+
+// Load a state record into the bf16 operand tile [D][D] (row f) and return
+// row f's last entry (z_f or r_f) in *last.  Rows outside [0, D) skip.
+template <int D>
+__device__ __forceinline__ void load_state_row(const float* rec, int frow, uint8_t* tile,
+                                               float* last) {
+    using namespace sm100;
+    for (int q = 0; q < D / 8; ++q) {
+        float v8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v8[t] = rec ? rec[size_t(frow) * D + q * 8 + t] : 0.f;
+        *reinterpret_cast<uint4*>(tile + tile_chunk_off(D, frow, q)) =
+            make_uint4(pack_bf16(v8[0], v8[1]), pack_bf16(v8[2], v8[3]), pack_bf16(v8[4], v8[5]),
+                       pack_bf16(v8[6], v8[7]));
+    }
+    *last = rec ? rec[size_t(D) * D + frow] : 0.f;
+}
+
+// Write 16 fp32 TMEM values of row `row` as bf16 into a row tile.
+__device__ __forceinline__ void store_row16_bf16(uint8_t* tile, int rows, int row, int col0,
+                                                 const float* v) {
+    using namespace sm100;
+    *reinterpret_cast<uint4*>(tile + tile_chunk_off(rows, row, col0 >> 3)) =
+        make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                   pack_bf16(v[6], v[7]));
+    *reinterpret_cast<uint4*>(tile + tile_chunk_off(rows, row, (col0 >> 3) + 1)) =
+        make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]), pack_bf16(v[12], v[13]),
+                   pack_bf16(v[14], v[15]));
+}
+
+// Read 8 bf16 values (columns 8q..8q+7) of row `row` of a row tile.
+__device__ __forceinline__ void load_chunk8(const uint8_t* tile, int rows, int row, int q,
+                                            float* out) {
+    using namespace sm100;
+    const uint4 x = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(rows, row, q));
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        const float2 f = unpack_bf16(w[t]);
+        out[2 * t] = f.x;
+        out[2 * t + 1] = f.y;
+    }
+}
+
+// ======================================================================
+// Pass 1: dQ (token order), g and dg saved for pass 2.
+// ======================================================================
+template <int D, int C, int PHI, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ BwdParams prm) {
+    using namespace sm100;
+    using Cfg = Bwd1Cfg<D, C>;
+    constexpr int NS = Cfg::NSTAGE;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* phi_done = bars + NS;
+    uint64_t* empty = bars + 2 * NS;     // released by the epilogue (count 128)
+    uint64_t* p_ready = bars + 3 * NS;   // commit: P, A S, A z
+    uint64_t* pt_ready = p_ready + 1;    // 128: masked P in X
+    uint64_t* o_ready = p_ready + 2;     // commit: num complete
+    uint64_t* du_ready = p_ready + 3;    // 128: dU, DG written
+    uint64_t* w_ready = p_ready + 4;     // commit: dU V^T
+    uint64_t* wt_ready = p_ready + 5;    // 128: W' in X
+    uint64_t* da_ready = p_ready + 6;    // commit: dA, state updates
+    uint64_t* s_ready = p_ready + 7;     // 128: state operand for next chunk
+    uint64_t* drain = p_ready + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int tok0 = seg * prm.seg_len;
+    const int tok1 = min(prm.N, tok0 + prm.seg_len);
+    const int nchunks = (tok1 - tok0 + C - 1) / C;
+    const float* st_in =
+        prm.state_in ? prm.state_in + size_t(prm.in_per_head ? head : blockIdx.x) * size_t(D * D + D)
+                     : nullptr;
+    const bool rec = prm.rec_out != nullptr;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&phi_done[s], 128);
+            mbar_init(&empty[s], 128);
+        }
+        mbar_init(p_ready, 1);
+        mbar_init(pt_ready, 128);
+        mbar_init(o_ready, 1);
+        mbar_init(du_ready, 128);
+        mbar_init(w_ready, 1);
+        mbar_init(wt_ready, 128);
+        mbar_init(da_ready, 1);
+        mbar_init(s_ready, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::T_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&prm.tm_q);
+            tma_prefetch_desc(&prm.tm_k);
+            tma_prefetch_desc(&prm.tm_v);
+            tma_prefetch_desc(&prm.tm_do);
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS;
+                if (c >= NS && !mbar_wait(&empty[s], ((c / NS) - 1) & 1, abort_flag)) break;
+                uint8_t* st = smem + s * Cfg::STAGE;
+                mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
+                const int row = tok0 + c * C;
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
+                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row, head);
+                    tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
+                                head);
+                    tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
+                                head);
+                }
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - NS); c < issued; ++c)
+                mbar_wait_drain(&full[c % NS], (c / NS) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t tP = tmem + Cfg::T_P, tO = tmem + Cfg::T_O, tOZ = tmem + Cfg::T_OZ;
+            const uint32_t tS = tmem + Cfg::T_S, tZ = tmem + Cfg::T_Z;
+            const uint32_t tR = tmem + Cfg::T_R, tRZ = tmem + Cfg::T_RZ;
+            const uint32_t sprev = sbase + Cfg::OFF_SPREV, zop = sbase + Cfg::OFF_ZOP;
+            const uint32_t eop = sbase + Cfg::OFF_E, xop = sbase + Cfg::OFF_X;
+            const uint32_t duop = sbase + Cfg::OFF_DU, dgop = sbase + Cfg::OFF_DG;
+            constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);   // [C x C] from two K-major
+            constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);
+            constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);
+            constexpr uint32_t idOZ = idesc_bf16(C, 16, 0, 0);
+            constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);
+            constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);
+            const bool has_init = st_in != nullptr;
+            bool ok = true;
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c % NS;
+                const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
+                const uint32_t vs = qs + 2 * Cfg::TILE;
+                if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait(s_ready, c & 1, abort_flag))) break;
+                tc_fence_after();
+                if (CAUSAL) {
+#pragma unroll
+                    for (int k = 0; k < D; k += 16)
+                        umma_bf16(tP, desc_kmajor(qs, C, k), desc_kmajor(ks, C, k), idCC, k > 0);
+                }
+#pragma unroll
+                for (int k = 0; k < D; k += 16) {
+                    umma_bf16(tO, desc_kmajor(qs, C, k), desc_mnmajor(sprev, D, k), idCD_mn, k > 0);
+                    umma_bf16(tOZ, desc_kmajor(qs, C, k), desc_kmajor(zop, 16, k), idOZ, k > 0);
+                }
+                if (CAUSAL) {
+                    umma_commit(p_ready);
+                    if (!(ok = mbar_wait(pt_ready, c & 1, abort_flag))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(vs, C, k), idCD_mn, 1);
+                }
+                umma_commit(o_ready);
+                if (!(ok = mbar_wait(du_ready, c & 1, abort_flag))) break;
+                tc_fence_after();
+                if (CAUSAL) {
+                    // W = dU V^T
+#pragma unroll
+                    for (int k = 0; k < D; k += 16)
+                        umma_bf16(tP, desc_kmajor(duop, C, k), desc_kmajor(vs, C, k), idCC, k > 0);
+                    umma_commit(w_ready);
+                    if (!(ok = mbar_wait(wt_ready, c & 1, abort_flag))) break;
+                    tc_fence_after();
+                    // dA = W' B
+#pragma unroll
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(ks, C, k), idCD_mn, k > 0);
+                }
+                // dA += dU S^T
+#pragma unroll
+                for (int k = 0; k < D; k += 16)
+                    umma_bf16(tO, desc_kmajor(duop, C, k), desc_kmajor(sprev, D, k), idCD_k,
+                              (CAUSAL || k > 0) ? 1u : 0u);
+                if (CAUSAL) {
+                    // S += B^T V, z += B^T 1
+#pragma unroll
+                    for (int k = 0; k < C; k += 16) {
+                        const uint32_t acc = (c > 0 || has_init || k > 0) ? 1u : 0u;
+                        umma_bf16(tS, desc_mnmajor(ks, C, k), desc_mnmajor(vs, C, k), idDD, acc);
+                        umma_bf16(tZ, desc_mnmajor(ks, C, k), desc_kmajor(eop, 16, k), idD16, acc);
+                    }
+                }
+                if (rec) {
+                    // R += A^T dU, r += A^T [dg_hi; dg_lo]
+#pragma unroll
+                    for (int k = 0; k < C; k += 16) {
+                        const uint32_t acc = (c > 0 || k > 0) ? 1u : 0u;
+                        umma_bf16(tR, desc_mnmajor(qs, C, k), desc_mnmajor(duop, C, k), idDD, acc);
+                        umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgop, 16, k), idD16, acc);
+                    }
+                }
+                umma_commit(da_ready);
+            }
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+    } else if (warp < 6) {
+        // feature map on Q and K (dO is used as loaded)
+        const int u = tid - 64;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS;
+            if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
+            uint8_t* st = smem + s * Cfg::STAGE;
+            const int nvalid = min(C, tok1 - (tok0 + c * C));
+            for (int r = u; r < 2 * C; r += 128) {
+                const bool isk = r >= C;
+                const int row = isk ? r - C : r;
+                uint8_t* tile = st + (isk ? Cfg::TILE : 0);
+                const bool zero = row >= nvalid;
+#pragma unroll
+                for (int q = 0; q < D / 8; ++q) {
+                    uint4* p = reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q));
+                    uint4 x = *p;
+                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 f = unpack_bf16(w[t]);
+                        w[t] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
+                    }
+                    *p = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&phi_done[s]);
+        }
+    } else {
+        const int e = tid - 192;
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int irow = acc_row<C>(sp, lane);
+        const int frow = acc_row<D>(sp, lane);
+        uint8_t* sprev = smem + Cfg::OFF_SPREV;
+        uint8_t* zop = smem + Cfg::OFF_ZOP;
+        uint8_t* eop = smem + Cfg::OFF_E;
+        uint8_t* xop = smem + Cfg::OFF_X;
+        uint8_t* duop = smem + Cfg::OFF_DU;
+        uint8_t* dgop = smem + Cfg::OFF_DG;
+        uint8_t* stg = smem + Cfg::OFF_STG;
+        float* zf = reinterpret_cast<float*>(smem + Cfg::OFF_ZF);
+        __nv_bfloat16* zop_h = reinterpret_cast<__nv_bfloat16*>(zop);
+        __nv_bfloat16* dg_h = reinterpret_cast<__nv_bfloat16*>(dgop);
+        float* gb = prm.gbuf + size_t(head) * prm.N;
+        float* dgb = prm.dgbuf + size_t(head) * prm.N;
+
+        for (int idx = e; idx < 16 * C; idx += 128) {
+            const int r = idx / C, cc = idx % C;
+            *reinterpret_cast<__nv_bfloat16*>(eop + tile_off(16, r, cc)) =
+                __float2bfloat16_rn(r == 0 ? 1.f : 0.f);
+            dg_h[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
+        }
+        for (int idx = e; idx < 16 * D; idx += 128) {
+            const int r = idx / D, cc = idx % D;
+            zop_h[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
+        }
+        named_bar_sync(1, 128);
+        if (frow >= 0) {
+            float z0;
+            load_state_row<D>(st_in, frow, sprev, &z0);
+            const __nv_bfloat16 zh = __float2bfloat16_rn(z0);
+            zop_h[tile_off(16, 0, frow) / 2] = zh;
+            zop_h[tile_off(16, 1, frow) / 2] = __float2bfloat16_rn(z0 - __bfloat162float(zh));
+            zf[frow] = z0;
+        }
+        if (CAUSAL && st_in) {
+            for (int cc = 0; cc < D; cc += 16) {
+                float v16[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    v16[t] = frow >= 0 ? st_in[size_t(frow) * D + cc + t] : 0.f;
+                tmem_st16(tmem + lane_base + Cfg::T_S + cc, v16);
+            }
+            float z16[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) z16[t] = (t == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+            tmem_st16(tmem + lane_base + Cfg::T_Z, z16);
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(s_ready);
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS;
+            const uint8_t* qt = smem + s * Cfg::STAGE;
+            const uint8_t* dot = qt + 3 * Cfg::TILE;
+            const int row0 = tok0 + c * C;
+            const int nvalid = min(C, tok1 - row0);
+            const bool valid = irow >= 0 && irow < nvalid;
+            float den_intra = 0.f;
+            if (CAUSAL) {
+                if (!named_bar_all(1, 128, mbar_wait(p_ready, c & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int j0 = 0; j0 < C; j0 += 32) {
+                    float pv[32];
+                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0, pv);
+                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0 + 16, pv + 16);
+                    tmem_wait_ld();
+                    if (irow >= 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int j = j0 + q * 8 + 2 * t;
+                                w[t] = pack_bf16(j <= irow ? pv[q * 8 + 2 * t] : 0.f,
+                                                 j + 1 <= irow ? pv[q * 8 + 2 * t + 1] : 0.f);
+                                const float2 r = unpack_bf16(w[t]);
+                                den_intra += r.x + r.y;
+                            }
+                            *reinterpret_cast<uint4*>(xop + tile_chunk_off(C, irow, (j0 >> 3) + q)) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(pt_ready);
+            }
+            // ---- o, g, du, dg
+            if (!named_bar_all(1, 128, mbar_wait(o_ready, c & 1, abort_flag))) break;
+            tc_fence_after();
+            float oz[16];
+            tmem_ld16(tmem + lane_base + Cfg::T_OZ, oz);
+            tmem_wait_ld();
+            const float g = den_intra + oz[0] + oz[1];
+            const float ginv = 1.f / g;
+            float dotp = 0.f;
+#pragma unroll 1
+            for (int v0 = 0; v0 < D; v0 += 16) {
+                float ov[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_O + v0, ov);
+                tmem_wait_ld();
+                if (irow >= 0) {
+                    float d8a[8], d8b[8];
+                    load_chunk8(dot, C, irow, v0 >> 3, d8a);
+                    load_chunk8(dot, C, irow, (v0 >> 3) + 1, d8b);
+                    float du16[16];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        dotp = fmaf(d8a[t], ov[t] * ginv, dotp);
+                        dotp = fmaf(d8b[t], ov[8 + t] * ginv, dotp);
+                        du16[t] = valid ? d8a[t] * ginv : 0.f;
+                        du16[8 + t] = valid ? d8b[t] * ginv : 0.f;
+                    }
+                    store_row16_bf16(duop, C, irow, v0, du16);
+                }
+            }
+            const float dg = valid ? -dotp * ginv : 0.f;
+            if (irow >= 0) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(dg);
+                dg_h[tile_off(16, 0, irow) / 2] = h;
+                dg_h[tile_off(16, 1, irow) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
+            }
+            if (valid) {
+                gb[row0 + irow] = g;
+                dgb[row0 + irow] = dg;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(du_ready);
+            if (CAUSAL) {
+                // ---- W' = (dU V^T + dg) masked
+                if (!named_bar_all(1, 128, mbar_wait(w_ready, c & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int j0 = 0; j0 < C; j0 += 32) {
+                    float wv[32];
+                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0, wv);
+                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0 + 16, wv + 16);
+                    tmem_wait_ld();
+                    if (irow >= 0) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t w[4];
+#pragma unroll
+                            for (int t = 0; t < 4; ++t) {
+                                const int j = j0 + q * 8 + 2 * t;
+                                w[t] = pack_bf16(j <= irow ? wv[q * 8 + 2 * t] + dg : 0.f,
+                                                 j + 1 <= irow ? wv[q * 8 + 2 * t + 1] + dg : 0.f);
+                            }
+                            *reinterpret_cast<uint4*>(xop + tile_chunk_off(C, irow, (j0 >> 3) + q)) =
+                                make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(wt_ready);
+            }
+            // ---- dQ = (dA + dg z) * phi'(q)
+            if (!named_bar_all(1, 128, mbar_wait(da_ready, c & 1, abort_flag))) break;
+            tc_fence_after();
+            if (e == 0) bulk_wait_read0();
+            named_bar_sync(1, 128);
+#pragma unroll 1
+            for (int f0 = 0; f0 < D; f0 += 16) {
+                float av[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_O + f0, av);
+                tmem_wait_ld();
+                if (irow >= 0) {
+                    float a8a[8], a8b[8];
+                    load_chunk8(qt, C, irow, f0 >> 3, a8a);
+                    load_chunk8(qt, C, irow, (f0 >> 3) + 1, a8b);
+                    float dq16[16];
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) {
+                        dq16[t] = fmaf(dg, zf[f0 + t], av[t]) * dphi_from_phi<PHI>(a8a[t]);
+                        dq16[8 + t] = fmaf(dg, zf[f0 + 8 + t], av[8 + t]) * dphi_from_phi<PHI>(a8b[t]);
+                    }
+                    store_row16_bf16(stg, C, irow, f0, dq16);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);  // staging complete; every zf read done
+            mbar_arrive(&empty[s]);  // this thread is done with the stage
+            if (e == 0) {
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a)
+                    tma_store_3d(&prm.tm_dq, stg + a * C * 128, a * 64, row0, head);
+                bulk_commit();
+            }
+            // ---- next state operand; segment (R, r) on the last chunk
+            if (CAUSAL) {
+#pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 16) {
+                    float sv[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_S + v0, sv);
+                    tmem_wait_ld();
+                    if (frow >= 0) store_row16_bf16(sprev, D, frow, v0, sv);
+                }
+                float zv[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_Z, zv);
+                tmem_wait_ld();
+                if (frow >= 0) {
+                    const __nv_bfloat16 zh = __float2bfloat16_rn(zv[0]);
+                    zop_h[tile_off(16, 0, frow) / 2] = zh;
+                    zop_h[tile_off(16, 1, frow) / 2] = __float2bfloat16_rn(zv[0] - __bfloat162float(zh));
+                    zf[frow] = zv[0];
+                }
+            }
+            if (rec && c == nchunks - 1) {
+                float* out = prm.rec_out + size_t(blockIdx.x) * (D * D + D);
+#pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 16) {
+                    float rv[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
+                    tmem_wait_ld();
+                    if (frow >= 0)
+                        for (int t = 0; t < 16; ++t) out[size_t(frow) * D + v0 + t] = rv[t];
+                }
+                float rz[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
+                tmem_wait_ld();
+                if (frow >= 0) out[size_t(D) * D + frow] = rz[0] + rz[1];
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(s_ready);
+        }
+        if (e == 0) bulk_wait0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, Cfg::T_COLS);
+}
+
+// ======================================================================
+// Pass 2: dK, dV (reverse token order).
+// ======================================================================
+template <int D, int C, int PHI, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams prm) {
+    using namespace sm100;
+    using Cfg = Bwd2Cfg<D, C>;
+    constexpr int NS = Cfg::NSTAGE;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full = bars;
+    uint64_t* phi_done = bars + NS;
+    uint64_t* empty = bars + 2 * NS;    // released by the epilogue (count 128)
+    uint64_t* x_ready = bars + 3 * NS;  // commit: B A^T, V dU^T
+    uint64_t* xt_ready = x_ready + 1;   // 128: X1, X2 written
+    uint64_t* d_ready = x_ready + 2;    // commit: dV, dB, R
+    uint64_t* r_ready = x_ready + 3;    // 128: R operand for the next (earlier) chunk
+    uint64_t* drain = x_ready + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int tok0 = seg * prm.seg_len;
+    const int tok1 = min(prm.N, tok0 + prm.seg_len);
+    const int nchunks = (tok1 - tok0 + C - 1) / C;
+    const float* st_in =
+        prm.state_in ? prm.state_in + size_t(prm.in_per_head ? head : blockIdx.x) * size_t(D * D + D)
+                     : nullptr;
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&phi_done[s], 128);
+            mbar_init(&empty[s], 128);
+        }
+        mbar_init(x_ready, 1);
+        mbar_init(xt_ready, 128);
+        mbar_init(d_ready, 1);
+        mbar_init(r_ready, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::T_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // chunk processed at step t (reverse order)
+    auto chunk_of = [&](int t) { return nchunks - 1 - t; };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&prm.tm_q);
+            tma_prefetch_desc(&prm.tm_k);
+            tma_prefetch_desc(&prm.tm_v);
+            tma_prefetch_desc(&prm.tm_do);
+            int issued = 0;
+            for (int t = 0; t < nchunks; ++t) {
+                const int s = t % NS;
+                if (t >= NS && !mbar_wait(&empty[s], ((t / NS) - 1) & 1, abort_flag)) break;
+                uint8_t* st = smem + s * Cfg::STAGE;
+                mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
+                const int row = tok0 + chunk_of(t) * C;
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
+                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row, head);
+                    tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
+                                head);
+                    tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
+                                head);
+                }
+                issued = t + 1;
+            }
+            for (int t = max(0, issued - NS); t < issued; ++t)
+                mbar_wait_drain(&full[t % NS], (t / NS) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t t1 = tmem + Cfg::T_1, t2 = tmem + Cfg::T_2, t3 = tmem + Cfg::T_3;
+            const uint32_t t4 = tmem + Cfg::T_4, tR = tmem + Cfg::T_R, tRZ = tmem + Cfg::T_RZ;
+            const uint32_t rprev = sbase + Cfg::OFF_RPREV;
+            const uint32_t x1 = sbase + Cfg::OFF_X1, x2 = sbase + Cfg::OFF_X2;
+            constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);
+            constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);
+            constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);
+            constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);
+            constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);
+            const bool has_init = st_in != nullptr;
+            bool ok = true;
+            for (int t = 0; ok && t < nchunks; ++t) {
+                const int s = t % NS;
+                const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
+                const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                const uint32_t dgs = qs + Cfg::OFF_DGT;
+                if (!(ok = mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag))) break;
+                if (!(ok = mbar_wait(r_ready, t & 1, abort_flag))) break;
+                tc_fence_after();
+                if (CAUSAL) {
+#pragma unroll
+                    for (int k = 0; k < D; k += 16) {
+                        // B A^T and V dU^T
+                        umma_bf16(t1, desc_kmajor(ks, C, k), desc_kmajor(qs, C, k), idCC, k > 0);
+                        umma_bf16(t2, desc_kmajor(vs, C, k), desc_kmajor(dus, C, k), idCC, k > 0);
+                    }
+                    umma_commit(x_ready);
+                    if (!(ok = mbar_wait(xt_ready, t & 1, abort_flag))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < C; k += 16) {
+                        umma_bf16(t3, desc_kmajor(x1, C, k), desc_mnmajor(dus, C, k), idCD_mn, k > 0);
+                        umma_bf16(t4, desc_kmajor(x2, C, k), desc_mnmajor(qs, C, k), idCD_mn, k > 0);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < D; k += 16) {
+                    // dV += B R, dB += V R^T
+                    umma_bf16(t3, desc_kmajor(ks, C, k), desc_mnmajor(rprev, D, k), idCD_mn,
+                              (CAUSAL || k > 0) ? 1u : 0u);
+                    umma_bf16(t4, desc_kmajor(vs, C, k), desc_kmajor(rprev, D, k), idCD_k,
+                              (CAUSAL || k > 0) ? 1u : 0u);
+                }
+                if (CAUSAL) {
+#pragma unroll
+                    for (int k = 0; k < C; k += 16) {
+                        const uint32_t acc = (t > 0 || has_init || k > 0) ? 1u : 0u;
+                        umma_bf16(tR, desc_mnmajor(qs, C, k), desc_mnmajor(dus, C, k), idDD, acc);
+                        umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgs, 16, k), idD16, acc);
+                    }
+                }
+                umma_commit(d_ready);
+            }
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+    } else if (warp < 6) {
+        // phi on Q and K, dU = dO / g, DG rows = (dg_hi, dg_lo)
+        const int u = tid - 64;
+        for (int s = 0; s < NS; ++s) {
+            __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(smem + s * Cfg::STAGE + Cfg::OFF_DGT);
+            for (int idx = u; idx < 16 * C; idx += 128) {
+                const int r = idx / C, cc = idx % C;
+                dgt[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
+            }
+        }
+        const float* gb = prm.gbuf + size_t(head) * prm.N;
+        const float* dgb = prm.dgbuf + size_t(head) * prm.N;
+        for (int t = 0; t < nchunks; ++t) {
+            const int s = t % NS;
+            if (!mbar_wait(&full[s], (t / NS) & 1, abort_flag)) break;
+            uint8_t* st = smem + s * Cfg::STAGE;
+            const int row0 = tok0 + chunk_of(t) * C;
+            const int nvalid = min(C, tok1 - row0);
+            __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(st + Cfg::OFF_DGT);
+            float* dgf = reinterpret_cast<float*>(st + Cfg::OFF_DGF);
+            for (int r = u; r < 3 * C; r += 128) {
+                const int which = r / C;  // 0: Q, 1: K, 2: dO
+                const int row = r % C;
+                const bool zero = row >= nvalid;
+                uint8_t* tile = st + (which == 2 ? 3 : which) * Cfg::TILE;
+                float ginv = 0.f;
+                if (which == 2) {
+                    const float g = zero ? 1.f : gb[row0 + row];
+                    const float dg = zero ? 0.f : dgb[row0 + row];
+                    ginv = 1.f / g;
+                    const __nv_bfloat16 h = __float2bfloat16_rn(dg);
+                    dgt[tile_off(16, 0, row) / 2] = h;
+                    dgt[tile_off(16, 1, row) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
+                    dgf[row] = dg;
+                }
+#pragma unroll
+                for (int q = 0; q < D / 8; ++q) {
+                    uint4* p = reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q));
+                    uint4 x = *p;
+                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 f = unpack_bf16(w[k]);
+                        if (zero)
+                            w[k] = 0u;
+                        else if (which == 2)
+                            w[k] = pack_bf16(f.x * ginv, f.y * ginv);
+                        else
+                            w[k] = pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
+                    }
+                    *p = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&phi_done[s]);
+        }
+    } else {
+        const int e = tid - 192;
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int jrow = acc_row<C>(sp, lane);
+        const int frow = acc_row<D>(sp, lane);
+        uint8_t* rprev = smem + Cfg::OFF_RPREV;
+        float* rf = reinterpret_cast<float*>(smem + Cfg::OFF_RF);
+        uint8_t* x1 = smem + Cfg::OFF_X1;
+        uint8_t* x2 = smem + Cfg::OFF_X2;
+        uint8_t* stgv = smem + Cfg::OFF_STGV;
+        uint8_t* stgk = smem + Cfg::OFF_STGK;
+
+        if (frow >= 0) {
+            float r0;
+            load_state_row<D>(st_in, frow, rprev, &r0);
+            rf[frow] = r0;
+        }
+        if (CAUSAL && st_in) {
+            for (int cc = 0; cc < D; cc += 16) {
+                float v16[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    v16[t] = frow >= 0 ? st_in[size_t(frow) * D + cc + t] : 0.f;
+                tmem_st16(tmem + lane_base + Cfg::T_R + cc, v16);
+            }
+            float z16[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) z16[t] = (t == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+            tmem_st16(tmem + lane_base + Cfg::T_RZ, z16);
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(r_ready);
+
+        for (int t = 0; t < nchunks; ++t) {
+            const int s = t % NS;
+            const uint8_t* st = smem + s * Cfg::STAGE;
+            const uint8_t* kt = st + Cfg::TILE;
+            const float* dgf = reinterpret_cast<const float*>(st + Cfg::OFF_DGF);
+            const int row0 = tok0 + chunk_of(t) * C;
+            if (CAUSAL) {
+                if (!named_bar_all(1, 128, mbar_wait(x_ready, t & 1, abort_flag))) break;
+                tc_fence_after();
+                if (Cfg::STG_ALIAS) {
+                    if (e == 0) bulk_wait_read0();
+                    named_bar_sync(1, 128);
+                }
+#pragma unroll 1
+                for (int i0 = 0; i0 < C; i0 += 16) {
+                    float pv[16], wv[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_1 + i0, pv);
+                    tmem_ld16(tmem + lane_base + Cfg::T_2 + i0, wv);
+                    tmem_wait_ld();
+                    if (jrow >= 0) {
+                        float a16[16], b16[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int i = i0 + k;
+                            a16[k] = i >= jrow ? pv[k] : 0.f;
+                            b16[k] = i >= jrow ? wv[k] + dgf[i] : 0.f;
+                        }
+                        store_row16_bf16(x1, C, jrow, i0, a16);
+                        store_row16_bf16(x2, C, jrow, i0, b16);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(xt_ready);
+            }
+            if (!named_bar_all(1, 128, mbar_wait(d_ready, t & 1, abort_flag))) break;
+            tc_fence_after();
+            if (!Cfg::STG_ALIAS || !CAUSAL) {
+                if (e == 0) bulk_wait_read0();
+                named_bar_sync(1, 128);
+            }
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float dv16[16], db16[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_3 + c0, dv16);
+                tmem_ld16(tmem + lane_base + Cfg::T_4 + c0, db16);
+                tmem_wait_ld();
+                if (jrow >= 0) {
+                    float b8a[8], b8b[8];
+                    load_chunk8(kt, C, jrow, c0 >> 3, b8a);
+                    load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
+                    float dk16[16];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        dk16[k] = (db16[k] + rf[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
+                        dk16[8 + k] = (db16[8 + k] + rf[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
+                    }
+                    store_row16_bf16(stgv, C, jrow, c0, dv16);
+                    store_row16_bf16(stgk, C, jrow, c0, dk16);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);  // staging complete; every rf read done
+            mbar_arrive(&empty[s]);
+            if (e == 0) {
+#pragma unroll
+                for (int a = 0; a < D / 64; ++a) {
+                    tma_store_3d(&prm.tm_dv, stgv + a * C * 128, a * 64, row0, head);
+                    tma_store_3d(&prm.tm_dk, stgk + a * C * 128, a * 64, row0, head);
+                }
+                bulk_commit();
+            }
+            if (CAUSAL) {
+#pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 16) {
+                    float rv[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
+                    tmem_wait_ld();
+                    if (frow >= 0) store_row16_bf16(rprev, D, frow, v0, rv);
+                }
+                float rz[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
+                tmem_wait_ld();
+                if (frow >= 0) rf[frow] = rz[0] + rz[1];
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(r_ready);
+        }
+        if (e == 0) bulk_wait0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, Cfg::T_COLS);
+}
+
+}  // namespace la

@@ -30,6 +30,21 @@ state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks
     }
 }
 
+// rec[h][p] <- sum_{p' > p} rec[h][p'] (exclusive suffix, in place).
+__global__ void __launch_bounds__(kStateThreads)
+state_exclusive_rscan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head) {
+    const size_t h = blockIdx.x / blocks_per_head;
+    const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
+    if (e >= R) return;
+    float* base = rec + h * size_t(nseg) * R + e;
+    float run = 0.f;
+    for (int p = nseg - 1; p >= 0; --p) {
+        const float x = base[size_t(p) * R];
+        base[size_t(p) * R] = run;
+        run += x;
+    }
+}
+
 // out[h] <- sum_p rec[h][p]; out record stride R.
 __global__ void __launch_bounds__(kStateThreads)
 state_sum_kernel(const float* __restrict__ rec, float* __restrict__ out, int nseg, int R,

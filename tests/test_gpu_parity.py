@@ -199,3 +199,28 @@ def test_quadratic_form_small_fp32():
     for causal in (True, False):
         o = api.la_forward(q, k, v, causal)
         compare(o, oracle.quadratic(q, k, v, causal), torch.float32, "quadratic")
+
+
+def test_calls_from_another_host_thread():
+    # A fresh host thread (as torch's autograd worker is) must work: the
+    # library binds the current device's context before its driver calls.
+    import threading
+    q, k, v, dO = small(1, 2, 200, 64, torch.bfloat16, seed=9, dO=True)
+    out = {}
+
+    def worker():
+        try:
+            out["o"] = api.la_forward(q, k, v, True)
+            out["g"] = api.la_backward(q, k, v, dO, True)
+            torch.cuda.synchronize()
+        except Exception as e:  # surfaced below
+            out["err"] = e
+
+    t = threading.Thread(target=worker)
+    t.start()
+    t.join()
+    assert "err" not in out, out.get("err")
+    rq, rk, rv = oracle.backward(q, k, v, dO, True, oracle.PHI_ELU1)
+    compare(out["o"], oracle.forward(q, k, v, True, oracle.PHI_ELU1)[0], torch.bfloat16, "o")
+    for name, g, r in zip(("dq", "dk", "dv"), out["g"], (rq, rk, rv)):
+        compare(g, r, torch.bfloat16, name)
