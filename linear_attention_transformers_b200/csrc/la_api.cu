@@ -15,6 +15,7 @@
 
 #include "la_chunk_bwd.cuh"
 #include "la_chunk_fwd.cuh"
+#include "la_chunk_fwd64.cuh"
 #include "la_common.cuh"
 #include "la_decode.cuh"
 #include "la_generic.cuh"
@@ -194,8 +195,8 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
 template <int D, int C, int PHI, int MODE>
 la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st,
                        const char* name) {
-    auto kern = la::chunk_fwd_kernel<D, C, PHI, MODE>;
-    constexpr int smem = la::ChunkCfg<D, C>::SMEM;
+    auto kern = D == 64 ? la::chunk_fwd64_kernel<PHI, MODE> : la::chunk_fwd_kernel<D, C, PHI, MODE>;
+    constexpr int smem = D == 64 ? la::Chunk64Cfg::SMEM : la::ChunkCfg<D, C>::SMEM;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
         return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope(name, st);

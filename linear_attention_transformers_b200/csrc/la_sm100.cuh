@@ -58,14 +58,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+// One try_wait with a suspend-time hint: the warp sleeps in hardware until the
+// phase completes or about `hint_ns` pass, instead of spinning and taking
+// issue slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
+                                              uint32_t hint_ns = 200000u) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
@@ -78,7 +82,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile 
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if ((it & 3u) == 0) {
             if (*abort) return false;
             if (global_ns() - t0 > kWaitLimitNs) {
                 *abort = 1;
@@ -95,7 +99,7 @@ __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 63u && global_ns() - t0 > kWaitLimitNs) {
+        if ((it & 3u) == 3u && global_ns() - t0 > kWaitLimitNs) {
             atomicOr(&g_device_error, 1u);
             return false;
         }
@@ -249,6 +253,17 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile, int rows, int k) 
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile, int rows, int k) {
     return sdesc_sw128(tile + uint32_t(k) * 128u, uint32_t(rows) * 128u, 1024);
 }
+
+// Base descriptors (k = 0) and the constant offsets that step them along K:
+// adding kstep_*() to a base descriptor moves its start address field.
+__device__ __forceinline__ uint64_t desc_k_base(uint32_t tile) { return sdesc_sw128(tile, 16, 1024); }
+__device__ __forceinline__ uint64_t desc_mn_base(uint32_t tile, int rows) {
+    return sdesc_sw128(tile, uint32_t(rows) * 128u, 1024);
+}
+__host__ __device__ constexpr uint64_t kstep_k(int rows, int k) {
+    return uint64_t(((k / 64) * rows * 128 + (k % 64) * 2) >> 4);
+}
+__host__ __device__ constexpr uint64_t kstep_mn(int k) { return uint64_t((k * 128) >> 4); }
 
 // Instruction descriptor: kind::f16 with bf16 A/B, fp32 D, dense.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {

@@ -1,0 +1,97 @@
+// la_tile_ops.cuh — elementwise passes over swizzled bf16 row tiles in
+// shared memory (see la_sm100.cuh for the layout), shared by the chunked
+// kernels.
+#pragma once
+
+#include "la_common.cuh"
+#include "la_sm100.cuh"
+
+namespace la {
+
+// Apply the feature map in place to a [C][D] bf16 row tile.  The T threads
+// calling this split the tile's C*D/8 16-byte chunks evenly; each thread
+// loads all of its chunks before it computes so their latencies overlap.
+// Rows >= nvalid are written as zero when `zero_tail` (a partial last chunk:
+// those keys must not reach the state).
+template <int PHI, int C, int D, int T>
+__device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool zero_tail) {
+    using namespace sm100;
+    constexpr int CH = D / 8;
+    constexpr int PER = (C * CH) / T;
+    static_assert(PER >= 1 && (C * CH) % T == 0 && CH % PER == 0, "work split");
+    const int first = t * PER;
+    const int row = first / CH, q0 = first % CH;
+    uint4 x[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        x[i] = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q0 + i));
+    const bool zero = zero_tail && row >= nvalid;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16(w[k]);
+            w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
+        }
+        x[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + i)) = x[i];
+}
+
+// Scale rows of a [C][D] bf16 row tile in place: row r times rs[r] (rows >=
+// nvalid become zero).  Same work split as phi_tile.
+template <int C, int D, int T>
+__device__ __forceinline__ void scale_tile_rows(uint8_t* tile, int t, int nvalid, const float* rs) {
+    using namespace sm100;
+    constexpr int CH = D / 8;
+    constexpr int PER = (C * CH) / T;
+    static_assert(PER >= 1 && (C * CH) % T == 0 && CH % PER == 0, "work split");
+    const int first = t * PER;
+    const int row = first / CH, q0 = first % CH;
+    uint4 x[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        x[i] = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q0 + i));
+    const float sc = row < nvalid ? rs[row] : 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16(w[k]);
+            w[k] = pack_bf16(f.x * sc, f.y * sc);
+        }
+        x[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + i)) = x[i];
+}
+
+// Write n x 16 fp32 values of row `row` (columns col0..col0+16n-1) as bf16
+// into a row tile with `rows` rows.
+template <int NV>
+__device__ __forceinline__ void store_row_bf16(uint8_t* tile, int rows, int row, int col0,
+                                               const float* v) {
+    using namespace sm100;
+#pragma unroll
+    for (int j = 0; j < NV / 8; ++j) {
+        const float* x = v + 8 * j;
+        *reinterpret_cast<uint4*>(tile + tile_chunk_off(rows, row, (col0 >> 3) + j)) =
+            make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                       pack_bf16(x[6], x[7]));
+    }
+}
+
+// Load NV consecutive TMEM columns of this thread's lane (NV multiple of 16).
+template <int NV>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, float* v) {
+#pragma unroll
+    for (int j = 0; j < NV / 16; ++j) sm100::tmem_ld16(taddr + 16 * j, v + 16 * j);
+    sm100::tmem_wait_ld();
+}
+
+}  // namespace la
