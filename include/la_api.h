@@ -138,6 +138,34 @@ LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void
                          const void *v, void *o, int64_t B, int64_t H, int64_t D,
                          la_dtype dt, la_phi phi, la_stream_t stream);
 
+/*
+ * la_backward_noalloc — la_backward without a caller-provided workspace, for
+ * callers that cannot allocate device memory at call time: code running
+ * inside a CUDA stream capture, under a memory-pool or allocator policy that
+ * forbids new allocations, or in plugins handed only their input and output
+ * buffers.  The paper has no counterpart to this entry point; it exists for
+ * those callers only.
+ *
+ * Instead of a workspace it uses one scratch array of LA_NOALLOC_MAX_BYTES
+ * bytes that the library reserves statically in device memory; every GPU
+ * that loads the library holds that array until the process exits.
+ * Arguments and results are exactly those of la_backward.  The first call
+ * on a device resolves the array's device address (a runtime call); make
+ * that first call before any stream capture.  Calls whose scratch need
+ * (la_workspace_size(LA_OP_BACKWARD, ...)) exceeds LA_NOALLOC_MAX_BYTES are
+ * rejected with LA_ERR_WORKSPACE and nothing is launched.  All calls share
+ * the one array and it keeps the last call's contents, so calls that
+ * overlap on the GPU (other streams, other host threads) race: serialise
+ * them.  No device memory is allocated or freed by this call.
+ */
+#define LA_NOALLOC_MAX_BYTES (64u << 20)
+
+LA_EXPORT la_status la_backward_noalloc(const void *q, const void *k, const void *v,
+                                        const void *dO, void *dq, void *dk, void *dv,
+                                        int64_t B, int64_t H, int64_t N, int64_t D,
+                                        la_dtype dt, int causal, la_phi phi,
+                                        la_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 LA_EXPORT const char *la_status_string(la_status status);
 

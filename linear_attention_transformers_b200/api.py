@@ -77,6 +77,9 @@ def load_library(path: str | None = None):
         lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
                                     vp, sz, vp]
         lib.la_backward.restype = ci
+        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci,
+                                            ci, ci, vp]
+        lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
         lib.la_status_string.argtypes = [ci]
@@ -200,6 +203,31 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
                          B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
                          ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
+    return dq, dk, dv
+
+
+def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None,
+                        dv=None, stream=None):
+    """la_backward on the library's static device scratch (no workspace).
+
+    For callers that cannot allocate device memory during the call; see
+    la_backward_noalloc in include/la_api.h for the limits (a fixed maximum
+    scratch size, one shared scratch array: overlapping calls race).  Output
+    tensors must be passed in to avoid allocation here as well.
+    """
+    lib = load_library()
+    _check_qkv("la_backward_noalloc", q, k, v, dO)
+    if q.dim() != 4:
+        raise ValueError("la_backward_noalloc: tensors must be [B, H, N, D]")
+    B, H, N, D = q.shape
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _check_qkv("la_backward_noalloc", q, dq, dk, dv)
+    st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, H, N, D, DTYPE[q.dtype], int(bool(causal)),
+                                 _phi(phi), _stream_handle(stream))
+    _check("la_backward_noalloc", st)
     return dq, dk, dv
 
 

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "la_chunk_bwd.cuh"
 #include "la_chunk_fwd.cuh"
@@ -545,6 +546,38 @@ struct DecodeOp {
 
 }  // namespace
 
+// ------------------------------------------------------------ static scratch
+// Scratch for la_backward_noalloc: a fixed array in device memory, reserved
+// when the library's device code is loaded on a GPU.  Host code must not use
+// the symbol as an address; the device address comes from
+// cudaGetSymbolAddress, resolved once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[LA_NOALLOC_MAX_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (resolved on
+// the first call for that device).
+la_status static_scratch(void** out) {
+    int dev = 0;
+    if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch))
+            return cuda_fail("cudaGetSymbolAddress", e);
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return LA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int la_version(void) { return LA_API_VERSION; }
@@ -645,6 +678,27 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     float* dgbuf = reinterpret_cast<float*>(ws + w.dg_off);
     return dispatch<BwdOp>(dt, phi, q, k, v, dO, dq, dk, dv, heads, N, D, causal ? 1 : 0, gbuf,
                            dgbuf, st);
+}
+
+la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
+                              void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
+                              int64_t D, la_dtype dt, int causal, la_phi phi,
+                              la_stream_t stream) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
+    if (need > size_t(LA_NOALLOC_MAX_BYTES)) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "la_backward_noalloc: needs %zu bytes of scratch, limit %u", need,
+                 unsigned(LA_NOALLOC_MAX_BYTES));
+        return LA_ERR_WORKSPACE;
+    }
+    if ((s = bind_context()) != LA_OK) return s;
+    void* scratch = nullptr;
+    if ((s = static_scratch(&scratch)) != LA_OK) return s;
+    return la_backward(q, k, v, dO, dq, dk, dv, B, H, N, D, dt, causal, phi, scratch,
+                       size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 
 la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
