@@ -353,7 +353,7 @@ la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
         return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope(name, st);
-    kern<<<unsigned(grid), 320, smem, st>>>(prm);
+    kern<<<unsigned(grid), la::kBwdThreads, smem, st>>>(prm);
     return launch_status();
 }
 

@@ -32,6 +32,7 @@
 
 #include "la_common.cuh"
 #include "la_sm100.cuh"
+#include "la_tile_ops.cuh"
 
 namespace la {
 
@@ -78,7 +79,8 @@ struct Bwd2Cfg {
     static constexpr int TILE = C * D * 2;
     static constexpr int OFF_DGT = 4 * TILE;           // in-stage: DG operand [16][C]
     static constexpr int OFF_DGF = 4 * TILE + 16 * C * 2;  // in-stage: dg float [C]
-    static constexpr int STAGE = ((OFF_DGF + C * 4) + 1023) / 1024 * 1024;
+    static constexpr int OFF_RINV = OFF_DGF + C * 4;       // in-stage: 1/g float [C]
+    static constexpr int STAGE = ((OFF_RINV + C * 4) + 1023) / 1024 * 1024;
     static constexpr int OFF_RPREV = NSTAGE * STAGE;
     static constexpr int OFF_RF = OFF_RPREV + D * D * 2;
     static constexpr int OFF_X1 = OFF_RF + 1024;
@@ -153,8 +155,10 @@ __device__ __forceinline__ void load_chunk8(const uint8_t* tile, int rows, int r
 // ======================================================================
 // Pass 1: dQ (token order), g and dg saved for pass 2.
 // ======================================================================
+constexpr int kBwdThreads = 448;  // producer, MMA, 8 phi warps, 4 epilogue warps
+
 template <int D, int C, int PHI, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ BwdParams prm) {
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd1Cfg<D, C>;
     constexpr int NS = Cfg::NSTAGE;
@@ -191,7 +195,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&phi_done[s], 128);
+            mbar_init(&phi_done[s], 256);
             mbar_init(&empty[s], 128);
         }
         mbar_init(p_ready, 1);
@@ -327,37 +331,23 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
         }
-    } else if (warp < 6) {
-        // feature map on Q and K (dO is used as loaded)
-        const int u = tid - 64;
+    } else if (warp < 10) {
+        // feature map on Q and K (dO is used as loaded); 8 warps, batched loads
+        const int u = tid - 64;  // 0..255
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
             uint8_t* st = smem + s * Cfg::STAGE;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
-            for (int r = u; r < 2 * C; r += 128) {
-                const bool isk = r >= C;
-                const int row = isk ? r - C : r;
-                uint8_t* tile = st + (isk ? Cfg::TILE : 0);
-                const bool zero = row >= nvalid;
-#pragma unroll
-                for (int q = 0; q < D / 8; ++q) {
-                    uint4* p = reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q));
-                    uint4 x = *p;
-                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 f = unpack_bf16(w[t]);
-                        w[t] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
-                    }
-                    *p = make_uint4(w[0], w[1], w[2], w[3]);
-                }
-            }
+            if (u < 128)
+                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+            else
+                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
         }
     } else {
-        const int e = tid - 192;
+        const int e = tid - 320;
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int irow = acc_row<C>(sp, lane);
@@ -603,7 +593,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dq_kernel(const __grid_constant__ 
 // Pass 2: dK, dV (reverse token order).
 // ======================================================================
 template <int D, int C, int PHI, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams prm) {
+__global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd2Cfg<D, C>;
     constexpr int NS = Cfg::NSTAGE;
@@ -635,7 +625,7 @@ __global__ void __launch_bounds__(320, 1) bwd_dkdv_kernel(const __grid_constant_
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&phi_done[s], 128);
+            mbar_init(&phi_done[s], 256);
             mbar_init(&empty[s], 128);
         }
         mbar_init(x_ready, 1);
@@ -743,12 +733,12 @@ __global__ void __launch_bounds__(320, 1) bwd_dkdv_kernel(const __grid_constant_
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
         }
-    } else if (warp < 6) {
-        // phi on Q and K, dU = dO / g, DG rows = (dg_hi, dg_lo)
-        const int u = tid - 64;
+    } else if (warp < 10) {
+        // phi on Q and K, dU = dO / g, DG rows = (dg_hi, dg_lo); 8 warps
+        const int u = tid - 64;  // 0..255
         for (int s = 0; s < NS; ++s) {
             __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(smem + s * Cfg::STAGE + Cfg::OFF_DGT);
-            for (int idx = u; idx < 16 * C; idx += 128) {
+            for (int idx = u; idx < 16 * C; idx += 256) {
                 const int r = idx / C, cc = idx % C;
                 dgt[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
             }
@@ -763,44 +753,27 @@ __global__ void __launch_bounds__(320, 1) bwd_dkdv_kernel(const __grid_constant_
             const int nvalid = min(C, tok1 - row0);
             __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(st + Cfg::OFF_DGT);
             float* dgf = reinterpret_cast<float*>(st + Cfg::OFF_DGF);
-            for (int r = u; r < 3 * C; r += 128) {
-                const int which = r / C;  // 0: Q, 1: K, 2: dO
-                const int row = r % C;
-                const bool zero = row >= nvalid;
-                uint8_t* tile = st + (which == 2 ? 3 : which) * Cfg::TILE;
-                float ginv = 0.f;
-                if (which == 2) {
-                    const float g = zero ? 1.f : gb[row0 + row];
-                    const float dg = zero ? 0.f : dgb[row0 + row];
-                    ginv = 1.f / g;
-                    const __nv_bfloat16 h = __float2bfloat16_rn(dg);
-                    dgt[tile_off(16, 0, row) / 2] = h;
-                    dgt[tile_off(16, 1, row) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
-                    dgf[row] = dg;
-                }
-#pragma unroll
-                for (int q = 0; q < D / 8; ++q) {
-                    uint4* p = reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q));
-                    uint4 x = *p;
-                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const float2 f = unpack_bf16(w[k]);
-                        if (zero)
-                            w[k] = 0u;
-                        else if (which == 2)
-                            w[k] = pack_bf16(f.x * ginv, f.y * ginv);
-                        else
-                            w[k] = pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
-                    }
-                    *p = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+            float* rinv = reinterpret_cast<float*>(st + Cfg::OFF_RINV);
+            if (u < C) {
+                const bool valid = u < nvalid;
+                const float dg = valid ? dgb[row0 + u] : 0.f;
+                rinv[u] = valid ? 1.f / gb[row0 + u] : 0.f;
+                const __nv_bfloat16 h = __float2bfloat16_rn(dg);
+                dgt[tile_off(16, 0, u) / 2] = h;
+                dgt[tile_off(16, 1, u) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
+                dgf[u] = dg;
             }
+            named_bar_sync(3, 256);  // rinv ready
+            if (u < 128)
+                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+            else
+                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+            scale_tile_rows<C, D, 256>(st + 3 * Cfg::TILE, u, nvalid, rinv);
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
         }
     } else {
-        const int e = tid - 192;
+        const int e = tid - 320;
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int jrow = acc_row<C>(sp, lane);
