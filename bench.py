@@ -4,8 +4,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step is one training pass of the attention layer on the timed workload
-(causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward followed by
-la_backward through the library's Python binding, inputs resident in HBM.
+(causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward (which also
+keeps the per-token denominators g) followed by la_backward given O and g,
+through the library's Python binding, inputs resident in HBM.
 The inputs (4 x 128 MiB) are larger than the 126 MB L2, so consecutive steps
 cannot serve each other from cache.  W untimed warm-up steps, then exactly K
 steps between two barrier + synchronize points, timed with CUDA events on the
@@ -76,8 +77,8 @@ def algorithmic_bytes(kernel: str, w) -> float:
     table = {
         "fwd_generic": 4 * t,           # q, k, v -> o
         "bwd_generic": 7 * t,           # q, k, v, dO -> dq, dk, dv
-        "chunk_causal": 4 * t,          # q, k, v -> o
-        "bwd_dq": 5 * t + 2 * n,        # q, k, v, dO -> dq, g, dg
+        "chunk_causal": 4 * t + n,      # q, k, v -> o, g
+        "bwd_dq": 6 * t + 2 * n,        # q, k, v, dO, o, g -> dq, dg
         "bwd_dkdv": 6 * t + 2 * n,      # q, k, v, dO, g, dg -> dk, dv
     }
     return float(table.get(kernel, 0.0))
@@ -268,6 +269,7 @@ def run_ours(args, world, rank, local):
     q, k, v, dO = (t for t in inputs.make_inputs(w, device=dev))
     B, H, N, D = q.shape
     o = torch.empty_like(q)
+    g = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws_f = api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal, w.dtype)
     ws_b = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, w.causal, w.dtype)
@@ -275,9 +277,10 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream)
+        # forward keeps its denominators g; backward reuses O and g
+        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream, g=g)
         api.la_backward(q, k, v, dO, w.causal, w.phi, dq=dq, dk=dk, dv=dv, workspace=ws,
-                        stream=stream)
+                        stream=stream, o=o, g=g)
 
     for _ in range(args.warmup):
         step()
@@ -325,6 +328,8 @@ def run_ours(args, world, rank, local):
                     "share_of_step": tot_ms / max(ms, 1e-9)}
     kernels = {k: {"launches": n, "total_ms": t, "share": t / max(ms, 1e-9)}
                for k, (n, t) in prof.items()}
+    # the method's minimum: forward reads q, k, v and writes o; backward reads
+    # q, k, v, dO and writes dq, dk, dv (22 bytes x D per token and head)
     step_bytes = algorithmic_bytes("fwd_generic", w) + algorithmic_bytes("bwd_generic", w)
     step_frac = (step_bytes / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"]
 

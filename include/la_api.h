@@ -100,26 +100,33 @@ LA_EXPORT size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, in
  * causal != 0 selects the prefix sums j <= i.  S_out [B, H, D, D] (row = key
  * feature f, column = value index) and z_out [B, H, D], float32, may each be
  * NULL; when given they receive the state after all N tokens (both modes),
- * which la_decode_step can continue from.  Workspace: see la_workspace_size;
- * may be NULL when that is 0.
+ * which la_decode_step can continue from.  g_out [B, H, N], float32, may be
+ * NULL; when given it receives the denominators g_i = phi(q_i) . z_i, which
+ * la_backward accepts together with o to skip recomputing the forward.
+ * Workspace: see la_workspace_size; may be NULL when that is 0.
  * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE,
  * LA_ERR_CUDA.  On error nothing has been launched except for LA_ERR_CUDA,
  * where earlier launches of the same call may have run.
  */
 LA_EXPORT la_status la_forward(const void *q, const void *k, const void *v, void *o,
-                     float *S_out, float *z_out,
+                     float *S_out, float *z_out, float *g_out,
                      int64_t B, int64_t H, int64_t N, int64_t D,
                      la_dtype dt, int causal, la_phi phi,
                      void *workspace, size_t workspace_bytes, la_stream_t stream);
 
 /*
  * Backward pass of L = sum(dO * O) for the same forward.  q, k, v, dO
- * (read) and dq, dk, dv (written): [B, H, N, D] of dtype `dt`.  The forward
- * is recomputed inside (no saved O or state is needed) and no N x D x D
- * tensor is ever stored: the prefix states are rebuilt chunk by chunk.
- * dq/dk/dv must not alias the inputs.  Errors as la_forward.
+ * (read) and dq, dk, dv (written): [B, H, N, D] of dtype `dt`.  o (the
+ * forward's output, [B, H, N, D] of dtype `dt`) and g (the forward's g_out,
+ * float32 [B, H, N]) are optional and go together: when both are NULL the
+ * forward quantities are recomputed inside; when both are given they are
+ * used instead (dU = dO/g and dg = -(dO . o)/g directly), which is faster.
+ * No N x D x D tensor is ever stored: the prefix states are rebuilt chunk by
+ * chunk.  dq/dk/dv must not alias the inputs.  Errors as la_forward; one of
+ * o, g without the other is LA_ERR_INVALID_ARG.
  */
 LA_EXPORT la_status la_backward(const void *q, const void *k, const void *v, const void *dO,
+                      const void *o, const float *g,
                       void *dq, void *dk, void *dv,
                       int64_t B, int64_t H, int64_t N, int64_t D,
                       la_dtype dt, int causal, la_phi phi,
@@ -161,7 +168,8 @@ LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void
 #define LA_NOALLOC_MAX_BYTES (64u << 20)
 
 LA_EXPORT la_status la_backward_noalloc(const void *q, const void *k, const void *v,
-                                        const void *dO, void *dq, void *dk, void *dv,
+                                        const void *dO, const void *o, const float *g,
+                                        void *dq, void *dk, void *dv,
                                         int64_t B, int64_t H, int64_t N, int64_t D,
                                         la_dtype dt, int causal, la_phi phi,
                                         la_stream_t stream);

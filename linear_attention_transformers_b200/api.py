@@ -71,14 +71,14 @@ def load_library(path: str | None = None):
         vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.la_workspace_size.argtypes = [ci, i64, i64, i64, i64, ci, ci]
         lib.la_workspace_size.restype = sz
-        lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp, sz,
-                                   vp]
+        lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp,
+                                   sz, vp]
         lib.la_forward.restype = ci
-        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
-                                    vp, sz, vp]
+        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci,
+                                    ci, ci, vp, sz, vp]
         lib.la_backward.restype = ci
-        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci,
-                                            ci, ci, vp]
+        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                            i64, ci, ci, ci, vp]
         lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
@@ -163,8 +163,12 @@ def _workspace(op, q, causal, workspace):
 
 
 def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=False,
-               workspace=None, stream=None):
-    """o = linear attention of q, k, v [B, H, N, D]; optionally the final (S, z)."""
+               workspace=None, stream=None, g=None):
+    """o = linear attention of q, k, v [B, H, N, D]; optionally the final (S, z).
+
+    ``g``: optional float32 [B, H, N] tensor that receives the denominators;
+    pass it with ``o`` to la_backward to skip the forward recompute there.
+    """
     lib = load_library()
     _check_qkv("la_forward", q, k, v)
     if q.dim() != 4:
@@ -178,17 +182,34 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     if return_state:
         S = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
         z = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
+                          or not g.is_contiguous() or g.device != q.device):
+        raise ValueError("la_forward: g must be contiguous float32 [B, H, N] on q's device")
     ws, ws_bytes = _workspace(LA_OP_FORWARD, q, causal, workspace)
-    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, H, N, D,
+    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g), B, H, N, D,
                         DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
                         _stream_handle(stream))
     _check("la_forward", st)
     return (o, S, z) if return_state else o
 
 
+def _check_saved(name, q, o, g):
+    if (o is None) != (g is None):
+        raise ValueError(f"{name}: pass both o and g (saved forward statistics) or neither")
+    if o is not None:
+        _check_qkv(name, q, o)
+        B, H, N, _ = q.shape
+        if g.dtype != torch.float32 or tuple(g.shape) != (B, H, N) or not g.is_contiguous():
+            raise ValueError(f"{name}: g must be contiguous float32 [B, H, N]")
+
+
 def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, dv=None,
-                workspace=None, stream=None):
-    """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi)."""
+                workspace=None, stream=None, o=None, g=None):
+    """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi).
+
+    ``o``, ``g``: the forward's output and denominators (la_forward(..., g=g));
+    when given, the backward does not recompute them.
+    """
     lib = load_library()
     _check_qkv("la_backward", q, k, v, dO)
     if q.dim() != 4:
@@ -198,8 +219,10 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward", q, dq, dk, dv)
+    _check_saved("la_backward", q, o, g)
     ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
-    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk), _ptr(dv),
+    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
+                         _ptr(dk), _ptr(dv),
                          B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
                          ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
@@ -207,7 +230,7 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
 
 
 def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None,
-                        dv=None, stream=None):
+                        dv=None, stream=None, o=None, g=None):
     """la_backward on the library's static device scratch (no workspace).
 
     For callers that cannot allocate device memory during the call; see
@@ -224,8 +247,9 @@ def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, d
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward_noalloc", q, dq, dk, dv)
-    st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, H, N, D, DTYPE[q.dtype], int(bool(causal)),
+    _check_saved("la_backward_noalloc", q, o, g)
+    st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), B, H, N, D, DTYPE[q.dtype], int(bool(causal)),
                                  _phi(phi), _stream_handle(stream))
     _check("la_backward_noalloc", st)
     return dq, dk, dv
@@ -280,13 +304,18 @@ class LinearAttention(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, causal=True, phi="elu1"):
-        ctx.save_for_backward(q, k, v)
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        B, H, N, _ = q.shape
+        g = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+        o = la_forward(q, k, v, causal, phi, g=g)
+        # the output and its denominators are kept so the backward need not
+        # recompute the forward
+        ctx.save_for_backward(q, k, v, o, g)
         ctx.causal, ctx.phi = causal, phi
-        return la_forward(q.contiguous(), k.contiguous(), v.contiguous(), causal, phi)
+        return o
 
     @staticmethod
     def backward(ctx, dO):
-        q, k, v = ctx.saved_tensors
-        dq, dk, dv = la_backward(q.contiguous(), k.contiguous(), v.contiguous(),
-                                 dO.contiguous(), ctx.causal, ctx.phi)
+        q, k, v, o, g = ctx.saved_tensors
+        dq, dk, dv = la_backward(q, k, v, dO.contiguous(), ctx.causal, ctx.phi, o=o, g=g)
         return dq, dk, dv, None, None

@@ -228,8 +228,8 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
 
 template <int D, int PHI>
 la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, float* S_out,
-                          float* z_out, int64_t heads, int64_t N, int causal, const FwdPlan& p,
-                          char* ws, cudaStream_t st) {
+                          float* z_out, float* g_out, int64_t heads, int64_t N, int causal,
+                          const FwdPlan& p, char* ws, cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
     la::ChunkParams prm;
     memset(&prm, 0, sizeof(prm));
@@ -237,6 +237,7 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
         !make_qkv_map(&prm.tm_v, v, heads, N, D, C) || !make_qkv_map(&prm.tm_o, o, heads, N, D, C))
         return LA_ERR_CUDA;
     prm.N = int(N);
+    prm.g_out = g_out;
     const int64_t R = int64_t(D) * D + D;
     float* rec = reinterpret_cast<float*>(ws + p.rec_off);
     la_status s;
@@ -290,11 +291,12 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
 
 template <int PHI>
 la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o, float* S_out,
-                            float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
-                            const FwdPlan& p, char* ws, cudaStream_t st) {
+                            float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
+                            int causal, const FwdPlan& p, char* ws, cudaStream_t st) {
     if (D == 64)
-        return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, heads, N, causal, p, ws, st);
-    return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, heads, N, causal, p, ws, st);
+        return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, causal, p, ws,
+                                        st);
+    return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, causal, p, ws, st);
 }
 
 
@@ -349,18 +351,19 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
 
 template <typename Kern>
 la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64_t grid,
-                            cudaStream_t st, const char* name) {
+                            cudaStream_t st, const char* name, int threads = la::kBwdThreads) {
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
         return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope(name, st);
-    kern<<<unsigned(grid), la::kBwdThreads, smem, st>>>(prm);
+    kern<<<unsigned(grid), threads, smem, st>>>(prm);
     return launch_status();
 }
 
 template <int D, int PHI>
-la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO, void* dq,
-                          void* dk, void* dv, int64_t heads, int64_t N, int causal,
-                          const BwdPlan& p, char* ws, cudaStream_t st) {
+la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO,
+                          const void* o_saved, const float* g_saved, void* dq, void* dk, void* dv,
+                          int64_t heads, int64_t N, int causal, const BwdPlan& p, char* ws,
+                          cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
     la::BwdParams prm;
     memset(&prm, 0, sizeof(prm));
@@ -371,8 +374,12 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
         !make_qkv_map(&prm.tm_dk, dk, heads, N, D, C) || !make_qkv_map(&prm.tm_dv, dv, heads, N, D, C))
         return LA_ERR_CUDA;
     prm.N = int(N);
-    prm.gbuf = reinterpret_cast<float*>(ws + p.g_off);
+    const bool saved = o_saved != nullptr && g_saved != nullptr;
+    // with saved statistics g is the caller's (read only); otherwise pass 1
+    // writes it to the workspace
+    prm.gbuf = saved ? const_cast<float*>(g_saved) : reinterpret_cast<float*>(ws + p.g_off);
     prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
+    prm.o_in = static_cast<const __nv_bfloat16*>(o_saved);
     const int64_t R = int64_t(D) * D + D;
     float* srec = reinterpret_cast<float*>(ws + p.srec_off);
     float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
@@ -406,8 +413,10 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
             p1.state_in = srec;
             p1.rec_out = rrec;
         }
-        if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true>, smem1, p1,
-                                   heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
+        if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
+                                           heads * p.seg.nseg, st, "bwd_dq")
+                       : launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, false>, smem1, p1,
+                                           heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
             return s;
         if (p.seg.nseg > 1) {
             if ((s = launch_state_kernel(3, rrec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
@@ -432,8 +441,10 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     p1.state_in = stot;
     p1.in_per_head = 1;
     p1.rec_out = rrec;
-    if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false>, smem1, p1,
-                               heads * p.qseg.nseg, st, "bwd_dq")) != LA_OK)
+    if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, true>, smem1, p1,
+                                       heads * p.qseg.nseg, st, "bwd_dq")
+                   : launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, false>, smem1, p1,
+                                       heads * p.qseg.nseg, st, "bwd_dq")) != LA_OK)
         return s;
     if ((s = launch_state_kernel(1, rrec, rtot, nullptr, nullptr, heads, p.qseg.nseg, D, st)) !=
         LA_OK)
@@ -445,19 +456,22 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
 }
 
 template <int PHI>
-la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO, void* dq,
-                            void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                            const BwdPlan& p, char* ws, cudaStream_t st) {
+la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO,
+                            const void* o_saved, const float* g_saved, void* dq, void* dk, void* dv,
+                            int64_t heads, int64_t N, int64_t D, int causal, const BwdPlan& p,
+                            char* ws, cudaStream_t st) {
     if (D == 64)
-        return run_bwd_chunked<64, PHI>(q, k, v, dO, dq, dk, dv, heads, N, causal, p, ws, st);
-    return run_bwd_chunked<128, PHI>(q, k, v, dO, dq, dk, dv, heads, N, causal, p, ws, st);
+        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, dq, dk, dv, heads, N,
+                                        causal, p, ws, st);
+    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, dq, dk, dv, heads, N, causal,
+                                     p, ws, st);
 }
 
 // ------------------------------------------------------------ generic path
 template <typename T, int PHI>
 la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
-                          float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
-                          cudaStream_t st) {
+                          float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
+                          int causal, cudaStream_t st) {
     auto kern = la::fwd_generic_kernel<T, PHI>;
     const size_t smem = la::generic_smem_bytes(int(D));
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -466,7 +480,7 @@ la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, 
     la::LaunchScope scope("fwd_generic", st);
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-        static_cast<T*>(o), S_out, z_out, int(N), int(D), causal);
+        static_cast<T*>(o), S_out, z_out, g_out, int(N), int(D), causal);
     return launch_status();
 }
 
@@ -520,9 +534,9 @@ la_status dispatch(la_dtype dt, la_phi phi, Args... args) {
 template <typename T, int PHI>
 struct FwdOp {
     static la_status run(const void* q, const void* k, const void* v, void* o, float* S_out,
-                         float* z_out, int64_t heads, int64_t N, int64_t D, int causal,
-                         cudaStream_t st) {
-        return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, heads, N, D, causal, st);
+                         float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
+                         int causal, cudaStream_t st) {
+        return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, D, causal, st);
     }
 };
 
@@ -610,13 +624,15 @@ size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, i
 }
 
 la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
-                     float* z_out, int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt,
-                     int causal, la_phi phi, void* workspace, size_t workspace_bytes,
+                     float* z_out, float* g_out, int64_t B, int64_t H, int64_t N, int64_t D,
+                     la_dtype dt, int causal, la_phi phi, void* workspace, size_t workspace_bytes,
                      la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
-    if ((S_out && !aligned16(S_out)) || (z_out && !aligned16(z_out))) return LA_ERR_INVALID_ARG;
+    if ((S_out && !aligned16(S_out)) || (z_out && !aligned16(z_out)) ||
+        (g_out && !aligned16(g_out)))
+        return LA_ERR_INVALID_ARG;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t heads = B * H;
@@ -638,18 +654,19 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
     if (plan.fast) {
         char* ws = static_cast<char*>(workspace);
         return phi == LA_PHI_ELU1
-                   ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, heads, N, D,
+                   ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, heads, N, D,
                                                  causal ? 1 : 0, plan, ws, st)
-                   : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, heads, N, D,
+                   : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, heads, N, D,
                                                      causal ? 1 : 0, plan, ws, st);
     }
-    return dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, heads, N, D, causal ? 1 : 0, st);
+    return dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D, causal ? 1 : 0,
+                           st);
 }
 
-la_status la_backward(const void* q, const void* k, const void* v, const void* dO, void* dq,
-                      void* dk, void* dv, int64_t B, int64_t H, int64_t N, int64_t D,
-                      la_dtype dt, int causal, la_phi phi, void* workspace,
-                      size_t workspace_bytes, la_stream_t stream) {
+la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
+                      const void* o, const float* g, void* dq, void* dk, void* dv, int64_t B,
+                      int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                      void* workspace, size_t workspace_bytes, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
@@ -659,6 +676,9 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
         (s = check_ptr(dq)) || (s = check_ptr(dk)) || (s = check_ptr(dv)))
         return s;
+    // saved forward statistics: both or neither
+    if ((o == nullptr) != (g == nullptr)) return LA_ERR_INVALID_ARG;
+    if (o && ((s = check_ptr(o)) || (s = check_ptr(g)))) return s;
     const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -667,9 +687,9 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     if (bp.fast) {
         char* wsp = static_cast<char*>(workspace);
         return phi == LA_PHI_ELU1
-                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, dq, dk, dv, heads, N, D,
+                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, dq, dk, dv, heads, N, D,
                                                  causal ? 1 : 0, bp, wsp, st)
-                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, dq, dk, dv, heads, N, D,
+                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, dq, dk, dv, heads, N, D,
                                                      causal ? 1 : 0, bp, wsp, st);
     }
     const BwdWorkspace w = plan_bwd(B, H, N);
@@ -681,9 +701,9 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
 }
 
 la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
-                              void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t N,
-                              int64_t D, la_dtype dt, int causal, la_phi phi,
-                              la_stream_t stream) {
+                              const void* o, const float* g, void* dq, void* dk, void* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, int causal,
+                              la_phi phi, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
@@ -697,7 +717,7 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
     if ((s = bind_context()) != LA_OK) return s;
     void* scratch = nullptr;
     if ((s = static_scratch(&scratch)) != LA_OK) return s;
-    return la_backward(q, k, v, dO, dq, dk, dv, B, H, N, D, dt, causal, phi, scratch,
+    return la_backward(q, k, v, dO, o, g, dq, dk, dv, B, H, N, D, dt, causal, phi, scratch,
                        size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 

@@ -47,13 +47,20 @@ struct BwdParams {
     float* gbuf;     // [heads][N] g_i (pass 1 writes, pass 2 reads)
     float* dgbuf;    // [heads][N] dg_i
     float* rec_out;  // pass 1: (R, r) of the block's tokens, record per block (nullable)
+    // pass 1 with saved forward statistics: the forward's output O (bf16
+    // [heads][N][D]); gbuf then holds the forward's denominators g.
+    const __nv_bfloat16* o_in;
 };
 
 template <int D, int C>
 struct Bwd1Cfg {
     static constexpr int NSTAGE = 2;
     static constexpr int TILE = C * D * 2;
-    static constexpr int STAGE = 4 * TILE;  // Q, K, V, dO
+    // Q, K, V, dO tiles, then (saved-statistics mode) the chunk's DG operand
+    // [16][C] and its dg values [C]
+    static constexpr int OFF_SDG = 4 * TILE;
+    static constexpr int OFF_SDGF = OFF_SDG + 16 * C * 2;
+    static constexpr int STAGE = ((OFF_SDGF + C * 4) + 1023) / 1024 * 1024;
     static constexpr int OFF_SPREV = NSTAGE * STAGE;
     static constexpr int OFF_ZOP = OFF_SPREV + D * D * 2;
     static constexpr int OFF_E = OFF_ZOP + 16 * D * 2;
@@ -157,7 +164,9 @@ __device__ __forceinline__ void load_chunk8(const uint8_t* tile, int rows, int r
 // ======================================================================
 constexpr int kBwdThreads = 448;  // producer, MMA, 8 phi warps, 4 epilogue warps
 
-template <int D, int C, int PHI, bool CAUSAL>
+// SAVED = the forward's O and g are given: no forward recompute; the
+// feature-map warps form dU = dO / g and dg = -(dO . O) / g directly.
+template <int D, int C, int PHI, bool CAUSAL, bool SAVED>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd1Cfg<D, C>;
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             const uint32_t tR = tmem + Cfg::T_R, tRZ = tmem + Cfg::T_RZ;
             const uint32_t sprev = sbase + Cfg::OFF_SPREV, zop = sbase + Cfg::OFF_ZOP;
             const uint32_t eop = sbase + Cfg::OFF_E, xop = sbase + Cfg::OFF_X;
-            const uint32_t duop = sbase + Cfg::OFF_DU, dgop = sbase + Cfg::OFF_DG;
+            const uint32_t duop_g = sbase + Cfg::OFF_DU, dgop_g = sbase + Cfg::OFF_DG;
             constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);   // [C x C] from two K-major
             constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);
             constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);
@@ -266,30 +275,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 const int s = c % NS;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE;
+                // dU and the DG operand: the scaled dO tile and the stage's DG
+                // (saved mode) or the epilogue-written tiles
+                const uint32_t duop = SAVED ? qs + 3 * Cfg::TILE : duop_g;
+                const uint32_t dgop = SAVED ? qs + Cfg::OFF_SDG : dgop_g;
                 if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
                 if (!(ok = mbar_wait(s_ready, c & 1, abort_flag))) break;
                 tc_fence_after();
-                if (CAUSAL) {
+                if (!SAVED) {
+                    if (CAUSAL) {
 #pragma unroll
-                    for (int k = 0; k < D; k += 16)
-                        umma_bf16(tP, desc_kmajor(qs, C, k), desc_kmajor(ks, C, k), idCC, k > 0);
-                }
+                        for (int k = 0; k < D; k += 16)
+                            umma_bf16(tP, desc_kmajor(qs, C, k), desc_kmajor(ks, C, k), idCC, k > 0);
+                    }
 #pragma unroll
-                for (int k = 0; k < D; k += 16) {
-                    umma_bf16(tO, desc_kmajor(qs, C, k), desc_mnmajor(sprev, D, k), idCD_mn, k > 0);
-                    umma_bf16(tOZ, desc_kmajor(qs, C, k), desc_kmajor(zop, 16, k), idOZ, k > 0);
-                }
-                if (CAUSAL) {
-                    umma_commit(p_ready);
-                    if (!(ok = mbar_wait(pt_ready, c & 1, abort_flag))) break;
+                    for (int k = 0; k < D; k += 16) {
+                        umma_bf16(tO, desc_kmajor(qs, C, k), desc_mnmajor(sprev, D, k), idCD_mn,
+                                  k > 0);
+                        umma_bf16(tOZ, desc_kmajor(qs, C, k), desc_kmajor(zop, 16, k), idOZ, k > 0);
+                    }
+                    if (CAUSAL) {
+                        umma_commit(p_ready);
+                        if (!(ok = mbar_wait(pt_ready, c & 1, abort_flag))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < C; k += 16)
+                            umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(vs, C, k), idCD_mn, 1);
+                    }
+                    umma_commit(o_ready);
+                    if (!(ok = mbar_wait(du_ready, c & 1, abort_flag))) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int k = 0; k < C; k += 16)
-                        umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(vs, C, k), idCD_mn, 1);
                 }
-                umma_commit(o_ready);
-                if (!(ok = mbar_wait(du_ready, c & 1, abort_flag))) break;
-                tc_fence_after();
                 if (CAUSAL) {
                     // W = dU V^T
 #pragma unroll
@@ -332,8 +348,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             mbar_wait_drain(drain, 0);
         }
     } else if (warp < 10) {
-        // feature map on Q and K (dO is used as loaded); 8 warps, batched loads
+        // feature map on Q and K (and, with saved statistics, dU and dg)
         const int u = tid - 64;  // 0..255
+        if (SAVED) {
+            for (int s = 0; s < NS; ++s) {
+                __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(smem + s * Cfg::STAGE + Cfg::OFF_SDG);
+                for (int idx = u; idx < 16 * C; idx += 256)
+                    dgt[tile_off(16, idx / C, idx % C) / 2] = __float2bfloat16_rn(0.f);
+            }
+        }
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
@@ -343,6 +366,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
             else
                 phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+            if (SAVED) {
+                // dU = dO / g in place, dg = -(dO . O) / g; 256 / C threads per row
+                constexpr int TPR = 256 / C;          // threads per row
+                constexpr int CHT = (D / 8) / TPR;    // 16-byte chunks per thread
+                const int r = u / TPR, part = u % TPR;
+                const bool valid = r < nvalid;
+                const size_t tok = size_t(head) * prm.N + size_t(tok0 + c * C + r);
+                uint8_t* dot_tile = st + 3 * Cfg::TILE;
+                uint4 x[CHT], ov[CHT];
+#pragma unroll
+                for (int j = 0; j < CHT; ++j) {
+                    x[j] = *reinterpret_cast<const uint4*>(dot_tile + tile_chunk_off(C, r, part * CHT + j));
+                    ov[j] = valid ? __ldg(reinterpret_cast<const uint4*>(prm.o_in + tok * D) + part * CHT + j)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+                }
+                const float g = valid ? prm.gbuf[tok] : 1.f;
+                float dotp = 0.f;
+#pragma unroll
+                for (int j = 0; j < CHT; ++j) {
+                    const uint32_t a[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+                    const uint32_t b[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 fa = unpack_bf16(a[t]), fb = unpack_bf16(b[t]);
+                        dotp = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, dotp));
+                    }
+                }
+#pragma unroll
+                for (int m = 1; m < TPR; m <<= 1) dotp += __shfl_xor_sync(0xffffffffu, dotp, m);
+                const float ginv = 1.f / g;
+                const float dg = valid ? -dotp * ginv : 0.f;
+#pragma unroll
+                for (int j = 0; j < CHT; ++j) {
+                    uint32_t w[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 f = unpack_bf16(w[t]);
+                        w[t] = valid ? pack_bf16(f.x * ginv, f.y * ginv) : 0u;
+                    }
+                    *reinterpret_cast<uint4*>(dot_tile + tile_chunk_off(C, r, part * CHT + j)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                if (part == 0) {
+                    __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(st + Cfg::OFF_SDG);
+                    const __nv_bfloat16 hi = __float2bfloat16_rn(dg);
+                    dgt[tile_off(16, 0, r) / 2] = hi;
+                    dgt[tile_off(16, 1, r) / 2] = __float2bfloat16_rn(dg - __bfloat162float(hi));
+                    reinterpret_cast<float*>(st + Cfg::OFF_SDGF)[r] = dg;
+                    if (valid) prm.dgbuf[tok] = dg;
+                }
+            }
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
         }
@@ -409,79 +483,86 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             const int row0 = tok0 + c * C;
             const int nvalid = min(C, tok1 - row0);
             const bool valid = irow >= 0 && irow < nvalid;
-            float den_intra = 0.f;
-            if (CAUSAL) {
-                if (!named_bar_all(1, 128, mbar_wait(p_ready, c & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll 1
-                for (int j0 = 0; j0 < C; j0 += 32) {
-                    float pv[32];
-                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0, pv);
-                    tmem_ld16(tmem + lane_base + Cfg::T_P + j0 + 16, pv + 16);
-                    tmem_wait_ld();
-                    if (irow >= 0) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int t = 0; t < 4; ++t) {
-                                const int j = j0 + q * 8 + 2 * t;
-                                w[t] = pack_bf16(j <= irow ? pv[q * 8 + 2 * t] : 0.f,
-                                                 j + 1 <= irow ? pv[q * 8 + 2 * t + 1] : 0.f);
-                                const float2 r = unpack_bf16(w[t]);
-                                den_intra += r.x + r.y;
+            float dg = 0.f;
+            if (SAVED) {
+                // dU and dg come with the stage (feature-map warps): wait for them
+                if (!named_bar_all(1, 128, mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
+                dg = irow >= 0 ? reinterpret_cast<const float*>(qt + Cfg::OFF_SDGF)[irow] : 0.f;
+            } else {
+                float den_intra = 0.f;
+                if (CAUSAL) {
+                    if (!named_bar_all(1, 128, mbar_wait(p_ready, c & 1, abort_flag))) break;
+                    tc_fence_after();
+    #pragma unroll 1
+                    for (int j0 = 0; j0 < C; j0 += 32) {
+                        float pv[32];
+                        tmem_ld16(tmem + lane_base + Cfg::T_P + j0, pv);
+                        tmem_ld16(tmem + lane_base + Cfg::T_P + j0 + 16, pv + 16);
+                        tmem_wait_ld();
+                        if (irow >= 0) {
+    #pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                uint32_t w[4];
+    #pragma unroll
+                                for (int t = 0; t < 4; ++t) {
+                                    const int j = j0 + q * 8 + 2 * t;
+                                    w[t] = pack_bf16(j <= irow ? pv[q * 8 + 2 * t] : 0.f,
+                                                     j + 1 <= irow ? pv[q * 8 + 2 * t + 1] : 0.f);
+                                    const float2 r = unpack_bf16(w[t]);
+                                    den_intra += r.x + r.y;
+                                }
+                                *reinterpret_cast<uint4*>(xop + tile_chunk_off(C, irow, (j0 >> 3) + q)) =
+                                    make_uint4(w[0], w[1], w[2], w[3]);
                             }
-                            *reinterpret_cast<uint4*>(xop + tile_chunk_off(C, irow, (j0 >> 3) + q)) =
-                                make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(pt_ready);
+                }
+                // ---- o, g, du, dg
+                if (!named_bar_all(1, 128, mbar_wait(o_ready, c & 1, abort_flag))) break;
+                tc_fence_after();
+                float oz[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_OZ, oz);
+                tmem_wait_ld();
+                const float g = den_intra + oz[0] + oz[1];
+                const float ginv = 1.f / g;
+                float dotp = 0.f;
+    #pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 16) {
+                    float ov[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_O + v0, ov);
+                    tmem_wait_ld();
+                    if (irow >= 0) {
+                        float d8a[8], d8b[8];
+                        load_chunk8(dot, C, irow, v0 >> 3, d8a);
+                        load_chunk8(dot, C, irow, (v0 >> 3) + 1, d8b);
+                        float du16[16];
+    #pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            dotp = fmaf(d8a[t], ov[t] * ginv, dotp);
+                            dotp = fmaf(d8b[t], ov[8 + t] * ginv, dotp);
+                            du16[t] = valid ? d8a[t] * ginv : 0.f;
+                            du16[8 + t] = valid ? d8b[t] * ginv : 0.f;
+                        }
+                        store_row16_bf16(duop, C, irow, v0, du16);
+                    }
+                }
+                dg = valid ? -dotp * ginv : 0.f;
+                if (irow >= 0) {
+                    const __nv_bfloat16 h = __float2bfloat16_rn(dg);
+                    dg_h[tile_off(16, 0, irow) / 2] = h;
+                    dg_h[tile_off(16, 1, irow) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
+                }
+                if (valid) {
+                    gb[row0 + irow] = g;
+                    dgb[row0 + irow] = dg;
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(pt_ready);
+                mbar_arrive(du_ready);
             }
-            // ---- o, g, du, dg
-            if (!named_bar_all(1, 128, mbar_wait(o_ready, c & 1, abort_flag))) break;
-            tc_fence_after();
-            float oz[16];
-            tmem_ld16(tmem + lane_base + Cfg::T_OZ, oz);
-            tmem_wait_ld();
-            const float g = den_intra + oz[0] + oz[1];
-            const float ginv = 1.f / g;
-            float dotp = 0.f;
-#pragma unroll 1
-            for (int v0 = 0; v0 < D; v0 += 16) {
-                float ov[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_O + v0, ov);
-                tmem_wait_ld();
-                if (irow >= 0) {
-                    float d8a[8], d8b[8];
-                    load_chunk8(dot, C, irow, v0 >> 3, d8a);
-                    load_chunk8(dot, C, irow, (v0 >> 3) + 1, d8b);
-                    float du16[16];
-#pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        dotp = fmaf(d8a[t], ov[t] * ginv, dotp);
-                        dotp = fmaf(d8b[t], ov[8 + t] * ginv, dotp);
-                        du16[t] = valid ? d8a[t] * ginv : 0.f;
-                        du16[8 + t] = valid ? d8b[t] * ginv : 0.f;
-                    }
-                    store_row16_bf16(duop, C, irow, v0, du16);
-                }
-            }
-            const float dg = valid ? -dotp * ginv : 0.f;
-            if (irow >= 0) {
-                const __nv_bfloat16 h = __float2bfloat16_rn(dg);
-                dg_h[tile_off(16, 0, irow) / 2] = h;
-                dg_h[tile_off(16, 1, irow) / 2] = __float2bfloat16_rn(dg - __bfloat162float(h));
-            }
-            if (valid) {
-                gb[row0 + irow] = g;
-                dgb[row0 + irow] = dg;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(du_ready);
             if (CAUSAL) {
                 // ---- W' = (dU V^T + dg) masked
                 if (!named_bar_all(1, 128, mbar_wait(w_ready, c & 1, abort_flag))) break;

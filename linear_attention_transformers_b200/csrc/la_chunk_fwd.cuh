@@ -56,6 +56,9 @@ struct ChunkParams {
     float* S_out;
     float* z_out;
     int64_t stride_S, stride_z;
+    // Optional [heads][N] output of the denominators g_i = phi(q_i) . z_i
+    // (CAUSAL and QUERY), which lets the backward skip recomputing them.
+    float* g_out;
 };
 
 template <int D, int C>
@@ -476,6 +479,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                 float oz[16];
                 tmem_load<16>(tO + D, oz);
                 const float inv = 1.f / (oz[0] + oz[1]);
+                if (prm.g_out && irow >= 0 && row0 + irow < tok1)
+                    prm.g_out[size_t(head) * prm.N + row0 + irow] = oz[0] + oz[1];
 #pragma unroll 1
                 for (int v0 = 0; v0 < D; v0 += 32) {
                     float ov[32];

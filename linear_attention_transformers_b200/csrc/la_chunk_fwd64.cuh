@@ -408,6 +408,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 float den[16];
                 tmem_load<16>(tO + 64, den);
                 const float inv = 1.f / (den[0] + den[1]);
+                if (prm.g_out && row0 + row < tok1)
+                    prm.g_out[size_t(head) * prm.N + row0 + row] = den[0] + den[1];
 #pragma unroll 1
                 for (int v0 = 0; v0 < D; v0 += 32) {
                     float ov[32];

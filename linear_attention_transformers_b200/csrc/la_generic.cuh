@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kGenericThreads)
 fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, T* __restrict__ o,
                    float* __restrict__ S_out, float* __restrict__ z_out,
-                   int N, int D, int causal) {
+                   float* __restrict__ g_out, int N, int D, int causal) {
     extern __shared__ float sm[];
     float* S = sm;
     float* z = S + D * D;
@@ -86,6 +86,7 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                 den = fmaf(a[f], z[f], den);
             }
             oh[row + e] = from_f32<T>(num / den);
+            if (g_out && e == 0) g_out[head * size_t(N) + i] = den;
         }
         __syncthreads();
     }

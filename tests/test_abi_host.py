@@ -47,13 +47,15 @@ def test_status_strings(lib):
 FAKE = 0x100000  # aligned, non-null, never dereferenced: every use below must fail validation
 
 
-def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=None, z=None, B=1, H=1, N=8, D=64, dt=1,
+def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=None, z=None, g=None, B=1, H=1, N=8, D=64, dt=1,
         causal=1, phi=0, ws=None, ws_bytes=0):
-    return lib.la_forward(q, k, v, o, S, z, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
+    return lib.la_forward(q, k, v, o, S, z, g, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
 
 
-def bwd(lib, p=FAKE, B=1, H=1, N=8, D=64, dt=1, causal=1, phi=0, ws=None, ws_bytes=0, dq=FAKE):
-    return lib.la_backward(p, p, p, p, dq, p, p, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
+def bwd(lib, p=FAKE, B=1, H=1, N=8, D=64, dt=1, causal=1, phi=0, ws=None, ws_bytes=0, dq=FAKE,
+        o=None, g=None):
+    return lib.la_backward(p, p, p, p, o, g, dq, p, p, B, H, N, D, dt, causal, phi, ws, ws_bytes,
+                           None)
 
 
 def test_rejects_bad_arguments_before_launch(lib):
@@ -68,6 +70,10 @@ def test_rejects_bad_arguments_before_launch(lib):
     assert fwd(lib, B=1 << 20, H=1 << 20, N=1 << 20) == api.LA_ERR_UNSUPPORTED
     assert bwd(lib, dq=None) == api.LA_ERR_INVALID_ARG
     assert bwd(lib, D=96) == api.LA_ERR_UNSUPPORTED
+    assert fwd(lib, g=FAKE + 4) == api.LA_ERR_INVALID_ARG         # misaligned g
+    # saved forward statistics go together: o without g is refused
+    need = lib.la_workspace_size(api.LA_OP_BACKWARD, 1, 1, 8, 64, 1, api.LA_BF16)
+    assert bwd(lib, o=FAKE, g=None, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
     p = FAKE
     assert lib.la_decode_step(p, p, p, p, p, None, 2, 2, 64, 1, 0, None) == api.LA_ERR_INVALID_ARG
     assert lib.la_decode_step(p, p, p, p, p, p, 2, 2, 40, 1, 0, None) == api.LA_ERR_UNSUPPORTED

@@ -57,14 +57,41 @@ def check_state(S, z, S_ref, z_ref, dtype):
 @pytest.mark.parametrize("N", [1, 129, 777])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
-def test_backward_small(dtype, D, N, causal, phi):
+@pytest.mark.parametrize("saved", [False, True])
+def test_backward_small(dtype, D, N, causal, phi, saved):
     q, k, v, dO = small(2, 2, N, D, dtype, seed=N * 11 + D, dO=True)
-    dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi)
+    if saved:
+        # the forward's output and denominators handed to the backward
+        g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+        o = api.la_forward(q, k, v, causal, phi, g=g)
+        dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi, o=o, g=g)
+    else:
+        dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi)
     torch.cuda.synchronize()
     rq, rk, rv = oracle.backward(q, k, v, dO, causal, PHIS[phi])
     compare(dq, rq, dtype, "dq")
     compare(dk, rk, dtype, "dk")
     compare(dv, rv, dtype, "dv")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("causal", [True, False])
+def test_forward_denominators(dtype, causal):
+    # g_i = phi(q_i) . z_i, the row sums of the unnormalised weights
+    q, k, v = small(2, 3, 300, 64, dtype, seed=12)
+    g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+    api.la_forward(q, k, v, causal, g=g)
+    torch.cuda.synchronize()
+    _, S, z = oracle.forward(q, k, v, causal)
+    a = oracle.phi_map(q)
+    ref = np.einsum("bhnf,bhnf->bhn", a, causal_prefix_z(k) if causal else
+                    np.broadcast_to(z[:, :, None, :], a.shape))
+    np.testing.assert_allclose(g.double().cpu().numpy(), ref, rtol=1e-2 if dtype ==
+                               torch.bfloat16 else 2e-5)
+
+
+def causal_prefix_z(k):
+    return np.cumsum(oracle.phi_map(k), axis=2)
 
 
 def test_unit_values_give_unit_output_on_gpu():
@@ -154,10 +181,13 @@ def run_workload(w, full_check: bool):
     dev_inputs = inputs.make_inputs(w, device=DEV if not full_check else "cpu")
     dev_inputs = [t.to(DEV) for t in dev_inputs]
     q, k, v = dev_inputs[:3]
-    o = api.la_forward(q, k, v, w.causal, w.phi)
+    # the launch configuration the benchmark times: the forward keeps its
+    # denominators and the backward uses them with the output
+    g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+    o = api.la_forward(q, k, v, w.causal, w.phi, g=g)
     grads = None
     if w.backward:
-        grads = api.la_backward(q, k, v, dev_inputs[3], w.causal, w.phi)
+        grads = api.la_backward(q, k, v, dev_inputs[3], w.causal, w.phi, o=o, g=g)
     torch.cuda.synchronize()
     api.la_get_device_error()
     if full_check:
