@@ -74,6 +74,9 @@ struct Bwd1Cfg {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int T_P = 0, T_O = C, T_OZ = C + D, T_S = C + D + 16, T_Z = C + 2 * D + 16;
+    // masked C x C operands (P~, W') packed in place in TMEM and read by MMAs
+    // with A from TMEM (needs M = C = 128 rows); otherwise through smem
+    static constexpr bool XT = C == 128 && D == 64;
     static constexpr int T_R = C + 2 * D + 32, T_RZ = C + 3 * D + 32;
     static constexpr int T_COLS = 512;
     static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
@@ -99,7 +102,13 @@ struct Bwd2Cfg {
     static constexpr int NBAR = 3 * NSTAGE + 5;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
-    static constexpr int T_1 = 0, T_2 = C, T_3 = 0, T_4 = D;
+    // X in TMEM (C = 128): X1, X2 are packed to bf16 in place over the low
+    // halves of T1, T2 and feed MMAs with A from TMEM; dV and dB accumulate in
+    // the high halves.  Otherwise X1, X2 go through shared memory and dV, dB
+    // reuse T1/T2's columns.
+    static constexpr bool XT = C == 128 && D == 64;
+    static constexpr int T_1 = 0, T_2 = C;
+    static constexpr int T_3 = XT ? C / 2 : 0, T_4 = XT ? C + C / 2 : D;
     static constexpr int T_R = (2 * C > 2 * D ? 2 * C : 2 * D), T_RZ = T_R + D;
     static constexpr int T_COLS = 512;
     static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
@@ -298,9 +307,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                         umma_commit(p_ready);
                         if (!(ok = mbar_wait(pt_ready, c & 1, abort_flag))) break;
                         tc_fence_after();
+                        if (Cfg::XT) {
 #pragma unroll
-                        for (int k = 0; k < C; k += 16)
-                            umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(vs, C, k), idCD_mn, 1);
+                            for (int k = 0; k < C; k += 16)
+                                umma_bf16_ts(tO, tP + k / 2, desc_mnmajor(vs, C, k), idCD_mn, 1);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < C; k += 16)
+                                umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(vs, C, k), idCD_mn,
+                                          1);
+                        }
                     }
                     umma_commit(o_ready);
                     if (!(ok = mbar_wait(du_ready, c & 1, abort_flag))) break;
@@ -315,9 +331,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     if (!(ok = mbar_wait(wt_ready, c & 1, abort_flag))) break;
                     tc_fence_after();
                     // dA = W' B
+                    if (Cfg::XT) {
 #pragma unroll
-                    for (int k = 0; k < C; k += 16)
-                        umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(ks, C, k), idCD_mn, k > 0);
+                        for (int k = 0; k < C; k += 16)
+                            umma_bf16_ts(tO, tP + k / 2, desc_mnmajor(ks, C, k), idCD_mn, k > 0);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < C; k += 16)
+                            umma_bf16(tO, desc_kmajor(xop, C, k), desc_mnmajor(ks, C, k), idCD_mn,
+                                      k > 0);
+                    }
                 }
                 // dA += dU S^T
 #pragma unroll
@@ -493,6 +516,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 if (CAUSAL) {
                     if (!named_bar_all(1, 128, mbar_wait(p_ready, c & 1, abort_flag))) break;
                     tc_fence_after();
+                    if (Cfg::XT) {
+                        const uint32_t reg = tmem + lane_base + Cfg::T_P;
+    #pragma unroll 1
+                        for (int j0 = 0; j0 < C; j0 += 32) {
+                            float pv[32];
+                            tmem_load<32>(reg + j0, pv);
+                            float pk[16];
+    #pragma unroll
+                            for (int t = 0; t < 16; ++t) {
+                                const int j = j0 + 2 * t;
+                                const uint32_t w = pack_bf16(j <= irow ? pv[2 * t] : 0.f,
+                                                             j + 1 <= irow ? pv[2 * t + 1] : 0.f);
+                                const float2 r = unpack_bf16(w);
+                                den_intra += r.x + r.y;
+                                pk[t] = __uint_as_float(w);
+                            }
+                            tmem_st16(reg + j0 / 2, pk);
+                        }
+                        tmem_wait_st();
+                    } else {
     #pragma unroll 1
                     for (int j0 = 0; j0 < C; j0 += 32) {
                         float pv[32];
@@ -515,6 +558,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                                     make_uint4(w[0], w[1], w[2], w[3]);
                             }
                         }
+                    }
                     }
                     fence_proxy_async_smem();
                     tc_fence_before();
@@ -567,6 +611,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 // ---- W' = (dU V^T + dg) masked
                 if (!named_bar_all(1, 128, mbar_wait(w_ready, c & 1, abort_flag))) break;
                 tc_fence_after();
+                if (Cfg::XT) {
+                    const uint32_t reg = tmem + lane_base + Cfg::T_P;
+#pragma unroll 1
+                    for (int j0 = 0; j0 < C; j0 += 32) {
+                        float wv[32];
+                        tmem_load<32>(reg + j0, wv);
+                        float pk[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            const int j = j0 + 2 * t;
+                            pk[t] = __uint_as_float(pack_bf16(j <= irow ? wv[2 * t] + dg : 0.f,
+                                                              j + 1 <= irow ? wv[2 * t + 1] + dg : 0.f));
+                        }
+                        tmem_st16(reg + j0 / 2, pk);
+                    }
+                    tmem_wait_st();
+                } else {
 #pragma unroll 1
                 for (int j0 = 0; j0 < C; j0 += 32) {
                     float wv[32];
@@ -587,6 +648,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                                 make_uint4(w[0], w[1], w[2], w[3]);
                         }
                     }
+                }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -787,10 +849,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     umma_commit(x_ready);
                     if (!(ok = mbar_wait(xt_ready, t & 1, abort_flag))) break;
                     tc_fence_after();
+                    if (Cfg::XT) {
 #pragma unroll
-                    for (int k = 0; k < C; k += 16) {
-                        umma_bf16(t3, desc_kmajor(x1, C, k), desc_mnmajor(dus, C, k), idCD_mn, k > 0);
-                        umma_bf16(t4, desc_kmajor(x2, C, k), desc_mnmajor(qs, C, k), idCD_mn, k > 0);
+                        for (int k = 0; k < C; k += 16) {
+                            umma_bf16_ts(t3, t1 + k / 2, desc_mnmajor(dus, C, k), idCD_mn, k > 0);
+                            umma_bf16_ts(t4, t2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, k > 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < C; k += 16) {
+                            umma_bf16(t3, desc_kmajor(x1, C, k), desc_mnmajor(dus, C, k), idCD_mn,
+                                      k > 0);
+                            umma_bf16(t4, desc_kmajor(x2, C, k), desc_mnmajor(qs, C, k), idCD_mn,
+                                      k > 0);
+                        }
                     }
                 }
 #pragma unroll
@@ -898,6 +970,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             if (CAUSAL) {
                 if (!named_bar_all(1, 128, mbar_wait(x_ready, t & 1, abort_flag))) break;
                 tc_fence_after();
+                if (Cfg::XT) {
+                    // mask and pack X1, X2 in place in TMEM (block i0 is read
+                    // before columns i0/2.. are overwritten)
+                    const uint32_t r1 = tmem + lane_base + Cfg::T_1;
+                    const uint32_t r2 = tmem + lane_base + Cfg::T_2;
+#pragma unroll 1
+                    for (int i0 = 0; i0 < C; i0 += 32) {
+                        float pv[32], wv[32];
+                        tmem_load<32>(r1 + i0, pv);
+                        tmem_load<32>(r2 + i0, wv);
+                        float a16[16], b16[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const int i = i0 + 2 * k;
+                            a16[k] = __uint_as_float(pack_bf16(i >= jrow ? pv[2 * k] : 0.f,
+                                                               i + 1 >= jrow ? pv[2 * k + 1] : 0.f));
+                            b16[k] = __uint_as_float(
+                                pack_bf16(i >= jrow ? wv[2 * k] + dgf[i] : 0.f,
+                                          i + 1 >= jrow ? wv[2 * k + 1] + dgf[i + 1] : 0.f));
+                        }
+                        tmem_st16(r1 + i0 / 2, a16);
+                        tmem_st16(r2 + i0 / 2, b16);
+                    }
+                    tmem_wait_st();
+                } else {
                 if (Cfg::STG_ALIAS) {
                     if (e == 0) bulk_wait_read0();
                     named_bar_sync(1, 128);
@@ -920,13 +1017,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                         store_row16_bf16(x2, C, jrow, i0, b16);
                     }
                 }
+                }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(xt_ready);
             }
             if (!named_bar_all(1, 128, mbar_wait(d_ready, t & 1, abort_flag))) break;
             tc_fence_after();
-            if (!Cfg::STG_ALIAS || !CAUSAL) {
+            if (Cfg::XT || !Cfg::STG_ALIAS || !CAUSAL) {
                 if (e == 0) bulk_wait_read0();
                 named_bar_sync(1, 128);
             }

@@ -13,7 +13,9 @@
 //                                              0..63 numerator, 64..65 the
 //                                              two halves of the denominator)
 //
-// "[V | 1]" is the V tile followed, at a per-stage descriptor stride, by one
+// The masked P~ is packed to bf16 in place over P in TMEM by the P warpgroup
+// and read back by tcgen05.mma with A from TMEM, so it never touches shared
+// memory.  "[V | 1]" is the V tile followed, at a per-stage descriptor stride, by one
 // constant 64-column atom whose first column is ones; the same atom serves as
 // extra M rows (state) and extra N columns (output).  Per chunk: 4 + 4 + 8 +
 // 8 = 24 MMAs (A B^T, A Sx^T, [V|1]^T B, P [V|1]).  The mathematics is the
@@ -94,7 +96,7 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&p_full[b], 1);
-            mbar_init(&p_free[b], 128);
+            mbar_init(&p_free[b], 1);  // P buffer consumed by the P~ [V|1] MMAs
             mbar_init(&o_full[b], 1);
             mbar_init(&o_free[b], 128);
         }
@@ -150,7 +152,6 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
             constexpr uint32_t idPV = idesc_bf16(C, 80, 0, 1); // (P.tril) [V|1]
             constexpr uint32_t idS = idesc_bf16(128, D, 1, 1); // [V|1]^T B
             const uint64_t dSx = desc_k_base(sbase + Cfg::OFF_SX);
-            const uint64_t dPt = desc_k_base(sbase + Cfg::OFF_PT);
             const uint32_t ones = sbase + Cfg::OFF_ONES;
             const bool has_init = st_in != nullptr;
             auto dq_of = [&](int s) { return desc_k_base(sbase + s * Cfg::STAGE); };
@@ -199,11 +200,13 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                     if (c + 1 < nchunks && !(ok = p_part(c + 1))) break;
                     if (!(ok = mbar_wait(pt_full, c & 1, abort_flag))) break;
                     tc_fence_after();
+                    // P~ is in TMEM (bf16 pairs over P's columns): A from TMEM
+                    const uint32_t tPt = tmem + Cfg::T_P + (c & 1) * C;
 #pragma unroll
                     for (int k = 0; k < C; k += 16)
-                        umma_bf16(tO, dPt + kstep_k(C, k), dvx + kstep_mn(k), idPV, 1);
+                        umma_bf16_ts(tO, tPt + k / 2, dvx + kstep_mn(k), idPV, 1);
                     umma_commit(&o_full[bo]);
-                    umma_commit(pt_free);
+                    umma_commit(&p_free[c & 1]);
                     umma_commit(&empty[s]);
                 }
             } else if (MODE == MODE_QUERY) {
@@ -262,28 +265,31 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
         }
     } else if (warp < 14) {
         if (MODE == MODE_CAUSAL) {
+            // mask P and pack it to bf16 pairs in place (TMEM): block j0 is
+            // read before columns j0/2.. are overwritten
             const int sp = warp & 3;
             const uint32_t lane_base = uint32_t(32 * sp) << 16;
             const int irow = 32 * sp + lane;
-            uint8_t* pt = smem + Cfg::OFF_PT;
             for (int c = 0; c < nchunks; ++c) {
                 const int b = c & 1;
-                bool ok = c == 0 || mbar_wait(pt_free, (c - 1) & 1, abort_flag);
-                ok = ok && mbar_wait(&p_full[b], (c >> 1) & 1, abort_flag);
-                if (!named_bar_all(1, 128, ok)) break;
+                if (!named_bar_all(1, 128, mbar_wait(&p_full[b], (c >> 1) & 1, abort_flag))) break;
                 tc_fence_after();
+                const uint32_t reg = tmem + lane_base + Cfg::T_P + b * C;
 #pragma unroll 1
                 for (int j0 = 0; j0 < C; j0 += 32) {
                     float pv[32];
-                    tmem_load<32>(tmem + lane_base + Cfg::T_P + b * C + j0, pv);
+                    tmem_load<32>(reg + j0, pv);
+                    float pk[16];
 #pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if (j0 + t > irow) pv[t] = 0.f;
-                    store_row_bf16<32>(pt, C, irow, j0, pv);
+                    for (int t = 0; t < 16; ++t) {
+                        const int j = j0 + 2 * t;
+                        pk[t] = __uint_as_float(pack_bf16(j <= irow ? pv[2 * t] : 0.f,
+                                                          j + 1 <= irow ? pv[2 * t + 1] : 0.f));
+                    }
+                    tmem_st16(reg + j0 / 2, pk);
                 }
+                tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&p_free[b]);
-                fence_proxy_async_smem();
                 mbar_arrive(pt_full);
             }
         }
