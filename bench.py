@@ -84,6 +84,46 @@ def algorithmic_bytes(kernel: str, w) -> float:
     return float(table.get(kernel, 0.0))
 
 
+# DRAM traffic per launch from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), per token and head so that it scales to the bench
+# workload; valid only while the kernel sources hash to `sources`.  The
+# capture ran at N = 4096 (the profiling size rule); traffic grows in
+# proportion to tokens for these kernels (each token's tiles are moved once).
+MEASURED_TRAFFIC = {
+    "bwd_dkdv": {"bytes_per_token_head": (272.695296e6 + 103.127296e6) / (8 * 16 * 4096),
+                 "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
+                 "profile": "profiles/bwd_dkdv_causal_b8h16n4096d64_bf16.md"},
+    "bwd_dq": {"bytes_per_token_head": (337.710080e6 + 55.305728e6) / (8 * 16 * 4096),
+               "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
+               "profile": "profiles/bwd_dq_causal_b8h16n4096d64_bf16.md"},
+    "chunk_causal": {"bytes_per_token_head": (201.389568e6 + 45.153024e6) / (8 * 16 * 4096),
+                     "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
+                     "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
+}
+
+
+def kernel_sources_hash() -> str:
+    """sha256 over the CUDA sources of the library (file names and bytes)."""
+    import hashlib
+    d = os.path.join(ROOT, "linear_attention_transformers_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel: str, w):
+    """Per-launch DRAM bytes of `kernel` on workload w, or None when no
+    capture exists for it or the kernel sources changed since."""
+    rec = MEASURED_TRAFFIC.get(kernel)
+    if rec is None or rec["sources"] != kernel_sources_hash():
+        return None
+    return rec["bytes_per_token_head"] * w.B * w.H * w.N
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons through NVML on a thread."""
 
@@ -322,7 +362,8 @@ def run_ours(args, world, rank, local):
         achieved = alg / avg_s / 1e9
         roofline = {"kernel": name, "bound": "hbm", "achieved": achieved,
                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": measured_traffic(name, w),
                     "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_s * 1e3,
                     "peak_source": f"{peaks_src} hbm_gbs",
                     "share_of_step": tot_ms / max(ms, 1e-9)}
