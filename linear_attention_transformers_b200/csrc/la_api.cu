@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "la_chunk_bwd.cuh"
+#include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
 #include "la_common.cuh"
@@ -424,8 +425,12 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                 return s;
             p2.state_in = rrec;
         }
-        return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
-                                 heads * p.seg.nseg, st, "bwd_dkdv");
+        if constexpr (D == 64)
+            return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI>, la::Bwd2x64Cfg::SMEM, p2,
+                                     heads * p.seg.nseg, st, "bwd_dkdv", la::kBwd64Threads);
+        else
+            return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
+                                     heads * p.seg.nseg, st, "bwd_dkdv");
     }
     float* stot = reinterpret_cast<float*>(ws + p.stot_off);
     float* rtot = reinterpret_cast<float*>(ws + p.rtot_off);

@@ -1,0 +1,455 @@
+// la_chunk_bwd64.cuh — causal backward pass 2 (dK, dV) for head size D = 64,
+// chunk C = 128, as a software pipeline over chunks.
+//
+// Same mathematics as bwd_dkdv_kernel in la_chunk_bwd.cuh (reverse token
+// order, R/r = suffix state of the later chunks):
+//
+//   X1 = (B A^T).M^T,  X2 = (V dU^T + 1 dg^T).M^T
+//   dV = X1 dU + B R,  dB = X2 A + V R^T + 1 r^T,  dK = dB * phi'(k)
+//   R += A^T dU,  r += A^T dg
+//
+// but laid out so that no chunk waits for the previous one to drain:
+//  * the raw products X1, X2, the packed masked operands (in place, bf16
+//    pairs, read by MMAs with A from TMEM), the dV/dB accumulators and the
+//    state accumulator each have their own TMEM columns, so the MMAs of chunk
+//    t+1 start while the epilogue still reads chunk t;
+//  * the state is accumulated transposed and augmented, R' = [dU | DG]^T A
+//    (M = 128: rows 0..63 = R^T, rows 64/65 = the r sums of the bf16 hi/lo
+//    halves of dg, read through a per-stage atom one descriptor stride after
+//    dU), so R and r take 8 MMAs per chunk instead of 16;
+//  * masking skips whole 32-column blocks (all-zero below the diagonal block,
+//    unmasked above it);
+//  * the producer also prefetches the next chunks' tiles into L2, so a stage
+//    that frees late still fills from L2.
+//
+// Warp roles (576 threads): 0 TMA producer, 1 MMA issuer (one thread), 2-9
+// feature map / dU scaling, 10-13 mask-and-pack of X1 and X2, 14-17 dV/dK
+// epilogue and state readout.  Every wait is bounded (la_sm100.cuh).
+#pragma once
+
+#include "la_chunk_bwd.cuh"
+
+namespace la {
+
+struct Bwd2x64Cfg {
+    static constexpr int C = 128, D = 64;
+    static constexpr int NSTAGE = 2;
+    static constexpr int TILE = C * D * 2;             // 16 KB
+    static constexpr int OFF_DGA = 4 * TILE;           // in-stage: [C][64] atom, cols 0/1 = dg hi/lo
+    static constexpr int OFF_DGF = OFF_DGA + TILE;     // in-stage: dg float [C]
+    static constexpr int OFF_RINV = OFF_DGF + C * 4;   // in-stage: 1/g float [C]
+    static constexpr int STAGE = ((OFF_RINV + C * 4) + 1023) / 1024 * 1024;
+    static constexpr int OFF_RX = NSTAGE * STAGE;      // R^T, bf16 [D][D] row tile (row v)
+    static constexpr int OFF_RF = OFF_RX + D * D * 2;  // r hi / lo sums, float [2][D]
+    static constexpr int OFF_STGV = OFF_RF + 1024;     // dV staging [C][D]
+    static constexpr int OFF_STGK = OFF_STGV + TILE;   // dK staging [C][D]
+    static constexpr int OFF_BAR = OFF_STGK + TILE;
+    static constexpr int NBAR = 3 * NSTAGE + 9;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    // TMEM columns
+    static constexpr int T_X1 = 0, T_X2 = C, T_DV = 2 * C, T_DB = 2 * C + D, T_R = 2 * C + 2 * D;
+    static constexpr int T_COLS = 512;
+    static_assert(T_R + D <= T_COLS, "TMEM budget");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(OFF_STGV % 1024 == 0 && OFF_RX % 1024 == 0, "swizzled tiles on 1 KB");
+};
+constexpr int kBwd64Threads = 576;
+
+// L2 prefetch of one tensor-map box (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+// Mask and pack one C x C product in place in TMEM (rows = key j in this
+// thread's lane, columns = query i; keep i >= j), optionally adding dg_i to
+// the kept entries.  Columns i, i+1 go to column i/2 as a bf16 pair.  Warp
+// `sp` holds rows 32sp..32sp+31, so 32-column block b is all-zero for b < sp,
+// the diagonal block for b == sp and unmasked for b > sp.  Block b is read
+// before columns 16b.. are written, and writes only reach columns of blocks
+// already read.
+__device__ __forceinline__ void mask_pack_upper(uint32_t reg, int sp, int jrow, const float* dgf) {
+    using namespace sm100;
+#pragma unroll 1
+    for (int b = 0; b < 4; ++b) {
+        const int i0 = 32 * b;
+        float pk[16];
+        if (b < sp) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) pk[t] = 0.f;
+        } else {
+            float v[32];
+            tmem_load<32>(reg + i0, v);
+            if (dgf) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const float4 d4 = reinterpret_cast<const float4*>(dgf + i0)[q];
+                    v[4 * q] += d4.x;
+                    v[4 * q + 1] += d4.y;
+                    v[4 * q + 2] += d4.z;
+                    v[4 * q + 3] += d4.w;
+                }
+            }
+            if (b == sp) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int i = i0 + 2 * t;
+                    pk[t] = __uint_as_float(
+                        pack_bf16(i >= jrow ? v[2 * t] : 0.f, i + 1 >= jrow ? v[2 * t + 1] : 0.f));
+                }
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) pk[t] = __uint_as_float(pack_bf16(v[2 * t], v[2 * t + 1]));
+            }
+        }
+        tmem_st16(reg + i0 / 2, pk);
+    }
+    tmem_wait_st();
+}
+
+template <int PHI>
+__global__ void __launch_bounds__(kBwd64Threads, 1)
+bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
+    using namespace sm100;
+    using Cfg = Bwd2x64Cfg;
+    constexpr int C = Cfg::C, D = Cfg::D, NS = Cfg::NSTAGE;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full = bars;                 // TMA
+    uint64_t* phi_done = bars + NS;        // 256 feature-map threads
+    uint64_t* empty = bars + 2 * NS;       // MMA commit + 128 epilogue threads
+    uint64_t* x1_full = bars + 3 * NS;     // commit: B A^T
+    uint64_t* x2_full = x1_full + 1;       // commit: V dU^T
+    uint64_t* x1p_full = x1_full + 2;      // 128: X1 packed
+    uint64_t* x2p_full = x1_full + 3;      // 128: X2 packed
+    uint64_t* d_full = x1_full + 4;        // commit: dV, dB complete
+    uint64_t* d_free = x1_full + 5;        // 128: dV, dB read
+    uint64_t* r_full = x1_full + 6;        // commit: state update complete
+    uint64_t* rx_full = x1_full + 7;       // 128: R^T operand and r written
+    uint64_t* drain = x1_full + 8;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int tok0 = seg * prm.seg_len;
+    const int tok1 = min(prm.N, tok0 + prm.seg_len);
+    const int nchunks = (tok1 - tok0 + C - 1) / C;
+    const float* st_in =
+        prm.state_in ? prm.state_in + size_t(prm.in_per_head ? head : blockIdx.x) * size_t(D * D + D)
+                     : nullptr;
+    // chunk processed at step t (reverse token order)
+    auto row_of = [&](int t) { return tok0 + (nchunks - 1 - t) * C; };
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&phi_done[s], 256);
+            mbar_init(&empty[s], 1 + 128);
+        }
+        mbar_init(x1_full, 1);
+        mbar_init(x2_full, 1);
+        mbar_init(x1p_full, 128);
+        mbar_init(x2p_full, 128);
+        mbar_init(d_full, 1);
+        mbar_init(d_free, 128);
+        mbar_init(r_full, 1);
+        mbar_init(rx_full, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::T_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&prm.tm_q);
+            tma_prefetch_desc(&prm.tm_k);
+            tma_prefetch_desc(&prm.tm_v);
+            tma_prefetch_desc(&prm.tm_do);
+            auto prefetch = [&](int t) {
+                if (t < nchunks) {
+                    const int row = row_of(t);
+                    tma_prefetch_l2_3d(&prm.tm_q, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_k, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_v, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_do, 0, row, head);
+                }
+            };
+            prefetch(NS);
+            int issued = 0;
+            for (int t = 0; t < nchunks; ++t) {
+                const int s = t % NS;
+                prefetch(t + NS + 1);
+                if (t >= NS && !mbar_wait(&empty[s], ((t / NS) - 1) & 1, abort_flag)) break;
+                uint8_t* st = smem + s * Cfg::STAGE;
+                mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
+                const int row = row_of(t);
+                tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, head);
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, head);
+                tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
+                issued = t + 1;
+            }
+            for (int t = max(0, issued - NS); t < issued; ++t)
+                mbar_wait_drain(&full[t % NS], (t / NS) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t tX1 = tmem + Cfg::T_X1, tX2 = tmem + Cfg::T_X2;
+            const uint32_t tDV = tmem + Cfg::T_DV, tDB = tmem + Cfg::T_DB, tR = tmem + Cfg::T_R;
+            const uint32_t rx = sbase + Cfg::OFF_RX;
+            constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);     // B A^T, V dU^T
+            constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);  // B operand rows = K
+            constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);   // B operand K-major
+            constexpr uint32_t idR = idesc_bf16(128, D, 1, 1);    // [dU | DG]^T A
+            const bool has_init = st_in != nullptr;
+            bool ok = true;
+            for (int t = 0; ok && t < nchunks; ++t) {
+                const int s = t % NS;
+                const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
+                const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                const uint32_t dga = qs + Cfg::OFF_DGA;
+                if (!(ok = mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag))) break;
+                tc_fence_after();
+                // X1 = B A^T, X2 = V dU^T (raw, fp32)
+#pragma unroll
+                for (int k = 0; k < D; k += 16)
+                    umma_bf16(tX1, desc_kmajor(ks, C, k), desc_kmajor(qs, C, k), idCC, k > 0);
+                umma_commit(x1_full);
+#pragma unroll
+                for (int k = 0; k < D; k += 16)
+                    umma_bf16(tX2, desc_kmajor(vs, C, k), desc_kmajor(dus, C, k), idCC, k > 0);
+                umma_commit(x2_full);
+                // dV = B R, dB = V R^T from the state of the later chunks
+                if (!(ok = mbar_wait(rx_full, t & 1, abort_flag))) break;
+                if (t > 0 && !(ok = mbar_wait(d_free, (t - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D; k += 16) {
+                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_kmajor(rx, D, k), idCD_k, k > 0);
+                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_mnmajor(rx, D, k), idCD_mn, k > 0);
+                }
+                // dV += X1 dU, dB += X2 A (A operands packed in TMEM)
+                if (!(ok = mbar_wait(x1p_full, t & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C; k += 16)
+                    umma_bf16_ts(tDV, tX1 + k / 2, desc_mnmajor(dus, C, k), idCD_mn, 1);
+                if (!(ok = mbar_wait(x2p_full, t & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C; k += 16)
+                    umma_bf16_ts(tDB, tX2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, 1);
+                umma_commit(d_full);
+                if (t + 1 < nchunks) {
+                    // R' += [dU | DG]^T A: the DG atom is one LBO after dU
+                    const uint64_t dudg = sdesc_sw128(dus, dga - dus, 1024);
+                    const uint64_t amn = desc_mn_base(qs, C);
+#pragma unroll
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tR, dudg + kstep_mn(k), amn + kstep_mn(k), idR,
+                                  (t > 0 || has_init || k > 0) ? 1u : 0u);
+                    umma_commit(r_full);
+                }
+                umma_commit(&empty[s]);
+            }
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+    } else if (warp < 10) {
+        // per chunk: dg (bf16 hi/lo into the DG atom, fp32 copy), 1/g, phi on Q
+        // and K in place, dU = dO / g in place
+        const int u = tid - 64;  // 0..255
+        for (int idx = u; idx < NS * (Cfg::TILE / 16); idx += 256) {
+            const int s = idx / (Cfg::TILE / 16), q = idx % (Cfg::TILE / 16);
+            reinterpret_cast<uint4*>(smem + s * Cfg::STAGE + Cfg::OFF_DGA)[q] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        const float* gb = prm.gbuf + size_t(head) * prm.N;
+        const float* dgb = prm.dgbuf + size_t(head) * prm.N;
+        // g and dg of the next chunk are loaded one chunk ahead
+        float g_nx = 1.f, dg_nx = 0.f;
+        auto load_gdg = [&](int t) {
+            if (u < C && t < nchunks) {
+                const int tok = row_of(t) + u;
+                if (tok < tok1) {
+                    g_nx = gb[tok];
+                    dg_nx = dgb[tok];
+                } else {
+                    g_nx = 1.f;
+                    dg_nx = 0.f;
+                }
+            }
+        };
+        load_gdg(0);
+        for (int t = 0; t < nchunks; ++t) {
+            const int s = t % NS;
+            const int row0 = row_of(t);
+            const int nvalid = min(C, tok1 - row0);
+            const float g = g_nx, dg = dg_nx;
+            load_gdg(t + 1);
+            if (!named_bar_all(3, 256, mbar_wait(&full[s], (t / NS) & 1, abort_flag))) break;
+            uint8_t* st = smem + s * Cfg::STAGE;
+            float* dgf = reinterpret_cast<float*>(st + Cfg::OFF_DGF);
+            float* rinv = reinterpret_cast<float*>(st + Cfg::OFF_RINV);
+            if (u < C) {
+                const bool valid = u < nvalid;
+                const float d = valid ? dg : 0.f;
+                rinv[u] = valid ? 1.f / g : 0.f;
+                const __nv_bfloat16 h = __float2bfloat16_rn(d);
+                const __nv_bfloat16 l = __float2bfloat16_rn(d - __bfloat162float(h));
+                const uint32_t w = uint32_t(__bfloat16_as_ushort(h)) |
+                                   (uint32_t(__bfloat16_as_ushort(l)) << 16);
+                *reinterpret_cast<uint4*>(st + Cfg::OFF_DGA + tile_chunk_off(C, u, 0)) =
+                    make_uint4(w, 0u, 0u, 0u);
+                dgf[u] = d;
+            }
+            named_bar_sync(3, 256);  // rinv ready
+            if (u < 128)
+                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+            else
+                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+            scale_tile_rows<C, D, 256>(st + 3 * Cfg::TILE, u, nvalid, rinv);
+            fence_proxy_async_smem();
+            mbar_arrive(&phi_done[s]);
+        }
+    } else if (warp < 14) {
+        // mask and pack X1 (keep i >= j) and X2 (+ dg_i) in place
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int jrow = 32 * sp + lane;
+        for (int t = 0; t < nchunks; ++t) {
+            const int s = t % NS;
+            const float* dgf = reinterpret_cast<const float*>(smem + s * Cfg::STAGE + Cfg::OFF_DGF);
+            if (!named_bar_all(1, 128, mbar_wait(x1_full, t & 1, abort_flag))) break;
+            tc_fence_after();
+            mask_pack_upper(tmem + lane_base + Cfg::T_X1, sp, jrow, nullptr);
+            tc_fence_before();
+            mbar_arrive(x1p_full);
+            if (!named_bar_all(1, 128, mbar_wait(x2_full, t & 1, abort_flag))) break;
+            tc_fence_after();
+            mask_pack_upper(tmem + lane_base + Cfg::T_X2, sp, jrow, dgf);
+            tc_fence_before();
+            mbar_arrive(x2p_full);
+        }
+    } else {
+        // dV / dK epilogue and the state readout
+        const int e = tid - 448;
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int jrow = 32 * sp + lane;
+        uint8_t* rx = smem + Cfg::OFF_RX;
+        float* rf = reinterpret_cast<float*>(smem + Cfg::OFF_RF);  // [2][D]
+        uint8_t* stgv = smem + Cfg::OFF_STGV;
+        uint8_t* stgk = smem + Cfg::OFF_STGK;
+
+        // initial state: R^T operand, r, and (with an initial state) R'
+        if (jrow < D) {
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float col[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    col[i] = st_in ? st_in[size_t(32 * h + i) * D + jrow] : 0.f;
+                store_row_bf16<32>(rx, D, jrow, 32 * h, col);
+            }
+        } else if (jrow < D + 2) {
+            for (int f = 0; f < D; ++f)
+                rf[(jrow - D) * D + f] = (st_in && jrow == D) ? st_in[size_t(D) * D + f] : 0.f;
+        }
+        if (st_in) {
+#pragma unroll 1
+            for (int f0 = 0; f0 < D; f0 += 16) {
+                float v16[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int f = f0 + i;
+                    v16[i] = jrow < D ? st_in[size_t(f) * D + jrow]
+                                      : (jrow == D ? st_in[size_t(D) * D + f] : 0.f);
+                }
+                tmem_st16(tmem + lane_base + Cfg::T_R + f0, v16);
+            }
+            tmem_wait_st();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(rx_full);
+
+        for (int t = 0; t < nchunks; ++t) {
+            const int s = t % NS;
+            const uint8_t* kt = smem + s * Cfg::STAGE + Cfg::TILE;
+            const int row0 = row_of(t);
+            if (!named_bar_all(2, 128, mbar_wait(d_full, t & 1, abort_flag))) break;
+            tc_fence_after();
+            if (e == 0) bulk_wait_read0();
+            named_bar_sync(2, 128);  // staging free
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+                float dv16[16], db16[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_DV + c0, dv16);
+                tmem_ld16(tmem + lane_base + Cfg::T_DB + c0, db16);
+                tmem_wait_ld();
+                float b8a[8], b8b[8];
+                load_chunk8(kt, C, jrow, c0 >> 3, b8a);
+                load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
+                float dk16[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int f = c0 + i;
+                    dk16[i] = (db16[i] + rf[f] + rf[D + f]) * dphi_from_phi<PHI>(b8a[i]);
+                    dk16[8 + i] = (db16[8 + i] + rf[f + 8] + rf[D + f + 8]) * dphi_from_phi<PHI>(b8b[i]);
+                }
+                store_row16_bf16(stgv, C, jrow, c0, dv16);
+                store_row16_bf16(stgk, C, jrow, c0, dk16);
+            }
+            tc_fence_before();
+            mbar_arrive(d_free);
+            fence_proxy_async_smem();
+            named_bar_sync(2, 128);  // staging complete, every rf and K-tile read done
+            mbar_arrive(&empty[s]);
+            if (e == 0) {
+                tma_store_3d(&prm.tm_dv, stgv, 0, row0, head);
+                tma_store_3d(&prm.tm_dk, stgk, 0, row0, head);
+                bulk_commit();
+            }
+            if (t + 1 == nchunks) break;
+            // state after this chunk -> operands of the next (earlier) chunk
+            if (!named_bar_all(2, 128, mbar_wait(r_full, t & 1, abort_flag))) break;
+            tc_fence_after();
+#pragma unroll 1
+            for (int h = 0; h < 2; ++h) {
+                float col[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_R + 32 * h, col);
+                if (jrow < D) {
+                    store_row_bf16<32>(rx, D, jrow, 32 * h, col);
+                } else if (jrow < D + 2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) rf[(jrow - D) * D + 32 * h + i] = col[i];
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(rx_full);
+        }
+        if (e == 0) bulk_wait0();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, Cfg::T_COLS);
+}
+
+}  // namespace la
