@@ -50,6 +50,9 @@ struct BwdParams {
     // pass 1 with saved forward statistics: the forward's output O (bf16
     // [heads][N][D]); gbuf then holds the forward's denominators g.
     const __nv_bfloat16* o_in;
+    // outputs as plain pointers, for kernels that store rows directly
+    __nv_bfloat16* dk_out;
+    __nv_bfloat16* dv_out;
 };
 
 template <int D, int C>
