@@ -11,20 +11,20 @@
 // but laid out so that no chunk waits for the previous one to drain:
 //  * the raw products X1, X2, the packed masked operands (in place, bf16
 //    pairs, read by MMAs with A from TMEM), the dV/dB accumulators and the
-//    state accumulator each have their own TMEM columns, so the MMAs of chunk
-//    t+1 start while the epilogue still reads chunk t;
-//  * the state is accumulated transposed and augmented, R' = [dU | DG]^T A
-//    (M = 128: rows 0..63 = R^T, rows 64/65 = the r sums of the bf16 hi/lo
-//    halves of dg, read through a per-stage atom one descriptor stride after
-//    dU), so R and r take 8 MMAs per chunk instead of 16;
+//    state accumulators each have their own TMEM columns, so the MMAs of
+//    chunk t+1 start while the epilogue still reads chunk t;
+//  * three input stages (q, k, v, dO tiles); dV and dK are staged in place
+//    over the chunk's V and K tiles (dead once dV, dB are complete) and
+//    stored by TMA from a warp of their own, which frees the stage once the
+//    store has read it; the producer also prefetches later chunks' tiles
+//    into L2;
 //  * masking skips whole 32-column blocks (all-zero below the diagonal block,
-//    unmasked above it);
-//  * the producer also prefetches the next chunks' tiles into L2, so a stage
-//    that frees late still fills from L2.
+//    unmasked above it).
 //
-// Warp roles (576 threads): 0 TMA producer, 1 MMA issuer (one thread), 2-9
+// Warp roles (608 threads): 0 TMA producer, 1 MMA issuer (one thread), 2-9
 // feature map / dU scaling, 10-13 mask-and-pack of X1 and X2, 14-17 dV/dK
-// epilogue and state readout.  Every wait is bounded (la_sm100.cuh).
+// epilogue and state readout, 18 TMA stores.  Every wait is bounded
+// (la_sm100.cuh).
 #pragma once
 
 #include "la_chunk_bwd.cuh"
@@ -33,28 +33,27 @@ namespace la {
 
 struct Bwd2x64Cfg {
     static constexpr int C = 128, D = 64;
-    static constexpr int NSTAGE = 2;
+    static constexpr int NSTAGE = 3;
     static constexpr int TILE = C * D * 2;             // 16 KB
-    static constexpr int OFF_DGA = 4 * TILE;           // in-stage: [C][64] atom, cols 0/1 = dg hi/lo
-    static constexpr int OFF_DGF = OFF_DGA + TILE;     // in-stage: dg float [C]
+    static constexpr int OFF_DG = 4 * TILE;            // in-stage: [16][C] K-major, rows 0/1 = dg hi/lo
+    static constexpr int OFF_DGF = OFF_DG + 16 * C * 2;  // in-stage: dg float [C]
     static constexpr int OFF_RINV = OFF_DGF + C * 4;   // in-stage: 1/g float [C]
     static constexpr int STAGE = ((OFF_RINV + C * 4) + 1023) / 1024 * 1024;
-    static constexpr int OFF_RX = NSTAGE * STAGE;      // R^T, bf16 [D][D] row tile (row v)
-    static constexpr int OFF_RF = OFF_RX + D * D * 2;  // r hi / lo sums, float [2][D]
-    static constexpr int OFF_STGV = OFF_RF + 1024;     // dV staging [C][D]
-    static constexpr int OFF_STGK = OFF_STGV + TILE;   // dK staging [C][D]
-    static constexpr int OFF_BAR = OFF_STGK + TILE;
-    static constexpr int NBAR = 3 * NSTAGE + 9;
+    static constexpr int OFF_RP = NSTAGE * STAGE;      // R, bf16 [D][D] row tile (row f)
+    static constexpr int OFF_RF = OFF_RP + D * D * 2;  // r, float [D]
+    static constexpr int OFF_BAR = OFF_RF + D * 4;
+    static constexpr int NBAR = 3 * NSTAGE + 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM columns
-    static constexpr int T_X1 = 0, T_X2 = C, T_DV = 2 * C, T_DB = 2 * C + D, T_R = 2 * C + 2 * D;
+    static constexpr int T_X1 = 0, T_X2 = C, T_DV = 2 * C, T_DB = 2 * C + D;
+    static constexpr int T_R = 2 * C + 2 * D, T_RZ = T_R + D;
     static constexpr int T_COLS = 512;
-    static_assert(T_R + D <= T_COLS, "TMEM budget");
+    static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
-    static_assert(OFF_STGV % 1024 == 0 && OFF_RX % 1024 == 0, "swizzled tiles on 1 KB");
+    static_assert(OFF_RP % 1024 == 0, "swizzled tiles on 1 KB");
 };
-constexpr int kBwd64Threads = 576;
+constexpr int kBwd64Threads = 608;
 
 // L2 prefetch of one tensor-map box (no shared memory, no completion).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
@@ -122,7 +121,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
     uint64_t* full = bars;                 // TMA
     uint64_t* phi_done = bars + NS;        // 256 feature-map threads
-    uint64_t* empty = bars + 2 * NS;       // MMA commit + 128 epilogue threads
+    uint64_t* empty = bars + 2 * NS;       // MMA commit + the store warp
     uint64_t* x1_full = bars + 3 * NS;     // commit: B A^T
     uint64_t* x2_full = x1_full + 1;       // commit: V dU^T
     uint64_t* x1p_full = x1_full + 2;      // 128: X1 packed
@@ -130,8 +129,9 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     uint64_t* d_full = x1_full + 4;        // commit: dV, dB complete
     uint64_t* d_free = x1_full + 5;        // 128: dV, dB read
     uint64_t* r_full = x1_full + 6;        // commit: state update complete
-    uint64_t* rx_full = x1_full + 7;       // 128: R^T operand and r written
+    uint64_t* rx_full = x1_full + 7;       // 128: R operand and r written
     uint64_t* drain = x1_full + 8;
+    uint64_t* staged = x1_full + 9;        // 128: dV, dK rows staged
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -150,7 +150,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&phi_done[s], 256);
-            mbar_init(&empty[s], 1 + 128);
+            mbar_init(&empty[s], 2);
         }
         mbar_init(x1_full, 1);
         mbar_init(x2_full, 1);
@@ -161,6 +161,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
         mbar_init(r_full, 1);
         mbar_init(rx_full, 128);
         mbar_init(drain, 1);
+        mbar_init(staged, 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -209,19 +210,21 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t tX1 = tmem + Cfg::T_X1, tX2 = tmem + Cfg::T_X2;
-            const uint32_t tDV = tmem + Cfg::T_DV, tDB = tmem + Cfg::T_DB, tR = tmem + Cfg::T_R;
-            const uint32_t rx = sbase + Cfg::OFF_RX;
+            const uint32_t tDV = tmem + Cfg::T_DV, tDB = tmem + Cfg::T_DB;
+            const uint32_t tR = tmem + Cfg::T_R, tRZ = tmem + Cfg::T_RZ;
+            const uint32_t rp = sbase + Cfg::OFF_RP;
             constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);     // B A^T, V dU^T
             constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);  // B operand rows = K
             constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);   // B operand K-major
-            constexpr uint32_t idR = idesc_bf16(128, D, 1, 1);    // [dU | DG]^T A
+            constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);     // A^T dU
+            constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);   // A^T [dg_hi; dg_lo]
             const bool has_init = st_in != nullptr;
             bool ok = true;
             for (int t = 0; ok && t < nchunks; ++t) {
                 const int s = t % NS;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
-                const uint32_t dga = qs + Cfg::OFF_DGA;
+                const uint32_t dgs = qs + Cfg::OFF_DG;
                 if (!(ok = mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag))) break;
                 tc_fence_after();
                 // X1 = B A^T, X2 = V dU^T (raw, fp32)
@@ -239,8 +242,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D; k += 16) {
-                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_kmajor(rx, D, k), idCD_k, k > 0);
-                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_mnmajor(rx, D, k), idCD_mn, k > 0);
+                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_mnmajor(rp, D, k), idCD_mn, k > 0);
+                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_kmajor(rp, D, k), idCD_k, k > 0);
                 }
                 // dV += X1 dU, dB += X2 A (A operands packed in TMEM)
                 if (!(ok = mbar_wait(x1p_full, t & 1, abort_flag))) break;
@@ -255,13 +258,13 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                     umma_bf16_ts(tDB, tX2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, 1);
                 umma_commit(d_full);
                 if (t + 1 < nchunks) {
-                    // R' += [dU | DG]^T A: the DG atom is one LBO after dU
-                    const uint64_t dudg = sdesc_sw128(dus, dga - dus, 1024);
-                    const uint64_t amn = desc_mn_base(qs, C);
+                    // R += A^T dU, r += A^T [dg_hi; dg_lo]
 #pragma unroll
-                    for (int k = 0; k < C; k += 16)
-                        umma_bf16(tR, dudg + kstep_mn(k), amn + kstep_mn(k), idR,
-                                  (t > 0 || has_init || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < C; k += 16) {
+                        const uint32_t acc = (t > 0 || has_init || k > 0) ? 1u : 0u;
+                        umma_bf16(tR, desc_mnmajor(qs, C, k), desc_mnmajor(dus, C, k), idDD, acc);
+                        umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgs, 16, k), idD16, acc);
+                    }
                     umma_commit(r_full);
                 }
                 umma_commit(&empty[s]);
@@ -273,9 +276,10 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
         // per chunk: dg (bf16 hi/lo into the DG atom, fp32 copy), 1/g, phi on Q
         // and K in place, dU = dO / g in place
         const int u = tid - 64;  // 0..255
-        for (int idx = u; idx < NS * (Cfg::TILE / 16); idx += 256) {
-            const int s = idx / (Cfg::TILE / 16), q = idx % (Cfg::TILE / 16);
-            reinterpret_cast<uint4*>(smem + s * Cfg::STAGE + Cfg::OFF_DGA)[q] = make_uint4(0u, 0u, 0u, 0u);
+        for (int idx = u; idx < NS * 16 * C; idx += 256) {
+            const int s = idx / (16 * C), r = (idx / C) % 16, cc = idx % C;
+            reinterpret_cast<__nv_bfloat16*>(smem + s * Cfg::STAGE + Cfg::OFF_DG)[tile_off(16, r, cc) / 2] =
+                __float2bfloat16_rn(0.f);
         }
         const float* gb = prm.gbuf + size_t(head) * prm.N;
         const float* dgb = prm.dgbuf + size_t(head) * prm.N;
@@ -308,12 +312,10 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const bool valid = u < nvalid;
                 const float d = valid ? dg : 0.f;
                 rinv[u] = valid ? 1.f / g : 0.f;
+                __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(st + Cfg::OFF_DG);
                 const __nv_bfloat16 h = __float2bfloat16_rn(d);
-                const __nv_bfloat16 l = __float2bfloat16_rn(d - __bfloat162float(h));
-                const uint32_t w = uint32_t(__bfloat16_as_ushort(h)) |
-                                   (uint32_t(__bfloat16_as_ushort(l)) << 16);
-                *reinterpret_cast<uint4*>(st + Cfg::OFF_DGA + tile_chunk_off(C, u, 0)) =
-                    make_uint4(w, 0u, 0u, 0u);
+                dgt[tile_off(16, 0, u) / 2] = h;
+                dgt[tile_off(16, 1, u) / 2] = __float2bfloat16_rn(d - __bfloat162float(h));
                 dgf[u] = d;
             }
             named_bar_sync(3, 256);  // rinv ready
@@ -344,43 +346,34 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             tc_fence_before();
             mbar_arrive(x2p_full);
         }
-    } else {
-        // dV / dK epilogue and the state readout
-        const int e = tid - 448;
+    } else if (warp < 18) {
+        // dV / dK epilogue (rows staged in place over the V and K tiles) and
+        // the state readout
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int jrow = 32 * sp + lane;
-        uint8_t* rx = smem + Cfg::OFF_RX;
-        float* rf = reinterpret_cast<float*>(smem + Cfg::OFF_RF);  // [2][D]
-        uint8_t* stgv = smem + Cfg::OFF_STGV;
-        uint8_t* stgk = smem + Cfg::OFF_STGK;
+        const int frow = acc_row<D>(sp, lane);  // row of the M = 64 state accumulators
+        uint8_t* rp = smem + Cfg::OFF_RP;
+        float* rf = reinterpret_cast<float*>(smem + Cfg::OFF_RF);
 
-        // initial state: R^T operand, r, and (with an initial state) R'
-        if (jrow < D) {
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float col[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    col[i] = st_in ? st_in[size_t(32 * h + i) * D + jrow] : 0.f;
-                store_row_bf16<32>(rx, D, jrow, 32 * h, col);
-            }
-        } else if (jrow < D + 2) {
-            for (int f = 0; f < D; ++f)
-                rf[(jrow - D) * D + f] = (st_in && jrow == D) ? st_in[size_t(D) * D + f] : 0.f;
+        // initial state: R operand, r, and (with an initial state) the accumulators
+        if (frow >= 0) {
+            float r0;
+            load_state_row<D>(st_in, frow, rp, &r0);
+            rf[frow] = r0;
         }
         if (st_in) {
 #pragma unroll 1
             for (int f0 = 0; f0 < D; f0 += 16) {
                 float v16[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int f = f0 + i;
-                    v16[i] = jrow < D ? st_in[size_t(f) * D + jrow]
-                                      : (jrow == D ? st_in[size_t(D) * D + f] : 0.f);
-                }
+                for (int i = 0; i < 16; ++i) v16[i] = frow >= 0 ? st_in[size_t(frow) * D + f0 + i] : 0.f;
                 tmem_st16(tmem + lane_base + Cfg::T_R + f0, v16);
             }
+            float z16[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) z16[i] = (i == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+            tmem_st16(tmem + lane_base + Cfg::T_RZ, z16);
             tmem_wait_st();
         }
         fence_proxy_async_smem();
@@ -389,12 +382,10 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
 
         for (int t = 0; t < nchunks; ++t) {
             const int s = t % NS;
-            const uint8_t* kt = smem + s * Cfg::STAGE + Cfg::TILE;
-            const int row0 = row_of(t);
+            uint8_t* kt = smem + s * Cfg::STAGE + Cfg::TILE;   // B, then dK
+            uint8_t* vt = smem + s * Cfg::STAGE + 2 * Cfg::TILE;  // dV
             if (!named_bar_all(2, 128, mbar_wait(d_full, t & 1, abort_flag))) break;
             tc_fence_after();
-            if (e == 0) bulk_wait_read0();
-            named_bar_sync(2, 128);  // staging free
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 16) {
                 float dv16[16], db16[16];
@@ -404,46 +395,65 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 float b8a[8], b8b[8];
                 load_chunk8(kt, C, jrow, c0 >> 3, b8a);
                 load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
+                float r16[16];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float4 x = reinterpret_cast<const float4*>(rf + c0)[q];
+                    r16[4 * q] = x.x;
+                    r16[4 * q + 1] = x.y;
+                    r16[4 * q + 2] = x.z;
+                    r16[4 * q + 3] = x.w;
+                }
                 float dk16[16];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int f = c0 + i;
-                    dk16[i] = (db16[i] + rf[f] + rf[D + f]) * dphi_from_phi<PHI>(b8a[i]);
-                    dk16[8 + i] = (db16[8 + i] + rf[f + 8] + rf[D + f + 8]) * dphi_from_phi<PHI>(b8b[i]);
+                    dk16[i] = (db16[i] + r16[i]) * dphi_from_phi<PHI>(b8a[i]);
+                    dk16[8 + i] = (db16[8 + i] + r16[8 + i]) * dphi_from_phi<PHI>(b8b[i]);
                 }
-                store_row16_bf16(stgv, C, jrow, c0, dv16);
-                store_row16_bf16(stgk, C, jrow, c0, dk16);
+                // this thread's row of B is read before it is overwritten
+                store_row16_bf16(vt, C, jrow, c0, dv16);
+                store_row16_bf16(kt, C, jrow, c0, dk16);
             }
             tc_fence_before();
             mbar_arrive(d_free);
             fence_proxy_async_smem();
-            named_bar_sync(2, 128);  // staging complete, every rf and K-tile read done
-            mbar_arrive(&empty[s]);
-            if (e == 0) {
-                tma_store_3d(&prm.tm_dv, stgv, 0, row0, head);
-                tma_store_3d(&prm.tm_dk, stgk, 0, row0, head);
-                bulk_commit();
-            }
+            mbar_arrive(staged);
             if (t + 1 == nchunks) break;
             // state after this chunk -> operands of the next (earlier) chunk
             if (!named_bar_all(2, 128, mbar_wait(r_full, t & 1, abort_flag))) break;
             tc_fence_after();
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float col[32];
-                tmem_load<32>(tmem + lane_base + Cfg::T_R + 32 * h, col);
-                if (jrow < D) {
-                    store_row_bf16<32>(rx, D, jrow, 32 * h, col);
-                } else if (jrow < D + 2) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) rf[(jrow - D) * D + 32 * h + i] = col[i];
-                }
+            for (int v0 = 0; v0 < D; v0 += 16) {
+                float rv[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
+                tmem_wait_ld();
+                if (frow >= 0) store_row16_bf16(rp, D, frow, v0, rv);
             }
+            float rz[16];
+            tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
+            tmem_wait_ld();
+            if (frow >= 0) rf[frow] = rz[0] + rz[1];
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(rx_full);
         }
-        if (e == 0) bulk_wait0();
+    } else if (warp == 18) {
+        // TMA stores of the staged dV, dK rows; the stage is free once they
+        // have been read
+        if (lane == 0) {
+            for (int t = 0; t < nchunks; ++t) {
+                const int s = t % NS;
+                const int row0 = row_of(t);
+                uint8_t* st = smem + s * Cfg::STAGE;
+                if (!mbar_wait(staged, t & 1, abort_flag)) break;
+                tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
+                tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(&empty[s]);
+            }
+            bulk_wait0();
+        }
     }
 
     tc_fence_before();
