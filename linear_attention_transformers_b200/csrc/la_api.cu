@@ -381,6 +381,8 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     prm.gbuf = saved ? const_cast<float*>(g_saved) : reinterpret_cast<float*>(ws + p.g_off);
     prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
     prm.o_in = static_cast<const __nv_bfloat16*>(o_saved);
+    prm.dk_out = static_cast<__nv_bfloat16*>(dk);
+    prm.dv_out = static_cast<__nv_bfloat16*>(dv);
     const int64_t R = int64_t(D) * D + D;
     float* srec = reinterpret_cast<float*>(ws + p.srec_off);
     float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
@@ -413,6 +415,16 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                 return s;
             p1.state_in = srec;
             p1.rec_out = rrec;
+        }
+        if constexpr (D == 64) {
+            // one segment per head with saved statistics: the pipelined pass
+            if (saved && p.seg.nseg == 1) {
+                if ((s = launch_bwd_kernel(la::bwd_dq64_kernel<PHI>, la::Bwd1x64Cfg::SMEM, p1,
+                                           heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
+                    return s;
+                return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI>, la::Bwd2x64Cfg::SMEM, p2,
+                                         heads, st, "bwd_dkdv", la::kBwd64Threads);
+            }
         }
         if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
                                            heads * p.seg.nseg, st, "bwd_dq")

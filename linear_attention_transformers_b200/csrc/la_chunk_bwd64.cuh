@@ -108,6 +108,38 @@ __device__ __forceinline__ void mask_pack_upper(uint32_t reg, int sp, int jrow, 
     tmem_wait_st();
 }
 
+// The same for a product with rows = query i and columns = key j, keeping
+// j <= i and adding the row's dg to the kept entries (pass 1's W').
+__device__ __forceinline__ void mask_pack_lower(uint32_t reg, int sp, int irow, float dg) {
+    using namespace sm100;
+#pragma unroll 1
+    for (int b = 0; b < 4; ++b) {
+        const int j0 = 32 * b;
+        float pk[16];
+        if (b > sp) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) pk[t] = 0.f;
+        } else {
+            float v[32];
+            tmem_load<32>(reg + j0, v);
+            if (b == sp) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int j = j0 + 2 * t;
+                    pk[t] = __uint_as_float(pack_bf16(j <= irow ? v[2 * t] + dg : 0.f,
+                                                      j + 1 <= irow ? v[2 * t + 1] + dg : 0.f));
+                }
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    pk[t] = __uint_as_float(pack_bf16(v[2 * t] + dg, v[2 * t + 1] + dg));
+            }
+        }
+        tmem_st16(reg + j0 / 2, pk);
+    }
+    tmem_wait_st();
+}
+
 template <int PHI>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
@@ -448,6 +480,353 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 if (!mbar_wait(staged, t & 1, abort_flag)) break;
                 tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
                 tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(&empty[s]);
+            }
+            bulk_wait0();
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, Cfg::T_COLS);
+}
+
+// ======================================================================
+// Pass 1 (dQ), causal, with the forward's saved O and g, one segment per
+// head.  Per chunk c (token order), S / z = state of the earlier chunks:
+//
+//   dU = dO / g,  dg = -(dO . o) / g          (feature-map warps)
+//   W  = dU V^T,  W' = (W + dg 1^T).M         (M: keep key j <= query i)
+//   dA = dU S^T + W' B,  dQ = (dA + dg z^T) * phi'(q)
+//   T  = [V | 1]^T B accumulated: rows 0..63 = S^T, row 64 = z^T
+//
+// A = phi(q) is not needed here (only phi'(q), formed in the epilogue from
+// the raw q tile, which then stages dQ in place).  Same warp roles and
+// hand-offs as bwd_dkdv64_kernel; W and dA are double-buffered in TMEM.
+// ======================================================================
+struct Bwd1x64Cfg {
+    static constexpr int C = 128, D = 64;
+    static constexpr int NSTAGE = 3;
+    static constexpr int TILE = C * D * 2;             // 16 KB
+    static constexpr int OFF_DGF = 4 * TILE;           // in-stage: dg float [C]
+    static constexpr int STAGE = ((OFF_DGF + C * 4) + 1023) / 1024 * 1024;
+    static constexpr int OFF_ONES = NSTAGE * STAGE;    // [C][64] atom, column 0 = 1
+    static constexpr int OFF_SX = OFF_ONES + TILE;     // S^T, bf16 [D][D] row tile (row v)
+    static constexpr int OFF_ZF = OFF_SX + D * D * 2;  // z, float [2][D] (by chunk parity)
+    static constexpr int OFF_BAR = OFF_ZF + 2 * D * 4;
+    static constexpr int NBAR = 3 * NSTAGE + 10;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 16 + 1024;
+    // TMEM columns: W [2][C], dA [2][D], T [D]
+    static constexpr int T_W = 0, T_DA = 2 * C, T_T = 2 * C + 2 * D;
+    static constexpr int T_COLS = 512;
+    static_assert(T_T + D <= T_COLS, "TMEM budget");
+    static_assert(SMEM <= 227 * 1024, "shared memory budget");
+    static_assert(OFF_ONES % 1024 == 0 && OFF_SX % 1024 == 0, "swizzled tiles on 1 KB");
+};
+
+template <int PHI>
+__global__ void __launch_bounds__(kBwd64Threads, 1)
+bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
+    using namespace sm100;
+    using Cfg = Bwd1x64Cfg;
+    constexpr int C = Cfg::C, D = Cfg::D, NS = Cfg::NSTAGE;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
+    uint64_t* full = bars;                // TMA
+    uint64_t* phi_done = bars + NS;       // 256 feature-map threads
+    uint64_t* empty = bars + 2 * NS;      // MMA commit + the store warp
+    uint64_t* w_full = bars + 3 * NS;     // commit: W
+    uint64_t* wp_full = w_full + 1;       // 128: W' packed
+    uint64_t* t_full = w_full + 2;        // commit: state update
+    uint64_t* sx_full = w_full + 3;       // 128: S^T operand and z written
+    uint64_t* da_full = w_full + 4;       // [2] commit: dA complete
+    uint64_t* da_free = w_full + 6;       // [2] 128: dA read
+    uint64_t* staged = w_full + 8;        // 128: dQ rows staged
+    uint64_t* drain = w_full + 9;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int tok0 = seg * prm.seg_len;
+    const int tok1 = min(prm.N, tok0 + prm.seg_len);
+    const int nchunks = (tok1 - tok0 + C - 1) / C;
+    auto row_of = [&](int c) { return tok0 + c * C; };
+
+    if (tid == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&phi_done[s], 256);
+            mbar_init(&empty[s], 2);
+        }
+        mbar_init(w_full, 1);
+        mbar_init(wp_full, 128);
+        mbar_init(t_full, 1);
+        mbar_init(sx_full, 128);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&da_full[b], 1);
+            mbar_init(&da_free[b], 128);
+        }
+        mbar_init(staged, 128);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, Cfg::T_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&prm.tm_q);
+            tma_prefetch_desc(&prm.tm_k);
+            tma_prefetch_desc(&prm.tm_v);
+            tma_prefetch_desc(&prm.tm_do);
+            auto prefetch = [&](int c) {
+                if (c < nchunks) {
+                    const int row = row_of(c);
+                    tma_prefetch_l2_3d(&prm.tm_q, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_k, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_v, 0, row, head);
+                    tma_prefetch_l2_3d(&prm.tm_do, 0, row, head);
+                }
+            };
+            prefetch(NS);
+            int issued = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS;
+                prefetch(c + NS + 1);
+                if (c >= NS && !mbar_wait(&empty[s], ((c / NS) - 1) & 1, abort_flag)) break;
+                uint8_t* st = smem + s * Cfg::STAGE;
+                mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
+                const int row = row_of(c);
+                tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, head);
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, head);
+                tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
+                issued = c + 1;
+            }
+            for (int c = max(0, issued - NS); c < issued; ++c)
+                mbar_wait_drain(&full[c % NS], (c / NS) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t tW = tmem + Cfg::T_W, tDA = tmem + Cfg::T_DA, tT = tmem + Cfg::T_T;
+            const uint32_t sx = sbase + Cfg::OFF_SX, ones = sbase + Cfg::OFF_ONES;
+            constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);     // dU V^T
+            constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);  // B operand rows = K
+            constexpr uint32_t idT = idesc_bf16(128, D, 1, 1);    // [V | 1]^T B
+            bool ok = true;
+            for (int c = 0; ok && c < nchunks; ++c) {
+                const int s = c % NS, b = c & 1;
+                const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
+                const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
+                tc_fence_after();
+                // W = dU V^T
+#pragma unroll
+                for (int k = 0; k < D; k += 16)
+                    umma_bf16(tW + b * C, desc_kmajor(dus, C, k), desc_kmajor(vs, C, k), idCC, k > 0);
+                umma_commit(w_full);
+                // dA = dU S^T (state of the earlier chunks), then the state update
+                if (!(ok = mbar_wait(sx_full, c & 1, abort_flag))) break;
+                if (c >= 2 && !(ok = mbar_wait(&da_free[b], ((c >> 1) - 1) & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D; k += 16)
+                    umma_bf16(tDA + b * D, desc_kmajor(dus, C, k), desc_mnmajor(sx, D, k), idCD_mn, k > 0);
+                if (c + 1 < nchunks) {
+                    const uint64_t dvx = sdesc_sw128(vs, ones - vs, 1024);
+                    const uint64_t dkm = desc_mn_base(ks, C);
+#pragma unroll
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tT, dvx + kstep_mn(k), dkm + kstep_mn(k), idT, (c > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(t_full);
+                }
+                // dA += W' B (W' packed in TMEM)
+                if (!(ok = mbar_wait(wp_full, c & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C; k += 16)
+                    umma_bf16_ts(tDA + b * D, tW + b * C + k / 2, desc_mnmajor(ks, C, k), idCD_mn, 1);
+                umma_commit(&da_full[b]);
+                umma_commit(&empty[s]);
+            }
+            umma_commit(drain);
+            mbar_wait_drain(drain, 0);
+        }
+    } else if (warp < 10) {
+        // warps 2-5: phi on K in place; warps 6-9: dU = dO / g in place and
+        // dg = -(dO . o) / g, one row per thread
+        const int u = tid - 64;  // 0..255
+        const int r = u - 128;   // row for the dU / dg threads
+        const float* gb = prm.gbuf + size_t(head) * prm.N;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS;
+            const int row0 = row_of(c);
+            const int nvalid = min(C, tok1 - row0);
+            // this row's o and g, loaded while the tiles land
+            float g = 1.f;
+            uint4 ov[8];
+            if (r >= 0) {
+                const bool valid = r < nvalid;
+                const uint4* orow =
+                    reinterpret_cast<const uint4*>(prm.o_in + (size_t(head) * prm.N + row0 + r) * D);
+                g = valid ? gb[row0 + r] : 1.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ov[j] = valid ? __ldg(orow + j) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (!named_bar_all(3, 256, mbar_wait(&full[s], (c / NS) & 1, abort_flag))) break;
+            uint8_t* st = smem + s * Cfg::STAGE;
+            if (u < 128) {
+                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u, nvalid, true);
+            } else {
+                uint8_t* dot = st + 3 * Cfg::TILE;
+                const bool valid = r < nvalid;
+                float dotp = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 x = *reinterpret_cast<const uint4*>(dot + tile_chunk_off(C, r, j));
+                    const uint32_t a[4] = {x.x, x.y, x.z, x.w};
+                    const uint32_t bb[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 fa = unpack_bf16(a[t]), fb = unpack_bf16(bb[t]);
+                        dotp = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, dotp));
+                    }
+                }
+                const float ginv = 1.f / g;
+                const float dg = valid ? -dotp * ginv : 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4* px = reinterpret_cast<uint4*>(dot + tile_chunk_off(C, r, j));
+                    const uint4 x = *px;
+                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const float2 f = unpack_bf16(w[t]);
+                        w[t] = valid ? pack_bf16(f.x * ginv, f.y * ginv) : 0u;
+                    }
+                    *px = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+                reinterpret_cast<float*>(st + Cfg::OFF_DGF)[r] = dg;
+                if (valid) prm.dgbuf[size_t(head) * prm.N + row0 + r] = dg;
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&phi_done[s]);
+        }
+    } else if (warp < 14) {
+        // W' = (W + dg) masked, packed in place
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int irow = 32 * sp + lane;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS, b = c & 1;
+            if (!named_bar_all(1, 128, mbar_wait(w_full, c & 1, abort_flag))) break;
+            tc_fence_after();
+            const float dg = reinterpret_cast<const float*>(smem + s * Cfg::STAGE + Cfg::OFF_DGF)[irow];
+            mask_pack_lower(tmem + lane_base + Cfg::T_W + b * C, sp, irow, dg);
+            tc_fence_before();
+            mbar_arrive(wp_full);
+        }
+    } else if (warp < 18) {
+        // state readout (S^T operand, z) and the dQ epilogue (staged in place
+        // over the raw q tile)
+        const int sp = warp & 3;
+        const uint32_t lane_base = uint32_t(32 * sp) << 16;
+        const int irow = 32 * sp + lane;  // token row; lane of T = v
+        uint8_t* sxp = smem + Cfg::OFF_SX;
+        uint8_t* ones = smem + Cfg::OFF_ONES;
+        float* zf = reinterpret_cast<float*>(smem + Cfg::OFF_ZF);  // [2][D]
+        {
+            float v8[8] = {1.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int q = 0; q < 8; ++q) store_row_bf16<8>(ones, C, irow, 8 * q, q == 0 ? v8 : z8);
+            if (irow < D) {
+                for (int q = 0; q < 8; ++q) store_row_bf16<8>(sxp, D, irow, 8 * q, z8);
+                zf[irow] = 0.f;
+                zf[D + irow] = 0.f;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(sx_full);
+
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS, b = c & 1;
+            uint8_t* qt = smem + s * Cfg::STAGE;
+            if (c + 1 < nchunks) {
+                // state after this chunk -> operands of the next chunk
+                if (!named_bar_all(2, 128, mbar_wait(t_full, c & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    float col[32];
+                    tmem_load<32>(tmem + lane_base + Cfg::T_T + 32 * h, col);
+                    if (irow < D) {
+                        store_row_bf16<32>(sxp, D, irow, 32 * h, col);
+                    } else if (irow == D) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) zf[((c + 1) & 1) * D + 32 * h + i] = col[i];
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(sx_full);
+            }
+            // dQ = (dA + dg z) * phi'(q)
+            if (!named_bar_all(2, 128, mbar_wait(&da_full[b], (c >> 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const float dg = reinterpret_cast<const float*>(qt + Cfg::OFF_DGF)[irow];
+            const float* z = zf + (c & 1) * D;
+#pragma unroll 1
+            for (int f0 = 0; f0 < D; f0 += 16) {
+                float av[16];
+                tmem_ld16(tmem + lane_base + Cfg::T_DA + b * D + f0, av);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    float q8[8];
+                    load_chunk8(qt, C, irow, (f0 >> 3) + h, q8);
+                    const float4 za = reinterpret_cast<const float4*>(z + f0 + 8 * h)[0];
+                    const float4 zb = reinterpret_cast<const float4*>(z + f0 + 8 * h)[1];
+                    const float z8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+                    uint32_t w[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        w[i] = pack_bf16(fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) * dphi_fast<PHI>(q8[2 * i]),
+                                         fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) *
+                                             dphi_fast<PHI>(q8[2 * i + 1]));
+                    // this thread's row of q is read before it is overwritten
+                    *reinterpret_cast<uint4*>(qt + tile_chunk_off(C, irow, (f0 >> 3) + h)) =
+                        make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&da_free[b]);
+            fence_proxy_async_smem();
+            mbar_arrive(staged);
+        }
+    } else if (warp == 18) {
+        // TMA stores of the staged dQ rows; the stage is free once they have
+        // been read
+        if (lane == 0) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS;
+                if (!mbar_wait(staged, c & 1, abort_flag)) break;
+                tma_store_3d(&prm.tm_dq, smem + s * Cfg::STAGE, 0, row_of(c), head);
                 bulk_commit();
                 bulk_wait_read0();
                 mbar_arrive(&empty[s]);
