@@ -74,6 +74,26 @@ def test_backward_small(dtype, D, N, causal, phi, saved):
     compare(dv, rv, dtype, "dv")
 
 
+@pytest.mark.parametrize("N", [1, 129, 700])
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+def test_fwd_bwd_one_segment_per_head(N, phi):
+    """128 heads put one segment on each head (the timed layout), which runs
+    the D = 64 kernels without a segment split; ragged N, both feature maps,
+    the forward's o and g handed to the backward, every head checked."""
+    q, k, v, dO = small(8, 16, N, 64, torch.bfloat16, seed=N + 5, dO=True)
+    g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
+    o = api.la_forward(q, k, v, True, phi, g=g)
+    dq, dk, dv = api.la_backward(q, k, v, dO, True, phi, o=o, g=g)
+    torch.cuda.synchronize()
+    api.la_get_device_error()
+    o_ref, _, _ = oracle.forward(q, k, v, True, PHIS[phi])
+    compare(o, o_ref, torch.bfloat16, "o")
+    rq, rk, rv = oracle.backward(q, k, v, dO, True, PHIS[phi])
+    compare(dq, rq, torch.bfloat16, "dq")
+    compare(dk, rk, torch.bfloat16, "dk")
+    compare(dv, rv, torch.bfloat16, "dv")
+
+
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("causal", [True, False])
 def test_forward_denominators(dtype, causal):
