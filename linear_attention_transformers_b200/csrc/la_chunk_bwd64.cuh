@@ -668,59 +668,55 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             mbar_wait_drain(drain, 0);
         }
     } else if (warp < 10) {
-        // warps 2-5: phi on K in place; warps 6-9: dU = dO / g in place and
-        // dg = -(dO . o) / g, one row per thread
+        // phi on K in place, then dU = dO / g in place and dg = -(dO . o) / g
+        // (two threads per row), all eight warps on each
         const int u = tid - 64;  // 0..255
-        const int r = u - 128;   // row for the dU / dg threads
+        const int r = u >> 1, part = u & 1;
         const float* gb = prm.gbuf + size_t(head) * prm.N;
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             const int row0 = row_of(c);
             const int nvalid = min(C, tok1 - row0);
+            const bool valid = r < nvalid;
             // this row's o and g, loaded while the tiles land
-            float g = 1.f;
-            uint4 ov[8];
-            if (r >= 0) {
-                const bool valid = r < nvalid;
-                const uint4* orow =
-                    reinterpret_cast<const uint4*>(prm.o_in + (size_t(head) * prm.N + row0 + r) * D);
-                g = valid ? gb[row0 + r] : 1.f;
+            const uint4* orow =
+                reinterpret_cast<const uint4*>(prm.o_in + (size_t(head) * prm.N + row0 + r) * D) + 4 * part;
+            const float g = valid ? gb[row0 + r] : 1.f;
+            uint4 ov[4];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) ov[j] = valid ? __ldg(orow + j) : make_uint4(0u, 0u, 0u, 0u);
-            }
+            for (int j = 0; j < 4; ++j) ov[j] = valid ? __ldg(orow + j) : make_uint4(0u, 0u, 0u, 0u);
             if (!named_bar_all(3, 256, mbar_wait(&full[s], (c / NS) & 1, abort_flag))) break;
             uint8_t* st = smem + s * Cfg::STAGE;
-            if (u < 128) {
-                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u, nvalid, true);
-            } else {
-                uint8_t* dot = st + 3 * Cfg::TILE;
-                const bool valid = r < nvalid;
-                float dotp = 0.f;
+            phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
+            uint8_t* dot = st + 3 * Cfg::TILE;
+            float dotp = 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 x = *reinterpret_cast<const uint4*>(dot + tile_chunk_off(C, r, j));
-                    const uint32_t a[4] = {x.x, x.y, x.z, x.w};
-                    const uint32_t bb[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
+            for (int j = 0; j < 4; ++j) {
+                const uint4 x = *reinterpret_cast<const uint4*>(dot + tile_chunk_off(C, r, 4 * part + j));
+                const uint32_t a[4] = {x.x, x.y, x.z, x.w};
+                const uint32_t bb[4] = {ov[j].x, ov[j].y, ov[j].z, ov[j].w};
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 fa = unpack_bf16(a[t]), fb = unpack_bf16(bb[t]);
-                        dotp = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, dotp));
-                    }
+                for (int t = 0; t < 4; ++t) {
+                    const float2 fa = unpack_bf16(a[t]), fb = unpack_bf16(bb[t]);
+                    dotp = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, dotp));
                 }
-                const float ginv = 1.f / g;
-                const float dg = valid ? -dotp * ginv : 0.f;
+            }
+            dotp += __shfl_xor_sync(0xffffffffu, dotp, 1);
+            const float ginv = 1.f / g;
+            const float dg = valid ? -dotp * ginv : 0.f;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint4* px = reinterpret_cast<uint4*>(dot + tile_chunk_off(C, r, j));
-                    const uint4 x = *px;
-                    uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            for (int j = 0; j < 4; ++j) {
+                uint4* px = reinterpret_cast<uint4*>(dot + tile_chunk_off(C, r, 4 * part + j));
+                const uint4 x = *px;
+                uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float2 f = unpack_bf16(w[t]);
-                        w[t] = valid ? pack_bf16(f.x * ginv, f.y * ginv) : 0u;
-                    }
-                    *px = make_uint4(w[0], w[1], w[2], w[3]);
+                for (int t = 0; t < 4; ++t) {
+                    const float2 f = unpack_bf16(w[t]);
+                    w[t] = valid ? pack_bf16(f.x * ginv, f.y * ginv) : 0u;
                 }
+                *px = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (part == 0) {
                 reinterpret_cast<float*>(st + Cfg::OFF_DGF)[r] = dg;
                 if (valid) prm.dgbuf[size_t(head) * prm.N + row0 + r] = dg;
             }
