@@ -5,7 +5,8 @@
 
 One step is one training pass of the attention layer on the timed workload
 (causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward (which also
-keeps the per-token denominators g) followed by la_backward given O and g,
+keeps the per-token denominators g and the feature maps phi(q), phi(k))
+followed by la_backward given O, g and the feature maps,
 through the library's Python binding, inputs resident in HBM.
 The inputs (4 x 128 MiB) are larger than the 126 MB L2, so consecutive steps
 cannot serve each other from cache.  W untimed warm-up steps, then exactly K
@@ -77,9 +78,10 @@ def algorithmic_bytes(kernel: str, w) -> float:
     table = {
         "fwd_generic": 4 * t,           # q, k, v -> o
         "bwd_generic": 7 * t,           # q, k, v, dO -> dq, dk, dv
-        "chunk_causal": 4 * t + n,      # q, k, v -> o, g
-        "bwd_dq": 6 * t + 2 * n,        # q, k, v, dO, o, g -> dq, dg
-        "bwd_dkdv": 6 * t + 2 * n,      # q, k, v, dO, g, dg -> dk, dv
+        "chunk_causal": 6 * t + n,      # q, k, v -> o, g, phi(q), phi(k)
+        "bwd_dq": 6 * t + 2 * n,        # phi(q), phi(k), v, dO, o, g -> dq, dg
+        "bwd_dkdv": 6 * t + 2 * n,      # phi(q), phi(k), v, dO, g, dg -> dk, dv
+        "phi_map": 4 * t,               # q, k -> phi(q), phi(k) (paths without a fused store)
     }
     return float(table.get(kernel, 0.0))
 
@@ -310,6 +312,10 @@ def run_ours(args, world, rank, local):
     B, H, N, D = q.shape
     o = torch.empty_like(q)
     g = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    # saved feature maps where the backward reads them (bf16, D = 64)
+    pq = pk = None
+    if api.backward_reads_phi(q.dtype, D):
+        pq, pk = torch.empty_like(q), torch.empty_like(q)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws_f = api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal, w.dtype)
     ws_b = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, w.causal, w.dtype)
@@ -317,10 +323,12 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        # forward keeps its denominators g; backward reuses O and g
-        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream, g=g)
+        # forward keeps its denominators g and feature maps; backward reuses
+        # O, g and phi(q), phi(k)
+        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream, g=g,
+                       phi_out=None if pq is None else (pq, pk))
         api.la_backward(q, k, v, dO, w.causal, w.phi, dq=dq, dk=dk, dv=dv, workspace=ws,
-                        stream=stream, o=o, g=g)
+                        stream=stream, o=o, g=g, phi_q=pq, phi_k=pk)
 
     for _ in range(args.warmup):
         step()

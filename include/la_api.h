@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define LA_API_VERSION 1
+#define LA_API_VERSION 2
 
 #if defined(__GNUC__)
 #define LA_EXPORT __attribute__((visibility("default")))
@@ -103,6 +103,10 @@ LA_EXPORT size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, in
  * which la_decode_step can continue from.  g_out [B, H, N], float32, may be
  * NULL; when given it receives the denominators g_i = phi(q_i) . z_i, which
  * la_backward accepts together with o to skip recomputing the forward.
+ * phi_q_out, phi_k_out ([B, H, N, D] of dtype `dt`) may both be NULL; when
+ * given (both) they receive phi(q) and phi(k) as the forward's products read
+ * them (rounded to `dt`), which la_backward accepts to skip evaluating the
+ * feature map again; one without the other is LA_ERR_INVALID_ARG.
  * Workspace: see la_workspace_size; may be NULL when that is 0.
  * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_WORKSPACE,
  * LA_ERR_CUDA.  On error nothing has been launched except for LA_ERR_CUDA,
@@ -110,6 +114,7 @@ LA_EXPORT size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, in
  */
 LA_EXPORT la_status la_forward(const void *q, const void *k, const void *v, void *o,
                      float *S_out, float *z_out, float *g_out,
+                     void *phi_q_out, void *phi_k_out,
                      int64_t B, int64_t H, int64_t N, int64_t D,
                      la_dtype dt, int causal, la_phi phi,
                      void *workspace, size_t workspace_bytes, la_stream_t stream);
@@ -121,12 +126,18 @@ LA_EXPORT la_status la_forward(const void *q, const void *k, const void *v, void
  * float32 [B, H, N]) are optional and go together: when both are NULL the
  * forward quantities are recomputed inside; when both are given they are
  * used instead (dU = dO/g and dg = -(dO . o)/g directly), which is faster.
+ * phi_q, phi_k (the forward's phi_q_out, phi_k_out) are optional as well,
+ * both or neither, and only together with o and g: when given, the head
+ * size 64 kernels read them in place of evaluating phi on q and k (phi'
+ * then comes from phi: min(phi, 1) for elu+1, 1 where phi exceeds the
+ * x <= 0 value for relu+eps); other paths ignore them.
  * No N x D x D tensor is ever stored: the prefix states are rebuilt chunk by
  * chunk.  dq/dk/dv must not alias the inputs.  Errors as la_forward; one of
- * o, g without the other is LA_ERR_INVALID_ARG.
+ * o, g without the other, one of phi_q, phi_k without the other, or them
+ * without o and g is LA_ERR_INVALID_ARG.
  */
 LA_EXPORT la_status la_backward(const void *q, const void *k, const void *v, const void *dO,
-                      const void *o, const float *g,
+                      const void *o, const float *g, const void *phi_q, const void *phi_k,
                       void *dq, void *dk, void *dv,
                       int64_t B, int64_t H, int64_t N, int64_t D,
                       la_dtype dt, int causal, la_phi phi,
@@ -169,6 +180,7 @@ LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void
 
 LA_EXPORT la_status la_backward_noalloc(const void *q, const void *k, const void *v,
                                         const void *dO, const void *o, const float *g,
+                                        const void *phi_q, const void *phi_k,
                                         void *dq, void *dk, void *dv,
                                         int64_t B, int64_t H, int64_t N, int64_t D,
                                         la_dtype dt, int causal, la_phi phi,

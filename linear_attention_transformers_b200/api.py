@@ -71,14 +71,14 @@ def load_library(path: str | None = None):
         vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.la_workspace_size.argtypes = [ci, i64, i64, i64, i64, ci, ci]
         lib.la_workspace_size.restype = sz
-        lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp,
-                                   sz, vp]
+        lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci,
+                                   ci, vp, sz, vp]
         lib.la_forward.restype = ci
-        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci,
-                                    ci, ci, vp, sz, vp]
+        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                    i64, ci, ci, ci, vp, sz, vp]
         lib.la_backward.restype = ci
-        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
-                                            i64, ci, ci, ci, vp]
+        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64,
+                                            i64, i64, ci, ci, ci, vp]
         lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
@@ -163,11 +163,13 @@ def _workspace(op, q, causal, workspace):
 
 
 def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=False,
-               workspace=None, stream=None, g=None):
+               workspace=None, stream=None, g=None, phi_out=None):
     """o = linear attention of q, k, v [B, H, N, D]; optionally the final (S, z).
 
     ``g``: optional float32 [B, H, N] tensor that receives the denominators;
     pass it with ``o`` to la_backward to skip the forward recompute there.
+    ``phi_out``: optional pair (pq, pk) of tensors shaped and typed like q
+    that receive phi(q), phi(k); pass them to la_backward with o and g.
     """
     lib = load_library()
     _check_qkv("la_forward", q, k, v)
@@ -185,17 +187,25 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
                           or not g.is_contiguous() or g.device != q.device):
         raise ValueError("la_forward: g must be contiguous float32 [B, H, N] on q's device")
+    pq = pk = None
+    if phi_out is not None:
+        pq, pk = phi_out
+        _check_qkv("la_forward", q, pq, pk)
     ws, ws_bytes = _workspace(LA_OP_FORWARD, q, causal, workspace)
-    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g), B, H, N, D,
-                        DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
-                        _stream_handle(stream))
+    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g), _ptr(pq),
+                        _ptr(pk), B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi),
+                        _ptr(ws), ws_bytes, _stream_handle(stream))
     _check("la_forward", st)
     return (o, S, z) if return_state else o
 
 
-def _check_saved(name, q, o, g):
+def _check_saved(name, q, o, g, phi_q=None, phi_k=None):
     if (o is None) != (g is None):
         raise ValueError(f"{name}: pass both o and g (saved forward statistics) or neither")
+    if (phi_q is None) != (phi_k is None) or (phi_q is not None and o is None):
+        raise ValueError(f"{name}: phi_q and phi_k go together, and only with o and g")
+    if phi_q is not None:
+        _check_qkv(name, q, phi_q, phi_k)
     if o is not None:
         _check_qkv(name, q, o)
         B, H, N, _ = q.shape
@@ -204,11 +214,13 @@ def _check_saved(name, q, o, g):
 
 
 def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, dv=None,
-                workspace=None, stream=None, o=None, g=None):
+                workspace=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
     """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi).
 
     ``o``, ``g``: the forward's output and denominators (la_forward(..., g=g));
-    when given, the backward does not recompute them.
+    when given, the backward does not recompute them.  ``phi_q``, ``phi_k``:
+    the forward's feature maps (la_forward(..., phi_out=(phi_q, phi_k))),
+    only with ``o`` and ``g``; when given, phi is not evaluated again.
     """
     lib = load_library()
     _check_qkv("la_backward", q, k, v, dO)
@@ -219,10 +231,10 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward", q, dq, dk, dv)
-    _check_saved("la_backward", q, o, g)
+    _check_saved("la_backward", q, o, g, phi_q, phi_k)
     ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
-    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
-                         _ptr(dk), _ptr(dv),
+    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(phi_q),
+                         _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
                          ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
@@ -230,7 +242,7 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
 
 
 def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None,
-                        dv=None, stream=None, o=None, g=None):
+                        dv=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
     """la_backward on the library's static device scratch (no workspace).
 
     For callers that cannot allocate device memory during the call; see
@@ -247,9 +259,10 @@ def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, d
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward_noalloc", q, dq, dk, dv)
-    _check_saved("la_backward_noalloc", q, o, g)
-    st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
-                                 _ptr(dk), _ptr(dv), B, H, N, D, DTYPE[q.dtype], int(bool(causal)),
+    _check_saved("la_backward_noalloc", q, o, g, phi_q, phi_k)
+    st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g),
+                                 _ptr(phi_q), _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N,
+                                 D, DTYPE[q.dtype], int(bool(causal)),
                                  _phi(phi), _stream_handle(stream))
     _check("la_backward_noalloc", st)
     return dq, dk, dv
@@ -299,6 +312,13 @@ def la_profile_collect() -> dict:
             for i in range(min(n, 64))}
 
 
+def backward_reads_phi(dtype, D: int) -> bool:
+    """True where la_backward reads saved phi(q), phi(k) instead of
+    evaluating the feature map (the bf16 head-size-64 kernels); elsewhere
+    they are ignored and asking the forward for them only costs a pass."""
+    return dtype == torch.bfloat16 and D == 64
+
+
 class LinearAttention(torch.autograd.Function):
     """torch autograd wrapper: forward and backward both run in liblinattn."""
 
@@ -307,15 +327,20 @@ class LinearAttention(torch.autograd.Function):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         B, H, N, _ = q.shape
         g = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-        o = la_forward(q, k, v, causal, phi, g=g)
-        # the output and its denominators are kept so the backward need not
-        # recompute the forward
-        ctx.save_for_backward(q, k, v, o, g)
+        pq = pk = None
+        if backward_reads_phi(q.dtype, q.shape[-1]):
+            pq, pk = torch.empty_like(q), torch.empty_like(k)
+        o = la_forward(q, k, v, causal, phi, g=g,
+                       phi_out=None if pq is None else (pq, pk))
+        # the output, its denominators and the feature maps are kept so the
+        # backward need not recompute the forward or evaluate phi again
+        ctx.save_for_backward(q, k, v, o, g, pq, pk)
         ctx.causal, ctx.phi = causal, phi
         return o
 
     @staticmethod
     def backward(ctx, dO):
-        q, k, v, o, g = ctx.saved_tensors
-        dq, dk, dv = la_backward(q, k, v, dO.contiguous(), ctx.causal, ctx.phi, o=o, g=g)
+        q, k, v, o, g, pq, pk = ctx.saved_tensors
+        dq, dk, dv = la_backward(q, k, v, dO.contiguous(), ctx.causal, ctx.phi, o=o, g=g,
+                                 phi_q=pq, phi_k=pk)
         return dq, dk, dv, None, None

@@ -21,6 +21,7 @@
 #include "la_common.cuh"
 #include "la_decode.cuh"
 #include "la_generic.cuh"
+#include "la_phi_map.cuh"
 #include "la_runtime.cuh"
 #include "la_sm100.cuh"
 #include "la_state.cuh"
@@ -202,7 +203,7 @@ la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
         return cuda_fail("cudaFuncSetAttribute", e);
     la::LaunchScope scope(name, st);
-    kern<<<unsigned(grid), la::kChunkThreads, smem, st>>>(prm);
+    kern<<<unsigned(grid), D == 64 ? la::kChunk64Threads : la::kChunkThreads, smem, st>>>(prm);
     return launch_status();
 }
 
@@ -229,8 +230,8 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
 
 template <int D, int PHI>
 la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, float* S_out,
-                          float* z_out, float* g_out, int64_t heads, int64_t N, int causal,
-                          const FwdPlan& p, char* ws, cudaStream_t st) {
+                          float* z_out, float* g_out, void* pq, void* pk, int64_t heads, int64_t N,
+                          int causal, const FwdPlan& p, char* ws, cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
     la::ChunkParams prm;
     memset(&prm, 0, sizeof(prm));
@@ -265,6 +266,13 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
         prm.z_out = z_out;
         prm.stride_S = int64_t(D) * D;
         prm.stride_z = D;
+        if (D == 64 && pq) {
+            // the D = 64 causal kernel stores its phi(q), phi(k) tiles itself
+            if (!make_qkv_map(&prm.tm_pq, pq, heads, N, D, C) ||
+                !make_qkv_map(&prm.tm_pk, pk, heads, N, D, C))
+                return LA_ERR_CUDA;
+            prm.store_phi = 1;
+        }
         return launch_chunk<D, C, PHI, la::MODE_CAUSAL>(prm, heads * p.seg.nseg, st, "chunk_causal");
     }
     // non-causal: segment sums -> totals -> query pass
@@ -292,12 +300,14 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
 
 template <int PHI>
 la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o, float* S_out,
-                            float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
-                            int causal, const FwdPlan& p, char* ws, cudaStream_t st) {
+                            float* z_out, float* g_out, void* pq, void* pk, int64_t heads,
+                            int64_t N, int64_t D, int causal, const FwdPlan& p, char* ws,
+                            cudaStream_t st) {
     if (D == 64)
-        return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, causal, p, ws,
-                                        st);
-    return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, causal, p, ws, st);
+        return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal,
+                                        p, ws, st);
+    return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal, p,
+                                     ws, st);
 }
 
 
@@ -362,7 +372,8 @@ la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64
 
 template <int D, int PHI>
 la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO,
-                          const void* o_saved, const float* g_saved, void* dq, void* dk, void* dv,
+                          const void* o_saved, const float* g_saved, const void* pq,
+                          const void* pk, void* dq, void* dk, void* dv,
                           int64_t heads, int64_t N, int causal, const BwdPlan& p, char* ws,
                           cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
@@ -383,6 +394,19 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     prm.o_in = static_cast<const __nv_bfloat16*>(o_saved);
     prm.dk_out = static_cast<__nv_bfloat16*>(dk);
     prm.dv_out = static_cast<__nv_bfloat16*>(dv);
+    // the D = 64 pipelined passes read phi(q), phi(k) through the q, k maps
+    // when the forward's feature maps are given
+    const bool pin = pq != nullptr;
+    CUtensorMap tm_pq, tm_pk;
+    if (pin && (!make_qkv_map(&tm_pq, pq, heads, N, D, C) || !make_qkv_map(&tm_pk, pk, heads, N, D, C)))
+        return LA_ERR_CUDA;
+    auto with_phi = [&](la::BwdParams b) {
+        if (pin) {
+            b.tm_q = tm_pq;
+            b.tm_k = tm_pk;
+        }
+        return b;
+    };
     const int64_t R = int64_t(D) * D + D;
     float* srec = reinterpret_cast<float*>(ws + p.srec_off);
     float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
@@ -419,11 +443,15 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
         if constexpr (D == 64) {
             // one segment per head with saved statistics: the pipelined pass
             if (saved && p.seg.nseg == 1) {
-                if ((s = launch_bwd_kernel(la::bwd_dq64_kernel<PHI>, la::Bwd1x64Cfg::SMEM, p1,
-                                           heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
+                if ((s = pin ? launch_bwd_kernel(la::bwd_dq64_kernel<PHI, true>, la::Bwd1x64Cfg::SMEM,
+                                                 with_phi(p1), heads, st, "bwd_dq", la::kBwd64Threads)
+                             : launch_bwd_kernel(la::bwd_dq64_kernel<PHI, false>, la::Bwd1x64Cfg::SMEM,
+                                                 p1, heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
                     return s;
-                return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI>, la::Bwd2x64Cfg::SMEM, p2,
-                                         heads, st, "bwd_dkdv", la::kBwd64Threads);
+                return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
+                                               with_phi(p2), heads, st, "bwd_dkdv", la::kBwd64Threads)
+                           : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
+                                               p2, heads, st, "bwd_dkdv", la::kBwd64Threads);
             }
         }
         if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
@@ -438,8 +466,12 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
             p2.state_in = rrec;
         }
         if constexpr (D == 64)
-            return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI>, la::Bwd2x64Cfg::SMEM, p2,
-                                     heads * p.seg.nseg, st, "bwd_dkdv", la::kBwd64Threads);
+            return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
+                                           with_phi(p2), heads * p.seg.nseg, st, "bwd_dkdv",
+                                           la::kBwd64Threads)
+                       : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
+                                           p2, heads * p.seg.nseg, st, "bwd_dkdv",
+                                           la::kBwd64Threads);
         else
             return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
                                      heads * p.seg.nseg, st, "bwd_dkdv");
@@ -474,14 +506,15 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
 
 template <int PHI>
 la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO,
-                            const void* o_saved, const float* g_saved, void* dq, void* dk, void* dv,
-                            int64_t heads, int64_t N, int64_t D, int causal, const BwdPlan& p,
-                            char* ws, cudaStream_t st) {
+                            const void* o_saved, const float* g_saved, const void* pq,
+                            const void* pk, void* dq, void* dk, void* dv, int64_t heads, int64_t N,
+                            int64_t D, int causal, const BwdPlan& p, char* ws, cudaStream_t st) {
     if (D == 64)
-        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, dq, dk, dv, heads, N,
-                                        causal, p, ws, st);
-    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, dq, dk, dv, heads, N, causal,
-                                     p, ws, st);
+        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
+                                        N, causal, p, ws, st);
+    // the D = 128 kernels evaluate the feature map themselves
+    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk, dv,
+                                     heads, N, causal, p, ws, st);
 }
 
 // ------------------------------------------------------------ generic path
@@ -568,6 +601,19 @@ struct BwdOp {
 };
 
 template <typename T, int PHI>
+struct PhiMapOp {
+    static la_status run(const void* q, const void* k, void* pq, void* pk, int64_t n,
+                         cudaStream_t st) {
+        la::LaunchScope scope("phi_map", st);
+        const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(kNumSM) * 16);
+        la::phi_map_kernel<T, PHI><<<unsigned(blocks), 256, 0, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<T*>(pq),
+            static_cast<T*>(pk), n);
+        return launch_status();
+    }
+};
+
+template <typename T, int PHI>
 struct DecodeOp {
     static la_status run(float* S, float* z, const void* q, const void* k, const void* v,
                          void* o, int64_t heads, int64_t D, cudaStream_t st) {
@@ -641,15 +687,17 @@ size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, i
 }
 
 la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
-                     float* z_out, float* g_out, int64_t B, int64_t H, int64_t N, int64_t D,
-                     la_dtype dt, int causal, la_phi phi, void* workspace, size_t workspace_bytes,
-                     la_stream_t stream) {
+                     float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
+                     int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                     void* workspace, size_t workspace_bytes, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
     if ((S_out && !aligned16(S_out)) || (z_out && !aligned16(z_out)) ||
         (g_out && !aligned16(g_out)))
         return LA_ERR_INVALID_ARG;
+    // feature-map outputs: both or neither
+    if ((phi_q_out == nullptr) != (phi_k_out == nullptr)) return LA_ERR_INVALID_ARG;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t heads = B * H;
@@ -664,24 +712,34 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
     }
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
+    if (phi_q_out && ((s = check_ptr(phi_q_out)) || (s = check_ptr(phi_k_out)))) return s;
     const FwdPlan plan = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
     if (plan.bytes > 0 && (workspace == nullptr || workspace_bytes < plan.bytes))
         return LA_ERR_WORKSPACE;
     if ((s = bind_context()) != LA_OK) return s;
+    // the D = 64 causal kernel stores phi(q), phi(k) from its own tiles;
+    // every other path writes them with one elementwise pass
+    const bool phi_fused = plan.fast && D == 64 && causal;
     if (plan.fast) {
         char* ws = static_cast<char*>(workspace);
-        return phi == LA_PHI_ELU1
-                   ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, heads, N, D,
-                                                 causal ? 1 : 0, plan, ws, st)
-                   : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, heads, N, D,
-                                                     causal ? 1 : 0, plan, ws, st);
+        void* pq = phi_fused ? phi_q_out : nullptr;
+        void* pk = phi_fused ? phi_k_out : nullptr;
+        s = phi == LA_PHI_ELU1
+                ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N,
+                                              D, causal ? 1 : 0, plan, ws, st)
+                : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads,
+                                                  N, D, causal ? 1 : 0, plan, ws, st);
+    } else {
+        s = dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D,
+                            causal ? 1 : 0, st);
     }
-    return dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D, causal ? 1 : 0,
-                           st);
+    if (s != LA_OK || phi_q_out == nullptr || phi_fused) return s;
+    return dispatch<PhiMapOp>(dt, phi, q, k, phi_q_out, phi_k_out, heads * N * D, st);
 }
 
 la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
-                      const void* o, const float* g, void* dq, void* dk, void* dv, int64_t B,
+                      const void* o, const float* g, const void* phi_q, const void* phi_k,
+                      void* dq, void* dk, void* dv, int64_t B,
                       int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
                       void* workspace, size_t workspace_bytes, la_stream_t stream) {
     la_status s;
@@ -696,6 +754,9 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     // saved forward statistics: both or neither
     if ((o == nullptr) != (g == nullptr)) return LA_ERR_INVALID_ARG;
     if (o && ((s = check_ptr(o)) || (s = check_ptr(g)))) return s;
+    // saved feature maps: both or neither, and only with o and g
+    if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
+    if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
     const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -704,10 +765,10 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     if (bp.fast) {
         char* wsp = static_cast<char*>(workspace);
         return phi == LA_PHI_ELU1
-                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, dq, dk, dv, heads, N, D,
-                                                 causal ? 1 : 0, bp, wsp, st)
-                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, dq, dk, dv, heads, N, D,
-                                                     causal ? 1 : 0, bp, wsp, st);
+                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
+                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st)
+                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
+                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st);
     }
     const BwdWorkspace w = plan_bwd(B, H, N);
     char* ws = static_cast<char*>(workspace);
@@ -718,7 +779,8 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
 }
 
 la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
-                              const void* o, const float* g, void* dq, void* dk, void* dv,
+                              const void* o, const float* g, const void* phi_q,
+                              const void* phi_k, void* dq, void* dk, void* dv,
                               int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, int causal,
                               la_phi phi, la_stream_t stream) {
     la_status s;
@@ -734,7 +796,8 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
     if ((s = bind_context()) != LA_OK) return s;
     void* scratch = nullptr;
     if ((s = static_scratch(&scratch)) != LA_OK) return s;
-    return la_backward(q, k, v, dO, o, g, dq, dk, dv, B, H, N, D, dt, causal, phi, scratch,
+    return la_backward(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, N, D, dt, causal, phi,
+                       scratch,
                        size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 

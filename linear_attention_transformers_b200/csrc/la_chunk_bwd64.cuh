@@ -140,7 +140,9 @@ __device__ __forceinline__ void mask_pack_lower(uint32_t reg, int sp, int irow, 
     tmem_wait_st();
 }
 
-template <int PHI>
+// PIN: the q and k maps hold phi(q), phi(k) from the forward (no feature
+// map is evaluated here).
+template <int PHI, bool PIN>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
@@ -351,10 +353,12 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 dgf[u] = d;
             }
             named_bar_sync(3, 256);  // rinv ready
-            if (u < 128)
-                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
-            else
-                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+            if constexpr (!PIN) {
+                if (u < 128)
+                    phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+                else
+                    phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+            }
             scale_tile_rows<C, D, 256>(st + 3 * Cfg::TILE, u, nvalid, rinv);
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
@@ -528,7 +532,7 @@ struct Bwd1x64Cfg {
     static_assert(OFF_ONES % 1024 == 0 && OFF_SX % 1024 == 0, "swizzled tiles on 1 KB");
 };
 
-template <int PHI>
+template <int PHI, bool PIN>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
@@ -687,7 +691,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             for (int j = 0; j < 4; ++j) ov[j] = valid ? __ldg(orow + j) : make_uint4(0u, 0u, 0u, 0u);
             if (!named_bar_all(3, 256, mbar_wait(&full[s], (c / NS) & 1, abort_flag))) break;
             uint8_t* st = smem + s * Cfg::STAGE;
-            phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
+            if constexpr (!PIN) phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
             uint8_t* dot = st + 3 * Cfg::TILE;
             float dotp = 0.f;
 #pragma unroll
@@ -801,10 +805,12 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                     const float z8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
                     uint32_t w[4];
 #pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        q8[i] = PIN ? dphi_from_phi<PHI>(q8[i]) : dphi_fast<PHI>(q8[i]);
+#pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        w[i] = pack_bf16(fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) * dphi_fast<PHI>(q8[2 * i]),
-                                         fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) *
-                                             dphi_fast<PHI>(q8[2 * i + 1]));
+                        w[i] = pack_bf16(fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) * q8[2 * i],
+                                         fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) * q8[2 * i + 1]);
                     // this thread's row of q is read before it is overwritten
                     *reinterpret_cast<uint4*>(qt + tile_chunk_off(C, irow, (f0 >> 3) + h)) =
                         make_uint4(w[0], w[1], w[2], w[3]);

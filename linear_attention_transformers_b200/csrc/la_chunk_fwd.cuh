@@ -59,6 +59,10 @@ struct ChunkParams {
     // Optional [heads][N] output of the denominators g_i = phi(q_i) . z_i
     // (CAUSAL and QUERY), which lets the backward skip recomputing them.
     float* g_out;
+    // Optional outputs phi(q), phi(k) (same layout as q, k): the bf16 tiles
+    // the products read, stored by TMA (D = 64 CAUSAL kernel, store_phi != 0).
+    CUtensorMap tm_pq, tm_pk;
+    int store_phi;
 };
 
 template <int D, int C>

@@ -50,8 +50,13 @@ struct Chunk64Cfg {
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
+// Warp 18 stores phi(q), phi(k) when asked (CAUSAL): it waits for the
+// feature map of each chunk, stores the two tiles by TMA and releases the
+// stage once the stores have read it.
+constexpr int kChunk64Threads = 608;
+
 template <int PHI, int MODE>
-__global__ void __launch_bounds__(kChunkThreads, 1)
+__global__ void __launch_bounds__(kChunk64Threads, 1)
 chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
     using namespace sm100;
     using Cfg = Chunk64Cfg;
@@ -92,7 +97,7 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&phi_done[s], 256);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], (MODE == MODE_CAUSAL && prm.store_phi) ? 2 : 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&p_full[b], 1);
@@ -293,7 +298,7 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 mbar_arrive(pt_full);
             }
         }
-    } else {
+    } else if (warp < 18) {
         const int e = tid - 448;
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
@@ -434,6 +439,20 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 }
             }
             if (e == 0) bulk_wait0();
+        }
+    } else if (warp == 18) {
+        if (MODE == MODE_CAUSAL && prm.store_phi && lane == 0) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS;
+                if (!mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag)) break;
+                const uint8_t* st = smem + s * Cfg::STAGE;
+                tma_store_3d(&prm.tm_pq, st, 0, tok0 + c * C, head);
+                tma_store_3d(&prm.tm_pk, st + Cfg::TILE, 0, tok0 + c * C, head);
+                bulk_commit();
+                bulk_wait_read0();
+                mbar_arrive(&empty[s]);
+            }
+            bulk_wait0();
         }
     }
 

@@ -35,7 +35,7 @@ def test_header_declares_the_documented_entry_points():
 def test_library_exports_every_declared_symbol(lib):
     missing = [n for n in declared_functions() if not hasattr(lib, n)]
     assert not missing, missing
-    assert lib.la_version() == 1
+    assert lib.la_version() == 2
 
 
 def test_status_strings(lib):
@@ -48,14 +48,15 @@ FAKE = 0x100000  # aligned, non-null, never dereferenced: every use below must f
 
 
 def fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, S=None, z=None, g=None, B=1, H=1, N=8, D=64, dt=1,
-        causal=1, phi=0, ws=None, ws_bytes=0):
-    return lib.la_forward(q, k, v, o, S, z, g, B, H, N, D, dt, causal, phi, ws, ws_bytes, None)
+        causal=1, phi=0, ws=None, ws_bytes=0, pq=None, pk=None):
+    return lib.la_forward(q, k, v, o, S, z, g, pq, pk, B, H, N, D, dt, causal, phi, ws, ws_bytes,
+                          None)
 
 
 def bwd(lib, p=FAKE, B=1, H=1, N=8, D=64, dt=1, causal=1, phi=0, ws=None, ws_bytes=0, dq=FAKE,
-        o=None, g=None):
-    return lib.la_backward(p, p, p, p, o, g, dq, p, p, B, H, N, D, dt, causal, phi, ws, ws_bytes,
-                           None)
+        o=None, g=None, pq=None, pk=None):
+    return lib.la_backward(p, p, p, p, o, g, pq, pk, dq, p, p, B, H, N, D, dt, causal, phi, ws,
+                           ws_bytes, None)
 
 
 def test_rejects_bad_arguments_before_launch(lib):
@@ -74,6 +75,11 @@ def test_rejects_bad_arguments_before_launch(lib):
     # saved forward statistics go together: o without g is refused
     need = lib.la_workspace_size(api.LA_OP_BACKWARD, 1, 1, 8, 64, 1, api.LA_BF16)
     assert bwd(lib, o=FAKE, g=None, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
+    # feature maps go together, and only with o and g
+    assert fwd(lib, pq=FAKE) == api.LA_ERR_INVALID_ARG
+    assert fwd(lib, pq=FAKE, pk=FAKE + 4) == api.LA_ERR_INVALID_ARG   # misaligned
+    assert bwd(lib, pq=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
+    assert bwd(lib, o=FAKE, g=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
     p = FAKE
     assert lib.la_decode_step(p, p, p, p, p, None, 2, 2, 64, 1, 0, None) == api.LA_ERR_INVALID_ARG
     assert lib.la_decode_step(p, p, p, p, p, p, 2, 2, 40, 1, 0, None) == api.LA_ERR_UNSUPPORTED

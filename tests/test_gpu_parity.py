@@ -57,14 +57,20 @@ def check_state(S, z, S_ref, z_ref, dtype):
 @pytest.mark.parametrize("N", [1, 129, 777])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
-@pytest.mark.parametrize("saved", [False, True])
+@pytest.mark.parametrize("saved", ["none", "o_g", "o_g_phi"])
 def test_backward_small(dtype, D, N, causal, phi, saved):
     q, k, v, dO = small(2, 2, N, D, dtype, seed=N * 11 + D, dO=True)
-    if saved:
-        # the forward's output and denominators handed to the backward
+    if saved != "none":
+        # the forward's output and denominators (and feature maps) handed to
+        # the backward
         g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
-        o = api.la_forward(q, k, v, causal, phi, g=g)
-        dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi, o=o, g=g)
+        if saved == "o_g_phi":
+            pq, pk = torch.empty_like(q), torch.empty_like(k)
+            o = api.la_forward(q, k, v, causal, phi, g=g, phi_out=(pq, pk))
+            dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi, o=o, g=g, phi_q=pq, phi_k=pk)
+        else:
+            o = api.la_forward(q, k, v, causal, phi, g=g)
+            dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi, o=o, g=g)
     else:
         dq, dk, dv = api.la_backward(q, k, v, dO, causal, phi)
     torch.cuda.synchronize()
@@ -76,14 +82,21 @@ def test_backward_small(dtype, D, N, causal, phi, saved):
 
 @pytest.mark.parametrize("N", [1, 129, 700])
 @pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
-def test_fwd_bwd_one_segment_per_head(N, phi):
+@pytest.mark.parametrize("with_phi", [False, True])
+def test_fwd_bwd_one_segment_per_head(N, phi, with_phi):
     """128 heads put one segment on each head (the timed layout), which runs
     the D = 64 kernels without a segment split; ragged N, both feature maps,
-    the forward's o and g handed to the backward, every head checked."""
+    the forward's o and g (and phi(q), phi(k)) handed to the backward, every
+    head checked."""
     q, k, v, dO = small(8, 16, N, 64, torch.bfloat16, seed=N + 5, dO=True)
     g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
-    o = api.la_forward(q, k, v, True, phi, g=g)
-    dq, dk, dv = api.la_backward(q, k, v, dO, True, phi, o=o, g=g)
+    if with_phi:
+        pq, pk = torch.empty_like(q), torch.empty_like(k)
+        o = api.la_forward(q, k, v, True, phi, g=g, phi_out=(pq, pk))
+        dq, dk, dv = api.la_backward(q, k, v, dO, True, phi, o=o, g=g, phi_q=pq, phi_k=pk)
+    else:
+        o = api.la_forward(q, k, v, True, phi, g=g)
+        dq, dk, dv = api.la_backward(q, k, v, dO, True, phi, o=o, g=g)
     torch.cuda.synchronize()
     api.la_get_device_error()
     o_ref, _, _ = oracle.forward(q, k, v, True, PHIS[phi])
@@ -92,6 +105,27 @@ def test_fwd_bwd_one_segment_per_head(N, phi):
     compare(dq, rq, torch.bfloat16, "dq")
     compare(dk, rk, torch.bfloat16, "dk")
     compare(dv, rv, torch.bfloat16, "dv")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("D", [32, 64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,H", [(2, 2), (8, 16)])
+def test_forward_feature_map_outputs(dtype, D, causal, B, H):
+    """phi(q), phi(k) written by the forward (stored from the D = 64 causal
+    kernel's own tiles, by an elementwise pass elsewhere) are the oracle's
+    feature map rounded to the tensor dtype: within half an ulp of it plus
+    the exponential's error."""
+    N = 300
+    q, k, v = small(B, H, N, D, dtype, seed=D + N)
+    pq, pk = torch.empty_like(q), torch.empty_like(k)
+    api.la_forward(q, k, v, causal, "elu1", phi_out=(pq, pk))
+    torch.cuda.synchronize()
+    rel = 2.0 ** -8 if dtype == torch.bfloat16 else 1e-6
+    for name, got, x in (("phi(q)", pq, q), ("phi(k)", pk, k)):
+        ref = oracle.phi_map(x, oracle.PHI_ELU1)
+        err = np.abs(got.double().cpu().numpy() - ref)
+        assert (err <= rel * np.abs(ref) + 1e-30).all(), f"{name}: max rel {np.max(err / ref):.3e}"
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -202,12 +236,14 @@ def run_workload(w, full_check: bool):
     dev_inputs = [t.to(DEV) for t in dev_inputs]
     q, k, v = dev_inputs[:3]
     # the launch configuration the benchmark times: the forward keeps its
-    # denominators and the backward uses them with the output
+    # denominators and feature maps and the backward uses them with the output
     g = torch.empty(q.shape[:3], dtype=torch.float32, device=DEV)
-    o = api.la_forward(q, k, v, w.causal, w.phi, g=g)
+    pq, pk = torch.empty_like(q), torch.empty_like(k)
+    o = api.la_forward(q, k, v, w.causal, w.phi, g=g, phi_out=(pq, pk))
     grads = None
     if w.backward:
-        grads = api.la_backward(q, k, v, dev_inputs[3], w.causal, w.phi, o=o, g=g)
+        grads = api.la_backward(q, k, v, dev_inputs[3], w.causal, w.phi, o=o, g=g, phi_q=pq,
+                                phi_k=pk)
     torch.cuda.synchronize()
     api.la_get_device_error()
     if full_check:
