@@ -235,15 +235,13 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);     // A^T dU
             constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);   // A^T [dg_hi; dg_lo]
             const bool has_init = st_in != nullptr;
-            bool ok = true;
-            for (int t = 0; ok && t < nchunks; ++t) {
+            // X1 = B A^T, X2 = V dU^T (raw, fp32) of step t
+            auto x_raw = [&](int t) -> bool {
                 const int s = t % NS;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
-                const uint32_t dgs = qs + Cfg::OFF_DG;
-                if (!(ok = mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag))) break;
+                if (!mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag)) return false;
                 tc_fence_after();
-                // X1 = B A^T, X2 = V dU^T (raw, fp32)
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
                     umma_bf16(tX1, desc_kmajor(ks, C, k), desc_kmajor(qs, C, k), idCC, k > 0);
@@ -252,28 +250,43 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 for (int k = 0; k < D; k += 16)
                     umma_bf16(tX2, desc_kmajor(vs, C, k), desc_kmajor(dus, C, k), idCC, k > 0);
                 umma_commit(x2_full);
-                // dV = B R, dB = V R^T from the state of the later chunks
-                if (!(ok = mbar_wait(rx_full, t & 1, abort_flag))) break;
+                return true;
+            };
+            // Order per step t (software-pipelined): dV = X1 dU and dB = X2 A
+            // first (they start the accumulators), then the state terms
+            // dV += B R, dB += V R^T, then step t+1's raw products, then the
+            // state update with step t.  The packed X1/X2 of step t are read
+            // before step t+1's raw products overwrite them (MMAs run in
+            // issue order); the state accumulator is read out (rx_full)
+            // before its next update.
+            bool ok = nchunks == 0 || x_raw(0);
+            for (int t = 0; ok && t < nchunks; ++t) {
+                const int s = t % NS;
+                const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
+                const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                const uint32_t dgs = qs + Cfg::OFF_DG;
                 if (t > 0 && !(ok = mbar_wait(d_free, (t - 1) & 1, abort_flag))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < D; k += 16) {
-                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_mnmajor(rp, D, k), idCD_mn, k > 0);
-                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_kmajor(rp, D, k), idCD_k, k > 0);
-                }
-                // dV += X1 dU, dB += X2 A (A operands packed in TMEM)
                 if (!(ok = mbar_wait(x1p_full, t & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C; k += 16)
-                    umma_bf16_ts(tDV, tX1 + k / 2, desc_mnmajor(dus, C, k), idCD_mn, 1);
+                    umma_bf16_ts(tDV, tX1 + k / 2, desc_mnmajor(dus, C, k), idCD_mn, k > 0);
                 if (!(ok = mbar_wait(x2p_full, t & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C; k += 16)
-                    umma_bf16_ts(tDB, tX2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, 1);
+                    umma_bf16_ts(tDB, tX2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, k > 0);
+                // dV += B R, dB += V R^T from the state of the later chunks
+                if (!(ok = mbar_wait(rx_full, t & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D; k += 16) {
+                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_mnmajor(rp, D, k), idCD_mn, 1);
+                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_kmajor(rp, D, k), idCD_k, 1);
+                }
                 umma_commit(d_full);
                 if (t + 1 < nchunks) {
+                    if (!(ok = x_raw(t + 1))) break;
                     // R += A^T dU, r += A^T [dg_hi; dg_lo]
 #pragma unroll
                     for (int k = 0; k < C; k += 16) {
@@ -314,13 +327,17 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             }
         };
         load_gdg(0);
+        // with the forward's feature maps (PIN) warps 2-5 also mask and pack
+        // X2 (the X warpgroup then packs X1 only); a failed wait there is
+        // carried into the next group barrier so all eight warps leave together
+        bool ok_x2 = true;
         for (int t = 0; t < nchunks; ++t) {
             const int s = t % NS;
             const int row0 = row_of(t);
             const int nvalid = min(C, tok1 - row0);
             const float g = g_nx, dg = dg_nx;
             load_gdg(t + 1);
-            if (!named_bar_all(3, 256, mbar_wait(&full[s], (t / NS) & 1, abort_flag))) break;
+            if (!named_bar_all(3, 256, ok_x2 && mbar_wait(&full[s], (t / NS) & 1, abort_flag))) break;
             uint8_t* st = smem + s * Cfg::STAGE;
             float* dgf = reinterpret_cast<float*>(st + Cfg::OFF_DGF);
             float* rinv = reinterpret_cast<float*>(st + Cfg::OFF_RINV);
@@ -344,9 +361,20 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             scale_tile_rows<C, D, 256>(st + 3 * Cfg::TILE, u, nvalid, rinv);
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
+            if (PIN && warp < 6) {
+                const int sp = warp & 3;
+                ok_x2 = named_bar_all(4, 128, mbar_wait(x2_full, t & 1, abort_flag));
+                if (ok_x2) {
+                    tc_fence_after();
+                    mask_pack_upper(tmem + (uint32_t(32 * sp) << 16) + Cfg::T_X2, sp, 32 * sp + lane,
+                                    dgf);
+                    tc_fence_before();
+                    mbar_arrive(x2p_full);
+                }
+            }
         }
     } else if (warp < 14) {
-        // mask and pack X1 (keep i >= j) and X2 (+ dg_i) in place
+        // mask and pack X1 (keep i >= j) and, without PIN, X2 (+ dg_i) in place
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int jrow = 32 * sp + lane;
@@ -358,6 +386,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             mask_pack_upper(tmem + lane_base + Cfg::T_X1, sp, jrow, nullptr);
             tc_fence_before();
             mbar_arrive(x1p_full);
+            if (PIN) continue;  // X2 is packed by feature-map warps 2-5
             if (!named_bar_all(1, 128, mbar_wait(x2_full, t & 1, abort_flag))) break;
             tc_fence_after();
             mask_pack_upper(tmem + lane_base + Cfg::T_X2, sp, jrow, dgf);
