@@ -8,6 +8,22 @@
 
 namespace la {
 
+// elu(x)+1 on a pair of bf16 values, to bf16: max(x, 0) + e^min(x, 0),
+// with the min/max and the final add on the packed pair (exact for bf16:
+// one of the two terms is 0 or, for x > 0, e^0 = 1 and 1 + x is exact in
+// fp32 before the add rounds), so only the exponential runs in fp32.  The
+// results equal rounding fp32 elu(x)+1 to bf16; about 5 instructions per
+// element instead of 6.5.
+__device__ __forceinline__ uint32_t phi2_elu1(uint32_t w) {
+    uint32_t m, big, r;
+    asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w), "r"(0u));
+    asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(big) : "r"(w), "r"(0u));
+    const uint32_t e = sm100::pack_bf16(exp_fast(__uint_as_float(m << 16)),
+                                        exp_fast(__uint_as_float(m & 0xffff0000u)));
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(e), "r"(big));
+    return r;
+}
+
 // Apply the feature map in place to a [C][D] bf16 row tile.  The T threads
 // calling this split the tile's C*D/8 16-byte chunks evenly; each thread
 // loads all of its chunks before it computes so their latencies overlap.
@@ -31,8 +47,12 @@ __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool 
         uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const float2 f = unpack_bf16(w[k]);
-            w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
+            if (PHI == PHI_ELU1) {
+                w[k] = zero ? 0u : phi2_elu1(w[k]);
+            } else {
+                const float2 f = unpack_bf16(w[k]);
+                w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
+            }
         }
         x[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }
