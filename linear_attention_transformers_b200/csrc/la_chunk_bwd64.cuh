@@ -235,20 +235,25 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);     // A^T dU
             constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);   // A^T [dg_hi; dg_lo]
             const bool has_init = st_in != nullptr;
+            // base descriptors (k = 0), stepped along K by constant offsets,
+            // so each MMA costs the issuing thread few instructions
+            const uint64_t krp = desc_k_base(rp), mrp = desc_mn_base(rp, D);
             // X1 = B A^T, X2 = V dU^T (raw, fp32) of step t
             auto x_raw = [&](int t) -> bool {
                 const int s = t % NS;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                const uint64_t kq = desc_k_base(qs), kk = desc_k_base(ks);
+                const uint64_t kv = desc_k_base(vs), kdu = desc_k_base(dus);
                 if (!mbar_wait(&phi_done[s], (t / NS) & 1, abort_flag)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
-                    umma_bf16(tX1, desc_kmajor(ks, C, k), desc_kmajor(qs, C, k), idCC, k > 0);
+                    umma_bf16(tX1, kk + kstep_k(C, k), kq + kstep_k(C, k), idCC, k > 0);
                 umma_commit(x1_full);
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
-                    umma_bf16(tX2, desc_kmajor(vs, C, k), desc_kmajor(dus, C, k), idCC, k > 0);
+                    umma_bf16(tX2, kv + kstep_k(C, k), kdu + kstep_k(C, k), idCC, k > 0);
                 umma_commit(x2_full);
                 return true;
             };
@@ -265,24 +270,26 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
                 const uint32_t dgs = qs + Cfg::OFF_DG;
+                const uint64_t mq = desc_mn_base(qs, C), mdu = desc_mn_base(dus, C);
+                const uint64_t kk = desc_k_base(ks), kv = desc_k_base(vs), kdg = desc_k_base(dgs);
                 if (t > 0 && !(ok = mbar_wait(d_free, (t - 1) & 1, abort_flag))) break;
                 if (!(ok = mbar_wait(x1p_full, t & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C; k += 16)
-                    umma_bf16_ts(tDV, tX1 + k / 2, desc_mnmajor(dus, C, k), idCD_mn, k > 0);
+                    umma_bf16_ts(tDV, tX1 + k / 2, mdu + kstep_mn(k), idCD_mn, k > 0);
                 if (!(ok = mbar_wait(x2p_full, t & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C; k += 16)
-                    umma_bf16_ts(tDB, tX2 + k / 2, desc_mnmajor(qs, C, k), idCD_mn, k > 0);
+                    umma_bf16_ts(tDB, tX2 + k / 2, mq + kstep_mn(k), idCD_mn, k > 0);
                 // dV += B R, dB += V R^T from the state of the later chunks
                 if (!(ok = mbar_wait(rx_full, t & 1, abort_flag))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D; k += 16) {
-                    umma_bf16(tDV, desc_kmajor(ks, C, k), desc_mnmajor(rp, D, k), idCD_mn, 1);
-                    umma_bf16(tDB, desc_kmajor(vs, C, k), desc_kmajor(rp, D, k), idCD_k, 1);
+                    umma_bf16(tDV, kk + kstep_k(C, k), mrp + kstep_mn(k), idCD_mn, 1);
+                    umma_bf16(tDB, kv + kstep_k(C, k), krp + kstep_k(D, k), idCD_k, 1);
                 }
                 umma_commit(d_full);
                 if (t + 1 < nchunks) {
@@ -291,8 +298,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
 #pragma unroll
                     for (int k = 0; k < C; k += 16) {
                         const uint32_t acc = (t > 0 || has_init || k > 0) ? 1u : 0u;
-                        umma_bf16(tR, desc_mnmajor(qs, C, k), desc_mnmajor(dus, C, k), idDD, acc);
-                        umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgs, 16, k), idD16, acc);
+                        umma_bf16(tR, mq + kstep_mn(k), mdu + kstep_mn(k), idDD, acc);
+                        umma_bf16(tRZ, mq + kstep_mn(k), kdg + kstep_k(16, k), idD16, acc);
                     }
                     umma_commit(r_full);
                 }
@@ -633,17 +640,20 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);     // dU V^T
             constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);  // B operand rows = K
             constexpr uint32_t idT = idesc_bf16(128, D, 1, 1);    // [V | 1]^T B
+            const uint64_t msx = desc_mn_base(sx, D);
             bool ok = true;
             for (int c = 0; ok && c < nchunks; ++c) {
                 const int s = c % NS, b = c & 1;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
+                // base descriptors (k = 0), stepped along K by constant offsets
+                const uint64_t kdu = desc_k_base(dus), kv = desc_k_base(vs), mk = desc_mn_base(ks, C);
                 if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
                 tc_fence_after();
                 // W = dU V^T
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
-                    umma_bf16(tW + b * C, desc_kmajor(dus, C, k), desc_kmajor(vs, C, k), idCC, k > 0);
+                    umma_bf16(tW + b * C, kdu + kstep_k(C, k), kv + kstep_k(C, k), idCC, k > 0);
                 umma_commit(w_full);
                 // dA = dU S^T (state of the earlier chunks), then the state update
                 if (!(ok = mbar_wait(sx_full, c & 1, abort_flag))) break;
@@ -651,7 +661,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
-                    umma_bf16(tDA + b * D, desc_kmajor(dus, C, k), desc_mnmajor(sx, D, k), idCD_mn, k > 0);
+                    umma_bf16(tDA + b * D, kdu + kstep_k(C, k), msx + kstep_mn(k), idCD_mn, k > 0);
                 if (c + 1 < nchunks) {
                     const uint64_t dvx = sdesc_sw128(vs, ones - vs, 1024);
                     const uint64_t dkm = desc_mn_base(ks, C);
@@ -665,7 +675,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C; k += 16)
-                    umma_bf16_ts(tDA + b * D, tW + b * C + k / 2, desc_mnmajor(ks, C, k), idCD_mn, 1);
+                    umma_bf16_ts(tDA + b * D, tW + b * C + k / 2, mk + kstep_mn(k), idCD_mn, 1);
                 umma_commit(&da_full[b]);
                 umma_commit(&empty[s]);
             }
