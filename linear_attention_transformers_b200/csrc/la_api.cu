@@ -147,12 +147,29 @@ constexpr int kNumSM = 148;
 bool fast_path(la_dtype dt, int64_t D) { return dt == LA_BF16 && (D == 64 || D == 128); }
 int chunk_len(int64_t D) { return D == 64 ? 128 : 64; }
 
-// Segments per head: enough blocks to cover the SMs twice when there are few
-// heads, at least two chunks per segment.
+// Segments per head.  Each chunked kernel holds one block per SM (its shared
+// memory), so a launch of heads * s blocks takes ceil(heads * s / SMs) waves
+// of ceil(nchunks / s) chunks each, plus a few chunks' worth of pipeline fill
+// per block; splitting (s > 1) also adds the segment-state pass, which reads
+// k and v again (about 0.3 of a chunk each).  Pick the s with the smallest
+// modelled makespan; 120 or more heads stay unsplit (one wave or close).
 int pick_nseg(int64_t heads, int64_t nchunks) {
-    if (heads >= 120) return 1;
-    const int64_t want = (2 * kNumSM + heads - 1) / heads;
-    return int(std::max<int64_t>(1, std::min<int64_t>(want, nchunks / 2)));
+    if (heads >= 120 || nchunks < 4) return 1;
+    constexpr double kFill = 3.0, kStatePass = 0.3;
+    int best = 1;
+    double best_cost = double((heads + kNumSM - 1) / kNumSM) * (double(nchunks) + kFill);
+    for (int64_t sg = 2; sg <= nchunks / 2; ++sg) {
+        const int64_t per = (nchunks + sg - 1) / sg;
+        const int64_t used = (nchunks + per - 1) / per;  // segments that are not empty
+        if (used != sg) continue;
+        const double waves = double((heads * sg + kNumSM - 1) / kNumSM);
+        const double cost = waves * ((1.0 + kStatePass) * double(per) + kFill);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = int(sg);
+        }
+    }
+    return best;
 }
 
 struct SegSplit {
