@@ -92,14 +92,14 @@ def algorithmic_bytes(kernel: str, w) -> float:
 # capture ran at N = 4096 (the profiling size rule); traffic grows in
 # proportion to tokens for these kernels (each token's tiles are moved once).
 MEASURED_TRAFFIC = {
-    "bwd_dkdv": {"bytes_per_token_head": (272.695296e6 + 103.127296e6) / (8 * 16 * 4096),
-                 "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
-                 "profile": "profiles/bwd_dkdv_causal_b8h16n4096d64_bf16.md"},
-    "bwd_dq": {"bytes_per_token_head": (337.710080e6 + 55.305728e6) / (8 * 16 * 4096),
-               "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
-               "profile": "profiles/bwd_dq_causal_b8h16n4096d64_bf16.md"},
-    "chunk_causal": {"bytes_per_token_head": (201.389568e6 + 45.153024e6) / (8 * 16 * 4096),
-                     "sources": "4de43d3835cff861aef5bc9c13852485c220eeb28a2e0355accad9ed8451f9c0",
+    "bwd_dkdv": {"bytes_per_token_head": (272.686336e6 + 101.973248e6) / (8 * 16 * 4096),
+                 "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
+                 "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
+    "bwd_dq": {"bytes_per_token_head": (337.681920e6 + 53.002496e6) / (8 * 16 * 4096),
+               "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
+               "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
+    "chunk_causal": {"bytes_per_token_head": (201.391104e6 + 156.569856e6) / (8 * 16 * 4096),
+                     "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
                      "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
 }
 
