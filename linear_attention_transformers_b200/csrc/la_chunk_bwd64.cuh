@@ -35,21 +35,22 @@ struct Bwd2x64Cfg {
     static constexpr int C = 128, D = 64;
     static constexpr int NSTAGE = 3;
     static constexpr int TILE = C * D * 2;             // 16 KB
-    static constexpr int OFF_DG = 4 * TILE;            // in-stage: [16][C] K-major, rows 0/1 = dg hi/lo
-    static constexpr int OFF_DGF = OFF_DG + 16 * C * 2;  // in-stage: dg float [C]
+    static constexpr int OFF_DGF = 4 * TILE;           // in-stage: dg float [C]
     static constexpr int OFF_RINV = OFF_DGF + C * 4;   // in-stage: 1/g float [C]
     static constexpr int STAGE = ((OFF_RINV + C * 4) + 1023) / 1024 * 1024;
     static constexpr int OFF_RP = NSTAGE * STAGE;      // R, bf16 [D][D] row tile (row f)
     static constexpr int OFF_RF = OFF_RP + D * D * 2;  // r, float [D]
-    static constexpr int OFF_BAR = OFF_RF + D * 4;
-    static constexpr int NBAR = 3 * NSTAGE + 10;
+    static constexpr int OFF_RPART = OFF_RF + D * 4;   // partial sums of A^T dg, float [2][D]
+    static constexpr int OFF_RCH = OFF_RPART + 2 * D * 4;  // A^T dg per step, ring of 4, float [4][D]
+    static constexpr int OFF_BAR = OFF_RCH + 4 * D * 4;
+    static constexpr int NBAR = 4 * NSTAGE + 12;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM columns
     static constexpr int T_X1 = 0, T_X2 = C, T_DV = 2 * C, T_DB = 2 * C + D;
-    static constexpr int T_R = 2 * C + 2 * D, T_RZ = T_R + D;
+    static constexpr int T_R = 2 * C + 2 * D;
     static constexpr int T_COLS = 512;
-    static_assert(T_RZ + 16 <= T_COLS, "TMEM budget");
+    static_assert(T_R + D <= T_COLS, "TMEM budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(OFF_RP % 1024 == 0, "swizzled tiles on 1 KB");
 };
@@ -158,7 +159,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     uint64_t* r_full = x1_full + 6;        // commit: state update complete
     uint64_t* rx_full = x1_full + 7;       // 128: R operand and r written
     uint64_t* drain = x1_full + 8;
-    uint64_t* staged = x1_full + 9;        // 128: dV, dK rows staged
+    uint64_t* rch_full = x1_full + 9;      // [2] 128: the step's A^T dg in the ring (by step parity)
+    uint64_t* staged = x1_full + 11;       // [NS] 128: dV, dK rows of the stage's step staged
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -188,7 +190,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
         mbar_init(r_full, 1);
         mbar_init(rx_full, 128);
         mbar_init(drain, 1);
-        mbar_init(staged, 128);
+        for (int i = 0; i < NS; ++i) mbar_init(&staged[i], 128);
+        for (int i = 0; i < 2; ++i) mbar_init(&rch_full[i], 128);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -227,13 +230,12 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
         if (lane == 0) {
             const uint32_t tX1 = tmem + Cfg::T_X1, tX2 = tmem + Cfg::T_X2;
             const uint32_t tDV = tmem + Cfg::T_DV, tDB = tmem + Cfg::T_DB;
-            const uint32_t tR = tmem + Cfg::T_R, tRZ = tmem + Cfg::T_RZ;
+            const uint32_t tR = tmem + Cfg::T_R;
             const uint32_t rp = sbase + Cfg::OFF_RP;
             constexpr uint32_t idCC = idesc_bf16(C, C, 0, 0);     // B A^T, V dU^T
             constexpr uint32_t idCD_mn = idesc_bf16(C, D, 0, 1);  // B operand rows = K
             constexpr uint32_t idCD_k = idesc_bf16(C, D, 0, 0);   // B operand K-major
             constexpr uint32_t idDD = idesc_bf16(D, D, 1, 1);     // A^T dU
-            constexpr uint32_t idD16 = idesc_bf16(D, 16, 1, 0);   // A^T [dg_hi; dg_lo]
             const bool has_init = st_in != nullptr;
             // base descriptors (k = 0), stepped along K by constant offsets,
             // so each MMA costs the issuing thread few instructions
@@ -269,9 +271,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const int s = t % NS;
                 const uint32_t qs = sbase + s * Cfg::STAGE, ks = qs + Cfg::TILE;
                 const uint32_t vs = qs + 2 * Cfg::TILE, dus = qs + 3 * Cfg::TILE;
-                const uint32_t dgs = qs + Cfg::OFF_DG;
                 const uint64_t mq = desc_mn_base(qs, C), mdu = desc_mn_base(dus, C);
-                const uint64_t kk = desc_k_base(ks), kv = desc_k_base(vs), kdg = desc_k_base(dgs);
+                const uint64_t kk = desc_k_base(ks), kv = desc_k_base(vs);
                 if (t > 0 && !(ok = mbar_wait(d_free, (t - 1) & 1, abort_flag))) break;
                 if (!(ok = mbar_wait(x1p_full, t & 1, abort_flag))) break;
                 tc_fence_after();
@@ -294,13 +295,11 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 umma_commit(d_full);
                 if (t + 1 < nchunks) {
                     if (!(ok = x_raw(t + 1))) break;
-                    // R += A^T dU, r += A^T [dg_hi; dg_lo]
+                    // R += A^T dU (r += A^T dg is summed by the feature-map warps)
 #pragma unroll
-                    for (int k = 0; k < C; k += 16) {
-                        const uint32_t acc = (t > 0 || has_init || k > 0) ? 1u : 0u;
-                        umma_bf16(tR, mq + kstep_mn(k), mdu + kstep_mn(k), idDD, acc);
-                        umma_bf16(tRZ, mq + kstep_mn(k), kdg + kstep_k(16, k), idD16, acc);
-                    }
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tR, mq + kstep_mn(k), mdu + kstep_mn(k), idDD,
+                                  (t > 0 || has_init || k > 0) ? 1u : 0u);
                     umma_commit(r_full);
                 }
                 umma_commit(&empty[s]);
@@ -309,14 +308,9 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             mbar_wait_drain(drain, 0);
         }
     } else if (warp < 10) {
-        // per chunk: dg (bf16 hi/lo into the DG atom, fp32 copy), 1/g, phi on Q
-        // and K in place, dU = dO / g in place
+        // per chunk: dg and 1/g, phi on Q and K in place (unless given),
+        // dU = dO / g in place
         const int u = tid - 64;  // 0..255
-        for (int idx = u; idx < NS * 16 * C; idx += 256) {
-            const int s = idx / (16 * C), r = (idx / C) % 16, cc = idx % C;
-            reinterpret_cast<__nv_bfloat16*>(smem + s * Cfg::STAGE + Cfg::OFF_DG)[tile_off(16, r, cc) / 2] =
-                __float2bfloat16_rn(0.f);
-        }
         const float* gb = prm.gbuf + size_t(head) * prm.N;
         const float* dgb = prm.dgbuf + size_t(head) * prm.N;
         // g and dg of the next chunk are loaded one chunk ahead
@@ -352,10 +346,6 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const bool valid = u < nvalid;
                 const float d = valid ? dg : 0.f;
                 rinv[u] = valid ? 1.f / g : 0.f;
-                __nv_bfloat16* dgt = reinterpret_cast<__nv_bfloat16*>(st + Cfg::OFF_DG);
-                const __nv_bfloat16 h = __float2bfloat16_rn(d);
-                dgt[tile_off(16, 0, u) / 2] = h;
-                dgt[tile_off(16, 1, u) / 2] = __float2bfloat16_rn(d - __bfloat162float(h));
                 dgf[u] = d;
             }
             named_bar_sync(3, 256);  // rinv ready
@@ -381,10 +371,13 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             }
         }
     } else if (warp < 14) {
-        // mask and pack X1 (keep i >= j) and, without PIN, X2 (+ dg_i) in place
+        // mask and pack X1 (keep i >= j) and, without PIN, X2 (+ dg_i) in
+        // place; sum the step's r term A^T dg
         const int sp = warp & 3;
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int jrow = 32 * sp + lane;
+        float* rpart = reinterpret_cast<float*>(smem + Cfg::OFF_RPART);
+        float* rch = reinterpret_cast<float*>(smem + Cfg::OFF_RCH);
         for (int t = 0; t < nchunks; ++t) {
             const int s = t % NS;
             const float* dgf = reinterpret_cast<const float*>(smem + s * Cfg::STAGE + Cfg::OFF_DGF);
@@ -393,6 +386,23 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             mask_pack_upper(tmem + lane_base + Cfg::T_X1, sp, jrow, nullptr);
             tc_fence_before();
             mbar_arrive(x1p_full);
+            {
+                // this step's r term A^T dg into ring slot t % 4 (read by the
+                // state readout of step t; the slot is written again at step
+                // t + 4, which cannot start before that readout): column f,
+                // half of the rows per thread, then the two halves summed
+                const int e = tid - 320, f = e & 63, r0 = (e >> 6) * 64;
+                const uint8_t* at = smem + s * Cfg::STAGE;
+                float acc = 0.f;
+#pragma unroll 8
+                for (int i = r0; i < r0 + 64; ++i)
+                    acc = fmaf(__bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(at + tile_off(C, i, f))),
+                               dgf[i], acc);
+                rpart[(e >> 6) * D + f] = acc;
+                named_bar_sync(1, 128);
+                if (e < D) rch[(t & 3) * D + e] = rpart[e] + rpart[D + e];
+                mbar_arrive(&rch_full[t & 1]);
+            }
             if (PIN) continue;  // X2 is packed by feature-map warps 2-5
             if (!named_bar_all(1, 128, mbar_wait(x2_full, t & 1, abort_flag))) break;
             tc_fence_after();
@@ -424,10 +434,6 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 for (int i = 0; i < 16; ++i) v16[i] = frow >= 0 ? st_in[size_t(frow) * D + f0 + i] : 0.f;
                 tmem_st16(tmem + lane_base + Cfg::T_R + f0, v16);
             }
-            float z16[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) z16[i] = (i == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
-            tmem_st16(tmem + lane_base + Cfg::T_RZ, z16);
             tmem_wait_st();
         }
         fence_proxy_async_smem();
@@ -471,7 +477,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             tc_fence_before();
             mbar_arrive(d_free);
             fence_proxy_async_smem();
-            mbar_arrive(staged);
+            mbar_arrive(&staged[s]);
             if (t + 1 == nchunks) break;
             // state after this chunk -> operands of the next (earlier) chunk
             if (!named_bar_all(2, 128, mbar_wait(r_full, t & 1, abort_flag))) break;
@@ -483,10 +489,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 tmem_wait_ld();
                 if (frow >= 0) store_row16_bf16(rp, D, frow, v0, rv);
             }
-            float rz[16];
-            tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
-            tmem_wait_ld();
-            if (frow >= 0) rf[frow] = rz[0] + rz[1];
+            if (!named_bar_all(2, 128, mbar_wait(&rch_full[t & 1], (t >> 1) & 1, abort_flag))) break;
+            if (frow >= 0) rf[frow] += reinterpret_cast<const float*>(smem + Cfg::OFF_RCH)[(t & 3) * D + frow];
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(rx_full);
@@ -499,7 +503,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const int s = t % NS;
                 const int row0 = row_of(t);
                 uint8_t* st = smem + s * Cfg::STAGE;
-                if (!mbar_wait(staged, t & 1, abort_flag)) break;
+                if (!mbar_wait(&staged[s], (t / NS) & 1, abort_flag)) break;
                 tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
                 tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
                 bulk_commit();
@@ -540,7 +544,7 @@ struct Bwd1x64Cfg {
     static constexpr int OFF_SX = OFF_ONES + TILE;     // S^T, bf16 [D][D] row tile (row v)
     static constexpr int OFF_ZF = OFF_SX + D * D * 2;  // z, float [2][D] (by chunk parity)
     static constexpr int OFF_BAR = OFF_ZF + 2 * D * 4;
-    static constexpr int NBAR = 3 * NSTAGE + 10;
+    static constexpr int NBAR = 4 * NSTAGE + 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // TMEM columns: W [2][C], dA [2][D], T [D]
@@ -571,8 +575,8 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
     uint64_t* sx_full = w_full + 3;       // 128: S^T operand and z written
     uint64_t* da_full = w_full + 4;       // [2] commit: dA complete
     uint64_t* da_free = w_full + 6;       // [2] 128: dA read
-    uint64_t* staged = w_full + 8;        // 128: dQ rows staged
-    uint64_t* drain = w_full + 9;
+    uint64_t* drain = w_full + 8;
+    uint64_t* staged = w_full + 9;        // [NS] 128: dQ rows of the stage's step staged
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -597,7 +601,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             mbar_init(&da_full[b], 1);
             mbar_init(&da_free[b], 128);
         }
-        mbar_init(staged, 128);
+        for (int i = 0; i < NS; ++i) mbar_init(&staged[i], 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -830,7 +834,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             tc_fence_before();
             mbar_arrive(&da_free[b]);
             fence_proxy_async_smem();
-            mbar_arrive(staged);
+            mbar_arrive(&staged[s]);
         }
     } else if (warp == 18) {
         // TMA stores of the staged dQ rows; the stage is free once they have
@@ -838,7 +842,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS;
-                if (!mbar_wait(staged, c & 1, abort_flag)) break;
+                if (!mbar_wait(&staged[s], (c / NS) & 1, abort_flag)) break;
                 tma_store_3d(&prm.tm_dq, smem + s * Cfg::STAGE, 0, row_of(c), head);
                 bulk_commit();
                 bulk_wait_read0();
