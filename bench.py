@@ -92,14 +92,14 @@ def algorithmic_bytes(kernel: str, w) -> float:
 # capture ran at N = 4096 (the profiling size rule); traffic grows in
 # proportion to tokens for these kernels (each token's tiles are moved once).
 MEASURED_TRAFFIC = {
-    "bwd_dkdv": {"bytes_per_token_head": (272.686336e6 + 101.973248e6) / (8 * 16 * 4096),
-                 "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
+    "bwd_dkdv": {"bytes_per_token_head": (272.682240e6 + 99.875584e6) / (8 * 16 * 4096),
+                 "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
                  "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
-    "bwd_dq": {"bytes_per_token_head": (337.681920e6 + 53.002496e6) / (8 * 16 * 4096),
-               "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
+    "bwd_dq": {"bytes_per_token_head": (337.682432e6 + 52.443904e6) / (8 * 16 * 4096),
+               "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
                "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
-    "chunk_causal": {"bytes_per_token_head": (201.391104e6 + 156.569856e6) / (8 * 16 * 4096),
-                     "sources": "db64f88cf86b087f9ff05d922a3bcc5fe7d7f2335b24cf1f2528f815add33cbb",
+    "chunk_causal": {"bytes_per_token_head": (201.390336e6 + 155.041536e6) / (8 * 16 * 4096),
+                     "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
                      "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
 }
 
