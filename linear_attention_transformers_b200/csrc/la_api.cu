@@ -215,13 +215,19 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
 template <int D, int C, int PHI, int MODE>
 la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st,
                        const char* name) {
-    auto kern = D == 64 ? la::chunk_fwd64_kernel<PHI, MODE> : la::chunk_fwd_kernel<D, C, PHI, MODE>;
-    constexpr int smem = D == 64 ? la::Chunk64Cfg::SMEM : la::ChunkCfg<D, C>::SMEM;
-    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
-        return cuda_fail("cudaFuncSetAttribute", e);
-    la::LaunchScope scope(name, st);
-    kern<<<unsigned(grid), D == 64 ? la::kChunk64Threads : la::kChunkThreads, smem, st>>>(prm);
-    return launch_status();
+    auto go = [&](auto kern, int smem, int threads) -> la_status {
+        if (cudaError_t e =
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem))
+            return cuda_fail("cudaFuncSetAttribute", e);
+        la::LaunchScope scope(name, st);
+        kern<<<unsigned(grid), threads, smem, st>>>(prm);
+        return launch_status();
+    };
+    if constexpr (D == 64)
+        return go(la::chunk_fwd64_kernel<PHI, MODE>, la::Chunk64Cfg::SMEM, la::kChunk64Threads);
+    else
+        return go(la::chunk_fwd_kernel<D, C, PHI, MODE>, la::ChunkCfg<D, C>::SMEM,
+                  la::kChunkThreads);
 }
 
 la_status launch_state_kernel(int which, float* rec, float* out, float* S, float* z,

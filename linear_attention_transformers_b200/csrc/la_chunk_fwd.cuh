@@ -6,31 +6,35 @@
 //          with A = phi(Q_c), B = phi(K_c) and the state S (D x D), z (D) of
 //          every earlier token:
 //              P   = A B^T                           (C x C)
-//              num = A S + (P . tril) V_c
-//              den = A z + (P . tril) 1              (both as 16-wide MMAs:
-//                                                     z split into two bf16 terms,
-//                                                     1 = a ones operand)
+//              [num | den] = A [S | z] + (P . tril) [V_c | 1]
 //              O_c = num / den
-//              S  += B^T V_c,   z += B^T 1           (fp32 accumulators in TMEM)
+//              [S | z] += B^T [V_c | 1]              (fp32 accumulators in TMEM)
 //          Inside a chunk this is the quadratic form, across chunks the
 //          associativity reorder (QK^T)V = Q(K^T V) of "Efficient Transformers
 //          Survey", Proposition "Linear Attention via Kernel Decomposition"
 //          (Intuition), with S and z carried chunk to chunk as in its "Why It
 //          Matters" paragraph.
-//  REDUCE  only S += B^T V, z += B^T 1 over the segment; writes the segment's
+//  REDUCE  only [S | z] += B^T [V | 1] over the segment; writes the segment's
 //          (S, z) record (non-causal totals, causal segment sums).
 //  QUERY   O = A S / (A z) against a fixed (S, z) record (the non-causal
 //          query pass: "each attention output costs O(md)").
+//
+// The denominator rides in the same MMAs as the numerator: the B operands
+// are 144 columns wide, [S | z_hi z_lo 0..] (z split into two bf16 terms)
+// and [V | 1] (V followed by a constant atom whose first column is ones), so
+// a chunk takes 8 (A B^T) + 8 (A [S|z]) + 4 (state) + 4 (P~ [V|1]) = 24
+// tcgen05.mma instructions; below N = 128 an instruction costs about the
+// same whatever its width, so the count is what matters.
 //
 // Warp roles (18 warps): a TMA producer warp; a single-thread tcgen05.mma
 // issuer; 8 feature-map warps that apply phi in place to the landed tiles;
 // a "P" warpgroup that masks P and writes it back as a bf16 operand; an "O"
 // warpgroup that converts the running state into the next chunk's bf16
-// operand and forms O = num / den, stored with TMA.  P and O accumulators
-// are double-buffered in TMEM so the next chunk's A B^T and the masking run
-// while the state of the current chunk is being converted; the only serial
-// chain per chunk is state conversion -> (A S, B^T V) MMAs.  All handshakes
-// are mbarriers with bounded waits.
+// operand and forms O = num / den, stored with TMA.  The O accumulator is
+// double-buffered in TMEM so the next chunk's products start while the
+// current O is being read; the serial chain per chunk is state conversion ->
+// (A [S|z], state) MMAs.  All handshakes are mbarriers with bounded waits.
+
 #pragma once
 
 #include "la_common.cuh"
@@ -65,31 +69,43 @@ struct ChunkParams {
     int store_phi;
 };
 
+// Shared-memory and TMEM plan of the kernel below (head size 128, 64-token
+// chunks).  Stage tiles live in 19 slots of one [C][64] bf16 atom (8 KB).
+// Slot 18 is the ones atom E; stage s puts its two V atoms at slots
+// 18 - 2 l_s and 18 - l_s (l = 1, 3, 7), so V atom 0, V atom 1 and E are
+// equally spaced and [V | 1] is a single MN-major operand whose atom stride
+// (LBO) is l_s slots; Q and K fill the remaining adjacent slot pairs.
 template <int D, int C>
 struct ChunkCfg {
+    static_assert(D == 128 && C == 64, "laid out for head size 128, 64-token chunks");
     static constexpr int NSTAGE = 3;
-    static constexpr int NO = (2 * C + 3 * (D + 16) <= 512) ? 2 : 1;  // O buffers in TMEM
-    static constexpr int TILE = C * D * 2;  // bytes of one [C][D] bf16 tile
-    static constexpr int STAGE = 3 * TILE;  // Q, K, V
-    static constexpr int OFF_SPREV = NSTAGE * STAGE;
-    static constexpr int OFF_ZOP = OFF_SPREV + D * D * 2;
-    static constexpr int OFF_E = OFF_ZOP + 16 * D * 2;
-    static constexpr int OFF_PT = OFF_E + 16 * C * 2;
-    static constexpr int OFF_OST = OFF_PT + C * C * 2;
+    static constexpr int NO = 2;            // O buffers in TMEM
+    static constexpr int ATOM = C * 128;    // one [C][64] bf16 atom
+    static constexpr int NSLOT = 19;
+    static constexpr int E_SLOT = 18;
+    __host__ __device__ static constexpr int q_slot(int s) { return s == 0 ? 0 : (s == 1 ? 5 : 9); }
+    __host__ __device__ static constexpr int k_slot(int s) { return s == 0 ? 2 : (s == 1 ? 7 : 13); }
+    __host__ __device__ static constexpr int v_l(int s) { return s == 0 ? 1 : (s == 1 ? 3 : 7); }
+    __host__ __device__ static constexpr int v_slot(int s, int a) {
+        return E_SLOT - (2 - a) * v_l(s);
+    }
+    // [D][192] row tile: S (columns 0..127), z_hi, z_lo (columns 128, 129)
+    static constexpr int OFF_SX = NSLOT * ATOM;
+    static constexpr int OFF_PT = OFF_SX + 3 * D * 128;  // [C][C] masked P
+    static constexpr int OFF_OST = OFF_PT + C * C * 2;   // [C][D] output staging
     static constexpr int OFF_BAR = OFF_OST + C * D * 2;
-    static constexpr int NBAR = 3 * NSTAGE + 9 + 2 * NO;
+    static constexpr int NBAR = 3 * NSTAGE + 7 + 2 * NO;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;  // + alignment slack
-    // TMEM columns: P[2], O[NO] (+16 for the denominator), S (+16 for z)
+    // TMEM columns: P, O[NO] (D + 16 each: numerator, then the two halves of
+    // the denominator), [S | z] (D + 16)
     static constexpr int T_P = 0;
-    static constexpr int T_O = 2 * C;
-    static constexpr int T_S = 2 * C + NO * (D + 16);
+    static constexpr int T_O = C;
+    static constexpr int T_S = C + NO * (D + 16);
     static constexpr int T_Z = T_S + D;
     static constexpr int T_COLS = 512;
     static_assert(T_Z + 16 <= T_COLS, "TMEM budget");
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
-    static_assert(C == 64 || C == 128, "chunk");
-    static_assert(D == 64 || D == 128, "head size");
 };
 
 constexpr int kChunkThreads = 576;  // producer, MMA, 8 phi warps, P and O warpgroups
@@ -108,14 +124,14 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
     uint64_t* full = bars;                // TMA landed                 (1 + tx)
     uint64_t* phi_done = bars + NS;       // phi applied                (256)
     uint64_t* empty = bars + 2 * NS;      // MMAs done with the stage   (commit)
-    uint64_t* p_full = bars + 3 * NS;     // [2] P = A B^T in TMEM      (commit)
-    uint64_t* p_free = p_full + 2;        // [2] P read by the P group  (128)
-    uint64_t* pt_full = p_full + 4;       // masked P in smem           (128)
-    uint64_t* pt_free = p_full + 5;       // masked P consumed          (commit)
-    uint64_t* s_full = p_full + 6;        // state operand written      (128)
-    uint64_t* s_done = p_full + 7;        // A S, state update done     (commit)
-    uint64_t* drain = p_full + 8;         // every MMA finished         (commit)
-    uint64_t* o_full = p_full + 9;        // [NO] O complete            (commit)
+    uint64_t* p_full = bars + 3 * NS;     // P = A B^T in TMEM          (commit)
+    uint64_t* p_free = p_full + 1;        // P read by the P group      (128)
+    uint64_t* pt_full = p_full + 2;       // masked P in smem           (128)
+    uint64_t* pt_free = p_full + 3;       // masked P consumed          (commit)
+    uint64_t* s_full = p_full + 4;        // state operand written      (128)
+    uint64_t* s_done = p_full + 5;        // A [S|z], state update done (commit)
+    uint64_t* drain = p_full + 6;         // every MMA finished         (commit)
+    uint64_t* o_full = p_full + 7;        // [NO] O complete            (commit)
     uint64_t* o_free = o_full + NO;       // [NO] O read                (128)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
@@ -138,10 +154,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
             mbar_init(&phi_done[s], 256);
             mbar_init(&empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&p_full[b], 1);
-            mbar_init(&p_free[b], 128);
-        }
+        mbar_init(p_full, 1);
+        mbar_init(p_free, 128);
         mbar_init(pt_full, 128);
         mbar_init(pt_free, 1);
         mbar_init(s_full, 128);
@@ -174,21 +188,22 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                 tma_prefetch_desc(&prm.tm_k);
                 tma_prefetch_desc(&prm.tm_v);
             }
-            constexpr uint32_t bytes = Cfg::TILE * ((kQ ? 1 : 0) + (kKV ? 2 : 0));
+            constexpr uint32_t bytes = 2 * Cfg::ATOM * ((kQ ? 1 : 0) + (kKV ? 2 : 0));
             int issued = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS;
                 if (c >= NS && !mbar_wait(&empty[s], ((c / NS) - 1) & 1, abort_flag)) break;
-                uint8_t* st = smem + s * Cfg::STAGE;
                 mbar_arrive_expect_tx(&full[s], bytes);
                 const int row = tok0 + c * C;
 #pragma unroll
-                for (int a = 0; a < D / 64; ++a) {
-                    if (kQ) tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
+                for (int a = 0; a < 2; ++a) {
+                    if (kQ)
+                        tma_load_3d(smem + (Cfg::q_slot(s) + a) * Cfg::ATOM, &prm.tm_q, &full[s],
+                                    a * 64, row, head);
                     if (kKV) {
-                        tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64,
-                                    row, head);
-                        tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s],
+                        tma_load_3d(smem + (Cfg::k_slot(s) + a) * Cfg::ATOM, &prm.tm_k, &full[s],
+                                    a * 64, row, head);
+                        tma_load_3d(smem + Cfg::v_slot(s, a) * Cfg::ATOM, &prm.tm_v, &full[s],
                                     a * 64, row, head);
                     }
                 }
@@ -201,71 +216,62 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idP = idesc_bf16(C, C, 0, 0);    // A B^T
-            constexpr uint32_t idO = idesc_bf16(C, D, 0, 1);    // A S ; (P.tril) V
-            constexpr uint32_t idOZ = idesc_bf16(C, 16, 0, 0);  // A [z_hi z_lo]^T ; (P.tril) 1
-            constexpr uint32_t idS = idesc_bf16(D, D, 1, 1);    // B^T V
-            constexpr uint32_t idSZ = idesc_bf16(D, 16, 1, 0);  // B^T 1
-            const uint64_t dSp = desc_mn_base(sbase + Cfg::OFF_SPREV, D);
-            const uint64_t dZo = desc_k_base(sbase + Cfg::OFF_ZOP);
-            const uint64_t dE = desc_k_base(sbase + Cfg::OFF_E);
+            constexpr uint32_t idP = idesc_bf16(C, C, 0, 0);       // A B^T
+            constexpr uint32_t idO = idesc_bf16(C, D + 16, 0, 1);  // A [S|z] ; P~ [V|1]
+            constexpr uint32_t idS = idesc_bf16(D, D + 16, 1, 1);  // B^T [V|1]
+            const uint64_t dSx = desc_mn_base(sbase + Cfg::OFF_SX, D);
             const uint64_t dPt = desc_k_base(sbase + Cfg::OFF_PT);
             const bool has_init = st_in != nullptr;
-            auto stage_q = [&](int s) { return desc_k_base(sbase + s * Cfg::STAGE); };
-            auto stage_k = [&](int s) { return desc_k_base(sbase + s * Cfg::STAGE + Cfg::TILE); };
+            auto stage_q = [&](int s) { return desc_k_base(sbase + Cfg::q_slot(s) * Cfg::ATOM); };
+            auto stage_k = [&](int s) { return desc_k_base(sbase + Cfg::k_slot(s) * Cfg::ATOM); };
             auto stage_kmn = [&](int s) {
-                return desc_mn_base(sbase + s * Cfg::STAGE + Cfg::TILE, C);
+                return desc_mn_base(sbase + Cfg::k_slot(s) * Cfg::ATOM, C);
             };
-            auto stage_vmn = [&](int s) {
-                return desc_mn_base(sbase + s * Cfg::STAGE + 2 * Cfg::TILE, C);
+            // [V | 1]: V atom 0, V atom 1 and the ones atom, l_s slots apart
+            auto stage_vx = [&](int s) {
+                return sdesc_sw128(sbase + Cfg::v_slot(s, 0) * Cfg::ATOM,
+                                   uint32_t(Cfg::v_l(s) * Cfg::ATOM), 1024);
             };
             bool ok = true;
-            // P = A B^T for chunk c into P buffer c & 1
+            // P = A B^T for chunk c (one TMEM buffer: the P group has read
+            // chunk c-1's long before chunk c's is issued)
             auto p_part = [&](int c) -> bool {
                 const int s = c % NS;
                 if (!mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag)) return false;
-                if (c >= 2 && !mbar_wait(&p_free[c & 1], ((c >> 1) - 1) & 1, abort_flag))
-                    return false;
+                if (c >= 1 && !mbar_wait(p_free, (c - 1) & 1, abort_flag)) return false;
                 tc_fence_after();
                 const uint64_t dq = stage_q(s), dk = stage_k(s);
-                const uint32_t tP = tmem + Cfg::T_P + (c & 1) * C;
+                const uint32_t tP = tmem + Cfg::T_P;
 #pragma unroll
                 for (int k = 0; k < D; k += 16)
                     umma_bf16(tP, dq + kstep_k(C, k), dk + kstep_k(C, k), idP, k > 0);
-                umma_commit(&p_full[c & 1]);
+                umma_commit(p_full);
                 return true;
             };
             if (MODE == MODE_CAUSAL) {
                 if (nchunks > 0) ok = p_part(0);
                 for (int c = 0; ok && c < nchunks; ++c) {
                     const int s = c % NS, bo = c % NO;
-                    const uint32_t tO = tmem + Cfg::T_O + bo * (D + 16), tOZ = tO + D;
+                    const uint32_t tO = tmem + Cfg::T_O + bo * (D + 16);
                     if (!(ok = mbar_wait(s_full, c & 1, abort_flag))) break;
                     if (c >= NO && !(ok = mbar_wait(&o_free[bo], ((c / NO) - 1) & 1, abort_flag)))
                         break;
                     tc_fence_after();
-                    const uint64_t dq = stage_q(s), dkm = stage_kmn(s), dvm = stage_vmn(s);
+                    const uint64_t dq = stage_q(s), dkm = stage_kmn(s), dvx = stage_vx(s);
 #pragma unroll
-                    for (int k = 0; k < D; k += 16) {
-                        umma_bf16(tO, dq + kstep_k(C, k), dSp + kstep_mn(k), idO, k > 0);
-                        umma_bf16(tOZ, dq + kstep_k(C, k), dZo + kstep_k(16, k), idOZ, k > 0);
-                    }
+                    for (int k = 0; k < D; k += 16)
+                        umma_bf16(tO, dq + kstep_k(C, k), dSx + kstep_mn(k), idO, k > 0);
 #pragma unroll
-                    for (int k = 0; k < C; k += 16) {
-                        const uint32_t acc = (c > 0 || has_init || k > 0) ? 1u : 0u;
-                        umma_bf16(tmem + Cfg::T_S, dkm + kstep_mn(k), dvm + kstep_mn(k), idS, acc);
-                        umma_bf16(tmem + Cfg::T_Z, dkm + kstep_mn(k), dE + kstep_k(16, k), idSZ,
-                                  acc);
-                    }
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tmem + Cfg::T_S, dkm + kstep_mn(k), dvx + kstep_mn(k), idS,
+                                  (c > 0 || has_init || k > 0) ? 1u : 0u);
                     umma_commit(s_done);
                     if (c + 1 < nchunks && !(ok = p_part(c + 1))) break;
                     if (!(ok = mbar_wait(pt_full, c & 1, abort_flag))) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int k = 0; k < C; k += 16) {
-                        umma_bf16(tO, dPt + kstep_k(C, k), dvm + kstep_mn(k), idO, 1);
-                        umma_bf16(tOZ, dPt + kstep_k(C, k), dE + kstep_k(16, k), idOZ, 1);
-                    }
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tO, dPt + kstep_k(C, k), dvx + kstep_mn(k), idO, 1);
                     umma_commit(&o_full[bo]);
                     umma_commit(pt_free);
                     umma_commit(&empty[s]);
@@ -274,17 +280,15 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                 ok = mbar_wait(s_full, 0, abort_flag);
                 for (int c = 0; ok && c < nchunks; ++c) {
                     const int s = c % NS, bo = c % NO;
-                    const uint32_t tO = tmem + Cfg::T_O + bo * (D + 16), tOZ = tO + D;
+                    const uint32_t tO = tmem + Cfg::T_O + bo * (D + 16);
                     if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
                     if (c >= NO && !(ok = mbar_wait(&o_free[bo], ((c / NO) - 1) & 1, abort_flag)))
                         break;
                     tc_fence_after();
                     const uint64_t dq = stage_q(s);
 #pragma unroll
-                    for (int k = 0; k < D; k += 16) {
-                        umma_bf16(tO, dq + kstep_k(C, k), dSp + kstep_mn(k), idO, k > 0);
-                        umma_bf16(tOZ, dq + kstep_k(C, k), dZo + kstep_k(16, k), idOZ, k > 0);
-                    }
+                    for (int k = 0; k < D; k += 16)
+                        umma_bf16(tO, dq + kstep_k(C, k), dSx + kstep_mn(k), idO, k > 0);
                     umma_commit(&o_full[bo]);
                     umma_commit(&empty[s]);
                 }
@@ -294,14 +298,11 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     const int s = c % NS;
                     if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
                     tc_fence_after();
-                    const uint64_t dkm = stage_kmn(s), dvm = stage_vmn(s);
+                    const uint64_t dkm = stage_kmn(s), dvx = stage_vx(s);
 #pragma unroll
-                    for (int k = 0; k < C; k += 16) {
-                        const uint32_t acc = (c > 0 || k > 0) ? 1u : 0u;
-                        umma_bf16(tmem + Cfg::T_S, dkm + kstep_mn(k), dvm + kstep_mn(k), idS, acc);
-                        umma_bf16(tmem + Cfg::T_Z, dkm + kstep_mn(k), dE + kstep_k(16, k), idSZ,
-                                  acc);
-                    }
+                    for (int k = 0; k < C; k += 16)
+                        umma_bf16(tmem + Cfg::T_S, dkm + kstep_mn(k), dvx + kstep_mn(k), idS,
+                                  (c > 0 || k > 0) ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 if (ok) umma_commit(s_done);
@@ -316,17 +317,18 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
-            uint8_t* st = smem + s * Cfg::STAGE;
+            uint8_t* qt = smem + Cfg::q_slot(s) * Cfg::ATOM;
+            uint8_t* kt = smem + Cfg::k_slot(s) * Cfg::ATOM;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
             if (MODE == MODE_CAUSAL) {
                 if (u < 128)
-                    phi_tile<PHI, C, D, 128>(st, u, nvalid, false);
+                    phi_tile<PHI, C, D, 128>(qt, u, nvalid, false);
                 else
-                    phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+                    phi_tile<PHI, C, D, 128>(kt, u - 128, nvalid, true);
             } else if (MODE == MODE_QUERY) {
-                phi_tile<PHI, C, D, 256>(st, u, nvalid, false);
+                phi_tile<PHI, C, D, 256>(qt, u, nvalid, false);
             } else {
-                phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
+                phi_tile<PHI, C, D, 256>(kt, u, nvalid, true);
             }
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
@@ -339,15 +341,14 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
             const int irow = acc_row<C>(sp, lane);
             uint8_t* pt = smem + Cfg::OFF_PT;
             for (int c = 0; c < nchunks; ++c) {
-                const int b = c & 1;
                 bool ok = c == 0 || mbar_wait(pt_free, (c - 1) & 1, abort_flag);
-                ok = ok && mbar_wait(&p_full[b], (c >> 1) & 1, abort_flag);
+                ok = ok && mbar_wait(p_full, c & 1, abort_flag);
                 if (!named_bar_all(1, 128, ok)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int j0 = 0; j0 < C; j0 += 32) {
                     float pv[32];
-                    tmem_load<32>(tmem + lane_base + Cfg::T_P + b * C + j0, pv);
+                    tmem_load<32>(tmem + lane_base + Cfg::T_P + j0, pv);
                     if (irow >= 0) {
 #pragma unroll
                         for (int t = 0; t < 32; ++t)
@@ -356,7 +357,7 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&p_free[b]);
+                mbar_arrive(p_free);
                 fence_proxy_async_smem();
                 mbar_arrive(pt_full);
             }
@@ -368,35 +369,38 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
         const uint32_t lane_base = uint32_t(32 * sp) << 16;
         const int irow = acc_row<C>(sp, lane);  // token row of this thread (or -1)
         const int frow = acc_row<D>(sp, lane);  // state row of this thread (or -1)
-        uint8_t* sprev = smem + Cfg::OFF_SPREV;
-        uint8_t* zop = smem + Cfg::OFF_ZOP;
-        uint8_t* eop = smem + Cfg::OFF_E;
+        uint8_t* sx = smem + Cfg::OFF_SX;
+        uint8_t* eop = smem + Cfg::E_SLOT * Cfg::ATOM;
         uint8_t* ost = smem + Cfg::OFF_OST;
-        __nv_bfloat16* zop_h = reinterpret_cast<__nv_bfloat16*>(zop);
 
-        // ---- constant ones operand E (row 0) and the zero rows of Zop
-        for (int idx = e; idx < 16 * C; idx += 128) {
-            const int r = idx / C, cc = idx % C;
-            *reinterpret_cast<__nv_bfloat16*>(eop + tile_off(16, r, cc)) =
-                __float2bfloat16_rn(r == 0 ? 1.f : 0.f);
+        // ---- constant ones atom E (column 0) and the zero z atom of Sx
+        for (int r = e; r < C + D; r += 128) {
+            float v8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            const float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            if (r < C) {
+                v8[0] = 1.f;
+                for (int q = 0; q < 8; ++q) store_row_bf16<8>(eop, C, r, 8 * q, q == 0 ? v8 : z8);
+            } else {
+                for (int q = 0; q < 8; ++q) store_row_bf16<8>(sx, D, r - C, D + 8 * q, z8);
+            }
         }
-        for (int idx = e; idx < 16 * D; idx += 128) {
-            const int r = idx / D, cc = idx % D;
-            zop_h[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
-        }
-        named_bar_sync(2, 128);  // zero rows written before rows 0/1 of Zop below
-        // ---- initial state: bf16 operand (+ TMEM accumulator in CAUSAL mode)
+        named_bar_sync(2, 128);  // zero z atom written before its columns 128/129 below
+        // ---- z into columns 128 (z_hi) and 129 (z_lo) of Sx, zeros after
         auto put_z = [&](float zf) {
-            const __nv_bfloat16 zh = __float2bfloat16_rn(zf);
-            zop_h[tile_off(16, 0, frow) / 2] = zh;
-            zop_h[tile_off(16, 1, frow) / 2] = __float2bfloat16_rn(zf - __bfloat162float(zh));
+            float z16[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) z16[t] = 0.f;
+            z16[0] = zf;
+            z16[1] = zf - __bfloat162float(__float2bfloat16_rn(zf));
+            store_row_bf16<16>(sx, D, frow, D, z16);
         };
+        // ---- initial state: bf16 operand (+ TMEM accumulator in CAUSAL mode)
         if (MODE != MODE_REDUCE && frow >= 0) {
             for (int q = 0; q < D / 8; ++q) {
                 float v8[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t) v8[t] = st_in ? st_in[size_t(frow) * D + q * 8 + t] : 0.f;
-                store_row_bf16<8>(sprev, D, frow, q * 8, v8);
+                store_row_bf16<8>(sx, D, frow, q * 8, v8);
             }
             put_z(st_in ? st_in[size_t(D) * D + frow] : 0.f);
         }
@@ -455,7 +459,7 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                             float sv[16];
                             tmem_load<16>(tmem + lane_base + Cfg::T_S + v0, sv);
                             if (frow >= 0) {
-                                store_row_bf16<16>(sprev, D, frow, v0, sv);
+                                store_row_bf16<16>(sx, D, frow, v0, sv);
                                 if (write_final)
                                     for (int t = 0; t < 16; ++t)
                                         prm.S_out[size_t(head) * prm.stride_S + size_t(frow) * D +
