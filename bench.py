@@ -92,14 +92,15 @@ def algorithmic_bytes(kernel: str, w) -> float:
 # capture ran at N = 4096 (the profiling size rule); traffic grows in
 # proportion to tokens for these kernels (each token's tiles are moved once).
 MEASURED_TRAFFIC = {
-    "bwd_dkdv": {"bytes_per_token_head": (272.682240e6 + 99.875584e6) / (8 * 16 * 4096),
-                 "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
+    "bwd_dkdv": {"bytes_per_token_head": (272.683008e6 + 99.865344e6) / (8 * 16 * 4096), "D": 64,
+                 "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
                  "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
-    "bwd_dq": {"bytes_per_token_head": (337.682432e6 + 52.443904e6) / (8 * 16 * 4096),
-               "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
+    "bwd_dq": {"bytes_per_token_head": (337.681664e6 + 52.509696e6) / (8 * 16 * 4096), "D": 64,
+               "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
                "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
-    "chunk_causal": {"bytes_per_token_head": (201.390336e6 + 155.041536e6) / (8 * 16 * 4096),
-                     "sources": "dd1ee4bcf3bae51e14ff6641abec47fbc60d74fa0dfa0b3dd21ba39517e10d11",
+    "chunk_causal": {"bytes_per_token_head": (201.406976e6 + 154.606080e6) / (8 * 16 * 4096),
+                     "D": 64,
+                     "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
                      "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
 }
 
@@ -119,9 +120,10 @@ def kernel_sources_hash() -> str:
 
 def measured_traffic(kernel: str, w):
     """Per-launch DRAM bytes of `kernel` on workload w, or None when no
-    capture exists for it or the kernel sources changed since."""
+    capture exists for it (at w's head size) or the kernel sources changed
+    since."""
     rec = MEASURED_TRAFFIC.get(kernel)
-    if rec is None or rec["sources"] != kernel_sources_hash():
+    if rec is None or rec["D"] != w.D or rec["sources"] != kernel_sources_hash():
         return None
     return rec["bytes_per_token_head"] * w.B * w.H * w.N
 
