@@ -14,6 +14,16 @@
 namespace la {
 
 constexpr int kStateThreads = 256;
+constexpr int kStateBatch = 8;  // segments whose loads are issued together
+
+// Up to kStateBatch elements p0, p0 + step, ... (n of them) of a column of
+// records, loaded before any is stored so their latencies overlap.
+__device__ __forceinline__ void load_batch(const float* base, int p0, int step, int n, size_t R,
+                                           float* x) {
+#pragma unroll
+    for (int i = 0; i < kStateBatch; ++i)
+        if (i < n) x[i] = base[size_t(p0 + i * step) * R];
+}
 
 // rec[h][p] <- sum_{p' < p} rec[h][p'] (exclusive prefix, in place).
 __global__ void __launch_bounds__(kStateThreads)
@@ -23,10 +33,16 @@ state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks
     if (e >= R) return;
     float* base = rec + h * size_t(nseg) * R + e;
     float run = 0.f;
-    for (int p = 0; p < nseg; ++p) {
-        const float x = base[size_t(p) * R];
-        base[size_t(p) * R] = run;
-        run += x;
+    for (int p0 = 0; p0 < nseg; p0 += kStateBatch) {
+        const int n = min(kStateBatch, nseg - p0);
+        float x[kStateBatch];
+        load_batch(base, p0, 1, n, R, x);
+#pragma unroll
+        for (int i = 0; i < kStateBatch; ++i)
+            if (i < n) {
+                base[size_t(p0 + i) * R] = run;
+                run += x[i];
+            }
     }
 }
 
@@ -38,10 +54,16 @@ state_exclusive_rscan_kernel(float* __restrict__ rec, int nseg, int R, int block
     if (e >= R) return;
     float* base = rec + h * size_t(nseg) * R + e;
     float run = 0.f;
-    for (int p = nseg - 1; p >= 0; --p) {
-        const float x = base[size_t(p) * R];
-        base[size_t(p) * R] = run;
-        run += x;
+    for (int p0 = nseg - 1; p0 >= 0; p0 -= kStateBatch) {
+        const int n = min(kStateBatch, p0 + 1);
+        float x[kStateBatch];
+        load_batch(base, p0, -1, n, R, x);
+#pragma unroll
+        for (int i = 0; i < kStateBatch; ++i)
+            if (i < n) {
+                base[size_t(p0 - i) * R] = run;
+                run += x[i];
+            }
     }
 }
 
@@ -54,7 +76,14 @@ state_sum_kernel(const float* __restrict__ rec, float* __restrict__ out, int nse
     if (e >= R) return;
     const float* base = rec + h * size_t(nseg) * R + e;
     float run = 0.f;
-    for (int p = 0; p < nseg; ++p) run += base[size_t(p) * R];
+    for (int p0 = 0; p0 < nseg; p0 += kStateBatch) {
+        const int n = min(kStateBatch, nseg - p0);
+        float x[kStateBatch];
+        load_batch(base, p0, 1, n, R, x);
+#pragma unroll
+        for (int i = 0; i < kStateBatch; ++i)
+            if (i < n) run += x[i];
+    }
     out[h * size_t(R) + e] = run;
 }
 
