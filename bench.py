@@ -88,42 +88,47 @@ def algorithmic_bytes(kernel: str, w) -> float:
 
 # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), per token and head so that it scales to the bench
-# workload; valid only while the kernel sources hash to `sources`.  The
-# capture ran at N = 4096 (the profiling size rule); traffic grows in
-# proportion to tokens for these kernels (each token's tiles are moved once).
+# workload; valid only while the sources the kernel is built and launched
+# from (`files`, under csrc/) hash to `sources`.  The capture ran at
+# N = 4096 (the profiling size rule); traffic grows in proportion to tokens
+# for these kernels (each token's tiles are moved once).
+_FWD64_FILES = ("la_chunk_fwd64.cuh", "la_chunk_fwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
+                "la_common.cuh", "la_api.cu")
+_BWD64_FILES = ("la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
+                "la_common.cuh", "la_api.cu")
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {"bytes_per_token_head": (272.683008e6 + 99.865344e6) / (8 * 16 * 4096), "D": 64,
-                 "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
+                 "files": _BWD64_FILES,
+                 "sources": "72c58888f0e4bfed567936cb2686b08bdd191285c3972ce0834ca1cc83a2d671",
                  "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
     "bwd_dq": {"bytes_per_token_head": (337.681664e6 + 52.509696e6) / (8 * 16 * 4096), "D": 64,
-               "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
+               "files": _BWD64_FILES,
+               "sources": "72c58888f0e4bfed567936cb2686b08bdd191285c3972ce0834ca1cc83a2d671",
                "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
     "chunk_causal": {"bytes_per_token_head": (201.406976e6 + 154.606080e6) / (8 * 16 * 4096),
-                     "D": 64,
-                     "sources": "7ce0b511db0660a061b8d035f492b0a75a95f39fc97b109e28a9854fa6ad9d67",
+                     "D": 64, "files": _FWD64_FILES,
+                     "sources": "276466c43a8e5d351119e9842a089875533e7d1c8e5277856323e21cd5ede0a4",
                      "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
 }
 
 
-def kernel_sources_hash() -> str:
-    """sha256 over the CUDA sources of the library (file names and bytes)."""
+def kernel_sources_hash(files) -> str:
+    """sha256 over the named CUDA sources of the library (names and bytes)."""
     import hashlib
     d = os.path.join(ROOT, "linear_attention_transformers_b200", "csrc")
     h = hashlib.sha256()
-    for name in sorted(os.listdir(d)):
-        if name.endswith((".cu", ".cuh")):
-            h.update(name.encode())
-            with open(os.path.join(d, name), "rb") as f:
-                h.update(f.read())
+    for name in sorted(files):
+        h.update(name.encode())
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()
 
 
 def measured_traffic(kernel: str, w):
     """Per-launch DRAM bytes of `kernel` on workload w, or None when no
-    capture exists for it (at w's head size) or the kernel sources changed
-    since."""
+    capture exists for it (at w's head size) or its sources changed since."""
     rec = MEASURED_TRAFFIC.get(kernel)
-    if rec is None or rec["D"] != w.D or rec["sources"] != kernel_sources_hash():
+    if rec is None or rec["D"] != w.D or rec["sources"] != kernel_sources_hash(rec["files"]):
         return None
     return rec["bytes_per_token_head"] * w.B * w.H * w.N
 
