@@ -19,8 +19,10 @@ The printed JSON line also carries:
                 measured launch time (CUDA events recorded by the library on
                 its launch stream during the timed steps) against the measured
                 HBM copy bandwidth;
-  e2e           the same metric with the inputs copied from pinned host
-                memory and the outputs read back inside the timed region;
+  e2e           the same metric with every step's inputs copied from pinned
+                host memory and its outputs (o, dq, dk, dv) read back inside
+                the timed region, consecutive steps pipelined over two copy
+                streams;
   cpu_baseline  the fp64 CPU oracle, as it stands, on a bounded sample;
   clocks        SM clocks and throttle reasons sampled during the timed steps.
 
@@ -389,37 +391,66 @@ def run_ours(args, world, rank, local):
     step_bytes = algorithmic_bytes("fwd_generic", w) + algorithmic_bytes("bwd_generic", w)
     step_frac = (step_bytes / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"]
 
-    # ---- end to end: pinned host inputs in, outputs back, every step
+    # ---- end to end: pinned host inputs in, outputs back, every step.  Steps
+    # are pipelined the way a streaming caller runs them: step t's inputs go
+    # up on one copy stream while step t-1 computes and step t-2's outputs
+    # come down on another (PCIe is full duplex), with two device buffer sets
+    # ordered by events.
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdO = (t.cpu().pin_memory() for t in (q, k, v, dO))
-        ho = [torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
+        hin = [t.cpu().pin_memory() for t in (q, k, v, dO)]
+        hout = [[torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
+                for _ in range(2)]
+        xin = [[q, k, v, dO], [torch.empty_like(t) for t in (q, k, v, dO)]]
+        yout = [[o, dq, dk, dv], [torch.empty_like(q) for _ in range(4)]]
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        in_ready = [torch.cuda.Event() for _ in range(2)]
+        cmp_done = [torch.cuda.Event() for _ in range(2)]
+        out_done = [torch.cuda.Event() for _ in range(2)]
         e2e_steps = max(3, min(args.steps, 10))
 
-        def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            k.copy_(hk, non_blocking=True)
-            v.copy_(hv, non_blocking=True)
-            dO.copy_(hdO, non_blocking=True)
-            step()
-            for dst, src in zip(ho, (o, dq, dk, dv)):
-                dst.copy_(src, non_blocking=True)
+        def e2e_step(t):
+            b = t % 2
+            xq, xk, xv, xdO = xin[b]
+            yo, ydq, ydk, ydv = yout[b]
+            with torch.cuda.stream(s_in):
+                if t >= 2:
+                    s_in.wait_event(cmp_done[b])  # step t-2 no longer reads xin[b]
+                for dst, src in zip(xin[b], hin):
+                    dst.copy_(src, non_blocking=True)
+                in_ready[b].record(s_in)
+            stream.wait_event(in_ready[b])
+            if t >= 2:
+                stream.wait_event(out_done[b])  # step t-2's outputs are on the host
+            api.la_forward(xq, xk, xv, w.causal, w.phi, o=yo, workspace=ws, stream=stream, g=g,
+                           phi_out=None if pq is None else (pq, pk))
+            api.la_backward(xq, xk, xv, xdO, w.causal, w.phi, dq=ydq, dk=ydk, dv=ydv,
+                            workspace=ws, stream=stream, o=yo, g=g, phi_q=pq, phi_k=pk)
+            cmp_done[b].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(cmp_done[b])
+                for dst, src in zip(hout[b], yout[b]):
+                    dst.copy_(src, non_blocking=True)
+                out_done[b].record(s_out)
 
-        e2e_step()
+        for t in range(2):
+            e2e_step(t)
         torch.cuda.synchronize(dev)
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        for t in range(e2e_steps):
+            e2e_step(t)
+        # the last step's outputs are the last work; s_out has waited on all of it
+        e1.record(s_out)
         torch.cuda.synchronize(dev)
         barrier(world)
         ems = max_over_ranks(e0.elapsed_time(e1), world)
         nbytes = q.numel() * q.element_size()
         e2e = {"value": world * tokens_per_step * e2e_steps / (ems / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
-               "steps": e2e_steps}
+               "steps": e2e_steps, "pipelined": "h2d, compute and d2h of consecutive steps overlap"}
+        api.la_get_device_error(stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
