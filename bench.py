@@ -101,15 +101,15 @@ _BWD64_FILES = ("la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "la
 MEASURED_TRAFFIC = {
     "bwd_dkdv": {"bytes_per_token_head": (272.683008e6 + 99.865344e6) / (8 * 16 * 4096), "D": 64,
                  "files": _BWD64_FILES,
-                 "sources": "72c58888f0e4bfed567936cb2686b08bdd191285c3972ce0834ca1cc83a2d671",
+                 "sources": "77a0c1180a9539723e3a666c8615670b382a898e6333731d6e90ea1e63d2d940",
                  "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
     "bwd_dq": {"bytes_per_token_head": (337.681664e6 + 52.509696e6) / (8 * 16 * 4096), "D": 64,
                "files": _BWD64_FILES,
-               "sources": "72c58888f0e4bfed567936cb2686b08bdd191285c3972ce0834ca1cc83a2d671",
+               "sources": "77a0c1180a9539723e3a666c8615670b382a898e6333731d6e90ea1e63d2d940",
                "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
     "chunk_causal": {"bytes_per_token_head": (201.406976e6 + 154.606080e6) / (8 * 16 * 4096),
                      "D": 64, "files": _FWD64_FILES,
-                     "sources": "276466c43a8e5d351119e9842a089875533e7d1c8e5277856323e21cd5ede0a4",
+                     "sources": "c623abd28e30c098899ffe21d4e05be3fcdb663f4db9e7fd1857be3cdd9901bf",
                      "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
 }
 

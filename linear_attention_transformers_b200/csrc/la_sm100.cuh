@@ -137,7 +137,7 @@ __device__ __forceinline__ bool named_bar_all(int id, int nthreads, bool pred) {
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
-// 3-D tiled load (no multicast) that completes a transaction on `bar`.
+// 3-D tiled load into this CTA's shared memory; completes a transaction on `bar`.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2) {
     asm volatile(
