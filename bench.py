@@ -4,25 +4,38 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step is one training pass of the attention layer on the timed workload
-(causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward (which also
-keeps the per-token denominators g and the feature maps phi(q), phi(k))
-followed by la_backward given O, g and the feature maps,
-through the library's Python binding, inputs resident in HBM.
-The inputs (4 x 128 MiB) are larger than the 126 MB L2, so consecutive steps
-cannot serve each other from cache.  W untimed warm-up steps, then exactly K
-steps between two barrier + synchronize points, timed with CUDA events on the
-launching stream; with several GPUs each rank runs its own replica (there is
-no exchange step in this op) and the max time over ranks is used.
+(causal, B=8, H=16, N=8192, D=64, bf16, phi = elu+1): la_forward, which also
+keeps the per-token denominators g and the final state (S, z), followed by
+la_backward given o, g and (S, z), through the library's Python binding,
+inputs resident in HBM.  The inputs (4 x 128 MiB) are larger than the 126 MB
+L2, so consecutive steps cannot serve each other from cache.  W untimed
+warm-up steps, then exactly K steps between two barrier + synchronize
+points, timed with CUDA events on the launching stream; with several GPUs
+each rank runs its own replica (there is no exchange step in this op) and
+the max time over ranks is used.
 
 The printed JSON line also carries:
-  roofline      the dominant kernel's algorithmic bytes per launch over its
-                measured launch time (CUDA events recorded by the library on
-                its launch stream during the timed steps) against the measured
-                HBM copy bandwidth;
-  e2e           the same metric with every step's inputs copied from pinned
-                host memory and its outputs (o, dq, dk, dv) read back inside
-                the timed region, consecutive steps pipelined over two copy
-                streams;
+  roofline      the dominant kernel: algorithmic bytes per launch (the
+                method's byte budget of the pass when the kernel is that
+                whole pass) over its measured launch time (CUDA events the
+                library records on its launch stream during the timed steps)
+                against the measured HBM copy bandwidth;
+  rows          step, forward and backward fractions of the method's byte
+                budget (forward 8 N D, backward 14 N D, step 22 N D bytes per
+                head in bf16; the slower of bytes at HBM peak and flops at
+                the bf16 MMA peak), the split timed with events between the
+                two calls;
+  kernels       per-kernel launch times and the fraction of each kernel's own
+                reads and writes;
+  graded        the other full-size workloads, each with its own clocks: the
+                long-context causal forward (B1 H32 N131072 D128), 1024
+                decode steps (B256 H32 D128, fp32 state in place) and the
+                1.4B-parameter LM layer shape forward + backward (B4 H16
+                N4096 D128) with both feature maps;
+  e2e           the headline metric with every step's inputs copied from
+                pinned host memory and its outputs (o, dq, dk, dv) read back
+                inside the timed region, consecutive steps pipelined over two
+                copy streams;
   cpu_baseline  the fp64 CPU oracle, as it stands, on a bounded sample;
   clocks        SM clocks and throttle reasons sampled during the timed steps.
 
@@ -66,52 +79,59 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def algorithmic_bytes(kernel: str, w) -> float:
-    """Bytes a launch of `kernel` must move at minimum for workload w.
-
-    Element size e; per head N*D elements per tensor.  forward: read q, k, v,
-    write o (4 tensors); backward: read q, k, v, dO, write dq, dk, dv (7).
-    Kernels that implement part of a pass are charged the tensors they must
-    touch (listed beside each name).
-    """
+def method_bytes(w, part: str) -> float:
+    """The method's minimum bytes for workload w (the per-head figures of the
+    method's byte budget, times heads): forward reads q, k, v and writes o
+    (4 tensors); backward reads q, k, v, dO and writes dq, dk, dv (7); the
+    step is both (11 tensors; 22 N D bytes per head in bf16)."""
     e = 2 if w.dtype == torch.bfloat16 else 4
     t = w.B * w.H * w.N * w.D * e  # bytes of one [B,H,N,D] tensor
+    return float({"forward": 4, "backward": 7, "step": 11}[part] * t)
+
+
+def method_flops(w, part: str) -> float:
+    """The method's multiply-add work: 4 N D^2 per head forward (state update
+    and query), 10 N D^2 backward."""
+    per = {"forward": 4, "backward": 10, "step": 14}[part]
+    return float(per * w.B * w.H * w.N * w.D * w.D)
+
+
+def own_bytes(kernel: str, w) -> float:
+    """Bytes one launch of `kernel` must move for workload w by its own
+    design (what it reads and writes), for the per-kernel fractions."""
+    e = 2 if w.dtype == torch.bfloat16 else 4
+    t = w.B * w.H * w.N * w.D * e
     n = w.B * w.H * w.N * 4  # one float32 per token (g or dg)
     table = {
         "fwd_generic": 4 * t,           # q, k, v -> o
         "bwd_generic": 7 * t,           # q, k, v, dO -> dq, dk, dv
-        "chunk_causal": 6 * t + n,      # q, k, v -> o, g, phi(q), phi(k)
+        "chunk_causal": 4 * t + n,      # q, k, v -> o, g (+2t with phi(q), phi(k) stored)
+        "bwd_fused": 8 * t + n,         # q, k, v, dO, o, g -> dq, dk, dv
         "bwd_dq": 6 * t + 2 * n,        # phi(q), phi(k), v, dO, o, g -> dq, dg
         "bwd_dkdv": 6 * t + 2 * n,      # phi(q), phi(k), v, dO, g, dg -> dk, dv
-        "phi_map": 4 * t,               # q, k -> phi(q), phi(k) (paths without a fused store)
+        "phi_map": 4 * t,               # q, k -> phi(q), phi(k)
     }
     return float(table.get(kernel, 0.0))
+
+
+def roofline_of(bytes_, flops, seconds, peaks, sustained=True):
+    """Roofline fraction of a timed region: the slower of bytes at the
+    measured HBM bandwidth and flops at the measured bf16 MMA rate."""
+    hbm = peaks["hbm_gbs"] * 1e9
+    tc = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * 1e12
+    t_roof = max(bytes_ / hbm, flops / tc)
+    return {"bound": "hbm" if bytes_ / hbm >= flops / tc else "tensor",
+            "achieved_gbs": bytes_ / seconds / 1e9, "frac": t_roof / seconds,
+            "algorithmic_bytes": bytes_, "flops": flops}
 
 
 # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), per token and head so that it scales to the bench
 # workload; valid only while the sources the kernel is built and launched
-# from (`files`, under csrc/) hash to `sources`.  The capture ran at
-# N = 4096 (the profiling size rule); traffic grows in proportion to tokens
-# for these kernels (each token's tiles are moved once).
-_FWD64_FILES = ("la_chunk_fwd64.cuh", "la_chunk_fwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
-                "la_common.cuh", "la_api.cu")
-_BWD64_FILES = ("la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
-                "la_common.cuh", "la_api.cu")
-MEASURED_TRAFFIC = {
-    "bwd_dkdv": {"bytes_per_token_head": (272.683008e6 + 99.865344e6) / (8 * 16 * 4096), "D": 64,
-                 "files": _BWD64_FILES,
-                 "sources": "77a0c1180a9539723e3a666c8615670b382a898e6333731d6e90ea1e63d2d940",
-                 "profile": "profiles/bwd_dkdv64_causal_b8h16n4096d64_bf16.md"},
-    "bwd_dq": {"bytes_per_token_head": (337.681664e6 + 52.509696e6) / (8 * 16 * 4096), "D": 64,
-               "files": _BWD64_FILES,
-               "sources": "77a0c1180a9539723e3a666c8615670b382a898e6333731d6e90ea1e63d2d940",
-               "profile": "profiles/bwd_dq64_causal_b8h16n4096d64_bf16.md"},
-    "chunk_causal": {"bytes_per_token_head": (201.406976e6 + 154.606080e6) / (8 * 16 * 4096),
-                     "D": 64, "files": _FWD64_FILES,
-                     "sources": "c623abd28e30c098899ffe21d4e05be3fcdb663f4db9e7fd1857be3cdd9901bf",
-                     "profile": "profiles/chunk_fwd64_causal_b8h16n4096d64_bf16.md"},
-}
+# from (`files`, under csrc/) hash to `sources`.  Captures run at a smaller
+# N (the profiling size rule); these kernels move each token's tiles once,
+# so traffic grows in proportion to tokens.
+MEASURED_TRAFFIC = {}
 
 
 def kernel_sources_hash(files) -> str:
@@ -312,84 +332,241 @@ def config_dict(w, gpus):
 
 
 # --------------------------------------------------------------------- ours
+def timed_region(fn, steps, stream, dev, world, sampler_index):
+    """Run fn() `steps` times between barrier + synchronize points, timed
+    with CUDA events on `stream`; returns (max-over-ranks ms, clocks)."""
+    sampler = ClockSampler(sampler_index)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with sampler:
+        ev0.record(stream)
+        for _ in range(steps):
+            fn()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    return max_over_ranks(ev0.elapsed_time(ev1), world), sampler.summary()
+
+
+class TrainStep:
+    """One forward + backward of workload w through the library's binding,
+    with every output and workspace preallocated: la_forward keeps o, the
+    denominators g and the final state (S, z) (and the feature maps where the
+    backward reads them); la_backward takes them."""
+
+    def __init__(self, api, w, dev, stream, tensors=None):
+        self.api, self.w, self.stream = api, w, stream
+        q, k, v, dO = tensors if tensors is not None else inputs.make_inputs(
+            w, device=dev, with_grad_out=True)
+        self.q, self.k, self.v, self.dO = q, k, v, dO
+        B, H, N, D = q.shape
+        self.o = torch.empty_like(q)
+        self.g = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        self.S = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+        self.z = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+        self.pq = self.pk = None
+        if api.backward_reads_phi(q.dtype, D):
+            self.pq, self.pk = torch.empty_like(q), torch.empty_like(q)
+        self.dq, self.dk, self.dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ws_f = api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal, w.dtype)
+        ws_b = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, w.causal, w.dtype)
+        self.ws = torch.empty(max(ws_f, ws_b, 256), dtype=torch.uint8, device=dev)
+
+    def forward(self, q=None, k=None, v=None, o=None):
+        a, w = self.api, self.w
+        a.la_forward(q if q is not None else self.q, k if k is not None else self.k,
+                     v if v is not None else self.v, w.causal, w.phi,
+                     o=o if o is not None else self.o, workspace=self.ws, stream=self.stream,
+                     g=self.g, phi_out=None if self.pq is None else (self.pq, self.pk),
+                     state_out=(self.S, self.z))
+
+    def backward(self, q=None, k=None, v=None, dO=None, o=None, grads=None):
+        a, w = self.api, self.w
+        dq, dk, dv = grads if grads is not None else (self.dq, self.dk, self.dv)
+        a.la_backward(q if q is not None else self.q, k if k is not None else self.k,
+                      v if v is not None else self.v, dO if dO is not None else self.dO,
+                      w.causal, w.phi, dq=dq, dk=dk, dv=dv, workspace=self.ws,
+                      stream=self.stream, o=o if o is not None else self.o, g=self.g,
+                      phi_q=self.pq, phi_k=self.pk, S=self.S, z=self.z)
+
+    def __call__(self):
+        self.forward()
+        self.backward()
+
+
+def split_times(step, steps, stream):
+    """Forward and backward milliseconds per step, from CUDA events recorded
+    between the two calls on the launching stream (a separate, untimed-by-
+    the-headline pass over the same steps)."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * steps)]
+    for i in range(steps):
+        evs[3 * i].record(stream)
+        step.forward()
+        evs[3 * i + 1].record(stream)
+        step.backward()
+        evs[3 * i + 2].record(stream)
+    torch.cuda.synchronize()
+    f = sum(evs[3 * i].elapsed_time(evs[3 * i + 1]) for i in range(steps)) / steps
+    b = sum(evs[3 * i + 1].elapsed_time(evs[3 * i + 2]) for i in range(steps)) / steps
+    return f, b
+
+
+def graded_train(api, w, dev, stream, world, peaks, steps=20, warmup=5):
+    """A forward + backward workload at its full size: ms per step, tokens/s
+    and the roofline fractions of the step, the forward and the backward."""
+    step = TrainStep(api, w, dev, stream)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    api.la_get_device_error(stream)
+    ms, clocks = timed_region(step, steps, stream, dev, world, dev.index or 0)
+    f_ms, b_ms = split_times(step, max(3, steps // 2), stream)
+    api.la_get_device_error(stream)
+    out = {"workload": w.name, "ms_per_step": ms / steps,
+           "tokens_per_s": world * w.B * w.N * steps / (ms / 1e3),
+           "step": roofline_of(method_bytes(w, "step"), method_flops(w, "step"),
+                               ms / steps / 1e3, peaks),
+           "forward": dict(ms=f_ms, **roofline_of(method_bytes(w, "forward"),
+                                                  method_flops(w, "forward"), f_ms / 1e3, peaks)),
+           "backward": dict(ms=b_ms, **roofline_of(method_bytes(w, "backward"),
+                                                   method_flops(w, "backward"), b_ms / 1e3,
+                                                   peaks)),
+           "clocks": clocks}
+    del step
+    torch.cuda.empty_cache()
+    return out
+
+
+def graded_forward(api, w, dev, stream, world, peaks, steps=10, warmup=3):
+    """The causal forward alone at full size (the long-context workload)."""
+    q, k, v = inputs.make_inputs(w, device=dev, with_grad_out=False)
+    o = torch.empty_like(q)
+    B, H, N, D = q.shape
+    ws = torch.empty(max(256, api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal,
+                                                    w.dtype)), dtype=torch.uint8, device=dev)
+
+    def fwd():
+        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        fwd()
+    torch.cuda.synchronize(dev)
+    api.la_get_device_error(stream)
+    ms, clocks = timed_region(fwd, steps, stream, dev, world, dev.index or 0)
+    api.la_get_device_error(stream)
+    out = {"workload": w.name, "ms_per_call": ms / steps,
+           "tokens_per_s": world * w.B * w.N * steps / (ms / 1e3),
+           "forward": roofline_of(method_bytes(w, "forward"), method_flops(w, "forward"),
+                                  ms / steps / 1e3, peaks),
+           "clocks": clocks}
+    del q, k, v, o, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def graded_decode(api, dev, stream, world, peaks, reps=3, warmup=2):
+    """`steps` recurrent decode steps at batch B (fp32 state in place), each
+    step one la_decode_step over every (b, h); timed over whole runs of all
+    steps."""
+    cfg = inputs.DECODE
+    B, H, D, steps = cfg["B"], cfg["H"], cfg["D"], cfg["steps"]
+    q, k, v = inputs.make_decode_inputs(B, H, D, steps, cfg["seed"], device=dev)
+    S = torch.zeros(B, H, D, D, device=dev)
+    z = torch.zeros(B, H, D, device=dev)
+    outs = torch.empty(steps, B, H, D, dtype=q.dtype, device=dev)
+
+    def run():
+        for t in range(steps):
+            api.la_decode_step(S, z, q[t], k[t], v[t], o=outs[t], stream=stream)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize(dev)
+    api.la_get_device_error(stream)
+    ms, clocks = timed_region(run, reps, stream, dev, world, dev.index or 0)
+    api.la_get_device_error(stream)
+    s_step = ms / reps / steps / 1e3
+    # per head and step: S and z read and written in float32, q, k, v read
+    # and o written in bf16
+    bytes_step = B * H * (2 * 4 * (D * D + D) + 4 * D * 2)
+    flops_step = B * H * 4 * D * D
+    out = {"workload": f"decode_b{B}h{H}d{D}_x{steps}_bf16", "us_per_step": s_step * 1e6,
+           "steps_per_s": world / s_step, "tokens_per_s": world * B / s_step,
+           "step": roofline_of(bytes_step, flops_step, s_step, peaks), "clocks": clocks}
+    del q, k, v, S, z, outs
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     from linear_attention_transformers_b200 import api
     w = workload_from_args(args)
     dev = torch.device("cuda", local)
     api.load_library()
-    q, k, v, dO = (t for t in inputs.make_inputs(w, device=dev))
-    B, H, N, D = q.shape
-    o = torch.empty_like(q)
-    g = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    # saved feature maps where the backward reads them (bf16, D = 64)
-    pq = pk = None
-    if api.backward_reads_phi(q.dtype, D):
-        pq, pk = torch.empty_like(q), torch.empty_like(q)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws_f = api.la_workspace_size(api.LA_OP_FORWARD, B, H, N, D, w.causal, w.dtype)
-    ws_b = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, w.causal, w.dtype)
-    ws = torch.empty(max(ws_f, ws_b, 256), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-
-    def step():
-        # forward keeps its denominators g and feature maps; backward reuses
-        # O, g and phi(q), phi(k)
-        api.la_forward(q, k, v, w.causal, w.phi, o=o, workspace=ws, stream=stream, g=g,
-                       phi_out=None if pq is None else (pq, pk))
-        api.la_backward(q, k, v, dO, w.causal, w.phi, dq=dq, dk=dk, dv=dv, workspace=ws,
-                        stream=stream, o=o, g=g, phi_q=pq, phi_k=pk)
+    peaks, peaks_src = load_peaks()
+    step = TrainStep(api, w, dev, stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
     api.la_get_device_error(stream)
 
-    # ---- timed region
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    # ---- timed region (the headline)
     api.la_profile_enable(True)
     api.la_profile_collect()
     launches0 = api.la_launch_count()
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with sampler:
-        ev0.record(stream)
-        for _ in range(args.steps):
-            step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-    barrier(world)
+    ms_max, clocks = timed_region(step, args.steps, stream, dev, world,
+                                  dev.index if dev.index is not None else 0)
     launches = api.la_launch_count() - launches0
     prof = api.la_profile_collect()
     api.la_profile_enable(False)
     api.la_get_device_error(stream)
-    ms = ev0.elapsed_time(ev1)
-    ms_max = max_over_ranks(ms, world)
     tokens_per_step = w.B * w.N
     value = world * tokens_per_step * args.steps / (ms_max / 1e3)
+    s_step = ms_max / args.steps / 1e3
 
-    # ---- dominant kernel roofline
-    peaks, peaks_src = load_peaks()
-    dom = max(prof.items(), key=lambda kv: kv[1][1]) if prof else None
+    # ---- forward / backward split (events between the calls, own pass)
+    f_ms, b_ms = split_times(step, min(args.steps, 20), stream)
+    rows = {
+        "step": roofline_of(method_bytes(w, "step"), method_flops(w, "step"), s_step, peaks),
+        "forward": dict(ms=f_ms, **roofline_of(method_bytes(w, "forward"),
+                                               method_flops(w, "forward"), f_ms / 1e3, peaks)),
+        "backward": dict(ms=b_ms, **roofline_of(method_bytes(w, "backward"),
+                                                method_flops(w, "backward"), b_ms / 1e3, peaks)),
+    }
+
+    # ---- dominant kernel: the library's own per-launch CUDA events (recorded
+    # on its launch stream during the timed steps).  Its algorithmic bytes are
+    # the method's byte budget of the pass it computes when it is that whole
+    # pass (the single-pass backward: 7 tensors; the causal forward: 4), else
+    # the bytes of its own design (a kernel that is part of a pass).
+    kernels = {}
+    for name, (n, tot) in prof.items():
+        avg_s = tot / n / 1e3
+        ob = own_bytes(name, w)
+        kernels[name] = {"launches": n, "total_ms": tot, "share": tot / max(ms_max, 1e-9),
+                         "avg_ms": avg_s * 1e3, "own_bytes": ob,
+                         "own_frac": (ob / avg_s / 1e9) / peaks["hbm_gbs"] if ob else None}
     roofline = None
-    if dom:
-        name, (n_launch, tot_ms) = dom
-        avg_s = tot_ms / n_launch / 1e3
-        alg = algorithmic_bytes(name, w)
+    if prof:
+        name, (n, tot) = max(prof.items(), key=lambda kv: kv[1][1])
+        avg_s = tot / n / 1e3
+        whole = {"bwd_fused": "backward", "chunk_causal": "forward"}
+        part = whole.get(name)
+        alg = method_bytes(w, part) if part else own_bytes(name, w)
         achieved = alg / avg_s / 1e9
         roofline = {"kernel": name, "bound": "hbm", "achieved": achieved,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"],
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                     "traffic": measured_traffic(name, w),
-                    "algorithmic_bytes_per_launch": alg, "avg_launch_ms": avg_s * 1e3,
-                    "peak_source": f"{peaks_src} hbm_gbs",
-                    "share_of_step": tot_ms / max(ms, 1e-9)}
-    kernels = {k: {"launches": n, "total_ms": t, "share": t / max(ms, 1e-9)}
-               for k, (n, t) in prof.items()}
-    # the method's minimum: forward reads q, k, v and writes o; backward reads
-    # q, k, v, dO and writes dq, dk, dv (22 bytes x D per token and head)
-    step_bytes = algorithmic_bytes("fwd_generic", w) + algorithmic_bytes("bwd_generic", w)
-    step_frac = (step_bytes / (ms / args.steps / 1e3) / 1e9) / peaks["hbm_gbs"]
+                    "algorithmic_bytes_per_launch": alg,
+                    "algorithmic_bytes_basis": (f"method {part}: {7 if part == 'backward' else 4}"
+                                                " tensors of B*H*N*D bf16" if part else
+                                                "the kernel's own reads and writes"),
+                    "avg_launch_ms": avg_s * 1e3,
+                    "peak_source": f"{peaks_src} hbm_gbs (of {peaks_src})",
+                    "share_of_step": tot / max(ms_max, 1e-9)}
 
     # ---- end to end: pinned host inputs in, outputs back, every step.  Steps
     # are pipelined the way a streaming caller runs them: step t's inputs go
@@ -398,11 +575,12 @@ def run_ours(args, world, rank, local):
     # ordered by events.
     e2e = None
     if not args.no_e2e:
+        q, k, v, dO = step.q, step.k, step.v, step.dO
         hin = [t.cpu().pin_memory() for t in (q, k, v, dO)]
         hout = [[torch.empty(q.shape, dtype=q.dtype, pin_memory=True) for _ in range(4)]
                 for _ in range(2)]
         xin = [[q, k, v, dO], [torch.empty_like(t) for t in (q, k, v, dO)]]
-        yout = [[o, dq, dk, dv], [torch.empty_like(q) for _ in range(4)]]
+        yout = [[step.o, step.dq, step.dk, step.dv], [torch.empty_like(q) for _ in range(4)]]
         s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         in_ready = [torch.cuda.Event() for _ in range(2)]
         cmp_done = [torch.cuda.Event() for _ in range(2)]
@@ -422,10 +600,8 @@ def run_ours(args, world, rank, local):
             stream.wait_event(in_ready[b])
             if t >= 2:
                 stream.wait_event(out_done[b])  # step t-2's outputs are on the host
-            api.la_forward(xq, xk, xv, w.causal, w.phi, o=yo, workspace=ws, stream=stream, g=g,
-                           phi_out=None if pq is None else (pq, pk))
-            api.la_backward(xq, xk, xv, xdO, w.causal, w.phi, dq=ydq, dk=ydk, dv=ydv,
-                            workspace=ws, stream=stream, o=yo, g=g, phi_q=pq, phi_k=pk)
+            step.forward(xq, xk, xv, o=yo)
+            step.backward(xq, xk, xv, xdO, o=yo, grads=(ydq, ydk, ydv))
             cmp_done[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(cmp_done[b])
@@ -451,6 +627,22 @@ def run_ours(args, world, rank, local):
                "h2d_bytes_per_step": 4 * nbytes, "d2h_bytes_per_step": 4 * nbytes,
                "steps": e2e_steps, "pipelined": "h2d, compute and d2h of consecutive steps overlap"}
         api.la_get_device_error(stream)
+        del hin, hout, xin, yout
+    del step
+    torch.cuda.empty_cache()
+
+    # ---- the other graded workloads, each at full size with its own clocks
+    graded = None
+    if not args.no_graded and not args.shape:
+        graded = {
+            "long_causal_fwd": graded_forward(api, inputs.WORKLOADS[
+                "causal_fwd_b1h32n131072d128_bf16"], dev, stream, world, peaks),
+            "decode": graded_decode(api, dev, stream, world, peaks),
+            "lm_layer_relu": graded_train(api, inputs.WORKLOADS[
+                "causal_fwdbwd_b4h16n4096d128_relu_bf16"], dev, stream, world, peaks),
+            "lm_layer_elu": graded_train(api, inputs.WORKLOADS[
+                "causal_fwdbwd_b4h16n4096d128_elu_bf16"], dev, stream, world, peaks),
+        }
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -464,13 +656,14 @@ def run_ours(args, world, rank, local):
             "dtype": "bf16", "data": "synthetic",
             "config": config_dict(w, world),
             "roofline": roofline,
-            "step_roofline": {"bound": "hbm", "algorithmic_bytes_per_step": step_bytes,
-                              "frac": step_frac, "peak": peaks["hbm_gbs"], "unit": "GB/s"},
+            "step_roofline": rows["step"],
+            "rows": rows,
             "kernels": kernels,
             "gpu_launches": int(launches),
             "e2e": e2e,
             "cpu_baseline": cpu,
-            "clocks": sampler.summary(),
+            "clocks": clocks,
+            "graded": graded,
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -484,6 +677,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graded", action="store_true",
+                    help="skip the other full-size workloads (long forward, decode, LM layer)")
     ap.add_argument("--shape", default="", help="B,H,N,D override (profiling runs only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:

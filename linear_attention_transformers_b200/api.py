@@ -74,11 +74,11 @@ def load_library(path: str | None = None):
         lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci,
                                    ci, vp, sz, vp]
         lib.la_forward.restype = ci
-        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
-                                    i64, ci, ci, ci, vp, sz, vp]
+        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64,
+                                    i64, i64, ci, ci, ci, vp, sz, vp]
         lib.la_backward.restype = ci
-        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64,
-                                            i64, i64, ci, ci, ci, vp]
+        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                            i64, i64, i64, i64, ci, ci, ci, vp]
         lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
@@ -163,13 +163,16 @@ def _workspace(op, q, causal, workspace):
 
 
 def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=False,
-               workspace=None, stream=None, g=None, phi_out=None):
+               workspace=None, stream=None, g=None, phi_out=None, state_out=None):
     """o = linear attention of q, k, v [B, H, N, D]; optionally the final (S, z).
 
     ``g``: optional float32 [B, H, N] tensor that receives the denominators;
     pass it with ``o`` to la_backward to skip the forward recompute there.
     ``phi_out``: optional pair (pq, pk) of tensors shaped and typed like q
     that receive phi(q), phi(k); pass them to la_backward with o and g.
+    ``state_out``: optional pair (S, z) of float32 tensors [B, H, D, D] and
+    [B, H, D] that receive the final state (instead of allocating them, as
+    ``return_state`` does); pass them to la_backward as S, z.
     """
     lib = load_library()
     _check_qkv("la_forward", q, k, v)
@@ -181,7 +184,14 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     else:
         _check_qkv("la_forward", q, o)
     S = z = None
-    if return_state:
+    if state_out is not None:
+        S, z = state_out
+        for nm, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+            if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
+                    or t.device != q.device:
+                raise ValueError(f"la_forward: {nm} must be contiguous float32 {shape} on q's "
+                                 "device")
+    elif return_state:
         S = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
         z = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
     if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
@@ -199,11 +209,19 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     return (o, S, z) if return_state else o
 
 
-def _check_saved(name, q, o, g, phi_q=None, phi_k=None):
+def _check_saved(name, q, o, g, phi_q=None, phi_k=None, S=None, z=None):
     if (o is None) != (g is None):
         raise ValueError(f"{name}: pass both o and g (saved forward statistics) or neither")
     if (phi_q is None) != (phi_k is None) or (phi_q is not None and o is None):
         raise ValueError(f"{name}: phi_q and phi_k go together, and only with o and g")
+    if (S is None) != (z is None) or (S is not None and o is None):
+        raise ValueError(f"{name}: S and z (final state) go together, and only with o and g")
+    if S is not None:
+        B, H, _, D = q.shape
+        for nm, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+            if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
+                    or t.device != q.device:
+                raise ValueError(f"{name}: {nm} must be contiguous float32 {shape} on q's device")
     if phi_q is not None:
         _check_qkv(name, q, phi_q, phi_k)
     if o is not None:
@@ -214,13 +232,16 @@ def _check_saved(name, q, o, g, phi_q=None, phi_k=None):
 
 
 def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, dv=None,
-                workspace=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
+                workspace=None, stream=None, o=None, g=None, phi_q=None, phi_k=None, S=None,
+                z=None):
     """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi).
 
     ``o``, ``g``: the forward's output and denominators (la_forward(..., g=g));
     when given, the backward does not recompute them.  ``phi_q``, ``phi_k``:
     the forward's feature maps (la_forward(..., phi_out=(phi_q, phi_k))),
     only with ``o`` and ``g``; when given, phi is not evaluated again.
+    ``S``, ``z``: the forward's final state (la_forward(..., return_state=True)),
+    only with ``o`` and ``g``; the single-pass causal backward starts from it.
     """
     lib = load_library()
     _check_qkv("la_backward", q, k, v, dO)
@@ -231,10 +252,10 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward", q, dq, dk, dv)
-    _check_saved("la_backward", q, o, g, phi_q, phi_k)
+    _check_saved("la_backward", q, o, g, phi_q, phi_k, S, z)
     ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
     st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(phi_q),
-                         _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(phi_k), _ptr(S), _ptr(z), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
                          ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
@@ -242,26 +263,28 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
 
 
 def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None,
-                        dv=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
+                        dv=None, stream=None, o=None, g=None, phi_q=None, phi_k=None, S=None,
+                        z=None):
     """la_backward on the library's static device scratch (no workspace).
 
     For callers that cannot allocate device memory during the call; see
     la_backward_noalloc in include/la_api.h for the limits (a fixed maximum
-    scratch size, one shared scratch array: overlapping calls race).  Output
-    tensors must be passed in to avoid allocation here as well.
+    scratch size, one shared scratch array: overlapping calls race).  The
+    output tensors dq, dk, dv are required: this wrapper allocates nothing
+    either, and raises ValueError when one of them is missing.
     """
     lib = load_library()
     _check_qkv("la_backward_noalloc", q, k, v, dO)
     if q.dim() != 4:
         raise ValueError("la_backward_noalloc: tensors must be [B, H, N, D]")
+    if dq is None or dk is None or dv is None:
+        raise ValueError("la_backward_noalloc: pass dq, dk and dv (it allocates nothing)")
     B, H, N, D = q.shape
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward_noalloc", q, dq, dk, dv)
-    _check_saved("la_backward_noalloc", q, o, g, phi_q, phi_k)
+    _check_saved("la_backward_noalloc", q, o, g, phi_q, phi_k, S, z)
     st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g),
-                                 _ptr(phi_q), _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N,
+                                 _ptr(phi_q), _ptr(phi_k), _ptr(S), _ptr(z), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, H, N,
                                  D, DTYPE[q.dtype], int(bool(causal)),
                                  _phi(phi), _stream_handle(stream))
     _check("la_backward_noalloc", st)

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "la_chunk_bwd.cuh"
@@ -142,7 +143,26 @@ bool make_qkv_map(CUtensorMap* m, const void* base, int64_t heads, int64_t N, in
 }
 
 // ------------------------------------------------------------ chunked path
-constexpr int kNumSM = 148;
+// Streaming multiprocessors of the current device (queried once per device
+// and cached; 148, the B200's count, where no device answers, so that sizing
+// calls made without a GPU still plan like the launches will).
+constexpr int kDefaultSMs = 148;
+int num_sms() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return kDefaultSMs;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return kDefaultSMs;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
 
 bool fast_path(la_dtype dt, int64_t D) { return dt == LA_BF16 && (D == 64 || D == 128); }
 int chunk_len(int64_t D) { return D == 64 ? 128 : 64; }
@@ -154,7 +174,8 @@ int chunk_len(int64_t D) { return D == 64 ? 128 : 64; }
 // k and v again (about 0.3 of a chunk each).  Pick the s with the smallest
 // modelled makespan; 120 or more heads stay unsplit (one wave or close).
 int pick_nseg(int64_t heads, int64_t nchunks) {
-    if (heads >= 120 || nchunks < 4) return 1;
+    const int kNumSM = num_sms();
+    if (heads >= kNumSM * 120 / 148 || nchunks < 4) return 1;
     constexpr double kFill = 3.0, kStatePass = 0.3;
     int best = 1;
     double best_cost = double((heads + kNumSM - 1) / kNumSM) * (double(nchunks) + kFill);
@@ -197,6 +218,7 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
     p.C = chunk_len(D);
     const int64_t heads = B * H;
     const int64_t nch = (N + p.C - 1) / p.C;
+    const int kNumSM = num_sms();
     p.seg = split(N, p.C, pick_nseg(heads, nch));
     const size_t R = size_t(D) * D + D;
     if (causal) {
@@ -351,6 +373,7 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     p.C = chunk_len(D);
     const int64_t heads = B * H;
     const int64_t nch = (N + p.C - 1) / p.C;
+    const int kNumSM = num_sms();
     const size_t R = size_t(D) * D + D;
     const size_t tok = size_t(heads) * size_t(N) * sizeof(float);
     size_t off = 0;
@@ -628,7 +651,7 @@ struct PhiMapOp {
     static la_status run(const void* q, const void* k, void* pq, void* pk, int64_t n,
                          cudaStream_t st) {
         la::LaunchScope scope("phi_map", st);
-        const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(kNumSM) * 16);
+        const int64_t blocks = std::min<int64_t>((n + 255) / 256, int64_t(num_sms()) * 16);
         la::phi_map_kernel<T, PHI><<<unsigned(blocks), 256, 0, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<T*>(pq),
             static_cast<T*>(pk), n);
@@ -664,7 +687,12 @@ void* g_scratch_ptr[kMaxDevices] = {};
 la_status static_scratch(void** out) {
     int dev = 0;
     if (cudaError_t e = cudaGetDevice(&dev)) return cuda_fail("cudaGetDevice", e);
-    if (dev < 0 || dev >= kMaxDevices) return LA_ERR_UNSUPPORTED;
+    if (dev < 0 || dev >= kMaxDevices) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "la_backward_noalloc: device index %d beyond the %d devices it tracks", dev,
+                 kMaxDevices);
+        return LA_ERR_UNSUPPORTED;
+    }
     std::lock_guard<std::mutex> g(g_scratch_mu);
     if (!g_scratch_ptr[dev]) {
         void* p = nullptr;
@@ -762,6 +790,7 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
 
 la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
                       const void* o, const float* g, const void* phi_q, const void* phi_k,
+                      const float* S_final, const float* z_final,
                       void* dq, void* dk, void* dv, int64_t B,
                       int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
                       void* workspace, size_t workspace_bytes, la_stream_t stream) {
@@ -780,6 +809,9 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     // saved feature maps: both or neither, and only with o and g
     if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
     if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
+    // the forward's final state: both or neither, and only with o and g
+    if ((S_final == nullptr) != (z_final == nullptr) || (S_final && !o)) return LA_ERR_INVALID_ARG;
+    if (S_final && ((s = check_ptr(S_final)) || (s = check_ptr(z_final)))) return s;
     const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -803,7 +835,8 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
 
 la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
                               const void* o, const float* g, const void* phi_q,
-                              const void* phi_k, void* dq, void* dk, void* dv,
+                              const void* phi_k, const float* S_final, const float* z_final,
+                              void* dq, void* dk, void* dv,
                               int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, int causal,
                               la_phi phi, la_stream_t stream) {
     la_status s;
@@ -819,9 +852,8 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
     if ((s = bind_context()) != LA_OK) return s;
     void* scratch = nullptr;
     if ((s = static_scratch(&scratch)) != LA_OK) return s;
-    return la_backward(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, N, D, dt, causal, phi,
-                       scratch,
-                       size_t(LA_NOALLOC_MAX_BYTES), stream);
+    return la_backward(q, k, v, dO, o, g, phi_q, phi_k, S_final, z_final, dq, dk, dv, B, H, N, D,
+                       dt, causal, phi, scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 
 la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,

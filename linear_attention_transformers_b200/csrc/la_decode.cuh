@@ -28,6 +28,7 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
     constexpr int RG = 8;        // row groups
     constexpr int RPT = D / RG;  // rows per thread
     constexpr int NT = 2 * D;
+    constexpr bool kExact = sizeof(T) == sizeof(float);
     static_assert(CG * RG == NT, "thread layout");
     __shared__ float a_s[D], b_s[D];
     __shared__ float4 v_s4[CG];
@@ -46,8 +47,11 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
 
     float znew = 0.f;
     if (tid < D) {
-        const float af = phi_fast<PHI>(to_f32(q[h * D + tid]));
-        const float bf = phi_fast<PHI>(to_f32(k[h * D + tid]));
+        // float32 tensors take libm's expf, as the float32 forward and
+        // backward do; bf16 ones the base-2 form (rounded away right after)
+        const float xq = to_f32(q[h * D + tid]), xk = to_f32(k[h * D + tid]);
+        const float af = kExact ? phi_exact<PHI>(xq) : phi_fast<PHI>(xq);
+        const float bf = kExact ? phi_exact<PHI>(xk) : phi_fast<PHI>(xk);
         a_s[tid] = af;
         b_s[tid] = bf;
         reinterpret_cast<float*>(v_s4)[tid] = to_f32(v[h * D + tid]);

@@ -5,8 +5,8 @@ inside a CUDA stream capture, code running under an allocator policy that
 forbids new allocations, or a plugin that only receives its input and output
 buffers.  For them la_backward_noalloc runs la_backward on a scratch array
 the library reserves statically in device memory.  This file checks, through
-the C ABI, that two calls in a row give the same gradients as la_backward
-with a caller-provided workspace (the second call on different shapes, so
+the C ABI, that two calls in a row give bit-identical gradients to
+la_backward with a caller-provided workspace (the second call on different shapes, so
 stale scratch contents from the first call would show), and that a call
 needing more scratch than the fixed maximum is refused before any launch.
 
@@ -18,10 +18,13 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from linear_attention_transformers_b200 import api, inputs
 from parity_util import compare
 
 pytestmark = pytest.mark.gpu
+
+PHIS = {"elu1": oracle.PHI_ELU1, "relu_eps": oracle.PHI_RELU_EPS}
 
 
 def _call_noalloc(lib, q, k, v, dO, dq, dk, dv, causal, phi):
@@ -30,7 +33,7 @@ def _call_noalloc(lib, q, k, v, dO, dq, dk, dv, causal, phi):
     return lib.la_backward_noalloc(
         ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
         ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(dO.data_ptr()), None, None, None, None,
-        ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+        None, None, ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
         ctypes.c_void_p(dv.data_ptr()), B, H, N, D, api.DTYPE[q.dtype], int(causal),
         api.PHI[phi], ctypes.c_void_p(stream))
 
@@ -50,8 +53,13 @@ def test_noalloc_backward_matches_workspace_backward(first, second):
         assert st == api.LA_OK, api.la_status_string(st)
         torch.cuda.synchronize()
         api.la_get_device_error()
+        # the same deterministic kernels on the same inputs: bit for bit
         for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-            compare(g, r.double().cpu().numpy(), torch.bfloat16, f"call {call} {name}")
+            assert torch.equal(g, r), f"call {call} {name}: differs from la_backward"
+        # and the reference call itself is right
+        refs = oracle.backward(q, k, v, dO, causal, PHIS[phi])
+        for name, r, o in zip(("dq", "dk", "dv"), ref, refs):
+            compare(r, o, torch.bfloat16, f"call {call} la_backward {name}")
 
 
 def test_noalloc_rejects_sizes_beyond_the_limit():
@@ -60,8 +68,8 @@ def test_noalloc_rejects_sizes_beyond_the_limit():
     need = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, True, torch.bfloat16)
     assert need > (64 << 20)
     fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check fails first
-    st = lib.la_backward_noalloc(fake, fake, fake, fake, None, None, None, None, fake, fake, fake,
-                                 B, H, N, D,
+    st = lib.la_backward_noalloc(fake, fake, fake, fake, None, None, None, None, None, None,
+                                 fake, fake, fake, B, H, N, D,
                                  api.LA_BF16, 1, 0, None)
     assert st == api.LA_ERR_WORKSPACE
     assert "limit" in api.la_last_error()
