@@ -336,10 +336,15 @@ def la_profile_collect() -> dict:
 
 
 def backward_reads_phi(dtype, D: int) -> bool:
-    """True where la_backward reads saved phi(q), phi(k) instead of
-    evaluating the feature map (the bf16 head-size-64 kernels); elsewhere
-    they are ignored and asking the forward for them only costs a pass."""
-    return dtype == torch.bfloat16 and D == 64
+    """Whether saving phi(q), phi(k) in the forward pays off for la_backward.
+
+    The single-pass causal backward (bf16, head size 64) evaluates the
+    feature map from q and k itself (it needs phi(k) - c rounded once, from
+    k), and the other paths read the maps in one of two passes at most, so
+    the forward's extra write never pays back: False everywhere.  la_forward
+    still writes them on request (phi_out) and la_backward still accepts
+    them."""
+    return False
 
 
 class LinearAttention(torch.autograd.Function):

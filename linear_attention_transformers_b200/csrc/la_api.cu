@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "la_chunk_bwd.cuh"
+#include "la_bwd_fused64.cuh"
 #include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
@@ -359,10 +360,18 @@ la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o
 // ------------------------------------------------------------ chunked backward
 struct BwdPlan {
     bool fast = false;
+    // causal, head size 64, one segment per head: the single-pass kernel
+    // (with saved o and g); fin_off holds the final state when the caller
+    // does not pass it
+    bool fused = false;
+    size_t fin_off = 0;
     int C = 0;
     SegSplit seg;   // causal: segments of both passes; non-causal: reduce split
     SegSplit qseg;  // non-causal: split of the two gradient passes
     size_t g_off = 0, dg_off = 0, srec_off = 0, stot_off = 0, rrec_off = 0, rtot_off = 0;
+    // without the forward's o and g, la_backward first runs the forward into
+    // o (o_off) and g (g_off) with the forward's own workspace at fwd_off
+    size_t o_off = 0, fwd_off = 0;
     size_t bytes = 0;
 };
 
@@ -384,6 +393,11 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     p.seg = split(N, p.C, pick_nseg(heads, nch));
     if (causal) {
         p.qseg = p.seg;
+        if (D == 64 && p.seg.nseg == 1) {
+            p.fused = true;
+            p.fin_off = off;
+            off += round_up(size_t(heads) * R * 4, 256);
+        }
         if (p.seg.nseg > 1) {
             p.srec_off = off;
             off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
@@ -402,6 +416,10 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
         p.rtot_off = off;
         off += round_up(size_t(heads) * R * 4, 256);
     }
+    p.o_off = off;
+    off += round_up(size_t(heads) * size_t(N) * size_t(D) * 2, 256);
+    p.fwd_off = off;
+    off += round_up(plan_fwd(B, H, N, D, causal, dt).bytes, 256);
     p.bytes = off;
     return p;
 }
@@ -419,9 +437,9 @@ la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64
 template <int D, int PHI>
 la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO,
                           const void* o_saved, const float* g_saved, const void* pq,
-                          const void* pk, void* dq, void* dk, void* dv,
-                          int64_t heads, int64_t N, int causal, const BwdPlan& p, char* ws,
-                          cudaStream_t st) {
+                          const void* pk, const float* S_fin, const float* z_fin, void* dq,
+                          void* dk, void* dv, int64_t heads, int64_t N, int causal,
+                          const BwdPlan& p, char* ws, cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
     la::BwdParams prm;
     memset(&prm, 0, sizeof(prm));
@@ -432,10 +450,10 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
         !make_qkv_map(&prm.tm_dk, dk, heads, N, D, C) || !make_qkv_map(&prm.tm_dv, dv, heads, N, D, C))
         return LA_ERR_CUDA;
     prm.N = int(N);
-    const bool saved = o_saved != nullptr && g_saved != nullptr;
-    // with saved statistics g is the caller's (read only); otherwise pass 1
-    // writes it to the workspace
-    prm.gbuf = saved ? const_cast<float*>(g_saved) : reinterpret_cast<float*>(ws + p.g_off);
+    // the forward's o and g: the caller's, or computed into the workspace
+    // by la_backward before this runs
+    if (o_saved == nullptr || g_saved == nullptr) return LA_ERR_INVALID_ARG;
+    prm.gbuf = const_cast<float*>(g_saved);
     prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
     prm.o_in = static_cast<const __nv_bfloat16*>(o_saved);
     prm.dk_out = static_cast<__nv_bfloat16*>(dk);
@@ -471,7 +489,39 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     red.S_out = srec;
     red.z_out = srec + D * D;
     red.stride_S = red.stride_z = R;
+    // the dQ products use the centred key features phi(k) - c, and so do
+    // the states they start from
+    red.center = 1;
 
+    if constexpr (D == 64) {
+        if (causal && p.fused) {
+            // one pass from the last chunk to the first, starting from the
+            // centred final state (sum of (phi(k) - c) v^T and of phi(k) - c)
+            // summed here with the same bf16 features the pass subtracts.
+            // The kernel evaluates phi on q and k itself (saved feature maps
+            // are not used: phi(k) - c is rounded once, from k).
+            (void)S_fin;
+            (void)z_fin;
+            la::BwdParams f = prm;
+            f.seg_len = int(N);
+            f.nseg = 1;
+            float* fin = reinterpret_cast<float*>(ws + p.fin_off);
+            la::ChunkParams r = red;
+            r.seg_len = int(N);
+            r.nseg = 1;
+            r.S_out = fin;
+            r.z_out = fin + D * D;
+            r.stride_S = r.stride_z = R;
+            r.center = 1;
+            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads, st, "chunk_reduce")) != LA_OK)
+                return s;
+            f.S_fin = fin;
+            f.z_fin = fin + D * D;
+            f.stride_S = f.stride_z = R;
+            return launch_bwd_kernel(la::bwd_fused64_kernel<PHI>, la::BwdFused64Cfg::SMEM, f, heads,
+                                     st, "bwd_fused", la::kBwdFused64Threads);
+        }
+    }
     if (causal) {
         la::BwdParams p1 = prm, p2 = prm;
         p1.seg_len = p2.seg_len = p.seg.seg_len;
@@ -486,24 +536,8 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
             p1.state_in = srec;
             p1.rec_out = rrec;
         }
-        if constexpr (D == 64) {
-            // one segment per head with saved statistics: the pipelined pass
-            if (saved && p.seg.nseg == 1) {
-                if ((s = pin ? launch_bwd_kernel(la::bwd_dq64_kernel<PHI, true>, la::Bwd1x64Cfg::SMEM,
-                                                 with_phi(p1), heads, st, "bwd_dq", la::kBwd64Threads)
-                             : launch_bwd_kernel(la::bwd_dq64_kernel<PHI, false>, la::Bwd1x64Cfg::SMEM,
-                                                 p1, heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
-                    return s;
-                return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
-                                               with_phi(p2), heads, st, "bwd_dkdv", la::kBwd64Threads)
-                           : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
-                                               p2, heads, st, "bwd_dkdv", la::kBwd64Threads);
-            }
-        }
-        if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
-                                           heads * p.seg.nseg, st, "bwd_dq")
-                       : launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, false>, smem1, p1,
-                                           heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
+        if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
+                                   heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
             return s;
         if (p.seg.nseg > 1) {
             if ((s = launch_state_kernel(3, rrec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
@@ -536,10 +570,8 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     p1.state_in = stot;
     p1.in_per_head = 1;
     p1.rec_out = rrec;
-    if ((s = saved ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, true>, smem1, p1,
-                                       heads * p.qseg.nseg, st, "bwd_dq")
-                   : launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, false>, smem1, p1,
-                                       heads * p.qseg.nseg, st, "bwd_dq")) != LA_OK)
+    if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, true>, smem1, p1,
+                               heads * p.qseg.nseg, st, "bwd_dq")) != LA_OK)
         return s;
     if ((s = launch_state_kernel(1, rrec, rtot, nullptr, nullptr, heads, p.qseg.nseg, D, st)) !=
         LA_OK)
@@ -553,14 +585,15 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
 template <int PHI>
 la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO,
                             const void* o_saved, const float* g_saved, const void* pq,
-                            const void* pk, void* dq, void* dk, void* dv, int64_t heads, int64_t N,
-                            int64_t D, int causal, const BwdPlan& p, char* ws, cudaStream_t st) {
+                            const void* pk, const float* S_fin, const float* z_fin, void* dq,
+                            void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
+                            const BwdPlan& p, char* ws, cudaStream_t st) {
     if (D == 64)
-        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
-                                        N, causal, p, ws, st);
+        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, S_fin, z_fin, dq,
+                                        dk, dv, heads, N, causal, p, ws, st);
     // the D = 128 kernels evaluate the feature map themselves
-    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk, dv,
-                                     heads, N, causal, p, ws, st);
+    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, nullptr,
+                                     nullptr, dq, dk, dv, heads, N, causal, p, ws, st);
 }
 
 // ------------------------------------------------------------ generic path
@@ -819,11 +852,30 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     if ((s = bind_context()) != LA_OK) return s;
     if (bp.fast) {
         char* wsp = static_cast<char*>(workspace);
+        if (o == nullptr) {
+            // the chunked backward reads the forward's o and g: compute them
+            // here (into the workspace) when the caller has not kept them
+            const FwdPlan fp = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
+            void* o_ws = wsp + bp.o_off;
+            float* g_ws = reinterpret_cast<float*>(wsp + bp.g_off);
+            s = phi == LA_PHI_ELU1
+                    ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o_ws, nullptr, nullptr, g_ws, nullptr,
+                                                  nullptr, heads, N, D, causal ? 1 : 0, fp,
+                                                  wsp + bp.fwd_off, st)
+                    : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o_ws, nullptr, nullptr, g_ws,
+                                                      nullptr, nullptr, heads, N, D,
+                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st);
+            if (s != LA_OK) return s;
+            o = o_ws;
+            g = g_ws;
+        }
         return phi == LA_PHI_ELU1
-                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st)
-                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st);
+                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, S_final,
+                                                 z_final, dq, dk, dv, heads, N, D,
+                                                 causal ? 1 : 0, bp, wsp, st)
+                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, S_final,
+                                                     z_final, dq, dk, dv, heads, N, D,
+                                                     causal ? 1 : 0, bp, wsp, st);
     }
     const BwdWorkspace w = plan_bwd(B, H, N);
     char* ws = static_cast<char*>(workspace);

@@ -53,6 +53,11 @@ struct BwdParams {
     // outputs as plain pointers, for kernels that store rows directly
     __nv_bfloat16* dk_out;
     __nv_bfloat16* dv_out;
+    // single-pass backward: the forward's final state, S [D][D] (row = key
+    // feature) at S_fin + head * stride_S and z [D] at z_fin + head * stride_z
+    const float* S_fin;
+    const float* z_fin;
+    int64_t stride_S, stride_z;
 };
 
 template <int D, int C>
@@ -388,10 +393,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
             uint8_t* st = smem + s * Cfg::STAGE;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
+            // q -> phi(q); k -> phi(k) - c (the centred key features: see
+            // the epilogue's all-ones correction)
             if (u < 128)
                 phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
             else
-                phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
+                phi_tile<PHI, C, D, 128, true>(st + Cfg::TILE, u - 128, nvalid, true);
             if (SAVED) {
                 // dU = dO / g in place, dg = -(dO . O) / g; 256 / C threads per row
                 constexpr int TPR = 256 / C;          // threads per row
@@ -657,11 +664,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 tc_fence_before();
                 mbar_arrive(wt_ready);
             }
-            // ---- dQ = (dA + dg z) * phi'(q)
+            // ---- dQ = (T + t 1) * phi'(q): T = dA + dg z formed with the
+            // centred key features phi(k) - c, which differ from the true dA
+            // only along the all-ones vector; that component is restored from
+            // <dA_i, a_i> = 0 (t = -(T . a_i) / (1 . a_i)).
             if (!named_bar_all(1, 128, mbar_wait(da_ready, c & 1, abort_flag))) break;
             tc_fence_after();
             if (e == 0) bulk_wait_read0();
             named_bar_sync(1, 128);
+            constexpr float kc = phi_center<PHI>();
+            float tcoef = 0.f;
+            if (kc != 0.f) {
+                float dot = 0.f, sa = 0.f;
+#pragma unroll 1
+                for (int f0 = 0; f0 < D; f0 += 16) {
+                    float av[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_O + f0, av);
+                    tmem_wait_ld();
+                    if (irow >= 0) {
+                        float a8a[8], a8b[8];
+                        load_chunk8(qt, C, irow, f0 >> 3, a8a);
+                        load_chunk8(qt, C, irow, (f0 >> 3) + 1, a8b);
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            dot = fmaf(fmaf(dg, zf[f0 + t], av[t]), a8a[t], dot);
+                            dot = fmaf(fmaf(dg, zf[f0 + 8 + t], av[8 + t]), a8b[t], dot);
+                            sa += a8a[t] + a8b[t];
+                        }
+                    }
+                }
+                tcoef = irow >= 0 ? -kc * dot / sa : 0.f;
+            }
 #pragma unroll 1
             for (int f0 = 0; f0 < D; f0 += 16) {
                 float av[16];
@@ -674,8 +707,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     float dq16[16];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
-                        dq16[t] = fmaf(dg, zf[f0 + t], av[t]) * dphi_from_phi<PHI>(a8a[t]);
-                        dq16[8 + t] = fmaf(dg, zf[f0 + 8 + t], av[8 + t]) * dphi_from_phi<PHI>(a8b[t]);
+                        dq16[t] = (fmaf(dg, zf[f0 + t], av[t]) + tcoef) * dphi_from_phi<PHI>(a8a[t]);
+                        dq16[8 + t] =
+                            (fmaf(dg, zf[f0 + 8 + t], av[8 + t]) + tcoef) * dphi_from_phi<PHI>(a8b[t]);
                     }
                     store_row16_bf16(stg, C, irow, f0, dq16);
                 }

@@ -67,6 +67,9 @@ struct ChunkParams {
     // the products read, stored by TMA (D = 64 CAUSAL kernel, store_phi != 0).
     CUtensorMap tm_pq, tm_pk;
     int store_phi;
+    // REDUCE: sum phi(k) - phi_center (the centred state the backward's dQ
+    // products use) instead of phi(k)
+    int center;
 };
 
 // Shared-memory and TMEM plan of the kernel below (head size 128, 64-token
@@ -327,6 +330,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     phi_tile<PHI, C, D, 128>(kt, u - 128, nvalid, true);
             } else if (MODE == MODE_QUERY) {
                 phi_tile<PHI, C, D, 256>(qt, u, nvalid, false);
+            } else if (prm.center) {
+                phi_tile<PHI, C, D, 256, true>(kt, u, nvalid, true);
             } else {
                 phi_tile<PHI, C, D, 256>(kt, u, nvalid, true);
             }

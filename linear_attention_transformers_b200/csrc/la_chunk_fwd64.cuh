@@ -262,6 +262,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                     phi_tile<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true);
             } else if (MODE == MODE_QUERY) {
                 phi_tile<PHI, C, D, 256>(st, u, nvalid, false);
+            } else if (prm.center) {
+                phi_tile<PHI, C, D, 256, true>(st + Cfg::TILE, u, nvalid, true);
             } else {
                 phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
             }

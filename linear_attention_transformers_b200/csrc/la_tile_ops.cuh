@@ -24,12 +24,37 @@ __device__ __forceinline__ uint32_t phi2_elu1(uint32_t w) {
     return r;
 }
 
+// The same map less its value at 0 minus the x > 0 slope's offset:
+// elu(x) = phi(x) - 1 (x for x > 0, exp(x) - 1 otherwise), to bf16.  The
+// exponential and the subtraction run in fp32 before the one rounding, so
+// the small deviations of phi from 1 keep bf16's relative precision instead
+// of being rounded against the 1.
+__device__ __forceinline__ uint32_t phi2_elu1_centered(uint32_t w) {
+    uint32_t m, big, r;
+    asm("min.NaN.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(w), "r"(0u));
+    asm("max.NaN.bf16x2 %0, %1, %2;" : "=r"(big) : "r"(w), "r"(0u));
+    const uint32_t e = sm100::pack_bf16(exp_fast(__uint_as_float(m << 16)) - 1.f,
+                                        exp_fast(__uint_as_float(m & 0xffff0000u)) - 1.f);
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(e), "r"(big));
+    return r;
+}
+
+// The constant c with phi = c + (a map whose typical values are small): the
+// feature vectors of elu(x)+1 on small inputs sit near the all-ones vector,
+// so products of them are formed from phi - 1 plus rank-one terms in c;
+// relu(x)+1e-6 has no such offset.
+template <int PHI>
+__host__ __device__ constexpr float phi_center() {
+    return PHI == PHI_ELU1 ? 1.f : 0.f;
+}
+
 // Apply the feature map in place to a [C][D] bf16 row tile.  The T threads
 // calling this split the tile's C*D/8 16-byte chunks evenly; each thread
 // loads all of its chunks before it computes so their latencies overlap.
 // Rows >= nvalid are written as zero when `zero_tail` (a partial last chunk:
-// those keys must not reach the state).
-template <int PHI, int C, int D, int T>
+// those keys must not reach the state).  CENTER: write phi - phi_center
+// instead (see phi2_elu1_centered).
+template <int PHI, int C, int D, int T, bool CENTER = false>
 __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool zero_tail) {
     using namespace sm100;
     constexpr int CH = D / 8;
@@ -48,7 +73,7 @@ __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool 
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (PHI == PHI_ELU1) {
-                w[k] = zero ? 0u : phi2_elu1(w[k]);
+                w[k] = zero ? 0u : (CENTER ? phi2_elu1_centered(w[k]) : phi2_elu1(w[k]));
             } else {
                 const float2 f = unpack_bf16(w[k]);
                 w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x), phi_fast<PHI>(f.y));
@@ -59,6 +84,24 @@ __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool 
 #pragma unroll
     for (int i = 0; i < PER; ++i)
         *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + i)) = x[i];
+}
+
+// Sum of row `row` of a [C][D] bf16 row tile (fp32, fixed order).
+template <int C, int D>
+__device__ __forceinline__ float tile_row_sum(const uint8_t* tile, int row) {
+    using namespace sm100;
+    float acc = 0.f;
+#pragma unroll
+    for (int q = 0; q < D / 8; ++q) {
+        const uint4 x = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q));
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16(w[k]);
+            acc += f.x + f.y;
+        }
+    }
+    return acc;
 }
 
 // Scale rows of a [C][D] bf16 row tile in place: row r times rs[r] (rows >=

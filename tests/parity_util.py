@@ -66,9 +66,11 @@ def ratios(g, r):
     return rms_ratio, max_ratio, float(err.max()), max_rel
 
 
-def compare(gpu, ref, dtype, what=""):
+def compare(gpu, ref, dtype, what="", elementwise=True):
     """Assert elementwise and normalised parity; return (max_abs, max_rel,
-    err_rms/ref_rms, max_err/max_ref)."""
+    err_rms/ref_rms, max_err/max_ref).  elementwise=False skips the output
+    tolerance (for sums such as the final state, bounded against their own
+    scale by the caller)."""
     atol, rtol = TOL[dtype]
     eps_rms, eps_max = NORM[dtype]
     g = gpu.detach().to("cpu").double().numpy() if isinstance(gpu, torch.Tensor) else \
@@ -85,7 +87,7 @@ def compare(gpu, ref, dtype, what=""):
     bad = err > atol + rtol * np.abs(r)
     summary = (f"max_abs={max_abs:.3e} max_rel={max_rel:.3e} err_rms/ref_rms={rms_ratio:.3e} "
                f"max_err/max_ref={max_ratio:.3e}")
-    if bad.any():
+    if elementwise and bad.any():
         idx = np.unravel_index(np.argmax(err - (atol + rtol * np.abs(r))), err.shape)
         raise AssertionError(
             f"{what}: {int(bad.sum())}/{bad.size} elements out of tolerance "
@@ -103,7 +105,9 @@ def check_state(S, z, S_ref, z_ref, dtype):
     state's own scale (2e-5 for float32 inputs; for bf16 inputs the tensor
     cores sum phi(k) rounded to bf16, a relative error of at most 2^-9 per
     term that adds up like a random walk, bounded here by 4e-3 of the scale),
-    plus the normalised bound of compare()."""
+    plus the normalised bound of compare() (its elementwise output tolerance
+    is an absolute bound for outputs of order one and does not apply to sums
+    over N tokens)."""
     rel = 2e-5 if dtype == torch.float32 else 4e-3
     for name, got, ref in (("S", S, S_ref), ("z", z, z_ref)):
         g = got.double().cpu().numpy()
@@ -111,4 +115,4 @@ def check_state(S, z, S_ref, z_ref, dtype):
         err = np.abs(g - ref)
         assert (err <= rel * scale + 1e-6).all(), \
             f"final {name}: max err {err.max():.3e} vs {rel:.1e} of scale {scale:.3e}"
-        compare(got, ref, dtype, f"final {name}")
+        compare(got, ref, dtype, f"final {name}", elementwise=False)
