@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define LA_API_VERSION 3
+#define LA_API_VERSION 2
 
 #if defined(__GNUC__)
 #define LA_EXPORT __attribute__((visibility("default")))
@@ -131,24 +131,16 @@ LA_EXPORT la_status la_forward(const void *q, const void *k, const void *v, void
  * size 64 kernels read them in place of evaluating phi on q and k (phi'
  * then comes from phi: min(phi, 1) for elu+1, 1 where phi exceeds the
  * x <= 0 value for relu+eps); other paths ignore them.
- * S_final [B, H, D, D] and z_final [B, H, D] (float32; the forward's S_out,
- * z_out: the state after all N tokens) are optional, both or neither, and
- * only together with o and g.  The causal single-pass backward (bf16, head
- * size 64) walks the chunks from last to first and needs them: it forms
- * each chunk's prefix state as the final state minus the suffix it has
- * accumulated, which keeps one read of every input and one write of every
- * gradient.  Without them it first sums the final state itself (one more
- * read of k and v, into the workspace); other paths ignore them.  They
- * must be the final state of the same forward (same inputs and feature map).
+ * The tensor-core dQ products use the centred key features phi(k) - 1
+ * (elu+1) so that bf16 operands keep phi's small deviations from 1; they
+ * are evaluated from k, never from a saved phi(k).
  * No N x D x D tensor is ever stored: the prefix and suffix states are
  * rebuilt chunk by chunk.  dq/dk/dv must not alias the inputs.  Errors as
- * la_forward; one of a pair (o/g, phi_q/phi_k, S_final/z_final) without the
- * other, or phi_q/phi_k or S_final/z_final without o and g, is
- * LA_ERR_INVALID_ARG.
+ * la_forward; one of o, g without the other, one of phi_q, phi_k without
+ * the other, or them without o and g is LA_ERR_INVALID_ARG.
  */
 LA_EXPORT la_status la_backward(const void *q, const void *k, const void *v, const void *dO,
                       const void *o, const float *g, const void *phi_q, const void *phi_k,
-                      const float *S_final, const float *z_final,
                       void *dq, void *dk, void *dv,
                       int64_t B, int64_t H, int64_t N, int64_t D,
                       la_dtype dt, int causal, la_phi phi,
@@ -192,7 +184,6 @@ LA_EXPORT la_status la_decode_step(float *S, float *z, const void *q, const void
 LA_EXPORT la_status la_backward_noalloc(const void *q, const void *k, const void *v,
                                         const void *dO, const void *o, const float *g,
                                         const void *phi_q, const void *phi_k,
-                                        const float *S_final, const float *z_final,
                                         void *dq, void *dk, void *dv,
                                         int64_t B, int64_t H, int64_t N, int64_t D,
                                         la_dtype dt, int causal, la_phi phi,

@@ -74,11 +74,11 @@ def load_library(path: str | None = None):
         lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci,
                                    ci, vp, sz, vp]
         lib.la_forward.restype = ci
-        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64,
-                                    i64, i64, ci, ci, ci, vp, sz, vp]
+        lib.la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                    i64, ci, ci, ci, vp, sz, vp]
         lib.la_backward.restype = ci
-        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
-                                            i64, i64, i64, i64, ci, ci, ci, vp]
+        lib.la_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64,
+                                            i64, i64, ci, ci, ci, vp]
         lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
@@ -209,19 +209,11 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     return (o, S, z) if return_state else o
 
 
-def _check_saved(name, q, o, g, phi_q=None, phi_k=None, S=None, z=None):
+def _check_saved(name, q, o, g, phi_q=None, phi_k=None):
     if (o is None) != (g is None):
         raise ValueError(f"{name}: pass both o and g (saved forward statistics) or neither")
     if (phi_q is None) != (phi_k is None) or (phi_q is not None and o is None):
         raise ValueError(f"{name}: phi_q and phi_k go together, and only with o and g")
-    if (S is None) != (z is None) or (S is not None and o is None):
-        raise ValueError(f"{name}: S and z (final state) go together, and only with o and g")
-    if S is not None:
-        B, H, _, D = q.shape
-        for nm, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
-            if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
-                    or t.device != q.device:
-                raise ValueError(f"{name}: {nm} must be contiguous float32 {shape} on q's device")
     if phi_q is not None:
         _check_qkv(name, q, phi_q, phi_k)
     if o is not None:
@@ -232,16 +224,13 @@ def _check_saved(name, q, o, g, phi_q=None, phi_k=None, S=None, z=None):
 
 
 def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, dv=None,
-                workspace=None, stream=None, o=None, g=None, phi_q=None, phi_k=None, S=None,
-                z=None):
+                workspace=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
     """dq, dk, dv of sum(dO * O) for O = la_forward(q, k, v, causal, phi).
 
     ``o``, ``g``: the forward's output and denominators (la_forward(..., g=g));
     when given, the backward does not recompute them.  ``phi_q``, ``phi_k``:
     the forward's feature maps (la_forward(..., phi_out=(phi_q, phi_k))),
     only with ``o`` and ``g``; when given, phi is not evaluated again.
-    ``S``, ``z``: the forward's final state (la_forward(..., return_state=True)),
-    only with ``o`` and ``g``; the single-pass causal backward starts from it.
     """
     lib = load_library()
     _check_qkv("la_backward", q, k, v, dO)
@@ -252,10 +241,10 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
     dk = torch.empty_like(q) if dk is None else dk
     dv = torch.empty_like(q) if dv is None else dv
     _check_qkv("la_backward", q, dq, dk, dv)
-    _check_saved("la_backward", q, o, g, phi_q, phi_k, S, z)
+    _check_saved("la_backward", q, o, g, phi_q, phi_k)
     ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
     st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(phi_q),
-                         _ptr(phi_k), _ptr(S), _ptr(z), _ptr(dq), _ptr(dk), _ptr(dv),
+                         _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv),
                          B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
                          ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
@@ -263,8 +252,7 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
 
 
 def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None,
-                        dv=None, stream=None, o=None, g=None, phi_q=None, phi_k=None, S=None,
-                        z=None):
+                        dv=None, stream=None, o=None, g=None, phi_q=None, phi_k=None):
     """la_backward on the library's static device scratch (no workspace).
 
     For callers that cannot allocate device memory during the call; see
@@ -281,10 +269,9 @@ def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, d
         raise ValueError("la_backward_noalloc: pass dq, dk and dv (it allocates nothing)")
     B, H, N, D = q.shape
     _check_qkv("la_backward_noalloc", q, dq, dk, dv)
-    _check_saved("la_backward_noalloc", q, o, g, phi_q, phi_k, S, z)
+    _check_saved("la_backward_noalloc", q, o, g, phi_q, phi_k)
     st = lib.la_backward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g),
-                                 _ptr(phi_q), _ptr(phi_k), _ptr(S), _ptr(z), _ptr(dq), _ptr(dk),
-                                 _ptr(dv), B, H, N,
+                                 _ptr(phi_q), _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N,
                                  D, DTYPE[q.dtype], int(bool(causal)),
                                  _phi(phi), _stream_handle(stream))
     _check("la_backward_noalloc", st)
@@ -336,15 +323,11 @@ def la_profile_collect() -> dict:
 
 
 def backward_reads_phi(dtype, D: int) -> bool:
-    """Whether saving phi(q), phi(k) in the forward pays off for la_backward.
-
-    The single-pass causal backward (bf16, head size 64) evaluates the
-    feature map from q and k itself (it needs phi(k) - c rounded once, from
-    k), and the other paths read the maps in one of two passes at most, so
-    the forward's extra write never pays back: False everywhere.  la_forward
-    still writes them on request (phi_out) and la_backward still accepts
-    them."""
-    return False
+    """True where la_backward reads saved phi(q), phi(k) instead of
+    evaluating the feature map (the bf16 head-size-64 passes: phi(q) in
+    pass 1, both in pass 2); elsewhere they are ignored and asking the
+    forward for them only costs a pass."""
+    return dtype == torch.bfloat16 and D == 64
 
 
 class LinearAttention(torch.autograd.Function):

@@ -16,7 +16,6 @@
 #include <mutex>
 
 #include "la_chunk_bwd.cuh"
-#include "la_bwd_fused64.cuh"
 #include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
@@ -360,11 +359,6 @@ la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o
 // ------------------------------------------------------------ chunked backward
 struct BwdPlan {
     bool fast = false;
-    // causal, head size 64, one segment per head: the single-pass kernel
-    // (with saved o and g); fin_off holds the final state when the caller
-    // does not pass it
-    bool fused = false;
-    size_t fin_off = 0;
     int C = 0;
     SegSplit seg;   // causal: segments of both passes; non-causal: reduce split
     SegSplit qseg;  // non-causal: split of the two gradient passes
@@ -393,11 +387,6 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     p.seg = split(N, p.C, pick_nseg(heads, nch));
     if (causal) {
         p.qseg = p.seg;
-        if (D == 64 && p.seg.nseg == 1) {
-            p.fused = true;
-            p.fin_off = off;
-            off += round_up(size_t(heads) * R * 4, 256);
-        }
         if (p.seg.nseg > 1) {
             p.srec_off = off;
             off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
@@ -437,9 +426,8 @@ la_status launch_bwd_kernel(Kern kern, int smem, const la::BwdParams& prm, int64
 template <int D, int PHI>
 la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO,
                           const void* o_saved, const float* g_saved, const void* pq,
-                          const void* pk, const float* S_fin, const float* z_fin, void* dq,
-                          void* dk, void* dv, int64_t heads, int64_t N, int causal,
-                          const BwdPlan& p, char* ws, cudaStream_t st) {
+                          const void* pk, void* dq, void* dk, void* dv, int64_t heads,
+                          int64_t N, int causal, const BwdPlan& p, char* ws, cudaStream_t st) {
     constexpr int C = D == 64 ? 128 : 64;
     la::BwdParams prm;
     memset(&prm, 0, sizeof(prm));
@@ -493,35 +481,6 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     // the states they start from
     red.center = 1;
 
-    if constexpr (D == 64) {
-        if (causal && p.fused) {
-            // one pass from the last chunk to the first, starting from the
-            // centred final state (sum of (phi(k) - c) v^T and of phi(k) - c)
-            // summed here with the same bf16 features the pass subtracts.
-            // The kernel evaluates phi on q and k itself (saved feature maps
-            // are not used: phi(k) - c is rounded once, from k).
-            (void)S_fin;
-            (void)z_fin;
-            la::BwdParams f = prm;
-            f.seg_len = int(N);
-            f.nseg = 1;
-            float* fin = reinterpret_cast<float*>(ws + p.fin_off);
-            la::ChunkParams r = red;
-            r.seg_len = int(N);
-            r.nseg = 1;
-            r.S_out = fin;
-            r.z_out = fin + D * D;
-            r.stride_S = r.stride_z = R;
-            r.center = 1;
-            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads, st, "chunk_reduce")) != LA_OK)
-                return s;
-            f.S_fin = fin;
-            f.z_fin = fin + D * D;
-            f.stride_S = f.stride_z = R;
-            return launch_bwd_kernel(la::bwd_fused64_kernel<PHI>, la::BwdFused64Cfg::SMEM, f, heads,
-                                     st, "bwd_fused", la::kBwdFused64Threads);
-        }
-    }
     if (causal) {
         la::BwdParams p1 = prm, p2 = prm;
         p1.seg_len = p2.seg_len = p.seg.seg_len;
@@ -535,6 +494,23 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                 return s;
             p1.state_in = srec;
             p1.rec_out = rrec;
+        }
+        if constexpr (D == 64) {
+            // one segment per head: the pipelined passes (pass 1 reads the
+            // forward's phi(q) when given, and k itself: it centres phi(k))
+            if (p.seg.nseg == 1) {
+                la::BwdParams q1 = p1;
+                if (pin) q1.tm_q = tm_pq;
+                if ((s = pin ? launch_bwd_kernel(la::bwd_dq64_kernel<PHI, true>, la::Bwd1x64Cfg::SMEM,
+                                                 q1, heads, st, "bwd_dq", la::kBwd64Threads)
+                             : launch_bwd_kernel(la::bwd_dq64_kernel<PHI, false>, la::Bwd1x64Cfg::SMEM,
+                                                 q1, heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
+                    return s;
+                return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
+                                               with_phi(p2), heads, st, "bwd_dkdv", la::kBwd64Threads)
+                           : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
+                                               p2, heads, st, "bwd_dkdv", la::kBwd64Threads);
+            }
         }
         if ((s = launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, p1,
                                    heads * p.seg.nseg, st, "bwd_dq")) != LA_OK)
@@ -585,15 +561,15 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
 template <int PHI>
 la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO,
                             const void* o_saved, const float* g_saved, const void* pq,
-                            const void* pk, const float* S_fin, const float* z_fin, void* dq,
-                            void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                            const BwdPlan& p, char* ws, cudaStream_t st) {
+                            const void* pk, void* dq, void* dk, void* dv, int64_t heads,
+                            int64_t N, int64_t D, int causal, const BwdPlan& p, char* ws,
+                            cudaStream_t st) {
     if (D == 64)
-        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, S_fin, z_fin, dq,
-                                        dk, dv, heads, N, causal, p, ws, st);
+        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
+                                        N, causal, p, ws, st);
     // the D = 128 kernels evaluate the feature map themselves
-    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, nullptr,
-                                     nullptr, dq, dk, dv, heads, N, causal, p, ws, st);
+    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk, dv,
+                                     heads, N, causal, p, ws, st);
 }
 
 // ------------------------------------------------------------ generic path
@@ -823,7 +799,6 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
 
 la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
                       const void* o, const float* g, const void* phi_q, const void* phi_k,
-                      const float* S_final, const float* z_final,
                       void* dq, void* dk, void* dv, int64_t B,
                       int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
                       void* workspace, size_t workspace_bytes, la_stream_t stream) {
@@ -842,9 +817,6 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     // saved feature maps: both or neither, and only with o and g
     if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
     if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
-    // the forward's final state: both or neither, and only with o and g
-    if ((S_final == nullptr) != (z_final == nullptr) || (S_final && !o)) return LA_ERR_INVALID_ARG;
-    if (S_final && ((s = check_ptr(S_final)) || (s = check_ptr(z_final)))) return s;
     const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -870,12 +842,10 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
             g = g_ws;
         }
         return phi == LA_PHI_ELU1
-                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, S_final,
-                                                 z_final, dq, dk, dv, heads, N, D,
-                                                 causal ? 1 : 0, bp, wsp, st)
-                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, S_final,
-                                                     z_final, dq, dk, dv, heads, N, D,
-                                                     causal ? 1 : 0, bp, wsp, st);
+                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
+                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st)
+                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
+                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st);
     }
     const BwdWorkspace w = plan_bwd(B, H, N);
     char* ws = static_cast<char*>(workspace);
@@ -887,8 +857,7 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
 
 la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
                               const void* o, const float* g, const void* phi_q,
-                              const void* phi_k, const float* S_final, const float* z_final,
-                              void* dq, void* dk, void* dv,
+                              const void* phi_k, void* dq, void* dk, void* dv,
                               int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, int causal,
                               la_phi phi, la_stream_t stream) {
     la_status s;
@@ -904,8 +873,8 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
     if ((s = bind_context()) != LA_OK) return s;
     void* scratch = nullptr;
     if ((s = static_scratch(&scratch)) != LA_OK) return s;
-    return la_backward(q, k, v, dO, o, g, phi_q, phi_k, S_final, z_final, dq, dk, dv, B, H, N, D,
-                       dt, causal, phi, scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
+    return la_backward(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, N, D, dt, causal, phi,
+                       scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 
 la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,

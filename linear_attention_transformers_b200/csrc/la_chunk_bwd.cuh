@@ -53,11 +53,6 @@ struct BwdParams {
     // outputs as plain pointers, for kernels that store rows directly
     __nv_bfloat16* dk_out;
     __nv_bfloat16* dv_out;
-    // single-pass backward: the forward's final state, S [D][D] (row = key
-    // feature) at S_fin + head * stride_S and z [D] at z_fin + head * stride_z
-    const float* S_fin;
-    const float* z_fin;
-    int64_t stride_S, stride_z;
 };
 
 template <int D, int C>

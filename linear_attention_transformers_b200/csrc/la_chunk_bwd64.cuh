@@ -531,7 +531,12 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
 //
 // No product reads A = phi(q): the epilogue forms phi'(q) from the q tile
 // (raw q, or with PIN the forward's phi(q), phi' = dphi_from_phi) and then
-// stages dQ in place over it.  Same warp roles and hand-offs as
+// stages dQ in place over it.  The k tile always comes from k and holds the
+// centred features B = phi(k) - c (phi_center): with elu+1 on small inputs
+// phi(k) is close to 1 and its bf16 rounding would lose most of phi(k) - 1.
+// W' B and dU S^T (S, z summed from the same centred features) then differ
+// from the true dA only along the all-ones vector, which the epilogue
+// restores exactly from <dA_i, phi(q_i)> = 0.  Same warp roles and hand-offs as
 // bwd_dkdv64_kernel; W and dA are double-buffered in TMEM.
 // ======================================================================
 struct Bwd1x64Cfg {
@@ -706,7 +711,9 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             for (int j = 0; j < 4; ++j) ov[j] = valid ? __ldg(orow + j) : make_uint4(0u, 0u, 0u, 0u);
             if (!named_bar_all(3, 256, mbar_wait(&full[s], (c / NS) & 1, abort_flag))) break;
             uint8_t* st = smem + s * Cfg::STAGE;
-            if constexpr (!PIN) phi_tile<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true);
+            // k -> phi(k) - c, the centred key features (from k even when the
+            // forward's phi(k) is available: it is rounded once, from k)
+            phi_tile<PHI, C, D, 256, true>(st + Cfg::TILE, u, nvalid, true);
             uint8_t* dot = st + 3 * Cfg::TILE;
             float dotp = 0.f;
 #pragma unroll
@@ -801,11 +808,38 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 tc_fence_before();
                 mbar_arrive(sx_full);
             }
-            // dQ = (dA + dg z) * phi'(q)
+            // dQ = (T + t 1) * phi'(q): T = dA + dg z formed with the centred
+            // key features, which differ from the true dA only along the
+            // all-ones vector; t restores that component from
+            // <dA_i, a_i> = 0 (t = -(T . a_i) / (1 . a_i)).  a = phi(q): the
+            // forward's map (PIN) or evaluated here from q.
             if (!named_bar_all(2, 128, mbar_wait(&da_full[b], (c >> 1) & 1, abort_flag))) break;
             tc_fence_after();
             const float dg = reinterpret_cast<const float*>(qt + Cfg::OFF_DGF)[irow];
             const float* z = zf + (c & 1) * D;
+            constexpr float kc = phi_center<PHI>();
+            float tcoef = 0.f;
+            if (kc != 0.f) {
+                float dot = 0.f, sa = 0.f;
+#pragma unroll 1
+                for (int f0 = 0; f0 < D; f0 += 16) {
+                    float av[16];
+                    tmem_ld16(tmem + lane_base + Cfg::T_DA + b * D + f0, av);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        float a8[8];
+                        load_chunk8(qt, C, irow, (f0 >> 3) + h, a8);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float a = PIN ? a8[i] : phi_fast<PHI>(a8[i]);
+                            dot = fmaf(fmaf(dg, z[f0 + 8 * h + i], av[8 * h + i]), a, dot);
+                            sa += a;
+                        }
+                    }
+                }
+                tcoef = -kc * dot / sa;
+            }
 #pragma unroll 1
             for (int f0 = 0; f0 < D; f0 += 16) {
                 float av[16];
@@ -824,8 +858,9 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                         q8[i] = PIN ? dphi_from_phi<PHI>(q8[i]) : dphi_fast<PHI>(q8[i]);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        w[i] = pack_bf16(fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) * q8[2 * i],
-                                         fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) * q8[2 * i + 1]);
+                        w[i] = pack_bf16((fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) + tcoef) * q8[2 * i],
+                                         (fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) + tcoef) *
+                                             q8[2 * i + 1]);
                     // this thread's row of q is read before it is overwritten
                     *reinterpret_cast<uint4*>(qt + tile_chunk_off(C, irow, (f0 >> 3) + h)) =
                         make_uint4(w[0], w[1], w[2], w[3]);

@@ -111,6 +111,15 @@ __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// Wait of a whole thread group (a named barrier `id` of `nthreads`) for a
+// phase: only `leader` polls the mbarrier; the others park on the named
+// barrier (parked warps issue nothing, so the group's wait does not take
+// issue slots from the warps that are working), then every thread takes the
+// completed phase with one try_wait (its acquire).  Returns false for every
+// thread when the leader's wait gave up.
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           int id, int nthreads, bool leader);
+
 // ----------------------------------------------------------------- proxies
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -131,6 +140,15 @@ __device__ __forceinline__ bool named_bar_all(int id, int nthreads, bool pred) {
         : "r"(uint32_t(pred)), "r"(id), "r"(nthreads)
         : "memory");
     return r != 0;
+}
+
+__device__ __forceinline__ bool group_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                           int id, int nthreads, bool leader) {
+    bool ok = true;
+    if (leader) ok = mbar_wait(bar, parity, abort);
+    ok = named_bar_all(id, nthreads, ok);
+    if (ok) (void)mbar_try_wait(bar, parity);
+    return ok;
 }
 
 // --------------------------------------------------------------------- TMA

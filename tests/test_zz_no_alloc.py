@@ -33,7 +33,7 @@ def _call_noalloc(lib, q, k, v, dO, dq, dk, dv, causal, phi):
     return lib.la_backward_noalloc(
         ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
         ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(dO.data_ptr()), None, None, None, None,
-        None, None, ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
+        ctypes.c_void_p(dq.data_ptr()), ctypes.c_void_p(dk.data_ptr()),
         ctypes.c_void_p(dv.data_ptr()), B, H, N, D, api.DTYPE[q.dtype], int(causal),
         api.PHI[phi], ctypes.c_void_p(stream))
 
@@ -68,8 +68,8 @@ def test_noalloc_rejects_sizes_beyond_the_limit():
     need = api.la_workspace_size(api.LA_OP_BACKWARD, B, H, N, D, True, torch.bfloat16)
     assert need > (64 << 20)
     fake = ctypes.c_void_p(0x100000)  # never dereferenced: the size check fails first
-    st = lib.la_backward_noalloc(fake, fake, fake, fake, None, None, None, None, None, None,
-                                 fake, fake, fake, B, H, N, D,
+    st = lib.la_backward_noalloc(fake, fake, fake, fake, None, None, None, None, fake, fake, fake,
+                                 B, H, N, D,
                                  api.LA_BF16, 1, 0, None)
     assert st == api.LA_ERR_WORKSPACE
     assert "limit" in api.la_last_error()
