@@ -210,6 +210,19 @@ LA_EXPORT const char *la_last_error(void);
 LA_EXPORT la_status la_get_device_error(la_stream_t stream);
 
 /*
+ * Failure-detection self-test.  Launches one thread block of `nthreads`
+ * threads (1..1024) that all wait, through the same bounded wait the
+ * chunked kernels use, on an mbarrier that nothing arrives at.  The wait
+ * gives up after its limit (1 s), records the failure in the device error
+ * word (so a following la_get_device_error returns LA_ERR_DEVICE_TIMEOUT and
+ * clears it), every other waiting thread leaves as soon as it sees the
+ * block's abort flag, and the kernel returns: a stuck pipeline ends with an
+ * error status instead of hanging the GPU.  Asynchronous on `stream`.
+ * Errors: LA_ERR_INVALID_ARG (nthreads out of range), LA_ERR_CUDA.
+ */
+LA_EXPORT la_status la_selftest_wait_timeout(int nthreads, la_stream_t stream);
+
+/*
  * Launch accounting.  la_launch_count() is the number of kernels this
  * library has launched since it was loaded (counted on the host at launch).
  *

@@ -88,6 +88,8 @@ def load_library(path: str | None = None):
         lib.la_last_error.restype = ctypes.c_char_p
         lib.la_get_device_error.argtypes = [vp]
         lib.la_get_device_error.restype = ci
+        lib.la_selftest_wait_timeout.argtypes = [ci, vp]
+        lib.la_selftest_wait_timeout.restype = ci
         lib.la_version.argtypes = []
         lib.la_version.restype = ci
         lib.la_launch_count.argtypes = []
@@ -301,6 +303,14 @@ def la_decode_step(S, z, q, k, v, phi="elu1", o=None, stream=None):
 def la_get_device_error(stream=None) -> None:
     """Synchronise the stream and raise if a bounded device-side wait gave up."""
     _check("la_get_device_error", load_library().la_get_device_error(_stream_handle(stream)))
+
+
+def la_selftest_wait_timeout(nthreads: int = 256, stream=None) -> None:
+    """Launch the failure-detection self-test (a bounded device wait that is
+    made to run out); la_get_device_error then raises with status
+    LA_ERR_DEVICE_TIMEOUT."""
+    _check("la_selftest_wait_timeout",
+           load_library().la_selftest_wait_timeout(int(nthreads), _stream_handle(stream)))
 
 
 def la_launch_count() -> int:

@@ -932,6 +932,16 @@ int la_profile_collect(la_profile_entry* out, int max_entries) {
     return int(agg.size());
 }
 
+la_status la_selftest_wait_timeout(int nthreads, la_stream_t stream) {
+    if (nthreads < 1 || nthreads > 1024) return LA_ERR_INVALID_ARG;
+    la_status s;
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    la::LaunchScope scope("wait_timeout_selftest", st);
+    la::wait_timeout_selftest_kernel<<<1, unsigned(nthreads), 0, st>>>();
+    return launch_status();
+}
+
 la_status la_get_device_error(la_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return LA_ERR_CUDA;

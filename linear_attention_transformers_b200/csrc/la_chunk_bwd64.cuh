@@ -822,18 +822,17 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             if (kc != 0.f) {
                 float dot = 0.f, sa = 0.f;
 #pragma unroll 1
-                for (int f0 = 0; f0 < D; f0 += 16) {
-                    float av[16];
-                    tmem_ld16(tmem + lane_base + Cfg::T_DA + b * D + f0, av);
-                    tmem_wait_ld();
+                for (int f0 = 0; f0 < D; f0 += 32) {
+                    float tv[32];
+                    tmem_load<32>(tmem + lane_base + Cfg::T_DA + b * D + f0, tv);
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
+                    for (int q = 0; q < 4; ++q) {
                         float a8[8];
-                        load_chunk8(qt, C, irow, (f0 >> 3) + h, a8);
+                        load_chunk8(qt, C, irow, (f0 >> 3) + q, a8);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float a = PIN ? a8[i] : phi_fast<PHI>(a8[i]);
-                            dot = fmaf(fmaf(dg, z[f0 + 8 * h + i], av[8 * h + i]), a, dot);
+                            dot = fmaf(fmaf(dg, z[f0 + 8 * q + i], tv[8 * q + i]), a, dot);
                             sa += a;
                         }
                     }
@@ -841,28 +840,26 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 tcoef = -kc * dot / sa;
             }
 #pragma unroll 1
-            for (int f0 = 0; f0 < D; f0 += 16) {
-                float av[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_DA + b * D + f0, av);
-                tmem_wait_ld();
+            for (int f0 = 0; f0 < D; f0 += 32) {
+                float tv[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_DA + b * D + f0, tv);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int q = 0; q < 4; ++q) {
                     float q8[8];
-                    load_chunk8(qt, C, irow, (f0 >> 3) + h, q8);
-                    const float4 za = reinterpret_cast<const float4*>(z + f0 + 8 * h)[0];
-                    const float4 zb = reinterpret_cast<const float4*>(z + f0 + 8 * h)[1];
-                    const float z8[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+                    load_chunk8(qt, C, irow, (f0 >> 3) + q, q8);
                     uint32_t w[4];
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         q8[i] = PIN ? dphi_from_phi<PHI>(q8[i]) : dphi_fast<PHI>(q8[i]);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        w[i] = pack_bf16((fmaf(dg, z8[2 * i], av[8 * h + 2 * i]) + tcoef) * q8[2 * i],
-                                         (fmaf(dg, z8[2 * i + 1], av[8 * h + 2 * i + 1]) + tcoef) *
+                    for (int i = 0; i < 4; ++i) {
+                        const int f = f0 + 8 * q + 2 * i;
+                        w[i] = pack_bf16((fmaf(dg, z[f], tv[8 * q + 2 * i]) + tcoef) * q8[2 * i],
+                                         (fmaf(dg, z[f + 1], tv[8 * q + 2 * i + 1]) + tcoef) *
                                              q8[2 * i + 1]);
+                    }
                     // this thread's row of q is read before it is overwritten
-                    *reinterpret_cast<uint4*>(qt + tile_chunk_off(C, irow, (f0 >> 3) + h)) =
+                    *reinterpret_cast<uint4*>(qt + tile_chunk_off(C, irow, (f0 >> 3) + q)) =
                         make_uint4(w[0], w[1], w[2], w[3]);
                 }
             }

@@ -339,4 +339,21 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 }
 
 }  // namespace sm100
+
+// One block whose threads wait on an mbarrier that nothing arrives at (the
+// bounded wait of the chunked kernels gives up, records the error and the
+// kernel returns).
+__global__ void wait_timeout_selftest_kernel() {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ volatile int abort_flag;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        abort_flag = 0;
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    (void)sm100::mbar_wait(&bar, 0, &abort_flag);
+    __syncthreads();
+}
+
 }  // namespace la

@@ -80,6 +80,8 @@ def test_rejects_bad_arguments_before_launch(lib):
     assert fwd(lib, pq=FAKE, pk=FAKE + 4) == api.LA_ERR_INVALID_ARG   # misaligned
     assert bwd(lib, pq=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
     assert bwd(lib, o=FAKE, g=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
+    assert lib.la_selftest_wait_timeout(0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_selftest_wait_timeout(2048, None) == api.LA_ERR_INVALID_ARG
     p = FAKE
     assert lib.la_decode_step(p, p, p, p, p, None, 2, 2, 64, 1, 0, None) == api.LA_ERR_INVALID_ARG
     assert lib.la_decode_step(p, p, p, p, p, p, 2, 2, 40, 1, 0, None) == api.LA_ERR_UNSUPPORTED
