@@ -15,6 +15,14 @@ Functions (all arrays [B, H, N, D] contiguous, D innermost):
   backward(q, k, v, dO, causal, phi)       -> dq, dk, dv
   decode_step(S, z, q, k, v, phi)          -> o   (updates S, z in place)
   phi_map(x, phi), dphi_map(x, phi)        -> elementwise feature map / slope
+  forward_gqa / backward_gqa / decode_step_gqa: the same with k, v on fewer
+  (key/value) heads, each shared by a group of query heads
+  forward_decay(q, k, v, gamma, phi)       -> o, S_final, z_final  (causal)
+  quadratic_decay(q, k, v, gamma, phi)     -> o   (small N only)
+  backward_decay(q, k, v, dO, gamma, phi)  -> dq, dk, dv
+  decode_step_decay(S, z, q, k, v, gamma, phi) -> o  (updates S, z in place)
+      the decayed (gated) recurrence S_i = gamma S_{i-1} + b_i v_i^T, z_i =
+      gamma z_{i-1} + b_i with one gamma in [0, 1] per head (gamma [H])
 """
 from __future__ import annotations
 
@@ -60,10 +68,16 @@ def _load():
             lib.oracle_quadratic.argtypes = [P, P, P, P, i64, i64, i64, i64, ci, ci]
             lib.oracle_backward.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, i64, ci, ci]
             lib.oracle_decode_step.argtypes = [P, P, P, P, P, P, i64, i64, i64, ci]
+            lib.oracle_forward_decay.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, i64, ci]
+            lib.oracle_quadratic_decay.argtypes = [P, P, P, P, P, i64, i64, i64, i64, ci]
+            lib.oracle_backward_decay.argtypes = [P, P, P, P, P, P, P, P, i64, i64, i64, i64, ci]
+            lib.oracle_decode_step_decay.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, ci]
             lib.oracle_set_threads.argtypes = [ci]
             lib.oracle_max_threads.restype = ci
             for fn in ("oracle_forward", "oracle_quadratic", "oracle_backward",
-                       "oracle_decode_step", "oracle_set_threads"):
+                       "oracle_decode_step", "oracle_set_threads", "oracle_forward_decay",
+                       "oracle_quadratic_decay", "oracle_backward_decay",
+                       "oracle_decode_step_decay"):
                 getattr(lib, fn).restype = None
             _lib = lib
     return _lib
@@ -134,6 +148,123 @@ def decode_step(S: np.ndarray, z: np.ndarray, q, k, v, phi: int = PHI_ELU1):
     o = np.empty_like(q)
     _load().oracle_decode_step(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
                                B, H, D, int(phi))
+    return o
+
+
+# ------------------------------------------------------- decayed (gated) LA
+def _gamma(gamma, H: int) -> np.ndarray:
+    g = np.ascontiguousarray(np.asarray(gamma, dtype=np.float64).reshape(-1))
+    if g.shape != (H,):
+        raise ValueError(f"gamma must hold one factor per head ({H})")
+    if not ((g >= 0.0) & (g <= 1.0)).all():
+        raise ValueError("gamma must lie in [0, 1]")
+    return g
+
+
+def forward_decay(q, k, v, gamma, phi: int = PHI_ELU1):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, D = _shape4(q)
+    g = _gamma(gamma, H)
+    o = np.empty_like(q)
+    S = np.empty((B, H, D, D))
+    z = np.empty((B, H, D))
+    _load().oracle_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), _ptr(S), _ptr(z),
+                                 B, H, N, D, int(phi))
+    return o, S, z
+
+
+def quadratic_decay(q, k, v, gamma, phi: int = PHI_ELU1):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, D = _shape4(q)
+    g = _gamma(gamma, H)
+    o = np.empty_like(q)
+    _load().oracle_quadratic_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(o), B, H, N, D,
+                                   int(phi))
+    return o
+
+
+def backward_decay(q, k, v, dO, gamma, phi: int = PHI_ELU1):
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, N, D = _shape4(q)
+    g = _gamma(gamma, H)
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    _load().oracle_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(g), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), B, H, N, D, int(phi))
+    return dq, dk, dv
+
+
+def decode_step_decay(S: np.ndarray, z: np.ndarray, q, k, v, gamma, phi: int = PHI_ELU1):
+    """One decayed in-place step on float64 S [B,H,D,D], z [B,H,D]; q,k,v [B,H,D]."""
+    if S.dtype != np.float64 or not S.flags.c_contiguous:
+        raise TypeError("S must be a C-contiguous float64 array (updated in place)")
+    if z.dtype != np.float64 or not z.flags.c_contiguous:
+        raise TypeError("z must be a C-contiguous float64 array (updated in place)")
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, D = q.shape
+    g = _gamma(gamma, H)
+    o = np.empty_like(q)
+    _load().oracle_decode_step_decay(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                     _ptr(o), B, H, D, int(phi))
+    return o
+
+
+# ---------------------------------------------------- grouped key/value heads
+# Grouped-query / multi-query attention ("Attention Optimization", Advanced
+# Techniques: Multi-Query Attention and Grouped-Query Attention): Hkv
+# key/value heads, each shared by G = H / Hkv consecutive query heads.  By
+# definition this is the per-head attention above with every query head h
+# given k, v of head h // G: the functions below expand k, v to one copy
+# per query head and call the functions above; the gradient with respect to
+# a shared k or v is the sum over the query heads that read it.
+
+def expand_kv(x, H: int) -> np.ndarray:
+    """[B, Hkv, ...] -> [B, H, ...], head h taking head h // (H // Hkv)."""
+    x = _f64(x)
+    hkv = x.shape[1]
+    if hkv < 1 or H % hkv:
+        raise ValueError("H must be a multiple of the key/value heads")
+    return np.ascontiguousarray(np.repeat(x, H // hkv, axis=1))
+
+
+def group_sum(x, Hkv: int) -> np.ndarray:
+    """[B, H, ...] -> [B, Hkv, ...]: the sum over each group of H // Hkv heads."""
+    x = np.asarray(x, dtype=np.float64)
+    B, H = x.shape[:2]
+    return x.reshape(B, Hkv, H // Hkv, *x.shape[2:]).sum(axis=2)
+
+
+def forward_gqa(q, k, v, causal: bool, phi: int = PHI_ELU1):
+    """o [B, H, N, D] and the final state per key/value head."""
+    q = _f64(q)
+    H, Hkv = q.shape[1], _f64(k).shape[1]
+    o, S, z = forward(q, expand_kv(k, H), expand_kv(v, H), causal, phi)
+    G = H // Hkv
+    return o, np.ascontiguousarray(S[:, ::G]), np.ascontiguousarray(z[:, ::G])
+
+
+def backward_gqa(q, k, v, dO, causal: bool, phi: int = PHI_ELU1):
+    """dq [B, H, N, D]; dk, dv [B, Hkv, N, D] summed over each group."""
+    q = _f64(q)
+    H, Hkv = q.shape[1], _f64(k).shape[1]
+    dq, dk, dv = backward(q, expand_kv(k, H), expand_kv(v, H), dO, causal, phi)
+    return dq, group_sum(dk, Hkv), group_sum(dv, Hkv)
+
+
+def decode_step_gqa(S: np.ndarray, z: np.ndarray, q, k, v, phi: int = PHI_ELU1):
+    """One step with per-key/value-head state S [B, Hkv, D, D], z [B, Hkv, D]
+    (updated in place); q [B, H, D], k, v [B, Hkv, D]; returns o [B, H, D].
+    The state is updated once per key/value head, then every query head of
+    the group reads it."""
+    q = _f64(q)
+    H, Hkv = q.shape[1], S.shape[1]
+    G = H // Hkv
+    # every query head steps its own copy of its group's state (all copies
+    # of a group receive the same update), then one copy per group is kept
+    S_x = np.ascontiguousarray(np.repeat(S, G, axis=1))
+    z_x = np.ascontiguousarray(np.repeat(z, G, axis=1))
+    o = decode_step(S_x, z_x, q, expand_kv(k, H), expand_kv(v, H), phi)
+    S[...] = S_x[:, ::G]
+    z[...] = z_x[:, ::G]
     return o
 
 

@@ -18,7 +18,14 @@ the wrong feature-map branch) fails at least one of them:
   incrementally) reproduces the causal forward and its final state;
 - S is D x D and z has D entries (section Exercises, ExerciseCore);
 - the backward matches central finite differences of L = sum(dO * O), and
-  satisfies the homogeneity / linearity identities of the definition.
+  satisfies the homogeneity / linearity identities of the definition;
+- grouped key/value heads: finite differences through the shared k, v;
+  multi-query heads are independent single-head attentions; the grouped
+  decode continues the grouped forward;
+- decayed (gated) recurrence: gamma = 1 is the causal oracle; recurrence ==
+  decayed quadratic form; gamma = 0 returns v; identical keys give the
+  bias-corrected exponential moving average of v; the final state is the
+  gamma^(N-1-j)-weighted sum; finite differences; decode continues it.
 """
 import numpy as np
 import pytest
@@ -239,3 +246,180 @@ def test_backward_d1_has_no_query_gradient():
     for causal in (True, False):
         dq, _, _ = oracle.backward(q, k, v, dO, causal, PHI_ELU1)
         assert np.abs(dq).max() < 1e-13
+
+
+# ---------------------------------------------------- grouped key/value heads
+
+def _gqa_inputs(B, H, Hkv, N, D, seed):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((B, H, N, D)) * 0.5
+    k = g.standard_normal((B, Hkv, N, D)) * 0.5
+    v = g.standard_normal((B, Hkv, N, D))
+    dO = g.standard_normal((B, H, N, D))
+    return q, k, v, dO
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_gqa_backward_matches_finite_differences(causal):
+    # the gradient with respect to a k or v shared by a group is checked
+    # against central differences of sum(dO * O) through the grouped forward
+    B, H, Hkv, N, D = 1, 4, 2, 6, 3
+    q, k, v, dO = _gqa_inputs(B, H, Hkv, N, D, 41)
+    dq, dk, dv = oracle.backward_gqa(q, k, v, dO, causal, oracle.PHI_ELU1)
+    loss = lambda q_, k_, v_: float((dO * oracle.forward_gqa(q_, k_, v_, causal)[0]).sum())  # noqa
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": (xp, k, v), "k": (q, xp, v), "v": (q, k, xp)}[name]
+            args_m = {"q": (xm, k, v), "k": (q, xm, v), "v": (q, k, xm)}[name]
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8, err_msg=name)
+
+
+def test_mqa_heads_are_independent_single_head_attentions():
+    # one key/value head shared by all query heads: each query head's output
+    # is the single-head attention of that query against the shared k, v
+    B, H, N, D = 2, 3, 9, 4
+    q, k, v, _ = _gqa_inputs(B, H, 1, N, D, 42)
+    o, S, z = oracle.forward_gqa(q, k, v, True)
+    for h in range(H):
+        o1, S1, z1 = oracle.forward(q[:, h:h + 1], k, v, True)
+        np.testing.assert_allclose(o[:, h:h + 1], o1, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(S, S1, rtol=1e-13)
+    np.testing.assert_allclose(z, z1, rtol=1e-13)
+    # the quadratic form with the shared k, v gives the same outputs
+    qd = oracle.quadratic(q, np.repeat(k, H, 1), np.repeat(v, H, 1), True)
+    np.testing.assert_allclose(o, qd, rtol=1e-12)
+
+
+def test_gqa_decode_continues_the_grouped_forward():
+    B, H, Hkv, T, D = 2, 4, 2, 7, 3
+    q, k, v, _ = _gqa_inputs(B, H, Hkv, T, D, 43)
+    o_ref, S_ref, z_ref = oracle.forward_gqa(q, k, v, True)
+    S = np.zeros((B, Hkv, D, D))
+    z = np.zeros((B, Hkv, D))
+    for t in range(T):
+        o = oracle.decode_step_gqa(S, z, q[:, :, t], k[:, :, t], v[:, :, t])
+        np.testing.assert_allclose(o, o_ref[:, :, t], rtol=1e-12)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12)
+    np.testing.assert_allclose(z, z_ref, rtol=1e-12)
+
+
+# ------------------------------------------------------- decayed (gated) LA
+# S_i = gamma S_{i-1} + b_i v_i^T, z_i = gamma z_{i-1} + b_i, one gamma per
+# head ("Efficient Transformers Survey", Common Confusions, "Watch Out": the
+# gating and decay factors linear-attention models add).
+
+def test_decay_one_is_the_causal_oracle():
+    q, k, v, dO = (rnd((2, 3, 37, 8), 300 + i, 0.5) for i in range(4))
+    g = np.ones(3)
+    o1, S1, z1 = oracle.forward_decay(q, k, v, g)
+    o0, S0, z0 = oracle.forward(q, k, v, True)
+    np.testing.assert_allclose(o1, o0, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(S1, S0, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(z1, z0, rtol=0, atol=1e-12)
+    for a, b in zip(oracle.backward_decay(q, k, v, dO, g), oracle.backward(q, k, v, dO, True)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+def test_decay_recurrence_equals_decayed_quadratic_form(phi):
+    q, k, v = (rnd((2, 4, 41, 8), 310 + i, 0.6) for i in range(3))
+    g = np.array([0.0, 0.35, 0.9, 0.999])
+    o, _, _ = oracle.forward_decay(q, k, v, g, phi)
+    np.testing.assert_allclose(o, oracle.quadratic_decay(q, k, v, g, phi), rtol=1e-11, atol=1e-13)
+
+
+def test_decay_zero_returns_the_values():
+    # gamma = 0 keeps only j = i: o_i = (a_i . b_i) v_i / (a_i . b_i) = v_i.
+    # A normaliser z left undecayed would give a different answer.
+    q, k, v = (rnd((1, 2, 23, 8), 320 + i) for i in range(3))
+    o, S, z = oracle.forward_decay(q, k, v, np.zeros(2))
+    np.testing.assert_allclose(o, v, rtol=1e-13, atol=1e-14)
+    # the final state is the last token's b v^T alone
+    b = oracle.phi_map(k[:, :, -1])
+    np.testing.assert_allclose(S, b[..., :, None] * v[:, :, -1][..., None, :], rtol=1e-13)
+
+
+@pytest.mark.parametrize("gamma", [0.5, 0.9])
+def test_decay_identical_keys_is_the_bias_corrected_moving_average(gamma):
+    # Identical keys: a_i . b_j = c_i for all j <= i, so o_i is the
+    # exponentially weighted average sum_j gamma^(i-j) v_j over the
+    # geometric sum (1 - gamma^(i+1)) / (1 - gamma), the recursion
+    # m_i = gamma m_{i-1} + (1 - gamma) v_i divided by 1 - gamma^(i+1).
+    N, D = 30, 4
+    q = rnd((1, 1, N, D), 330)
+    k = np.broadcast_to(rnd((1, 1, 1, D), 331), (1, 1, N, D)).copy()
+    v = rnd((1, 1, N, D), 332)
+    o, _, _ = oracle.forward_decay(q, k, v, np.array([gamma]))
+    m = np.zeros(D)
+    for i in range(N):
+        m = gamma * m + (1.0 - gamma) * v[0, 0, i]
+        np.testing.assert_allclose(o[0, 0, i], m / (1.0 - gamma ** (i + 1)), rtol=1e-12,
+                                   atol=1e-13)
+
+
+def test_decay_final_state_is_the_weighted_sum():
+    N, D, gamma = 19, 5, 0.8
+    q, k, v = (rnd((1, 1, N, D), 340 + i) for i in range(3))
+    _, S, z = oracle.forward_decay(q, k, v, np.array([gamma]))
+    b = oracle.phi_map(k)[0, 0]
+    w = gamma ** (N - 1 - np.arange(N))
+    np.testing.assert_allclose(S[0, 0], (b * w[:, None]).T @ v[0, 0], rtol=1e-12)
+    np.testing.assert_allclose(z[0, 0], (b * w[:, None]).sum(0), rtol=1e-12)
+
+
+def _fd_decay(q, k, v, dO, gamma, phi, h=1e-6):
+    def loss(q_, k_, v_):
+        return float((oracle.forward_decay(q_, k_, v_, gamma, phi)[0] * dO).sum())
+    grads = []
+    for which in range(3):
+        args = [q, k, v]
+        g = np.zeros_like(args[which])
+        it = np.nditer(g, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += h
+            minus[which][idx] -= h
+            g[idx] = (loss(*plus) - loss(*minus)) / (2 * h)
+        grads.append(g)
+    return grads
+
+
+@pytest.mark.parametrize("phi", [PHI_ELU1, PHI_RELU_EPS])
+def test_decay_backward_matches_finite_differences(phi):
+    q, k, v, dO = (rnd((1, 2, 7, 3), 350 + i, 0.7, away_from_zero=True) for i in range(4))
+    gamma = np.array([0.6, 0.95])
+    got = oracle.backward_decay(q, k, v, dO, gamma, phi)
+    ref = _fd_decay(q, k, v, dO, gamma, phi)
+    for name, a, b in zip("qkv", got, ref):
+        np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-8, err_msg=f"d{name}")
+
+
+def test_decay_decode_continues_the_decayed_forward():
+    B, H, N, D, T0 = 2, 3, 25, 8, 17
+    q, k, v = (rnd((B, H, N, D), 360 + i, 0.5) for i in range(3))
+    gamma = np.array([0.2, 0.7, 1.0])
+    o, S_ref, z_ref = oracle.forward_decay(q, k, v, gamma)
+    _, S, z = oracle.forward_decay(q[:, :, :T0], k[:, :, :T0], v[:, :, :T0], gamma)
+    for t in range(T0, N):
+        o_t = oracle.decode_step_decay(S, z, q[:, :, t], k[:, :, t], v[:, :, t], gamma)
+        np.testing.assert_allclose(o_t, o[:, :, t], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-12)
+    np.testing.assert_allclose(z, z_ref, rtol=1e-12)
+
+
+def test_decay_rejects_out_of_range_factors():
+    q = rnd((1, 2, 3, 4), 370)
+    with pytest.raises(ValueError):
+        oracle.forward_decay(q, q, q, np.array([0.5, 1.5]))
+    with pytest.raises(ValueError):
+        oracle.forward_decay(q, q, q, np.array([0.5]))
