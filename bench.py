@@ -29,7 +29,8 @@ The printed JSON line also carries:
                 reads and writes;
   graded        the other full-size workloads, each with its own clocks: the
                 long-context causal forward (B1 H32 N131072 D128), 1024
-                decode steps (B256 H32 D128, fp32 state in place) and the
+                decode steps (B256 H32 D128, fp32 state in place), the same
+                with grouped-query attention (8 key/value heads) and the
                 1.4B-parameter LM layer shape forward + backward (B4 H16
                 N4096 D128) with both feature maps;
   e2e           the headline metric with every step's inputs copied from
@@ -464,15 +465,20 @@ def graded_forward(api, w, dev, stream, world, peaks, steps=10, warmup=3):
     return out
 
 
-def graded_decode(api, dev, stream, world, peaks, reps=3, warmup=2):
+def graded_decode(api, dev, stream, world, peaks, reps=3, warmup=2, grouped=False):
     """`steps` recurrent decode steps at batch B (fp32 state in place), each
     step one la_decode_step over every (b, h); timed over whole runs of all
-    steps."""
-    cfg = inputs.DECODE
+    steps.  grouped: Hkv key/value heads, each state shared by H/Hkv query
+    heads."""
+    cfg = inputs.DECODE_GQA if grouped else inputs.DECODE
     B, H, D, steps = cfg["B"], cfg["H"], cfg["D"], cfg["steps"]
-    q, k, v = inputs.make_decode_inputs(B, H, D, steps, cfg["seed"], device=dev)
-    S = torch.zeros(B, H, D, D, device=dev)
-    z = torch.zeros(B, H, D, device=dev)
+    Hkv = cfg.get("Hkv", H)
+    if grouped:
+        q, k, v = inputs.make_decode_gqa_inputs(B, H, Hkv, D, steps, cfg["seed"], device=dev)
+    else:
+        q, k, v = inputs.make_decode_inputs(B, H, D, steps, cfg["seed"], device=dev)
+    S = torch.zeros(B, Hkv, D, D, device=dev)
+    z = torch.zeros(B, Hkv, D, device=dev)
     outs = torch.empty(steps, B, H, D, dtype=q.dtype, device=dev)
 
     def run():
@@ -486,11 +492,12 @@ def graded_decode(api, dev, stream, world, peaks, reps=3, warmup=2):
     ms, clocks = timed_region(run, reps, stream, dev, world, dev.index or 0)
     api.la_get_device_error(stream)
     s_step = ms / reps / steps / 1e3
-    # per head and step: S and z read and written in float32, q, k, v read
-    # and o written in bf16
-    bytes_step = B * H * (2 * 4 * (D * D + D) + 4 * D * 2)
-    flops_step = B * H * 4 * D * D
-    out = {"workload": f"decode_b{B}h{H}d{D}_x{steps}_bf16", "us_per_step": s_step * 1e6,
+    # per key/value head and step: S and z read and written in float32, k, v
+    # read in bf16; per query head q read and o written in bf16
+    bytes_step = B * Hkv * (2 * 4 * (D * D + D) + 2 * D * 2) + B * H * 2 * D * 2
+    flops_step = B * Hkv * 2 * D * D + B * H * 2 * D * D
+    name = f"decode_b{B}h{H}" + (f"kv{Hkv}" if grouped else "") + f"d{D}_x{steps}_bf16"
+    out = {"workload": name, "us_per_step": s_step * 1e6,
            "steps_per_s": world / s_step, "tokens_per_s": world * B / s_step,
            "step": roofline_of(bytes_step, flops_step, s_step, peaks), "clocks": clocks}
     del q, k, v, S, z, outs
@@ -639,6 +646,7 @@ def run_ours(args, world, rank, local):
             "long_causal_fwd": graded_forward(api, inputs.WORKLOADS[
                 "causal_fwd_b1h32n131072d128_bf16"], dev, stream, world, peaks),
             "decode": graded_decode(api, dev, stream, world, peaks),
+            "decode_gqa": graded_decode(api, dev, stream, world, peaks, grouped=True),
             "lm_layer_relu": graded_train(api, inputs.WORKLOADS[
                 "causal_fwdbwd_b4h16n4096d128_relu_bf16"], dev, stream, world, peaks),
             "lm_layer_elu": graded_train(api, inputs.WORKLOADS[

@@ -189,6 +189,41 @@ LA_EXPORT la_status la_backward_noalloc(const void *q, const void *k, const void
                                         la_dtype dt, int causal, la_phi phi,
                                         la_stream_t stream);
 
+/*
+ * Grouped key/value heads (grouped-query and multi-query attention, "Attention
+ * Optimization", Advanced Techniques: Multi-Query Attention and Grouped-Query
+ * Attention).  The same operations with Hkv key/value heads shared by the H
+ * query heads: Hkv >= 1 divides H, G = H / Hkv, and query head h of batch b
+ * reads k, v head h / G (heads h = 0..G-1 share head 0, and so on).  q, o,
+ * dO, dq, g: [B, H, N, D] (g: [B, H, N]) as before; k, v, dk, dv:
+ * [B, Hkv, N, D]; the state S_out / z_out and the decode state S, z are per
+ * key/value head: [B, Hkv, D, D] and [B, Hkv, D] (the state depends on k, v
+ * only); decode q and o are [B, H, D] and k, v [B, Hkv, D].  dk and dv are
+ * the sums over each group's query heads (formed per query head in the
+ * workspace and added in a fixed order).  The decode step updates each
+ * key/value head's state once and answers the group's G queries from it, so
+ * its state traffic is that of Hkv heads.  Hkv == H is exactly the call
+ * without the suffix.  phi_q/phi_k (in or out) with Hkv < H is
+ * LA_ERR_UNSUPPORTED; Hkv < 1 or H % Hkv != 0 is LA_ERR_INVALID_ARG.
+ */
+LA_EXPORT size_t la_workspace_size_gqa(la_op op, int64_t B, int64_t H, int64_t Hkv, int64_t N,
+                                       int64_t D, int causal, la_dtype dt);
+LA_EXPORT la_status la_forward_gqa(const void *q, const void *k, const void *v, void *o,
+                                   float *S_out, float *z_out, float *g_out,
+                                   void *phi_q_out, void *phi_k_out,
+                                   int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D,
+                                   la_dtype dt, int causal, la_phi phi,
+                                   void *workspace, size_t workspace_bytes, la_stream_t stream);
+LA_EXPORT la_status la_backward_gqa(const void *q, const void *k, const void *v, const void *dO,
+                                    const void *o, const float *g, const void *phi_q,
+                                    const void *phi_k, void *dq, void *dk, void *dv,
+                                    int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D,
+                                    la_dtype dt, int causal, la_phi phi,
+                                    void *workspace, size_t workspace_bytes, la_stream_t stream);
+LA_EXPORT la_status la_decode_step_gqa(float *S, float *z, const void *q, const void *k,
+                                       const void *v, void *o, int64_t B, int64_t H, int64_t Hkv,
+                                       int64_t D, la_dtype dt, la_phi phi, la_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 LA_EXPORT const char *la_status_string(la_status status);
 

@@ -10,7 +10,11 @@ raises ``RuntimeError``.
     la_forward(q, k, v, causal=True, phi="elu1", ...)        -> o [, S, z]
     la_backward(q, k, v, dO, causal=True, phi="elu1", ...)   -> dq, dk, dv
     la_decode_step(S, z, q, k, v, phi="elu1", ...)           -> o   (S, z in place)
-    la_workspace_size(op, B, H, N, D, causal, dtype)         -> bytes
+    la_workspace_size(op, B, H, N, D, causal, dtype, Hkv)    -> bytes
+
+k and v may have fewer heads than q (grouped-query / multi-query attention:
+Hkv key/value heads shared by groups of H / Hkv query heads); the group size
+is read from their shapes.
     la_get_device_error(stream=None)                         -> raises on a device timeout
     LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
 """
@@ -71,6 +75,16 @@ def load_library(path: str | None = None):
         vp, i64, ci, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
         lib.la_workspace_size.argtypes = [ci, i64, i64, i64, i64, ci, ci]
         lib.la_workspace_size.restype = sz
+        lib.la_workspace_size_gqa.argtypes = [ci, i64, i64, i64, i64, i64, ci, ci]
+        lib.la_workspace_size_gqa.restype = sz
+        lib.la_forward_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                       i64, ci, ci, ci, vp, sz, vp]
+        lib.la_forward_gqa.restype = ci
+        lib.la_backward_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64,
+                                        i64, i64, ci, ci, ci, vp, sz, vp]
+        lib.la_backward_gqa.restype = ci
+        lib.la_decode_step_gqa.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, vp]
+        lib.la_decode_step_gqa.restype = ci
         lib.la_forward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci,
                                    ci, vp, sz, vp]
         lib.la_forward.restype = ci
@@ -149,14 +163,28 @@ def _check_qkv(name: str, ref: torch.Tensor, *ts: torch.Tensor) -> None:
 
 
 def la_workspace_size(op: int, B: int, H: int, N: int, D: int, causal: bool,
-                      dtype: torch.dtype) -> int:
-    return int(load_library().la_workspace_size(int(op), B, H, N, D, int(bool(causal)),
-                                                DTYPE[dtype]))
+                      dtype: torch.dtype, Hkv: int | None = None) -> int:
+    return int(load_library().la_workspace_size_gqa(int(op), B, H, H if Hkv is None else Hkv, N,
+                                                    D, int(bool(causal)), DTYPE[dtype]))
 
 
-def _workspace(op, q, causal, workspace):
+def _check_kv(name: str, q: torch.Tensor, k: torch.Tensor, *ts: torch.Tensor) -> int:
+    """k (and v, dk, dv): [B, Hkv, N, D] like q but with Hkv heads dividing
+    q's; returns Hkv."""
+    _check_qkv(name, k, *ts)
+    if q.dim() != k.dim() or q.device != k.device or q.dtype != k.dtype:
+        raise ValueError(f"{name}: q and k need the same device, dtype and rank")
+    if q.dim() >= 3:
+        hq, hk = q.shape[1], k.shape[1]
+        if (q.shape[0], *q.shape[2:]) != (k.shape[0], *k.shape[2:]) or hk < 1 or hq % hk != 0:
+            raise ValueError(f"{name}: k, v must be [B, Hkv, ...] with Hkv dividing q's heads")
+        return int(hk)
+    return 1
+
+
+def _workspace(op, q, causal, workspace, Hkv=None):
     B, H, N, D = q.shape
-    need = la_workspace_size(op, B, H, N, D, causal, q.dtype)
+    need = la_workspace_size(op, B, H, N, D, causal, q.dtype, Hkv)
     if need == 0:
         return None, 0
     if workspace is None:
@@ -177,9 +205,10 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     ``return_state`` does); pass them to la_backward as S, z.
     """
     lib = load_library()
-    _check_qkv("la_forward", q, k, v)
+    _check_qkv("la_forward", q)
     if q.dim() != 4:
         raise ValueError("la_forward: q, k, v must be [B, H, N, D]")
+    Hkv = _check_kv("la_forward", q, k, v)
     B, H, N, D = q.shape
     if o is None:
         o = torch.empty_like(q)
@@ -188,14 +217,14 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     S = z = None
     if state_out is not None:
         S, z = state_out
-        for nm, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+        for nm, t, shape in (("S", S, (B, Hkv, D, D)), ("z", z, (B, Hkv, D))):
             if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
                     or t.device != q.device:
                 raise ValueError(f"la_forward: {nm} must be contiguous float32 {shape} on q's "
                                  "device")
     elif return_state:
-        S = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
-        z = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+        S = torch.empty((B, Hkv, D, D), dtype=torch.float32, device=q.device)
+        z = torch.empty((B, Hkv, D), dtype=torch.float32, device=q.device)
     if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
                           or not g.is_contiguous() or g.device != q.device):
         raise ValueError("la_forward: g must be contiguous float32 [B, H, N] on q's device")
@@ -203,10 +232,11 @@ def la_forward(q, k, v, causal: bool = True, phi="elu1", o=None, return_state=Fa
     if phi_out is not None:
         pq, pk = phi_out
         _check_qkv("la_forward", q, pq, pk)
-    ws, ws_bytes = _workspace(LA_OP_FORWARD, q, causal, workspace)
-    st = lib.la_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g), _ptr(pq),
-                        _ptr(pk), B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi),
-                        _ptr(ws), ws_bytes, _stream_handle(stream))
+    ws, ws_bytes = _workspace(LA_OP_FORWARD, q, causal, workspace, Hkv)
+    st = lib.la_forward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g),
+                            _ptr(pq), _ptr(pk), B, H, Hkv, N, D, DTYPE[q.dtype],
+                            int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
+                            _stream_handle(stream))
     _check("la_forward", st)
     return (o, S, z) if return_state else o
 
@@ -235,20 +265,22 @@ def la_backward(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, dk=None, 
     only with ``o`` and ``g``; when given, phi is not evaluated again.
     """
     lib = load_library()
-    _check_qkv("la_backward", q, k, v, dO)
+    _check_qkv("la_backward", q, dO)
     if q.dim() != 4:
         raise ValueError("la_backward: tensors must be [B, H, N, D]")
+    Hkv = _check_kv("la_backward", q, k, v)
     B, H, N, D = q.shape
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
-    _check_qkv("la_backward", q, dq, dk, dv)
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(k) if dv is None else dv
+    _check_qkv("la_backward", q, dq)
+    _check_qkv("la_backward", k, dk, dv)
     _check_saved("la_backward", q, o, g, phi_q, phi_k)
-    ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace)
-    st = lib.la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(phi_q),
-                         _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv),
-                         B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws),
-                         ws_bytes, _stream_handle(stream))
+    ws, ws_bytes = _workspace(LA_OP_BACKWARD, q, causal, workspace, Hkv)
+    st = lib.la_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(phi_q),
+                             _ptr(phi_k), _ptr(dq), _ptr(dk), _ptr(dv),
+                             B, H, Hkv, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi),
+                             _ptr(ws), ws_bytes, _stream_handle(stream))
     _check("la_backward", st)
     return dq, dk, dv
 
@@ -283,19 +315,20 @@ def la_backward_noalloc(q, k, v, dO, causal: bool = True, phi="elu1", dq=None, d
 def la_decode_step(S, z, q, k, v, phi="elu1", o=None, stream=None):
     """One in-place recurrent step: S, z (float32) updated, o [B, H, D] returned."""
     lib = load_library()
-    _check_qkv("la_decode_step", q, k, v)
+    _check_qkv("la_decode_step", q)
     if q.dim() != 3:
         raise ValueError("la_decode_step: q, k, v must be [B, H, D]")
+    Hkv = _check_kv("la_decode_step", q, k, v)
     B, H, D = q.shape
-    for name, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+    for name, t, shape in (("S", S, (B, Hkv, D, D)), ("z", z, (B, Hkv, D))):
         if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
                 or t.device != q.device:
             raise ValueError(f"la_decode_step: {name} must be contiguous float32 {shape} "
                              "on the device of q")
     if o is None:
         o = torch.empty_like(q)
-    st = lib.la_decode_step(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, D,
-                            DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
+    st = lib.la_decode_step_gqa(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, Hkv,
+                                D, DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
     _check("la_decode_step", st)
     return o
 
@@ -349,7 +382,7 @@ class LinearAttention(torch.autograd.Function):
         B, H, N, _ = q.shape
         g = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
         pq = pk = None
-        if backward_reads_phi(q.dtype, q.shape[-1]):
+        if backward_reads_phi(q.dtype, q.shape[-1]) and k.shape[1] == H:
             pq, pk = torch.empty_like(q), torch.empty_like(k)
         o = la_forward(q, k, v, causal, phi, g=g,
                        phi_out=None if pq is None else (pq, pk))

@@ -56,6 +56,13 @@ la_status check_enums(la_dtype dt, la_phi phi) {
     return LA_OK;
 }
 
+// Key/value heads: at least one, and a divisor of the query heads.
+la_status check_group(int64_t H, int64_t Hkv) {
+    if (H == 0 && Hkv == 0) return LA_OK;  // no heads: nothing to launch
+    if (Hkv < 1 || H < 0 || H % Hkv != 0) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
 la_status check_ptr(const void* p) {
     if (p == nullptr || !aligned16(p)) return LA_ERR_INVALID_ARG;
     return LA_OK;
@@ -86,17 +93,23 @@ la_status launch_status() {
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // ------------------------------------------------------------ workspace plan
-// Backward: g and dg, float32 [B, H, N] each.
+// Backward: g and dg, float32 [B, H, N] each; with grouped key/value heads
+// also float32 dK, dV per query head [B, H, N, D] each.
 struct BwdWorkspace {
-    size_t g_off = 0, dg_off = 0, bytes = 0;
+    size_t g_off = 0, dg_off = 0, part_off = 0, bytes = 0;
 };
 
-BwdWorkspace plan_bwd(int64_t B, int64_t H, int64_t N) {
+BwdWorkspace plan_bwd(int64_t B, int64_t H, int64_t N, int64_t D = 0, int G = 1) {
     BwdWorkspace w;
     const size_t tok = size_t(B) * size_t(H) * size_t(N) * sizeof(float);
     w.g_off = 0;
     w.dg_off = round_up(tok, 256);
     w.bytes = w.dg_off + round_up(tok, 256);
+    if (G > 1) {
+        // float32 dK, dV per query head, summed per key/value group afterwards
+        w.part_off = w.bytes;
+        w.bytes += 2 * round_up(size_t(B) * size_t(H) * size_t(N) * size_t(D) * 4, 256);
+    }
     return w;
 }
 
@@ -253,7 +266,8 @@ la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st
 }
 
 la_status launch_state_kernel(int which, float* rec, float* out, float* S, float* z,
-                              int64_t heads, int nseg, int64_t D, cudaStream_t st) {
+                              int64_t heads, int nseg, int64_t D, cudaStream_t st,
+                              int rec_step = 1) {
     const int R = int(D * D + D);
     const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
     const unsigned grid = unsigned(heads * bph);
@@ -268,7 +282,8 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
         la::state_sum_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, out, nseg, R, bph);
     } else {
         la::LaunchScope scope("state_unpack", st);
-        la::state_unpack_kernel<<<grid, la::kStateThreads, 0, st>>>(out, S, z, int(D), bph);
+        la::state_unpack_kernel<<<grid, la::kStateThreads, 0, st>>>(out, S, z, int(D), bph,
+                                                                     rec_step);
     }
     return launch_status();
 }
@@ -276,15 +291,18 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
 template <int D, int PHI>
 la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, float* S_out,
                           float* z_out, float* g_out, void* pq, void* pk, int64_t heads, int64_t N,
-                          int causal, const FwdPlan& p, char* ws, cudaStream_t st) {
+                          int causal, const FwdPlan& p, char* ws, cudaStream_t st, int G) {
     constexpr int C = D == 64 ? 128 : 64;
+    const int64_t kv_heads = heads / G;
     la::ChunkParams prm;
     memset(&prm, 0, sizeof(prm));
-    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
-        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) || !make_qkv_map(&prm.tm_o, o, heads, N, D, C))
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_k, k, kv_heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, kv_heads, N, D, C) || !make_qkv_map(&prm.tm_o, o, heads, N, D, C))
         return LA_ERR_CUDA;
     prm.N = int(N);
     prm.g_out = g_out;
+    prm.kv_group = G;
     const int64_t R = int64_t(D) * D + D;
     float* rec = reinterpret_cast<float*>(ws + p.rec_off);
     la_status s;
@@ -333,8 +351,9 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
         return s;
     if ((s = launch_state_kernel(1, rec, tot, nullptr, nullptr, heads, p.seg.nseg, D, st)) != LA_OK)
         return s;
+    // the state of each key/value head: the record of its group's first query head
     if ((S_out || z_out) &&
-        (s = launch_state_kernel(2, nullptr, tot, S_out, z_out, heads, 1, D, st)) != LA_OK)
+        (s = launch_state_kernel(2, nullptr, tot, S_out, z_out, kv_heads, 1, D, st, G)) != LA_OK)
         return s;
     prm.seg_len = p.qseg.seg_len;
     prm.nseg = p.qseg.nseg;
@@ -347,12 +366,12 @@ template <int PHI>
 la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o, float* S_out,
                             float* z_out, float* g_out, void* pq, void* pk, int64_t heads,
                             int64_t N, int64_t D, int causal, const FwdPlan& p, char* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, int G) {
     if (D == 64)
         return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal,
-                                        p, ws, st);
+                                        p, ws, st, G);
     return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal, p,
-                                     ws, st);
+                                     ws, st, G);
 }
 
 
@@ -366,10 +385,13 @@ struct BwdPlan {
     // without the forward's o and g, la_backward first runs the forward into
     // o (o_off) and g (g_off) with the forward's own workspace at fwd_off
     size_t o_off = 0, fwd_off = 0;
+    // grouped key/value heads (G > 1): dK, dV per query head, summed per group
+    size_t part_off = 0;
     size_t bytes = 0;
 };
 
-BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
+BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt,
+                      int G = 1) {
     BwdPlan p;
     if (!fast_path(dt, D) || N == 0 || B * H == 0) return p;
     p.fast = true;
@@ -409,6 +431,10 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     off += round_up(size_t(heads) * size_t(N) * size_t(D) * 2, 256);
     p.fwd_off = off;
     off += round_up(plan_fwd(B, H, N, D, causal, dt).bytes, 256);
+    if (G > 1) {
+        p.part_off = off;
+        off += 2 * round_up(size_t(heads) * size_t(N) * size_t(D) * 4, 256);
+    }
     p.bytes = off;
     return p;
 }
@@ -427,16 +453,27 @@ template <int D, int PHI>
 la_status run_bwd_chunked(const void* q, const void* k, const void* v, const void* dO,
                           const void* o_saved, const float* g_saved, const void* pq,
                           const void* pk, void* dq, void* dk, void* dv, int64_t heads,
-                          int64_t N, int causal, const BwdPlan& p, char* ws, cudaStream_t st) {
+                          int64_t N, int causal, const BwdPlan& p, char* ws, cudaStream_t st,
+                          int G, float* dk_part, float* dv_part) {
     constexpr int C = D == 64 ? 128 : 64;
+    const int64_t kv_heads = heads / G;
+    // with grouped key/value heads the kernels store float32 partials per
+    // query head; the bf16 dK, dV maps (never stored through then) span the
+    // caller's key/value heads
+    const int64_t dkv_heads = G > 1 ? kv_heads : heads;
     la::BwdParams prm;
     memset(&prm, 0, sizeof(prm));
-    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
-        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) ||
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_k, k, kv_heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, kv_heads, N, D, C) ||
         !make_qkv_map(&prm.tm_do, dO, heads, N, D, C) ||
         !make_qkv_map(&prm.tm_dq, dq, heads, N, D, C) ||
-        !make_qkv_map(&prm.tm_dk, dk, heads, N, D, C) || !make_qkv_map(&prm.tm_dv, dv, heads, N, D, C))
+        !make_qkv_map(&prm.tm_dk, dk, dkv_heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dv, dv, dkv_heads, N, D, C))
         return LA_ERR_CUDA;
+    prm.kv_group = G;
+    prm.dk_part = G > 1 ? dk_part : nullptr;
+    prm.dv_part = G > 1 ? dv_part : nullptr;
     prm.N = int(N);
     // the forward's o and g: the caller's, or computed into the workspace
     // by la_backward before this runs
@@ -444,8 +481,6 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     prm.gbuf = const_cast<float*>(g_saved);
     prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
     prm.o_in = static_cast<const __nv_bfloat16*>(o_saved);
-    prm.dk_out = static_cast<__nv_bfloat16*>(dk);
-    prm.dv_out = static_cast<__nv_bfloat16*>(dv);
     // the D = 64 pipelined passes read phi(q), phi(k) through the q, k maps
     // when the forward's feature maps are given
     const bool pin = pq != nullptr;
@@ -480,6 +515,7 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     // the dQ products use the centred key features phi(k) - c, and so do
     // the states they start from
     red.center = 1;
+    red.kv_group = G;
 
     if (causal) {
         la::BwdParams p1 = prm, p2 = prm;
@@ -558,25 +594,47 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                              heads * p.qseg.nseg, st, "bwd_dkdv");
 }
 
+// dK or dV of each key/value head <- the sum of its group's float32
+// per-query-head partials (n = N*D elements per head, a multiple of 4).
+template <typename T>
+la_status launch_group_sum(const float* part, void* out, int64_t kv_heads, int64_t n, int G,
+                           cudaStream_t st) {
+    const int64_t total4 = kv_heads * n / 4;
+    const int64_t blocks = std::min<int64_t>((total4 + 255) / 256, int64_t(num_sms()) * 16);
+    la::LaunchScope scope("group_sum", st);
+    la::group_sum_kernel<T><<<unsigned(std::max<int64_t>(blocks, 1)), 256, 0, st>>>(
+        part, static_cast<T*>(out), n, G, total4);
+    return launch_status();
+}
+
 template <int PHI>
 la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const void* dO,
                             const void* o_saved, const float* g_saved, const void* pq,
                             const void* pk, void* dq, void* dk, void* dv, int64_t heads,
                             int64_t N, int64_t D, int causal, const BwdPlan& p, char* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, int G) {
+    // with grouped key/value heads each query head's dK, dV go to the
+    // workspace first, in float32, and are summed per group after the passes
+    const size_t part_bytes = round_up(size_t(heads) * size_t(N) * size_t(D) * 4, 256);
+    float* dk_p = G > 1 ? reinterpret_cast<float*>(ws + p.part_off) : nullptr;
+    float* dv_p = G > 1 ? reinterpret_cast<float*>(ws + p.part_off + part_bytes) : nullptr;
+    la_status s;
     if (D == 64)
-        return run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
-                                        N, causal, p, ws, st);
-    // the D = 128 kernels evaluate the feature map themselves
-    return run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk, dv,
-                                     heads, N, causal, p, ws, st);
+        s = run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
+                                     N, causal, p, ws, st, G, dk_p, dv_p);
+    else  // the D = 128 kernels evaluate the feature map themselves
+        s = run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk,
+                                      dv, heads, N, causal, p, ws, st, G, dk_p, dv_p);
+    if (s != LA_OK || G == 1) return s;
+    if ((s = launch_group_sum<__nv_bfloat16>(dk_p, dk, heads / G, N * D, G, st)) != LA_OK) return s;
+    return launch_group_sum<__nv_bfloat16>(dv_p, dv, heads / G, N * D, G, st);
 }
 
 // ------------------------------------------------------------ generic path
 template <typename T, int PHI>
 la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
                           float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
-                          int causal, cudaStream_t st) {
+                          int causal, cudaStream_t st, int G) {
     auto kern = la::fwd_generic_kernel<T, PHI>;
     const size_t smem = la::generic_smem_bytes(int(D));
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -585,16 +643,36 @@ la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, 
     la::LaunchScope scope("fwd_generic", st);
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-        static_cast<T*>(o), S_out, z_out, g_out, int(N), int(D), causal);
+        static_cast<T*>(o), S_out, z_out, g_out, int(N), int(D), causal, G);
     return launch_status();
 }
 
 template <typename T, int PHI>
 la_status run_bwd_generic(const void* q, const void* k, const void* v, const void* dO, void* dq,
                           void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                          float* gbuf, float* dgbuf, cudaStream_t st) {
-    auto kern = la::bwd_generic_kernel<T, PHI>;
+                          float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part) {
+    // with grouped key/value heads each query head's dK, dV go to `part`
+    // first, in float32, and are summed per group afterwards
+    const size_t part_bytes = round_up(size_t(heads) * size_t(N) * size_t(D) * 4, 256);
+    float* dk_p = reinterpret_cast<float*>(part);
+    float* dv_p = reinterpret_cast<float*>(part + part_bytes);
     const size_t smem = la::generic_smem_bytes(int(D)) + size_t(D) * sizeof(float);
+    if (G > 1) {
+        auto kern = la::bwd_generic_kernel<T, PHI, float>;
+        if (cudaError_t e = cudaFuncSetAttribute(
+                kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)))
+            return cuda_fail("cudaFuncSetAttribute", e);
+        la::LaunchScope scope("bwd_generic", st);
+        kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
+            static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
+            static_cast<const T*>(dO), static_cast<T*>(dq), dk_p, dv_p, gbuf, dgbuf, int(N),
+            int(D), causal, G);
+        la_status s = launch_status();
+        if (s != LA_OK) return s;
+        if ((s = launch_group_sum<T>(dk_p, dk, heads / G, N * D, G, st)) != LA_OK) return s;
+        return launch_group_sum<T>(dv_p, dv, heads / G, N * D, G, st);
+    }
+    auto kern = la::bwd_generic_kernel<T, PHI>;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              int(smem)))
         return cuda_fail("cudaFuncSetAttribute", e);
@@ -602,17 +680,30 @@ la_status run_bwd_generic(const void* q, const void* k, const void* v, const voi
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(dO), static_cast<T*>(dq), static_cast<T*>(dk), static_cast<T*>(dv),
-        gbuf, dgbuf, int(N), int(D), causal);
+        gbuf, dgbuf, int(N), int(D), causal, 1);
     return launch_status();
 }
 
 template <typename T, int PHI>
 la_status run_decode(float* S, float* z, const void* q, const void* k, const void* v, void* o,
-                     int64_t heads, int64_t D, cudaStream_t st) {
+                     int64_t heads, int64_t D, cudaStream_t st, int G) {
     const T* qq = static_cast<const T*>(q);
     const T* kk = static_cast<const T*>(k);
     const T* vv = static_cast<const T*>(v);
     T* oo = static_cast<T*>(o);
+    if (G > 1) {
+        // one block per key/value head: its state read once for the group
+        const unsigned grid = unsigned(heads / G);
+        la::LaunchScope scope("decode_step_gqa", st);
+        switch (D) {
+            case 16: la::decode_step_gqa_kernel<T, PHI, 16><<<grid, 32, 0, st>>>(S, z, qq, kk, vv, oo, G); break;
+            case 32: la::decode_step_gqa_kernel<T, PHI, 32><<<grid, 64, 0, st>>>(S, z, qq, kk, vv, oo, G); break;
+            case 64: la::decode_step_gqa_kernel<T, PHI, 64><<<grid, 128, 0, st>>>(S, z, qq, kk, vv, oo, G); break;
+            case 128: la::decode_step_gqa_kernel<T, PHI, 128><<<grid, 256, 0, st>>>(S, z, qq, kk, vv, oo, G); break;
+            default: return LA_ERR_UNSUPPORTED;
+        }
+        return launch_status();
+    }
     const unsigned grid = unsigned(heads);
     la::LaunchScope scope("decode_step", st);
     switch (D) {
@@ -640,8 +731,9 @@ template <typename T, int PHI>
 struct FwdOp {
     static la_status run(const void* q, const void* k, const void* v, void* o, float* S_out,
                          float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
-                         int causal, cudaStream_t st) {
-        return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, D, causal, st);
+                         int causal, cudaStream_t st, int G) {
+        return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, D, causal, st,
+                                       G);
     }
 };
 
@@ -649,9 +741,9 @@ template <typename T, int PHI>
 struct BwdOp {
     static la_status run(const void* q, const void* k, const void* v, const void* dO, void* dq,
                          void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                         float* gbuf, float* dgbuf, cudaStream_t st) {
+                         float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part) {
         return run_bwd_generic<T, PHI>(q, k, v, dO, dq, dk, dv, heads, N, D, causal, gbuf, dgbuf,
-                                       st);
+                                       st, G, part);
     }
 };
 
@@ -671,8 +763,8 @@ struct PhiMapOp {
 template <typename T, int PHI>
 struct DecodeOp {
     static la_status run(float* S, float* z, const void* q, const void* k, const void* v,
-                         void* o, int64_t heads, int64_t D, cudaStream_t st) {
-        return run_decode<T, PHI>(S, z, q, k, v, o, heads, D, st);
+                         void* o, int64_t heads, int64_t D, cudaStream_t st, int G) {
+        return run_decode<T, PHI>(S, z, q, k, v, o, heads, D, st, G);
     }
 };
 
@@ -733,40 +825,50 @@ const char* la_status_string(la_status s) {
     return "unknown status";
 }
 
-size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
-                         la_dtype dt) {
-    if (check_sizes(B, H, N, D) != LA_OK) return 0;
+size_t la_workspace_size_gqa(la_op op, int64_t B, int64_t H, int64_t Hkv, int64_t N, int64_t D,
+                             int causal, la_dtype dt) {
+    if (check_sizes(B, H, N, D) != LA_OK || check_group(H, Hkv) != LA_OK) return 0;
     if (dt != LA_F32 && dt != LA_BF16) return 0;
     if (B == 0 || H == 0 || N == 0) return 0;
+    const int G = int(H / Hkv);
     if (op == LA_OP_FORWARD) return plan_fwd(B, H, N, D, causal, dt).bytes;
     if (op == LA_OP_BACKWARD) {
-        const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal, dt);
-        return bp.fast ? bp.bytes : plan_bwd(B, H, N).bytes;
+        const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal, dt, G);
+        return bp.fast ? bp.bytes : plan_bwd(B, H, N, D, G).bytes;
     }
     return 0;
 }
 
-la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
-                     float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
-                     int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
-                     void* workspace, size_t workspace_bytes, la_stream_t stream) {
+size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                         la_dtype dt) {
+    return la_workspace_size_gqa(op, B, H, H, N, D, causal, dt);
+}
+
+la_status la_forward_gqa(const void* q, const void* k, const void* v, void* o, float* S_out,
+                         float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
+                         int64_t H, int64_t Hkv, int64_t N, int64_t D, la_dtype dt, int causal,
+                         la_phi phi, void* workspace, size_t workspace_bytes, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if ((s = check_group(H, Hkv)) != LA_OK) return s;
     if ((S_out && !aligned16(S_out)) || (z_out && !aligned16(z_out)) ||
         (g_out && !aligned16(g_out)))
         return LA_ERR_INVALID_ARG;
-    // feature-map outputs: both or neither
+    // feature-map outputs: both or neither, and one key map per query head
     if ((phi_q_out == nullptr) != (phi_k_out == nullptr)) return LA_ERR_INVALID_ARG;
+    if (phi_q_out && Hkv != H) return LA_ERR_UNSUPPORTED;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t heads = B * H;
+    const int G = int(H == 0 ? 1 : H / Hkv);
     if (heads == 0) return LA_OK;
     if (N == 0) {
         // nothing to attend over; a requested final state is all zero
-        if (S_out && cudaMemsetAsync(S_out, 0, size_t(heads * D * D) * 4, st) != cudaSuccess)
+        const int64_t kv_heads = B * Hkv;
+        if (S_out && cudaMemsetAsync(S_out, 0, size_t(kv_heads * D * D) * 4, st) != cudaSuccess)
             return LA_ERR_CUDA;
-        if (z_out && cudaMemsetAsync(z_out, 0, size_t(heads * D) * 4, st) != cudaSuccess)
+        if (z_out && cudaMemsetAsync(z_out, 0, size_t(kv_heads * D) * 4, st) != cudaSuccess)
             return LA_ERR_CUDA;
         return LA_OK;
     }
@@ -786,28 +888,38 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
         void* pk = phi_fused ? phi_k_out : nullptr;
         s = phi == LA_PHI_ELU1
                 ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N,
-                                              D, causal ? 1 : 0, plan, ws, st)
+                                              D, causal ? 1 : 0, plan, ws, st, G)
                 : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads,
-                                                  N, D, causal ? 1 : 0, plan, ws, st);
+                                                  N, D, causal ? 1 : 0, plan, ws, st, G);
     } else {
         s = dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D,
-                            causal ? 1 : 0, st);
+                            causal ? 1 : 0, st, G);
     }
     if (s != LA_OK || phi_q_out == nullptr || phi_fused) return s;
     return dispatch<PhiMapOp>(dt, phi, q, k, phi_q_out, phi_k_out, heads * N * D, st);
 }
 
-la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
-                      const void* o, const float* g, const void* phi_q, const void* phi_k,
-                      void* dq, void* dk, void* dv, int64_t B,
-                      int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
-                      void* workspace, size_t workspace_bytes, la_stream_t stream) {
+la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
+                     float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
+                     int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                     void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    return la_forward_gqa(q, k, v, o, S_out, z_out, g_out, phi_q_out, phi_k_out, B, H, H, N, D,
+                          dt, causal, phi, workspace, workspace_bytes, stream);
+}
+
+la_status la_backward_gqa(const void* q, const void* k, const void* v, const void* dO,
+                          const void* o, const float* g, const void* phi_q, const void* phi_k,
+                          void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv,
+                          int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                          void* workspace, size_t workspace_bytes, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if ((s = check_group(H, Hkv)) != LA_OK) return s;
     if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
     const int64_t heads = B * H;
     if (heads == 0 || N == 0) return LA_OK;
+    const int G = int(H / Hkv);
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
         (s = check_ptr(dq)) || (s = check_ptr(dk)) || (s = check_ptr(dv)))
         return s;
@@ -816,11 +928,12 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
     if (o && ((s = check_ptr(o)) || (s = check_ptr(g)))) return s;
     // saved feature maps: both or neither, and only with o and g
     if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
+    if (phi_q && G != 1) return LA_ERR_UNSUPPORTED;
     if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
-    const size_t need = la_workspace_size(LA_OP_BACKWARD, B, H, N, D, causal, dt);
+    const size_t need = la_workspace_size_gqa(LA_OP_BACKWARD, B, H, Hkv, N, D, causal, dt);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt);
+    const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt, G);
     if ((s = bind_context()) != LA_OK) return s;
     if (bp.fast) {
         char* wsp = static_cast<char*>(workspace);
@@ -833,26 +946,35 @@ la_status la_backward(const void* q, const void* k, const void* v, const void* d
             s = phi == LA_PHI_ELU1
                     ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o_ws, nullptr, nullptr, g_ws, nullptr,
                                                   nullptr, heads, N, D, causal ? 1 : 0, fp,
-                                                  wsp + bp.fwd_off, st)
+                                                  wsp + bp.fwd_off, st, G)
                     : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o_ws, nullptr, nullptr, g_ws,
                                                       nullptr, nullptr, heads, N, D,
-                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st);
+                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st, G);
             if (s != LA_OK) return s;
             o = o_ws;
             g = g_ws;
         }
         return phi == LA_PHI_ELU1
                    ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st)
+                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st, G)
                    : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st);
+                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st, G);
     }
-    const BwdWorkspace w = plan_bwd(B, H, N);
+    const BwdWorkspace w = plan_bwd(B, H, N, D, G);
     char* ws = static_cast<char*>(workspace);
     float* gbuf = reinterpret_cast<float*>(ws + w.g_off);
     float* dgbuf = reinterpret_cast<float*>(ws + w.dg_off);
     return dispatch<BwdOp>(dt, phi, q, k, v, dO, dq, dk, dv, heads, N, D, causal ? 1 : 0, gbuf,
-                           dgbuf, st);
+                           dgbuf, st, G, ws + w.part_off);
+}
+
+la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
+                      const void* o, const float* g, const void* phi_q, const void* phi_k,
+                      void* dq, void* dk, void* dv, int64_t B,
+                      int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                      void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    return la_backward_gqa(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, H, N, D, dt, causal,
+                           phi, workspace, workspace_bytes, stream);
 }
 
 la_status la_backward_noalloc(const void* q, const void* k, const void* v, const void* dO,
@@ -877,19 +999,26 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
                        scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 
-la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
-                         void* o, int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
-                         la_stream_t stream) {
+la_status la_decode_step_gqa(float* S, float* z, const void* q, const void* k, const void* v,
+                             void* o, int64_t B, int64_t H, int64_t Hkv, int64_t D, la_dtype dt,
+                             la_phi phi, la_stream_t stream) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, 1, D)) != LA_OK) return s;
+    if ((s = check_group(H, Hkv)) != LA_OK) return s;
     const int64_t heads = B * H;
     if (heads == 0) return LA_OK;
     if ((s = check_ptr(S)) || (s = check_ptr(z)) || (s = check_ptr(q)) || (s = check_ptr(k)) ||
         (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return dispatch<DecodeOp>(dt, phi, S, z, q, k, v, o, heads, D, st);
+    return dispatch<DecodeOp>(dt, phi, S, z, q, k, v, o, heads, D, st, int(H / Hkv));
+}
+
+la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
+                         void* o, int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
+                         la_stream_t stream) {
+    return la_decode_step_gqa(S, z, q, k, v, o, B, H, H, D, dt, phi, stream);
 }
 
 uint64_t la_launch_count(void) { return la::profiler().launches.load(); }

@@ -50,9 +50,13 @@ struct BwdParams {
     // pass 1 with saved forward statistics: the forward's output O (bf16
     // [heads][N][D]); gbuf then holds the forward's denominators g.
     const __nv_bfloat16* o_in;
-    // outputs as plain pointers, for kernels that store rows directly
-    __nv_bfloat16* dk_out;
-    __nv_bfloat16* dv_out;
+    // query heads per key/value head: k and v are read at head / kv_group
+    int kv_group;
+    // kv_group > 1: dK, dV of each query head in float32 ([heads][N][D]),
+    // stored by the epilogue threads in place of the bf16 tiles, so that the
+    // caller's sum over each group rounds to bf16 once
+    float* dk_part;
+    float* dv_part;
 };
 
 template <int D, int C>
@@ -157,6 +161,13 @@ __device__ __forceinline__ void store_row16_bf16(uint8_t* tile, int rows, int ro
                    pack_bf16(v[14], v[15]));
 }
 
+// Write 16 fp32 values to global memory (16-byte aligned destination).
+__device__ __forceinline__ void store16_f32(float* dst, const float* v) {
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
 // Read 8 bf16 values (columns 8q..8q+7) of row `row` of a row tile.
 __device__ __forceinline__ void load_chunk8(const uint8_t* tile, int rows, int row, int q,
                                             float* out) {
@@ -256,9 +267,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
                     tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
-                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row, head);
+                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row,
+                                kv_head_of(head, prm.kv_group));
                     tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
-                                head);
+                                kv_head_of(head, prm.kv_group));
                     tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
                                 head);
                 }
@@ -839,9 +851,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
                     tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
-                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row, head);
+                    tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row,
+                                kv_head_of(head, prm.kv_group));
                     tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
-                                head);
+                                kv_head_of(head, prm.kv_group));
                     tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
                                 head);
                 }
@@ -1076,14 +1089,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                         dk16[k] = (db16[k] + rf[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
                         dk16[8 + k] = (db16[8 + k] + rf[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
                     }
-                    store_row16_bf16(stgv, C, jrow, c0, dv16);
-                    store_row16_bf16(stgk, C, jrow, c0, dk16);
+                    if (prm.dk_part) {
+                        if (row0 + jrow < prm.N) {
+                            const size_t off = (size_t(head) * prm.N + row0 + jrow) * D + c0;
+                            store16_f32(prm.dv_part + off, dv16);
+                            store16_f32(prm.dk_part + off, dk16);
+                        }
+                    } else {
+                        store_row16_bf16(stgv, C, jrow, c0, dv16);
+                        store_row16_bf16(stgk, C, jrow, c0, dk16);
+                    }
                 }
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every rf read done
             mbar_arrive(&empty[s]);
-            if (e == 0) {
+            if (e == 0 && !prm.dk_part) {
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
                     tma_store_3d(&prm.tm_dv, stgv + a * C * 128, a * 64, row0, head);

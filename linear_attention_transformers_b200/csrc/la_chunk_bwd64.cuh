@@ -218,8 +218,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
                 const int row = row_of(t);
                 tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
-                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, head);
-                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, head);
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head_of(head, prm.kv_group));
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head_of(head, prm.kv_group));
                 tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
                 issued = t + 1;
             }
@@ -470,9 +470,17 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                     dk16[i] = (db16[i] + r16[i]) * dphi_from_phi<PHI>(b8a[i]);
                     dk16[8 + i] = (db16[8 + i] + r16[8 + i]) * dphi_from_phi<PHI>(b8b[i]);
                 }
-                // this thread's row of B is read before it is overwritten
-                store_row16_bf16(vt, C, jrow, c0, dv16);
-                store_row16_bf16(kt, C, jrow, c0, dk16);
+                if (prm.dk_part) {
+                    if (row_of(t) + jrow < prm.N) {
+                        const size_t off = (size_t(head) * prm.N + row_of(t) + jrow) * D + c0;
+                        store16_f32(prm.dv_part + off, dv16);
+                        store16_f32(prm.dk_part + off, dk16);
+                    }
+                } else {
+                    // this thread's row of B is read before it is overwritten
+                    store_row16_bf16(vt, C, jrow, c0, dv16);
+                    store_row16_bf16(kt, C, jrow, c0, dk16);
+                }
             }
             tc_fence_before();
             mbar_arrive(d_free);
@@ -504,10 +512,12 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const int row0 = row_of(t);
                 uint8_t* st = smem + s * Cfg::STAGE;
                 if (!mbar_wait(&staged[s], (t / NS) & 1, abort_flag)) break;
-                tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
-                tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
-                bulk_commit();
-                bulk_wait_read0();
+                if (!prm.dk_part) {  // float32 partials were stored by the epilogue
+                    tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
+                    tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
+                    bulk_commit();
+                    bulk_wait_read0();
+                }
                 mbar_arrive(&empty[s]);
             }
             bulk_wait0();
@@ -634,8 +644,8 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
                 const int row = row_of(c);
                 tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
-                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, head);
-                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, head);
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head_of(head, prm.kv_group));
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head_of(head, prm.kv_group));
                 tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
                 issued = c + 1;
             }

@@ -70,7 +70,12 @@ struct ChunkParams {
     // REDUCE: sum phi(k) - phi_center (the centred state the backward's dQ
     // products use) instead of phi(k)
     int center;
+    // query heads per key/value head (grouped-query attention; 1 = one each):
+    // query head `head` reads k, v head head / kv_group, and the final state
+    // (per key/value head) is written by the group's first query head
+    int kv_group;
 };
+
 
 // Shared-memory and TMEM plan of the kernel below (head size 128, 64-token
 // chunks).  Stage tiles live in 19 slots of one [C][64] bf16 atom (8 KB).
@@ -204,10 +209,11 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                         tma_load_3d(smem + (Cfg::q_slot(s) + a) * Cfg::ATOM, &prm.tm_q, &full[s],
                                     a * 64, row, head);
                     if (kKV) {
+                        const int kvh = kv_head_of(head, prm.kv_group);
                         tma_load_3d(smem + (Cfg::k_slot(s) + a) * Cfg::ATOM, &prm.tm_k, &full[s],
-                                    a * 64, row, head);
+                                    a * 64, row, kvh);
                         tma_load_3d(smem + Cfg::v_slot(s, a) * Cfg::ATOM, &prm.tm_v, &full[s],
-                                    a * 64, row, head);
+                                    a * 64, row, kvh);
                     }
                 }
                 issued = c + 1;
@@ -457,7 +463,9 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     if (!named_bar_all(2, 128, mbar_wait(s_done, c & 1, abort_flag))) break;
                     tc_fence_after();
                     const bool last = c == nchunks - 1;
-                    const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr;
+                    const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
+                                             writes_kv_state(head, prm.kv_group);
+                    const size_t sidx = size_t(kv_head_of(head, prm.kv_group));
                     if (!last || write_final) {
 #pragma unroll 1
                         for (int v0 = 0; v0 < D; v0 += 16) {
@@ -467,8 +475,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                                 store_row_bf16<16>(sx, D, frow, v0, sv);
                                 if (write_final)
                                     for (int t = 0; t < 16; ++t)
-                                        prm.S_out[size_t(head) * prm.stride_S + size_t(frow) * D +
-                                                  v0 + t] = sv[t];
+                                        prm.S_out[sidx * prm.stride_S + size_t(frow) * D + v0 + t] =
+                                            sv[t];
                             }
                         }
                         float zv[16];
@@ -476,7 +484,7 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                         if (frow >= 0) {
                             put_z(zv[0]);
                             if (write_final && prm.z_out)
-                                prm.z_out[size_t(head) * prm.stride_z + frow] = zv[0];
+                                prm.z_out[sidx * prm.stride_z + frow] = zv[0];
                         }
                     }
                     fence_proxy_async_smem();

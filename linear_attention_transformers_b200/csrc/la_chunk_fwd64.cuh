@@ -142,8 +142,9 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 const int row = tok0 + c * C;
                 if (kQ) tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
                 if (kKV) {
-                    tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, head);
-                    tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, head);
+                    const int kvh = kv_head_of(head, prm.kv_group);
+                    tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kvh);
+                    tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kvh);
                 }
                 issued = c + 1;
             }
@@ -395,7 +396,9 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                     if (!named_bar_all(2, 128, mbar_wait(s_done, c & 1, abort_flag))) break;
                     tc_fence_after();
                     const bool last = c == nchunks - 1;
-                    const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr;
+                    const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
+                                             writes_kv_state(head, prm.kv_group);
+                    const size_t sidx = size_t(kv_head_of(head, prm.kv_group));
                     if (!last || write_final) {
 #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {
@@ -403,9 +406,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                             tmem_load<32>(tmem + lane_base + Cfg::T_S + 32 * half, col);
                             put_state(row, half, col);
                             if (write_final)
-                                write_state(prm.S_out + size_t(head) * prm.stride_S,
-                                            prm.z_out ? prm.z_out + size_t(head) * prm.stride_z
-                                                      : nullptr,
+                                write_state(prm.S_out + sidx * prm.stride_S,
+                                            prm.z_out ? prm.z_out + sidx * prm.stride_z : nullptr,
                                             half, col);
                         }
                     }

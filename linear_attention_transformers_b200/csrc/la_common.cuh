@@ -56,6 +56,20 @@ __device__ __forceinline__ float dphi_fast(float x) {
     return x > 0.f ? 1.f : 0.f;
 }
 
+// ------------------------------------------------ grouped key/value heads
+// With grouped-query attention G = kv_group query heads share one key/value
+// head ("Attention Optimization", Advanced Techniques: Multi-Query and
+// Grouped-Query Attention): flattened query head `head` = b*H + h reads
+// key/value head b*Hkv + h/G = head / G, and the state (a function of k and
+// v only) belongs to that key/value head.
+__device__ __forceinline__ int kv_head_of(int head, int kv_group) {
+    return head / (kv_group > 0 ? kv_group : 1);
+}
+// The group's first query head writes the key/value head's state.
+__device__ __forceinline__ bool writes_kv_state(int head, int kv_group) {
+    return kv_group <= 1 || head % kv_group == 0;
+}
+
 // ---------------------------------------------------------------- elements
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -94,4 +94,104 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
     }
 }
 
+// The same step with G query heads per key/value head (grouped-query or
+// multi-query attention, "Attention Optimization", Advanced Techniques): one
+// block per key/value head updates its state once, S += phi(k) v^T and
+// z += phi(k), then answers the group's G queries from the updated state,
+// o_h = S^T phi(q_h) / (phi(q_h) . z).  The state, the step's dominant
+// traffic, is read and written once per group instead of once per query
+// head.  Queries are taken QB at a time with the updated state slice kept
+// in registers.
+template <typename T, int PHI, int D>
+__global__ void __launch_bounds__(2 * D)
+decode_step_gqa_kernel(float* __restrict__ S, float* __restrict__ z,
+                       const T* __restrict__ q, const T* __restrict__ k,
+                       const T* __restrict__ v, T* __restrict__ o, int G) {
+    constexpr int CG = D / 4;
+    constexpr int RG = 8;
+    constexpr int RPT = D / RG;
+    constexpr int NT = 2 * D;
+    constexpr int QB = 4;
+    constexpr bool kExact = sizeof(T) == sizeof(float);
+    static_assert(CG * RG == NT, "thread layout");
+    __shared__ float a_s[QB][D], b_s[D], z_s[D];
+    __shared__ float4 v_s4[CG];
+    __shared__ float4 part[QB][RG][CG];
+    __shared__ float den_s[QB];
+
+    const size_t hk = blockIdx.x;  // key/value head
+    const int tid = threadIdx.x;
+    const int cg = tid % CG, rg = tid / CG;
+    float4* Sh = reinterpret_cast<float4*>(S + hk * D * D);
+
+    float4 s[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) s[r] = __ldcs(Sh + (rg + RG * r) * CG + cg);
+    if (tid < D) {
+        const float xk = to_f32(k[hk * D + tid]);
+        const float bf = kExact ? phi_exact<PHI>(xk) : phi_fast<PHI>(xk);
+        b_s[tid] = bf;
+        reinterpret_cast<float*>(v_s4)[tid] = to_f32(v[hk * D + tid]);
+        const float zn = z[hk * D + tid] + bf;
+        z[hk * D + tid] = zn;
+        z_s[tid] = zn;
+    }
+    __syncthreads();
+    const float4 vv = v_s4[cg];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int f = rg + RG * r;
+        const float bf = b_s[f];
+        float4 x = s[r];
+        x.x = fmaf(bf, vv.x, x.x);
+        x.y = fmaf(bf, vv.y, x.y);
+        x.z = fmaf(bf, vv.z, x.z);
+        x.w = fmaf(bf, vv.w, x.w);
+        __stcs(Sh + f * CG + cg, x);
+        s[r] = x;
+    }
+    for (int g0 = 0; g0 < G; g0 += QB) {
+        const int nq = min(QB, G - g0);
+        __syncthreads();  // a_s, part, den_s of the previous batch are consumed
+        if (tid < D) {
+            for (int i = 0; i < nq; ++i) {
+                const float xq = to_f32(q[(hk * G + g0 + i) * D + tid]);
+                a_s[i][tid] = kExact ? phi_exact<PHI>(xq) : phi_fast<PHI>(xq);
+            }
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // denominators phi(q) . z, one warp, fixed order
+            for (int i = 0; i < nq; ++i) {
+                float d = 0.f;
+                for (int f = tid; f < D; f += 32) d = fmaf(a_s[i][f], z_s[f], d);
+                d = warp_sum(d);
+                if (tid == 0) den_s[i] = d;
+            }
+        }
+        for (int i = 0; i < nq; ++i) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
+                const float af = a_s[i][rg + RG * r];
+                acc.x = fmaf(af, s[r].x, acc.x);
+                acc.y = fmaf(af, s[r].y, acc.y);
+                acc.z = fmaf(af, s[r].z, acc.z);
+                acc.w = fmaf(af, s[r].w, acc.w);
+            }
+            part[i][rg][cg] = acc;
+        }
+        __syncthreads();
+        if (tid < D) {
+            const float* pf = reinterpret_cast<const float*>(&part[0][0][0]);
+            for (int i = 0; i < nq; ++i) {
+                float num = 0.f;
+#pragma unroll
+                for (int gr = 0; gr < RG; ++gr) num += pf[(i * RG + gr) * D + tid];
+                o[(hk * G + g0 + i) * D + tid] = from_f32<T>(num / den_s[i]);
+            }
+        }
+    }
+}
+
 }  // namespace la

@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kGenericThreads)
 fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, T* __restrict__ o,
                    float* __restrict__ S_out, float* __restrict__ z_out,
-                   float* __restrict__ g_out, int N, int D, int causal) {
+                   float* __restrict__ g_out, int N, int D, int causal, int G) {
     extern __shared__ float sm[];
     float* S = sm;
     float* z = S + D * D;
@@ -43,9 +43,10 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
     const int tid = threadIdx.x, nt = blockDim.x;
     const size_t head = blockIdx.x;
     const size_t base = head * size_t(N) * D;
+    const size_t kvh = head / size_t(G);  // key/value head of this query head
     const T* qh = q + base;
-    const T* kh = k + base;
-    const T* vh = v + base;
+    const T* kh = k + kvh * size_t(N) * D;
+    const T* vh = v + kvh * size_t(N) * D;
     T* oh = o + base;
 
     for (int t = tid; t < D * D; t += nt) S[t] = 0.f;
@@ -90,10 +91,14 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
         }
         __syncthreads();
     }
-    if (S_out)
-        for (int t = tid; t < D * D; t += nt) S_out[head * D * D + t] = S[t];
-    if (z_out)
-        for (int t = tid; t < D; t += nt) z_out[head * D + t] = z[t];
+    // the state belongs to the key/value head: its group's first query head
+    // writes it
+    if (head % G == 0) {
+        if (S_out)
+            for (int t = tid; t < D * D; t += nt) S_out[kvh * D * D + t] = S[t];
+        if (z_out)
+            for (int t = tid; t < D; t += nt) z_out[kvh * D + t] = z[t];
+    }
 }
 
 // Backward of sum(dO * O).  Sweep 1 (token order) rebuilds the forward
@@ -101,13 +106,15 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
 // dQ_i = (S_i du_i + z_i dg_i) * phi'(q_i), saving g and dg.  Sweep 2
 // (reverse order) accumulates R = sum a_i du_i^T and r = sum a_i dg_i over
 // the queries that see key j: dK_j = (R v_j + r) * phi'(k_j), dV_j = R^T b_j.
-template <typename T, int PHI>
+// TO: the dK, dV element type (float for per-query-head partials that the
+// caller sums over a key/value group before rounding).
+template <typename T, int PHI, typename TO = T>
 __global__ void __launch_bounds__(kGenericThreads)
 bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ dO,
-                   T* __restrict__ dq, T* __restrict__ dk, T* __restrict__ dv,
+                   T* __restrict__ dq, TO* __restrict__ dk, TO* __restrict__ dv,
                    float* __restrict__ gbuf, float* __restrict__ dgbuf,
-                   int N, int D, int causal) {
+                   int N, int D, int causal, int G) {
     extern __shared__ float sm[];
     float* M = sm;            // S in sweep 1, R in sweep 2
     float* zr = M + D * D;    // z in sweep 1, r in sweep 2
@@ -119,8 +126,11 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
     const int tid = threadIdx.x, nt = blockDim.x;
     const size_t head = blockIdx.x;
     const size_t base = head * size_t(N) * D;
-    const T *qh = q + base, *kh = k + base, *vh = v + base, *gh = dO + base;
-    T *dqh = dq + base, *dkh = dk + base, *dvh = dv + base;
+    // k, v of the query head's group; dK, dV are written per query head
+    const size_t kvbase = (head / size_t(G)) * size_t(N) * D;
+    const T *qh = q + base, *kh = k + kvbase, *vh = v + kvbase, *gh = dO + base;
+    T* dqh = dq + base;
+    TO *dkh = dk + base, *dvh = dv + base;
     float* gb = gbuf + head * size_t(N);
     float* dgb = dgbuf + head * size_t(N);
 
@@ -220,12 +230,12 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
         for (int f = tid; f < D; f += nt) {
             float db = zr[f];
             for (int e = 0; e < D; ++e) db = fmaf(M[f * D + e], vv[e], db);
-            dkh[row + f] = from_f32<T>(db * dphi_exact<PHI>(to_f32(kh[row + f])));
+            dkh[row + f] = from_f32<TO>(db * dphi_exact<PHI>(to_f32(kh[row + f])));
         }
         for (int e = tid; e < D; e += nt) {
             float acc = 0.f;
             for (int f = 0; f < D; ++f) acc = fmaf(M[f * D + e], b[f], acc);
-            dvh[row + e] = from_f32<T>(acc);
+            dvh[row + e] = from_f32<TO>(acc);
         }
         __syncthreads();
     }

@@ -87,19 +87,51 @@ state_sum_kernel(const float* __restrict__ rec, float* __restrict__ out, int nse
     out[h * size_t(R) + e] = run;
 }
 
-// Split records into the caller's S [h][D][D] and z [h][D] arrays.
+// Split records into the caller's S [h][D][D] and z [h][D] arrays; output
+// h takes record h * rec_step (with grouped key/value heads the records are
+// per query head and every group's first one holds the key/value head's
+// state).
 __global__ void __launch_bounds__(kStateThreads)
 state_unpack_kernel(const float* __restrict__ rec, float* __restrict__ S, float* __restrict__ z,
-                    int D, int blocks_per_head) {
+                    int D, int blocks_per_head, int rec_step) {
     const size_t h = blockIdx.x / blocks_per_head;
     const int R = D * D + D;
     const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
     if (e >= R) return;
-    const float x = rec[h * size_t(R) + e];
+    const float x = rec[h * size_t(rec_step) * size_t(R) + e];
     if (e < D * D) {
         if (S) S[h * size_t(D) * D + e] = x;
     } else if (z) {
         z[h * size_t(D) + (e - D * D)] = x;
+    }
+}
+
+// out[h][e] <- sum_{g < G} part[h*G + g][e] for the n elements of each head:
+// the float32 per-query-head dK, dV of a key/value head's group, added in a
+// fixed order and rounded once to the output type.  Four elements per
+// thread (n is a multiple of 4: n = N*D with D a multiple of 16).
+template <typename T>
+__global__ void __launch_bounds__(256)
+group_sum_kernel(const float* __restrict__ part, T* __restrict__ out, int64_t n, int G,
+                 int64_t total4) {
+    const int64_t stride = int64_t(gridDim.x) * blockDim.x;
+    const int64_t n4 = n / 4;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < total4; i += stride) {
+        const int64_t h = i / n4, e = i % n4;
+        const float4* src = reinterpret_cast<const float4*>(part) + h * G * n4 + e;
+        float4 acc = __ldcs(src);
+        for (int g = 1; g < G; ++g) {
+            const float4 x = __ldcs(src + g * n4);
+            acc.x += x.x;
+            acc.y += x.y;
+            acc.z += x.z;
+            acc.w += x.w;
+        }
+        T* dst = out + 4 * i;
+        dst[0] = from_f32<T>(acc.x);
+        dst[1] = from_f32<T>(acc.y);
+        dst[2] = from_f32<T>(acc.z);
+        dst[3] = from_f32<T>(acc.w);
     }
 }
 

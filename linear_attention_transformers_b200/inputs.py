@@ -75,6 +75,10 @@ WORKLOADS = {
 
 # recurrent decode: batch 256, 32 heads of 128, fp32 state updated in place
 DECODE = dict(B=256, H=32, D=128, steps=1024, seed=4, dtype=torch.bfloat16, phi=PHI_ELU1)
+# the same decode with grouped-query attention: 8 key/value heads, each
+# shared by 4 query heads (the state is 4x smaller)
+DECODE_GQA = dict(B=256, H=32, Hkv=8, D=128, steps=1024, seed=5, dtype=torch.bfloat16,
+                  phi=PHI_ELU1)
 
 
 def _gen(device, seed: int) -> torch.Generator:
@@ -102,6 +106,35 @@ def make_tensors(B, H, N, D, dtype, seed, device="cpu", scaled=True, with_grad_o
         if name != "dO" and scale != 1.0:
             t.mul_(scale)
         out.append(t.to(dtype).contiguous())
+    return tuple(out)
+
+
+def make_gqa_tensors(B, H, Hkv, N, D, dtype, seed, device="cpu", with_grad_out=False):
+    """Grouped key/value heads: q [B, H, N, D], k, v [B, Hkv, N, D] (and dO
+    [B, H, N, D]), drawn in that order from one generator seeded with
+    ``seed``; q, k, v scaled by 1/sqrt(D), dO not; then cast to ``dtype``."""
+    g = _gen(device, seed)
+    scale = 1.0 / math.sqrt(D)
+    shapes = [(B, H, N, D), (B, Hkv, N, D), (B, Hkv, N, D)] + (
+        [(B, H, N, D)] if with_grad_out else [])
+    out = []
+    for i, shape in enumerate(shapes):
+        t = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        if i < 3:
+            t.mul_(scale)
+        out.append(t.to(dtype).contiguous())
+    return tuple(out)
+
+
+def make_decode_gqa_inputs(B, H, Hkv, D, steps, seed, dtype=torch.bfloat16, device="cpu"):
+    """q [steps, B, H, D] and k, v [steps, B, Hkv, D] for grouped decode
+    steps (generator seed + 1000, scaled by 1/sqrt(D))."""
+    g = _gen(device, seed + 1000)
+    scale = 1.0 / math.sqrt(D)
+    out = []
+    for heads in (H, Hkv, Hkv):
+        t = torch.randn((steps, B, heads, D), generator=g, device=device, dtype=torch.float32)
+        out.append(t.mul_(scale).to(dtype).contiguous())
     return tuple(out)
 
 

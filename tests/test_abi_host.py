@@ -80,6 +80,20 @@ def test_rejects_bad_arguments_before_launch(lib):
     assert fwd(lib, pq=FAKE, pk=FAKE + 4) == api.LA_ERR_INVALID_ARG   # misaligned
     assert bwd(lib, pq=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
     assert bwd(lib, o=FAKE, g=FAKE, pk=FAKE, ws=FAKE, ws_bytes=need) == api.LA_ERR_INVALID_ARG
+    # grouped key/value heads: Hkv must divide H
+    p = FAKE
+    assert lib.la_forward_gqa(p, p, p, p, None, None, None, None, None, 1, 4, 3, 8, 64, 1, 1, 0,
+                              None, 0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_forward_gqa(p, p, p, p, None, None, None, None, None, 1, 4, 0, 8, 64, 1, 1, 0,
+                              None, 0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step_gqa(p, p, p, p, p, p, 2, 4, 3, 64, 1, 0, None) == \
+        api.LA_ERR_INVALID_ARG
+    # feature maps are per query head: not with shared key/value heads
+    assert lib.la_forward_gqa(p, p, p, p, None, None, None, p, p, 1, 4, 2, 8, 64, 1, 1, 0,
+                              None, 0, None) == api.LA_ERR_UNSUPPORTED
+    assert lib.la_workspace_size_gqa(api.LA_OP_BACKWARD, 1, 4, 3, 8, 64, 1, 1) == 0
+    assert lib.la_workspace_size_gqa(api.LA_OP_BACKWARD, 2, 4, 2, 1000, 64, 1, 1) > \
+        lib.la_workspace_size(api.LA_OP_BACKWARD, 2, 4, 1000, 64, 1, 1)
     assert lib.la_selftest_wait_timeout(0, None) == api.LA_ERR_INVALID_ARG
     assert lib.la_selftest_wait_timeout(2048, None) == api.LA_ERR_INVALID_ARG
     p = FAKE
