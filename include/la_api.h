@@ -224,6 +224,43 @@ LA_EXPORT la_status la_decode_step_gqa(float *S, float *z, const void *q, const 
                                        const void *v, void *o, int64_t B, int64_t H, int64_t Hkv,
                                        int64_t D, la_dtype dt, la_phi phi, la_stream_t stream);
 
+/*
+ * Decayed (gated) linear attention, causal.  The pages name gating and decay
+ * factors as the architectural change linear-attention models need to match
+ * softmax quality ("Efficient Transformers Survey", Common Confusions, "Watch
+ * Out: Linear attention is not a drop-in replacement") without fixing a form;
+ * these calls take the plainest one, a constant factor per head:
+ *     S_i = gamma_h S_{i-1} + phi(k_i) v_i^T,   z_i = gamma_h z_{i-1} + phi(k_i),
+ *     o_i = S_i^T phi(q_i) / (phi(q_i) . z_i),
+ * i.e. o_i averages v_j (j <= i) with weights gamma^(i-j) phi(q_i).phi(k_j).
+ * gamma: HOST array of H float32 factors in [0, 1] (read during the call,
+ * not kept), the same for every batch entry; gamma = 1 is the undecayed
+ * causal call, gamma = 0 returns o = v.  NULL, a factor outside [0, 1] or
+ * NaN is LA_ERR_INVALID_ARG; H > 256 is LA_ERR_UNSUPPORTED.  Layouts,
+ * g_out, S_out / z_out (the decayed state after token N), the saved o and g
+ * of la_backward_decay and the decode state are as in la_forward,
+ * la_backward and la_decode_step; the decode step scales (S, z) by gamma
+ * before adding the token.  There is no gradient with respect to gamma (a
+ * fixed per-head constant).  la_workspace_size_decay covers every gamma.
+ */
+LA_EXPORT size_t la_workspace_size_decay(la_op op, int64_t B, int64_t H, int64_t N, int64_t D,
+                                         la_dtype dt);
+LA_EXPORT la_status la_forward_decay(const void *q, const void *k, const void *v, void *o,
+                                     float *S_out, float *z_out, float *g_out,
+                                     const float *gamma, int64_t B, int64_t H, int64_t N,
+                                     int64_t D, la_dtype dt, la_phi phi,
+                                     void *workspace, size_t workspace_bytes, la_stream_t stream);
+LA_EXPORT la_status la_backward_decay(const void *q, const void *k, const void *v,
+                                      const void *dO, const void *o, const float *g,
+                                      void *dq, void *dk, void *dv, const float *gamma,
+                                      int64_t B, int64_t H, int64_t N, int64_t D,
+                                      la_dtype dt, la_phi phi,
+                                      void *workspace, size_t workspace_bytes, la_stream_t stream);
+LA_EXPORT la_status la_decode_step_decay(float *S, float *z, const void *q, const void *k,
+                                         const void *v, void *o, const float *gamma,
+                                         int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
+                                         la_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 LA_EXPORT const char *la_status_string(la_status status);
 

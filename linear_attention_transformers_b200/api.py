@@ -11,12 +11,16 @@ raises ``RuntimeError``.
     la_backward(q, k, v, dO, causal=True, phi="elu1", ...)   -> dq, dk, dv
     la_decode_step(S, z, q, k, v, phi="elu1", ...)           -> o   (S, z in place)
     la_workspace_size(op, B, H, N, D, causal, dtype, Hkv)    -> bytes
+    la_forward_decay(q, k, v, gamma, phi="elu1", ...)        -> o [, S, z]  (causal)
+    la_backward_decay(q, k, v, dO, gamma, phi="elu1", ...)   -> dq, dk, dv
+    la_decode_step_decay(S, z, q, k, v, gamma, ...)          -> o   (S, z in place)
+    la_get_device_error(stream=None)                         -> raises on a device timeout
+    LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
 
 k and v may have fewer heads than q (grouped-query / multi-query attention:
 Hkv key/value heads shared by groups of H / Hkv query heads); the group size
-is read from their shapes.
-    la_get_device_error(stream=None)                         -> raises on a device timeout
-    LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
+is read from their shapes.  The *_decay calls take one decay factor per head
+(gamma, H host values in [0, 1]): S_i = gamma S_{i-1} + phi(k_i) v_i^T.
 """
 from __future__ import annotations
 
@@ -96,6 +100,17 @@ def load_library(path: str | None = None):
         lib.la_backward_noalloc.restype = ci
         lib.la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step.restype = ci
+        fp = ctypes.POINTER(ctypes.c_float)
+        lib.la_workspace_size_decay.argtypes = [ci, i64, i64, i64, i64, ci]
+        lib.la_workspace_size_decay.restype = sz
+        lib.la_forward_decay.argtypes = [vp, vp, vp, vp, vp, vp, vp, fp, i64, i64, i64, i64, ci,
+                                         ci, vp, sz, vp]
+        lib.la_forward_decay.restype = ci
+        lib.la_backward_decay.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, fp, i64, i64, i64,
+                                          i64, ci, ci, vp, sz, vp]
+        lib.la_backward_decay.restype = ci
+        lib.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, vp, fp, i64, i64, i64, ci, ci, vp]
+        lib.la_decode_step_decay.restype = ci
         lib.la_status_string.argtypes = [ci]
         lib.la_status_string.restype = ctypes.c_char_p
         lib.la_last_error.argtypes = []
@@ -330,6 +345,107 @@ def la_decode_step(S, z, q, k, v, phi="elu1", o=None, stream=None):
     st = lib.la_decode_step_gqa(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o), B, H, Hkv,
                                 D, DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
     _check("la_decode_step", st)
+    return o
+
+
+# ------------------------------------------------------- decayed (gated) LA
+def _gamma(gamma, H: int):
+    """Per-head decay factors (host sequence, numpy array or tensor) as a
+    ctypes float array of length H; the library checks the range."""
+    if isinstance(gamma, torch.Tensor):
+        gamma = gamma.detach().to("cpu", torch.float32).reshape(-1).tolist()
+    vals = [float(x) for x in gamma]
+    if len(vals) != H:
+        raise ValueError(f"gamma must hold one factor per head ({H}), got {len(vals)}")
+    return (ctypes.c_float * H)(*vals)
+
+
+def la_workspace_size_decay(op: int, B: int, H: int, N: int, D: int, dtype: torch.dtype) -> int:
+    return int(load_library().la_workspace_size_decay(int(op), B, H, N, D, DTYPE[dtype]))
+
+
+def _workspace_decay(op, q, workspace):
+    B, H, N, D = q.shape
+    need = la_workspace_size_decay(op, B, H, N, D, q.dtype)
+    if need == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def la_forward_decay(q, k, v, gamma, phi="elu1", o=None, return_state=False, workspace=None,
+                     stream=None, g=None):
+    """Causal linear attention with a decay factor per head:
+    S_i = gamma S_{i-1} + phi(k_i) v_i^T, z_i = gamma z_{i-1} + phi(k_i).
+    ``gamma``: H factors in [0, 1] (host values).  ``g``: optional float32
+    [B, H, N] tensor receiving the denominators (pass with o to
+    la_backward_decay)."""
+    lib = load_library()
+    _check_qkv("la_forward_decay", q, k, v)
+    if q.dim() != 4:
+        raise ValueError("la_forward_decay: q, k, v must be [B, H, N, D]")
+    B, H, N, D = q.shape
+    gm = _gamma(gamma, H)
+    o = torch.empty_like(q) if o is None else o
+    _check_qkv("la_forward_decay", q, o)
+    S = z = None
+    if return_state:
+        S = torch.empty((B, H, D, D), dtype=torch.float32, device=q.device)
+        z = torch.empty((B, H, D), dtype=torch.float32, device=q.device)
+    if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
+                          or not g.is_contiguous() or g.device != q.device):
+        raise ValueError("la_forward_decay: g must be contiguous float32 [B, H, N] on q's device")
+    ws, ws_bytes = _workspace_decay(LA_OP_FORWARD, q, workspace)
+    st = lib.la_forward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), _ptr(g), gm,
+                              B, H, N, D, DTYPE[q.dtype], _phi(phi), _ptr(ws), ws_bytes,
+                              _stream_handle(stream))
+    _check("la_forward_decay", st)
+    return (o, S, z) if return_state else o
+
+
+def la_backward_decay(q, k, v, dO, gamma, phi="elu1", dq=None, dk=None, dv=None,
+                      workspace=None, stream=None, o=None, g=None):
+    """dq, dk, dv of sum(dO * O) for O = la_forward_decay(q, k, v, gamma, phi)
+    (no gradient with respect to gamma).  ``o``, ``g``: the forward's output
+    and denominators, both or neither."""
+    lib = load_library()
+    _check_qkv("la_backward_decay", q, k, v, dO)
+    if q.dim() != 4:
+        raise ValueError("la_backward_decay: tensors must be [B, H, N, D]")
+    B, H, N, D = q.shape
+    gm = _gamma(gamma, H)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _check_qkv("la_backward_decay", q, dq, dk, dv)
+    _check_saved("la_backward_decay", q, o, g)
+    ws, ws_bytes = _workspace_decay(LA_OP_BACKWARD, q, workspace)
+    st = lib.la_backward_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
+                               _ptr(dk), _ptr(dv), gm, B, H, N, D, DTYPE[q.dtype], _phi(phi),
+                               _ptr(ws), ws_bytes, _stream_handle(stream))
+    _check("la_backward_decay", st)
+    return dq, dk, dv
+
+
+def la_decode_step_decay(S, z, q, k, v, gamma, phi="elu1", o=None, stream=None):
+    """One decayed in-place step: S = gamma S + phi(k) v^T, z = gamma z +
+    phi(k), o = S^T phi(q) / (phi(q) . z); returns o [B, H, D]."""
+    lib = load_library()
+    _check_qkv("la_decode_step_decay", q, k, v)
+    if q.dim() != 3:
+        raise ValueError("la_decode_step_decay: q, k, v must be [B, H, D]")
+    B, H, D = q.shape
+    gm = _gamma(gamma, H)
+    for name, t, shape in (("S", S, (B, H, D, D)), ("z", z, (B, H, D))):
+        if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
+                or t.device != q.device:
+            raise ValueError(f"la_decode_step_decay: {name} must be contiguous float32 {shape} "
+                             "on the device of q")
+    o = torch.empty_like(q) if o is None else o
+    st = lib.la_decode_step_decay(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(o), gm, B, H,
+                                  D, DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
+    _check("la_decode_step_decay", st)
     return o
 
 

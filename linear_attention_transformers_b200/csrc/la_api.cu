@@ -542,8 +542,13 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                              : launch_bwd_kernel(la::bwd_dq64_kernel<PHI, false>, la::Bwd1x64Cfg::SMEM,
                                                  q1, heads, st, "bwd_dq", la::kBwd64Threads)) != LA_OK)
                     return s;
-                return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
-                                               with_phi(p2), heads, st, "bwd_dkdv", la::kBwd64Threads)
+                if (pin)
+                    return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
+                                             with_phi(p2), heads, st, "bwd_dkdv", la::kBwd64Threads);
+                return p2.dk_part
+                           ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false, true>,
+                                               la::Bwd2x64Cfg::SMEM, p2, heads, st, "bwd_dkdv",
+                                               la::kBwd64Threads)
                            : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
                                                p2, heads, st, "bwd_dkdv", la::kBwd64Threads);
             }
@@ -557,16 +562,25 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                 return s;
             p2.state_in = rrec;
         }
-        if constexpr (D == 64)
-            return pin ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
-                                           with_phi(p2), heads * p.seg.nseg, st, "bwd_dkdv",
-                                           la::kBwd64Threads)
+        if constexpr (D == 64) {
+            if (pin)
+                return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, true>, la::Bwd2x64Cfg::SMEM,
+                                         with_phi(p2), heads * p.seg.nseg, st, "bwd_dkdv",
+                                         la::kBwd64Threads);
+            return p2.dk_part
+                       ? launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false, true>,
+                                           la::Bwd2x64Cfg::SMEM, p2, heads * p.seg.nseg, st,
+                                           "bwd_dkdv", la::kBwd64Threads)
                        : launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM,
                                            p2, heads * p.seg.nseg, st, "bwd_dkdv",
                                            la::kBwd64Threads);
-        else
-            return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
-                                     heads * p.seg.nseg, st, "bwd_dkdv");
+        } else {
+            return p2.dk_part
+                       ? launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true, true>, smem2, p2,
+                                           heads * p.seg.nseg, st, "bwd_dkdv")
+                       : launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, p2,
+                                           heads * p.seg.nseg, st, "bwd_dkdv");
+        }
     }
     float* stot = reinterpret_cast<float*>(ws + p.stot_off);
     float* rtot = reinterpret_cast<float*>(ws + p.rtot_off);
@@ -590,8 +604,10 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
         return s;
     p2.state_in = rtot;
     p2.in_per_head = 1;
-    return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, false>, smem2, p2,
-                             heads * p.qseg.nseg, st, "bwd_dkdv");
+    return p2.dk_part ? launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, false, true>, smem2, p2,
+                                          heads * p.qseg.nseg, st, "bwd_dkdv")
+                      : launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, false>, smem2, p2,
+                                          heads * p.qseg.nseg, st, "bwd_dkdv");
 }
 
 // dK or dV of each key/value head <- the sum of its group's float32
@@ -634,7 +650,7 @@ la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const v
 template <typename T, int PHI>
 la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
                           float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
-                          int causal, cudaStream_t st, int G) {
+                          int causal, cudaStream_t st, int G, const la::DecayArg& dec) {
     auto kern = la::fwd_generic_kernel<T, PHI>;
     const size_t smem = la::generic_smem_bytes(int(D));
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -643,14 +659,15 @@ la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, 
     la::LaunchScope scope("fwd_generic", st);
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
-        static_cast<T*>(o), S_out, z_out, g_out, int(N), int(D), causal, G);
+        static_cast<T*>(o), S_out, z_out, g_out, int(N), int(D), causal, G, dec);
     return launch_status();
 }
 
 template <typename T, int PHI>
 la_status run_bwd_generic(const void* q, const void* k, const void* v, const void* dO, void* dq,
                           void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                          float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part) {
+                          float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part,
+                          const la::DecayArg& dec) {
     // with grouped key/value heads each query head's dK, dV go to `part`
     // first, in float32, and are summed per group afterwards
     const size_t part_bytes = round_up(size_t(heads) * size_t(N) * size_t(D) * 4, 256);
@@ -666,7 +683,7 @@ la_status run_bwd_generic(const void* q, const void* k, const void* v, const voi
         kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
             static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
             static_cast<const T*>(dO), static_cast<T*>(dq), dk_p, dv_p, gbuf, dgbuf, int(N),
-            int(D), causal, G);
+            int(D), causal, G, dec);
         la_status s = launch_status();
         if (s != LA_OK) return s;
         if ((s = launch_group_sum<T>(dk_p, dk, heads / G, N * D, G, st)) != LA_OK) return s;
@@ -680,13 +697,14 @@ la_status run_bwd_generic(const void* q, const void* k, const void* v, const voi
     kern<<<unsigned(heads), la::kGenericThreads, smem, st>>>(
         static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v),
         static_cast<const T*>(dO), static_cast<T*>(dq), static_cast<T*>(dk), static_cast<T*>(dv),
-        gbuf, dgbuf, int(N), int(D), causal, 1);
+        gbuf, dgbuf, int(N), int(D), causal, 1, dec);
     return launch_status();
 }
 
 template <typename T, int PHI>
 la_status run_decode(float* S, float* z, const void* q, const void* k, const void* v, void* o,
-                     int64_t heads, int64_t D, cudaStream_t st, int G) {
+                     int64_t heads, int64_t D, cudaStream_t st, int G,
+                     const la::DecayArg& dec) {
     const T* qq = static_cast<const T*>(q);
     const T* kk = static_cast<const T*>(k);
     const T* vv = static_cast<const T*>(v);
@@ -707,10 +725,10 @@ la_status run_decode(float* S, float* z, const void* q, const void* k, const voi
     const unsigned grid = unsigned(heads);
     la::LaunchScope scope("decode_step", st);
     switch (D) {
-        case 16: la::decode_step_kernel<T, PHI, 16><<<grid, 32, 0, st>>>(S, z, qq, kk, vv, oo); break;
-        case 32: la::decode_step_kernel<T, PHI, 32><<<grid, 64, 0, st>>>(S, z, qq, kk, vv, oo); break;
-        case 64: la::decode_step_kernel<T, PHI, 64><<<grid, 128, 0, st>>>(S, z, qq, kk, vv, oo); break;
-        case 128: la::decode_step_kernel<T, PHI, 128><<<grid, 256, 0, st>>>(S, z, qq, kk, vv, oo); break;
+        case 16: la::decode_step_kernel<T, PHI, 16><<<grid, 32, 0, st>>>(S, z, qq, kk, vv, oo, dec); break;
+        case 32: la::decode_step_kernel<T, PHI, 32><<<grid, 64, 0, st>>>(S, z, qq, kk, vv, oo, dec); break;
+        case 64: la::decode_step_kernel<T, PHI, 64><<<grid, 128, 0, st>>>(S, z, qq, kk, vv, oo, dec); break;
+        case 128: la::decode_step_kernel<T, PHI, 128><<<grid, 256, 0, st>>>(S, z, qq, kk, vv, oo, dec); break;
         default: return LA_ERR_UNSUPPORTED;
     }
     return launch_status();
@@ -731,9 +749,9 @@ template <typename T, int PHI>
 struct FwdOp {
     static la_status run(const void* q, const void* k, const void* v, void* o, float* S_out,
                          float* z_out, float* g_out, int64_t heads, int64_t N, int64_t D,
-                         int causal, cudaStream_t st, int G) {
+                         int causal, cudaStream_t st, int G, const la::DecayArg* dec) {
         return run_fwd_generic<T, PHI>(q, k, v, o, S_out, z_out, g_out, heads, N, D, causal, st,
-                                       G);
+                                       G, *dec);
     }
 };
 
@@ -741,9 +759,10 @@ template <typename T, int PHI>
 struct BwdOp {
     static la_status run(const void* q, const void* k, const void* v, const void* dO, void* dq,
                          void* dk, void* dv, int64_t heads, int64_t N, int64_t D, int causal,
-                         float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part) {
+                         float* gbuf, float* dgbuf, cudaStream_t st, int G, char* part,
+                         const la::DecayArg* dec) {
         return run_bwd_generic<T, PHI>(q, k, v, dO, dq, dk, dv, heads, N, D, causal, gbuf, dgbuf,
-                                       st, G, part);
+                                       st, G, part, *dec);
     }
 };
 
@@ -763,8 +782,9 @@ struct PhiMapOp {
 template <typename T, int PHI>
 struct DecodeOp {
     static la_status run(float* S, float* z, const void* q, const void* k, const void* v,
-                         void* o, int64_t heads, int64_t D, cudaStream_t st, int G) {
-        return run_decode<T, PHI>(S, z, q, k, v, o, heads, D, st, G);
+                         void* o, int64_t heads, int64_t D, cudaStream_t st, int G,
+                         const la::DecayArg* dec) {
+        return run_decode<T, PHI>(S, z, q, k, v, o, heads, D, st, G, *dec);
     }
 };
 
@@ -844,10 +864,42 @@ size_t la_workspace_size(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, i
     return la_workspace_size_gqa(op, B, H, H, N, D, causal, dt);
 }
 
-la_status la_forward_gqa(const void* q, const void* k, const void* v, void* o, float* S_out,
-                         float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
-                         int64_t H, int64_t Hkv, int64_t N, int64_t D, la_dtype dt, int causal,
-                         la_phi phi, void* workspace, size_t workspace_bytes, la_stream_t stream) {
+size_t la_workspace_size_decay(la_op op, int64_t B, int64_t H, int64_t N, int64_t D,
+                               la_dtype dt) {
+    if (check_sizes(B, H, N, D) != LA_OK) return 0;
+    if (dt != LA_F32 && dt != LA_BF16) return 0;
+    if (B == 0 || H == 0 || N == 0) return 0;
+    // enough for either path (the decay factors choose it)
+    if (op == LA_OP_FORWARD) return plan_fwd(B, H, N, D, 1, dt).bytes;
+    if (op == LA_OP_BACKWARD)
+        return std::max(plan_bwd_fast(B, H, N, D, 1, dt, 1).bytes, plan_bwd(B, H, N, D, 1).bytes);
+    return 0;
+}
+
+namespace {
+
+const la::DecayArg kNoDecay{};  // H = 0: no decay
+
+// Per-head decay factors from a host array: finite, in [0, 1], at most
+// kMaxDecayHeads heads.
+la_status make_decay(const float* gamma, int64_t H, la::DecayArg* out) {
+    if (gamma == nullptr) return LA_ERR_INVALID_ARG;
+    if (H > la::kMaxDecayHeads) return LA_ERR_UNSUPPORTED;
+    memset(out, 0, sizeof(*out));
+    for (int64_t h = 0; h < H; ++h) {
+        const float g = gamma[h];
+        if (!(g >= 0.f && g <= 1.f)) return LA_ERR_INVALID_ARG;  // NaN fails too
+        out->gamma[h] = g;
+    }
+    out->H = int(H);
+    return LA_OK;
+}
+
+la_status forward_impl(const void* q, const void* k, const void* v, void* o, float* S_out,
+                       float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
+                       int64_t H, int64_t Hkv, int64_t N, int64_t D, la_dtype dt, int causal,
+                       la_phi phi, void* workspace, size_t workspace_bytes, la_stream_t stream,
+                       const la::DecayArg& dec) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
@@ -875,7 +927,8 @@ la_status la_forward_gqa(const void* q, const void* k, const void* v, void* o, f
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
     if (phi_q_out && ((s = check_ptr(phi_q_out)) || (s = check_ptr(phi_k_out)))) return s;
-    const FwdPlan plan = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
+    // decayed calls run the token-sequential kernels
+    const FwdPlan plan = dec.H > 0 ? FwdPlan{} : plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
     if (plan.bytes > 0 && (workspace == nullptr || workspace_bytes < plan.bytes))
         return LA_ERR_WORKSPACE;
     if ((s = bind_context()) != LA_OK) return s;
@@ -893,10 +946,33 @@ la_status la_forward_gqa(const void* q, const void* k, const void* v, void* o, f
                                                   N, D, causal ? 1 : 0, plan, ws, st, G);
     } else {
         s = dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D,
-                            causal ? 1 : 0, st, G);
+                            causal ? 1 : 0, st, G, &dec);
     }
     if (s != LA_OK || phi_q_out == nullptr || phi_fused) return s;
     return dispatch<PhiMapOp>(dt, phi, q, k, phi_q_out, phi_k_out, heads * N * D, st);
+}
+
+}  // namespace
+
+la_status la_forward_gqa(const void* q, const void* k, const void* v, void* o, float* S_out,
+                         float* z_out, float* g_out, void* phi_q_out, void* phi_k_out, int64_t B,
+                         int64_t H, int64_t Hkv, int64_t N, int64_t D, la_dtype dt, int causal,
+                         la_phi phi, void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    return forward_impl(q, k, v, o, S_out, z_out, g_out, phi_q_out, phi_k_out, B, H, Hkv, N, D,
+                        dt, causal, phi, workspace, workspace_bytes, stream, kNoDecay);
+}
+
+la_status la_forward_decay(const void* q, const void* k, const void* v, void* o, float* S_out,
+                           float* z_out, float* g_out, const float* gamma, int64_t B, int64_t H,
+                           int64_t N, int64_t D, la_dtype dt, la_phi phi, void* workspace,
+                           size_t workspace_bytes, la_stream_t stream) {
+    la::DecayArg dec;
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if ((s = make_decay(gamma, H, &dec)) != LA_OK) return s;
+    return forward_impl(q, k, v, o, S_out, z_out, g_out, nullptr, nullptr, B, H, H, N, D, dt, 1,
+                        phi, workspace, workspace_bytes, stream, dec);
 }
 
 la_status la_forward(const void* q, const void* k, const void* v, void* o, float* S_out,
@@ -907,11 +983,14 @@ la_status la_forward(const void* q, const void* k, const void* v, void* o, float
                           dt, causal, phi, workspace, workspace_bytes, stream);
 }
 
-la_status la_backward_gqa(const void* q, const void* k, const void* v, const void* dO,
-                          const void* o, const float* g, const void* phi_q, const void* phi_k,
-                          void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv,
-                          int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
-                          void* workspace, size_t workspace_bytes, la_stream_t stream) {
+namespace {
+
+la_status backward_impl(const void* q, const void* k, const void* v, const void* dO,
+                        const void* o, const float* g, const void* phi_q, const void* phi_k,
+                        void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv,
+                        int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                        void* workspace, size_t workspace_bytes, la_stream_t stream,
+                        const la::DecayArg& dec) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
@@ -930,10 +1009,11 @@ la_status la_backward_gqa(const void* q, const void* k, const void* v, const voi
     if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
     if (phi_q && G != 1) return LA_ERR_UNSUPPORTED;
     if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
-    const size_t need = la_workspace_size_gqa(LA_OP_BACKWARD, B, H, Hkv, N, D, causal, dt);
+    // decayed calls run the token-sequential kernels
+    const BwdPlan bp = dec.H > 0 ? BwdPlan{} : plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt, G);
+    const size_t need = bp.fast ? bp.bytes : plan_bwd(B, H, N, D, G).bytes;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const BwdPlan bp = plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt, G);
     if ((s = bind_context()) != LA_OK) return s;
     if (bp.fast) {
         char* wsp = static_cast<char*>(workspace);
@@ -965,7 +1045,32 @@ la_status la_backward_gqa(const void* q, const void* k, const void* v, const voi
     float* gbuf = reinterpret_cast<float*>(ws + w.g_off);
     float* dgbuf = reinterpret_cast<float*>(ws + w.dg_off);
     return dispatch<BwdOp>(dt, phi, q, k, v, dO, dq, dk, dv, heads, N, D, causal ? 1 : 0, gbuf,
-                           dgbuf, st, G, ws + w.part_off);
+                           dgbuf, st, G, ws + w.part_off, &dec);
+}
+
+}  // namespace
+
+la_status la_backward_gqa(const void* q, const void* k, const void* v, const void* dO,
+                          const void* o, const float* g, const void* phi_q, const void* phi_k,
+                          void* dq, void* dk, void* dv, int64_t B, int64_t H, int64_t Hkv,
+                          int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                          void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    return backward_impl(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, Hkv, N, D, dt, causal,
+                         phi, workspace, workspace_bytes, stream, kNoDecay);
+}
+
+la_status la_backward_decay(const void* q, const void* k, const void* v, const void* dO,
+                            const void* o, const float* g, void* dq, void* dk, void* dv,
+                            const float* gamma, int64_t B, int64_t H, int64_t N, int64_t D,
+                            la_dtype dt, la_phi phi, void* workspace, size_t workspace_bytes,
+                            la_stream_t stream) {
+    la::DecayArg dec;
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if ((s = make_decay(gamma, H, &dec)) != LA_OK) return s;
+    return backward_impl(q, k, v, dO, o, g, nullptr, nullptr, dq, dk, dv, B, H, H, N, D, dt, 1,
+                         phi, workspace, workspace_bytes, stream, dec);
 }
 
 la_status la_backward(const void* q, const void* k, const void* v, const void* dO,
@@ -999,9 +1104,11 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
                        scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
 }
 
-la_status la_decode_step_gqa(float* S, float* z, const void* q, const void* k, const void* v,
-                             void* o, int64_t B, int64_t H, int64_t Hkv, int64_t D, la_dtype dt,
-                             la_phi phi, la_stream_t stream) {
+namespace {
+
+la_status decode_impl(float* S, float* z, const void* q, const void* k, const void* v, void* o,
+                      int64_t B, int64_t H, int64_t Hkv, int64_t D, la_dtype dt, la_phi phi,
+                      la_stream_t stream, const la::DecayArg& dec) {
     la_status s;
     if ((s = check_enums(dt, phi)) != LA_OK) return s;
     if ((s = check_sizes(B, H, 1, D)) != LA_OK) return s;
@@ -1012,7 +1119,26 @@ la_status la_decode_step_gqa(float* S, float* z, const void* q, const void* k, c
         (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return dispatch<DecodeOp>(dt, phi, S, z, q, k, v, o, heads, D, st, int(H / Hkv));
+    return dispatch<DecodeOp>(dt, phi, S, z, q, k, v, o, heads, D, st, int(H / Hkv), &dec);
+}
+
+}  // namespace
+
+la_status la_decode_step_gqa(float* S, float* z, const void* q, const void* k, const void* v,
+                             void* o, int64_t B, int64_t H, int64_t Hkv, int64_t D, la_dtype dt,
+                             la_phi phi, la_stream_t stream) {
+    return decode_impl(S, z, q, k, v, o, B, H, Hkv, D, dt, phi, stream, kNoDecay);
+}
+
+la_status la_decode_step_decay(float* S, float* z, const void* q, const void* k, const void* v,
+                               void* o, const float* gamma, int64_t B, int64_t H, int64_t D,
+                               la_dtype dt, la_phi phi, la_stream_t stream) {
+    la::DecayArg dec;
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, 1, D)) != LA_OK) return s;
+    if ((s = make_decay(gamma, H, &dec)) != LA_OK) return s;
+    return decode_impl(S, z, q, k, v, o, B, H, H, D, dt, phi, stream, dec);
 }
 
 la_status la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,

@@ -216,6 +216,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int kv_head = kv_head_of(head, prm.kv_group);  // k, v head of this query head
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
     const int nchunks = (tok1 - tok0 + C - 1) / C;
@@ -268,9 +269,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 for (int a = 0; a < D / 64; ++a) {
                     tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
                     tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row,
-                                kv_head_of(head, prm.kv_group));
+                                kv_head);
                     tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
-                                kv_head_of(head, prm.kv_group));
+                                kv_head);
                     tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
                                 head);
                 }
@@ -779,7 +780,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 // ======================================================================
 // Pass 2: dK, dV (reverse token order).
 // ======================================================================
-template <int D, int C, int PHI, bool CAUSAL>
+// PART: grouped key/value heads, dK and dV stored as float32 per-query-head
+// partials (prm.dk_part, dv_part) instead of the bf16 tiles.
+template <int D, int C, int PHI, bool CAUSAL, bool PART = false>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd2Cfg<D, C>;
@@ -802,6 +805,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int kv_head = kv_head_of(head, prm.kv_group);  // k, v head of this query head
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
     const int nchunks = (tok1 - tok0 + C - 1) / C;
@@ -852,9 +856,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 for (int a = 0; a < D / 64; ++a) {
                     tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
                     tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row,
-                                kv_head_of(head, prm.kv_group));
+                                kv_head);
                     tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
-                                kv_head_of(head, prm.kv_group));
+                                kv_head);
                     tma_load_3d(st + 3 * Cfg::TILE + a * C * 128, &prm.tm_do, &full[s], a * 64, row,
                                 head);
                 }
@@ -1089,7 +1093,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                         dk16[k] = (db16[k] + rf[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
                         dk16[8 + k] = (db16[8 + k] + rf[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
                     }
-                    if (prm.dk_part) {
+                    if constexpr (PART) {
                         if (row0 + jrow < prm.N) {
                             const size_t off = (size_t(head) * prm.N + row0 + jrow) * D + c0;
                             store16_f32(prm.dv_part + off, dv16);
@@ -1104,7 +1108,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every rf read done
             mbar_arrive(&empty[s]);
-            if (e == 0 && !prm.dk_part) {
+            if (e == 0 && !PART) {
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
                     tma_store_3d(&prm.tm_dv, stgv + a * C * 128, a * 64, row0, head);

@@ -136,7 +136,9 @@ __device__ __forceinline__ void mask_pack_lower(uint32_t reg, int sp, int irow, 
 
 // PIN: the q and k maps hold phi(q), phi(k) from the forward (no feature
 // map is evaluated here).
-template <int PHI, bool PIN>
+// PART: grouped key/value heads, dK and dV stored as float32 per-query-head
+// partials (prm.dk_part, dv_part) instead of the bf16 tiles.
+template <int PHI, bool PIN, bool PART = false>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
@@ -166,6 +168,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int kv_head = kv_head_of(head, prm.kv_group);  // k, v head of this query head
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
     const int nchunks = (tok1 - tok0 + C - 1) / C;
@@ -218,8 +221,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
                 const int row = row_of(t);
                 tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
-                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head_of(head, prm.kv_group));
-                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head_of(head, prm.kv_group));
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head);
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head);
                 tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
                 issued = t + 1;
             }
@@ -470,7 +473,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                     dk16[i] = (db16[i] + r16[i]) * dphi_from_phi<PHI>(b8a[i]);
                     dk16[8 + i] = (db16[8 + i] + r16[8 + i]) * dphi_from_phi<PHI>(b8b[i]);
                 }
-                if (prm.dk_part) {
+                if constexpr (PART) {
                     if (row_of(t) + jrow < prm.N) {
                         const size_t off = (size_t(head) * prm.N + row_of(t) + jrow) * D + c0;
                         store16_f32(prm.dv_part + off, dv16);
@@ -512,7 +515,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 const int row0 = row_of(t);
                 uint8_t* st = smem + s * Cfg::STAGE;
                 if (!mbar_wait(&staged[s], (t / NS) & 1, abort_flag)) break;
-                if (!prm.dk_part) {  // float32 partials were stored by the epilogue
+                if constexpr (!PART) {  // else the epilogue stored float32 partials
                     tma_store_3d(&prm.tm_dv, st + 2 * Cfg::TILE, 0, row0, head);
                     tma_store_3d(&prm.tm_dk, st + Cfg::TILE, 0, row0, head);
                     bulk_commit();
@@ -597,6 +600,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg, seg = blockIdx.x % prm.nseg;
+    const int kv_head = kv_head_of(head, prm.kv_group);  // k, v head of this query head
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
     const int nchunks = (tok1 - tok0 + C - 1) / C;
@@ -644,8 +648,8 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
                 const int row = row_of(c);
                 tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
-                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head_of(head, prm.kv_group));
-                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head_of(head, prm.kv_group));
+                tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head);
+                tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head);
                 tma_load_3d(st + 3 * Cfg::TILE, &prm.tm_do, &full[s], 0, row, head);
                 issued = c + 1;
             }

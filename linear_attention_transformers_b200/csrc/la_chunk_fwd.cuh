@@ -147,6 +147,10 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg;
+    // grouped key/value heads: the k, v head this query head reads, and
+    // whether it writes that head's final state (the group's first one does)
+    const int kv_head = kv_head_of(head, prm.kv_group);
+    const bool state_writer = writes_kv_state(head, prm.kv_group);
     const int seg = blockIdx.x % prm.nseg;
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
@@ -209,11 +213,10 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                         tma_load_3d(smem + (Cfg::q_slot(s) + a) * Cfg::ATOM, &prm.tm_q, &full[s],
                                     a * 64, row, head);
                     if (kKV) {
-                        const int kvh = kv_head_of(head, prm.kv_group);
                         tma_load_3d(smem + (Cfg::k_slot(s) + a) * Cfg::ATOM, &prm.tm_k, &full[s],
-                                    a * 64, row, kvh);
+                                    a * 64, row, kv_head);
                         tma_load_3d(smem + Cfg::v_slot(s, a) * Cfg::ATOM, &prm.tm_v, &full[s],
-                                    a * 64, row, kvh);
+                                    a * 64, row, kv_head);
                     }
                 }
                 issued = c + 1;
@@ -464,8 +467,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     tc_fence_after();
                     const bool last = c == nchunks - 1;
                     const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
-                                             writes_kv_state(head, prm.kv_group);
-                    const size_t sidx = size_t(kv_head_of(head, prm.kv_group));
+                                             state_writer;
+                    const size_t sidx = size_t(kv_head);
                     if (!last || write_final) {
 #pragma unroll 1
                         for (int v0 = 0; v0 < D; v0 += 16) {

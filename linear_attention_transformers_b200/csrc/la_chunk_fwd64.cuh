@@ -84,6 +84,10 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int head = blockIdx.x / prm.nseg;
+    // grouped key/value heads: the k, v head this query head reads, and
+    // whether it writes that head's final state (the group's first one does)
+    const int kv_head = kv_head_of(head, prm.kv_group);
+    const bool state_writer = writes_kv_state(head, prm.kv_group);
     const int seg = blockIdx.x % prm.nseg;
     const int tok0 = seg * prm.seg_len;
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
@@ -142,9 +146,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 const int row = tok0 + c * C;
                 if (kQ) tma_load_3d(st, &prm.tm_q, &full[s], 0, row, head);
                 if (kKV) {
-                    const int kvh = kv_head_of(head, prm.kv_group);
-                    tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kvh);
-                    tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kvh);
+                    tma_load_3d(st + Cfg::TILE, &prm.tm_k, &full[s], 0, row, kv_head);
+                    tma_load_3d(st + 2 * Cfg::TILE, &prm.tm_v, &full[s], 0, row, kv_head);
                 }
                 issued = c + 1;
             }
@@ -397,8 +400,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                     tc_fence_after();
                     const bool last = c == nchunks - 1;
                     const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
-                                             writes_kv_state(head, prm.kv_group);
-                    const size_t sidx = size_t(kv_head_of(head, prm.kv_group));
+                                             state_writer;
+                    const size_t sidx = size_t(kv_head);
                     if (!last || write_final) {
 #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {

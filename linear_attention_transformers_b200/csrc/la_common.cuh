@@ -70,6 +70,21 @@ __device__ __forceinline__ bool writes_kv_state(int head, int kv_group) {
     return kv_group <= 1 || head % kv_group == 0;
 }
 
+// ------------------------------------------------ decayed (gated) recurrence
+// S_i = gamma S_{i-1} + b_i v_i^T, z_i = gamma z_{i-1} + b_i with one gamma
+// per head (the gating / decay factors of "Efficient Transformers Survey",
+// Common Confusions, "Watch Out").  Passed by value to the kernels that take
+// it; H = 0 means no decay (gamma = 1, and gamma * x is then exactly x).
+constexpr int kMaxDecayHeads = 256;
+struct DecayArg {
+    int H;
+    float gamma[kMaxDecayHeads];
+};
+// gamma of flattened head b*H + h
+__device__ __forceinline__ float decay_of(const DecayArg& d, size_t head) {
+    return d.H > 0 ? d.gamma[head % size_t(d.H)] : 1.f;
+}
+
 // ---------------------------------------------------------------- elements
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }

@@ -2,7 +2,9 @@
 //     S += phi(k) v^T,  z += phi(k),  o = S^T phi(q) / (phi(q) . z)
 // ("Efficient Transformers Survey", Proposition "Linear Attention via Kernel
 // Decomposition", "Why It Matters": S and z updated token by token with
-// constant memory per step).
+// constant memory per step).  With a decay factor gamma per head (DecayArg)
+// the step is S = gamma S + phi(k) v^T, z = gamma z + phi(k); gamma = 1
+// gives bitwise the undecayed step.
 //
 // The step is a single streaming pass over the float32 state: each S element
 // is read once and written once (8 bytes per element), so the kernel is HBM
@@ -23,7 +25,7 @@ template <typename T, int PHI, int D>
 __global__ void __launch_bounds__(2 * D)
 decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
                    const T* __restrict__ q, const T* __restrict__ k,
-                   const T* __restrict__ v, T* __restrict__ o) {
+                   const T* __restrict__ v, T* __restrict__ o, const DecayArg dec) {
     constexpr int CG = D / 4;    // 16-byte column groups
     constexpr int RG = 8;        // row groups
     constexpr int RPT = D / RG;  // rows per thread
@@ -39,6 +41,7 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
     const int tid = threadIdx.x;
     const int cg = tid % CG, rg = tid / CG;
     float4* Sh = reinterpret_cast<float4*>(S + h * D * D);
+    const float gm = decay_of(dec, h);
 
     // Issue the state loads first; the vectors arrive while they are in flight.
     float4 s[RPT];
@@ -55,7 +58,7 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
         a_s[tid] = af;
         b_s[tid] = bf;
         reinterpret_cast<float*>(v_s4)[tid] = to_f32(v[h * D + tid]);
-        znew = z[h * D + tid] + bf;
+        znew = fmaf(gm, z[h * D + tid], bf);
         z[h * D + tid] = znew;
         znew *= af;  // this thread's term of phi(q) . z
     }
@@ -70,10 +73,10 @@ decode_step_kernel(float* __restrict__ S, float* __restrict__ z,
         const int f = rg + RG * r;
         const float bf = b_s[f], af = a_s[f];
         float4 x = s[r];
-        x.x = fmaf(bf, vv.x, x.x);
-        x.y = fmaf(bf, vv.y, x.y);
-        x.z = fmaf(bf, vv.z, x.z);
-        x.w = fmaf(bf, vv.w, x.w);
+        x.x = fmaf(bf, vv.x, gm * x.x);
+        x.y = fmaf(bf, vv.y, gm * x.y);
+        x.z = fmaf(bf, vv.z, gm * x.z);
+        x.w = fmaf(bf, vv.w, gm * x.w);
         __stcs(Sh + f * CG + cg, x);
         acc.x = fmaf(af, x.x, acc.x);
         acc.y = fmaf(af, x.y, acc.y);

@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(kGenericThreads)
 fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, T* __restrict__ o,
                    float* __restrict__ S_out, float* __restrict__ z_out,
-                   float* __restrict__ g_out, int N, int D, int causal, int G) {
+                   float* __restrict__ g_out, int N, int D, int causal, int G,
+                   const DecayArg dec) {
     extern __shared__ float sm[];
     float* S = sm;
     float* z = S + D * D;
@@ -48,6 +49,7 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
     const T* kh = k + kvh * size_t(N) * D;
     const T* vh = v + kvh * size_t(N) * D;
     T* oh = o + base;
+    const float gm = decay_of(dec, head);  // causal only: scales the state per token
 
     for (int t = tid; t < D * D; t += nt) S[t] = 0.f;
     for (int t = tid; t < D; t += nt) z[t] = 0.f;
@@ -76,8 +78,8 @@ fwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
         }
         __syncthreads();
         if (causal) {
-            for (int t = tid; t < D * D; t += nt) S[t] = fmaf(b[t / D], vv[t % D], S[t]);
-            for (int t = tid; t < D; t += nt) z[t] += b[t];
+            for (int t = tid; t < D * D; t += nt) S[t] = fmaf(b[t / D], vv[t % D], gm * S[t]);
+            for (int t = tid; t < D; t += nt) z[t] = fmaf(gm, z[t], b[t]);
             __syncthreads();
         }
         for (int e = tid; e < D; e += nt) {
@@ -114,7 +116,7 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
                    const T* __restrict__ v, const T* __restrict__ dO,
                    T* __restrict__ dq, TO* __restrict__ dk, TO* __restrict__ dv,
                    float* __restrict__ gbuf, float* __restrict__ dgbuf,
-                   int N, int D, int causal, int G) {
+                   int N, int D, int causal, int G, const DecayArg dec) {
     extern __shared__ float sm[];
     float* M = sm;            // S in sweep 1, R in sweep 2
     float* zr = M + D * D;    // z in sweep 1, r in sweep 2
@@ -133,6 +135,9 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
     TO *dkh = dk + base, *dvh = dv + base;
     float* gb = gbuf + head * size_t(N);
     float* dgb = dgbuf + head * size_t(N);
+    // decay (causal only): the prefix state S, z and the suffix sums R, r
+    // are scaled by gamma per token
+    const float gm = decay_of(dec, head);
 
     // ---------------- sweep 1
     for (int t = tid; t < D * D; t += nt) M[t] = 0.f;
@@ -162,8 +167,8 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
         }
         __syncthreads();
         if (causal) {
-            for (int t = tid; t < D * D; t += nt) M[t] = fmaf(b[t / D], vv[t % D], M[t]);
-            for (int t = tid; t < D; t += nt) zr[t] += b[t];
+            for (int t = tid; t < D * D; t += nt) M[t] = fmaf(b[t / D], vv[t % D], gm * M[t]);
+            for (int t = tid; t < D; t += nt) zr[t] = fmaf(gm, zr[t], b[t]);
             __syncthreads();
         }
         float g = 0.f;
@@ -223,8 +228,8 @@ bwd_generic_kernel(const T* __restrict__ q, const T* __restrict__ k,
         }
         __syncthreads();
         if (causal) {
-            for (int t = tid; t < D * D; t += nt) M[t] = fmaf(a[t / D], du[t % D], M[t]);
-            for (int t = tid; t < D; t += nt) zr[t] = fmaf(a[t], dg, zr[t]);
+            for (int t = tid; t < D * D; t += nt) M[t] = fmaf(a[t / D], du[t % D], gm * M[t]);
+            for (int t = tid; t < D; t += nt) zr[t] = fmaf(a[t], dg, gm * zr[t]);
             __syncthreads();
         }
         for (int f = tid; f < D; f += nt) {

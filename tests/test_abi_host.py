@@ -118,3 +118,32 @@ def test_empty_sizes_launch_nothing(lib):
     assert fwd(lib, N=0) == api.LA_OK
     assert bwd(lib, N=0) == api.LA_OK
     assert lib.la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 4, 64, 1, 0, None) == api.LA_OK
+
+
+def test_decay_factors_are_validated_before_launch(lib):
+    import ctypes
+    p = FAKE
+
+    def gam(*vals):
+        return (ctypes.c_float * len(vals))(*vals)
+
+    def fwd_decay(gamma, H=2, N=8, D=64):
+        return lib.la_forward_decay(p, p, p, p, None, None, None, gamma, 1, H, N, D, 1, 0, None,
+                                    0, None)
+
+    assert fwd_decay(None) == api.LA_ERR_INVALID_ARG
+    assert fwd_decay(gam(0.5, 1.5)) == api.LA_ERR_INVALID_ARG
+    assert fwd_decay(gam(0.5, float("nan"))) == api.LA_ERR_INVALID_ARG
+    assert fwd_decay(gam(-0.25, 0.5)) == api.LA_ERR_INVALID_ARG
+    assert fwd_decay(gam(*([0.9] * 257)), H=257) == api.LA_ERR_UNSUPPORTED
+    assert fwd_decay(gam(0.5, 0.9), D=40) == api.LA_ERR_UNSUPPORTED
+    # valid factors, no tokens: nothing to launch
+    assert fwd_decay(gam(0.5, 0.9), N=0) == api.LA_OK
+    assert lib.la_backward_decay(p, p, p, p, None, None, p, p, p, gam(1.2, 0.5), 1, 2, 8, 64, 1,
+                                 0, None, 0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step_decay(p, p, p, p, p, p, gam(0.5, 2.0), 1, 2, 64, 1, 0, None) == \
+        api.LA_ERR_INVALID_ARG
+    assert lib.la_decode_step_decay(p, p, p, p, p, None, gam(0.5, 0.5), 1, 2, 64, 1, 0, None) == \
+        api.LA_ERR_INVALID_ARG
+    assert lib.la_workspace_size_decay(api.LA_OP_BACKWARD, 2, 4, 1000, 64, api.LA_BF16) >= \
+        lib.la_workspace_size(api.LA_OP_BACKWARD, 2, 4, 1000, 64, 1, api.LA_BF16)

@@ -1,0 +1,106 @@
+"""GPU parity for decayed (gated) linear attention, S_i = gamma S_{i-1} +
+phi(k_i) v_i^T with one gamma per head: the forward, the backward and the
+decode step through the C ABI against the fp64 oracle's decayed functions
+(pinned on the CPU in tests/test_oracle_pins.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_transformers_b200 import api, inputs
+from parity_util import check_state, compare
+
+pytestmark = pytest.mark.gpu
+
+PHIS = {"elu1": oracle.PHI_ELU1, "relu_eps": oracle.PHI_RELU_EPS}
+
+
+def gammas(H, lo=0.5):
+    """H factors spread over [lo, 1], the last exactly 1."""
+    return np.linspace(lo, 1.0, H).astype(np.float32)
+
+
+def tensors(B, H, N, D, dtype, seed, dO=False):
+    return [t.cuda() for t in inputs.make_tensors(B, H, N, D, dtype, seed, with_grad_out=dO)]
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("D", [16, 32, 64, 128])
+@pytest.mark.parametrize("N", [1, 129, 777])
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+def test_decay_forward(dtype, D, N, phi):
+    B, H = 2, 4
+    q, k, v = tensors(B, H, N, D, dtype, seed=N + D)
+    gm = gammas(H, 0.3)
+    g = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    o, S, z = api.la_forward_decay(q, k, v, gm, phi, return_state=True, g=g)
+    torch.cuda.synchronize()
+    api.la_get_device_error()
+    o_ref, S_ref, z_ref = oracle.forward_decay(q, k, v, gm.astype(np.float64), PHIS[phi])
+    compare(o, o_ref, dtype, "o")
+    check_state(S, z, S_ref, z_ref, dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("D", [16, 64, 128])
+@pytest.mark.parametrize("N", [1, 129, 777])
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+@pytest.mark.parametrize("saved", [False, True])
+def test_decay_backward(dtype, D, N, phi, saved):
+    B, H = 2, 3
+    q, k, v, dO = tensors(B, H, N, D, dtype, seed=N + 3 * D, dO=True)
+    gm = gammas(H, 0.6)
+    if saved:
+        g = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+        o = api.la_forward_decay(q, k, v, gm, phi, g=g)
+        dq, dk, dv = api.la_backward_decay(q, k, v, dO, gm, phi, o=o, g=g)
+    else:
+        dq, dk, dv = api.la_backward_decay(q, k, v, dO, gm, phi)
+    torch.cuda.synchronize()
+    api.la_get_device_error()
+    rq, rk, rv = oracle.backward_decay(q, k, v, dO, gm.astype(np.float64), PHIS[phi])
+    compare(dq, rq, dtype, "dq")
+    compare(dk, rk, dtype, "dk")
+    compare(dv, rv, dtype, "dv")
+
+
+def test_decay_of_one_is_the_causal_call():
+    # gamma = 1 everywhere: the decayed call equals the plain causal one (the
+    # token-sequential kernels give bitwise the same numbers for float32)
+    q, k, v = tensors(1, 2, 300, 32, torch.float32, seed=5)
+    o1 = api.la_forward_decay(q, k, v, [1.0, 1.0])
+    o0 = api.la_forward(q, k, v, True)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, o1)
+
+
+def test_decay_zero_returns_the_values():
+    q, k, v = tensors(2, 2, 65, 64, torch.float32, seed=6)
+    o = api.la_forward_decay(q, k, v, [0.0, 0.0])
+    torch.cuda.synchronize()
+    compare(o, v.double().cpu().numpy(), torch.float32, "o = v")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("D", [16, 64, 128])
+def test_decay_decode_continues_the_decayed_forward(dtype, D):
+    B, H, T0, T1 = 3, 4, 50, 6
+    q, k, v = tensors(B, H, T0 + T1, D, dtype, seed=D)
+    gm = gammas(H, 0.7)
+    _, S, z = api.la_forward_decay(q[:, :, :T0].contiguous(), k[:, :, :T0].contiguous(),
+                                   v[:, :, :T0].contiguous(), gm, return_state=True)
+    o_ref, S_ref, z_ref = oracle.forward_decay(q, k, v, gm.astype(np.float64))
+    for t in range(T0, T0 + T1):
+        o_t = api.la_decode_step_decay(S, z, q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                       v[:, :, t].contiguous(), gm)
+        compare(o_t, o_ref[:, :, t], dtype, f"decode step {t}")
+    check_state(S, z, S_ref, z_ref, dtype)
+
+
+def test_decay_rejects_bad_factors():
+    q, k, v = tensors(1, 2, 16, 64, torch.bfloat16, seed=1)
+    for bad in ([0.5, 1.5], [0.5, float("nan")], [-0.1, 0.5]):
+        with pytest.raises(api.LinearAttentionError):
+            api.la_forward_decay(q, k, v, bad)
+    with pytest.raises(ValueError):
+        api.la_forward_decay(q, k, v, [0.5])
