@@ -247,7 +247,7 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
     return p;
 }
 
-template <int D, int C, int PHI, int MODE>
+template <int D, int C, int PHI, int MODE, bool DECAY = false>
 la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st,
                        const char* name) {
     auto go = [&](auto kern, int smem, int threads) -> la_status {
@@ -259,21 +259,30 @@ la_status launch_chunk(const la::ChunkParams& prm, int64_t grid, cudaStream_t st
         return launch_status();
     };
     if constexpr (D == 64)
-        return go(la::chunk_fwd64_kernel<PHI, MODE>, la::Chunk64Cfg::SMEM, la::kChunk64Threads);
+        return go(la::chunk_fwd64_kernel<PHI, MODE, DECAY>, la::Chunk64Cfg::SMEM,
+                  la::kChunk64Threads);
     else
-        return go(la::chunk_fwd_kernel<D, C, PHI, MODE>, la::ChunkCfg<D, C>::SMEM,
+        return go(la::chunk_fwd_kernel<D, C, PHI, MODE, DECAY>, la::ChunkCfg<D, C>::SMEM,
                   la::kChunkThreads);
 }
 
+const la::DecayArg kNoDecay{};  // H = 0: no decay
+
+// Smallest decay factor the chunked kernels take with C-token chunks: their
+// chunk-local factors reach gamma^(-C) (an unmasked product), kept <= 2^64.
+float chunk_gamma_min(int C) { return exp2f(-64.f / float(C)); }
+
 la_status launch_state_kernel(int which, float* rec, float* out, float* S, float* z,
                               int64_t heads, int nseg, int64_t D, cudaStream_t st,
-                              int rec_step = 1) {
+                              int rec_step = 1, const la::DecayArg& dec = kNoDecay,
+                              int seg_len = 0) {
     const int R = int(D * D + D);
     const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
     const unsigned grid = unsigned(heads * bph);
     if (which == 0) {
         la::LaunchScope scope("state_scan", st);
-        la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
+        la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph,
+                                                                            dec, seg_len);
     } else if (which == 3) {
         la::LaunchScope scope("state_rscan", st);
         la::state_exclusive_rscan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
@@ -291,9 +300,11 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
 template <int D, int PHI>
 la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, float* S_out,
                           float* z_out, float* g_out, void* pq, void* pk, int64_t heads, int64_t N,
-                          int causal, const FwdPlan& p, char* ws, cudaStream_t st, int G) {
+                          int causal, const FwdPlan& p, char* ws, cudaStream_t st, int G,
+                          const la::DecayArg& dec) {
     constexpr int C = D == 64 ? 128 : 64;
     const int64_t kv_heads = heads / G;
+    const bool decay = dec.H > 0;  // causal only (checked by the caller)
     la::ChunkParams prm;
     memset(&prm, 0, sizeof(prm));
     if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) ||
@@ -303,6 +314,7 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
     prm.N = int(N);
     prm.g_out = g_out;
     prm.kv_group = G;
+    prm.dec = dec;
     const int64_t R = int64_t(D) * D + D;
     float* rec = reinterpret_cast<float*>(ws + p.rec_off);
     la_status s;
@@ -314,11 +326,13 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
             r.S_out = rec;
             r.z_out = rec + D * D;
             r.stride_S = r.stride_z = R;
-            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
-                                                             "chunk_reduce")) != LA_OK)
+            if ((s = decay ? launch_chunk<D, C, PHI, la::MODE_REDUCE, true>(
+                                 r, heads * p.seg.nseg, st, "chunk_reduce")
+                           : launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
+                                                                     "chunk_reduce")) != LA_OK)
                 return s;
             if ((s = launch_state_kernel(0, rec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
-                                         st)) != LA_OK)
+                                         st, 1, dec, p.seg.seg_len)) != LA_OK)
                 return s;
             prm.state_in = rec;
             prm.in_per_head = 0;
@@ -336,6 +350,9 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
                 return LA_ERR_CUDA;
             prm.store_phi = 1;
         }
+        if (decay)
+            return launch_chunk<D, C, PHI, la::MODE_CAUSAL, true>(prm, heads * p.seg.nseg, st,
+                                                                  "chunk_causal");
         return launch_chunk<D, C, PHI, la::MODE_CAUSAL>(prm, heads * p.seg.nseg, st, "chunk_causal");
     }
     // non-causal: segment sums -> totals -> query pass
@@ -366,12 +383,12 @@ template <int PHI>
 la_status run_fwd_chunked_d(const void* q, const void* k, const void* v, void* o, float* S_out,
                             float* z_out, float* g_out, void* pq, void* pk, int64_t heads,
                             int64_t N, int64_t D, int causal, const FwdPlan& p, char* ws,
-                            cudaStream_t st, int G) {
+                            cudaStream_t st, int G, const la::DecayArg& dec = kNoDecay) {
     if (D == 64)
         return run_fwd_chunked<64, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal,
-                                        p, ws, st, G);
+                                        p, ws, st, G, dec);
     return run_fwd_chunked<128, PHI>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N, causal, p,
-                                     ws, st, G);
+                                     ws, st, G, dec);
 }
 
 
@@ -878,8 +895,6 @@ size_t la_workspace_size_decay(la_op op, int64_t B, int64_t H, int64_t N, int64_
 
 namespace {
 
-const la::DecayArg kNoDecay{};  // H = 0: no decay
-
 // Per-head decay factors from a host array: finite, in [0, 1], at most
 // kMaxDecayHeads heads.
 la_status make_decay(const float* gamma, int64_t H, la::DecayArg* out) {
@@ -927,8 +942,12 @@ la_status forward_impl(const void* q, const void* k, const void* v, void* o, flo
     if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
         return s;
     if (phi_q_out && ((s = check_ptr(phi_q_out)) || (s = check_ptr(phi_k_out)))) return s;
-    // decayed calls run the token-sequential kernels
-    const FwdPlan plan = dec.H > 0 ? FwdPlan{} : plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
+    // decayed calls run the chunked kernels when every factor is within
+    // their range, the token-sequential ones otherwise
+    bool chunked = true;
+    for (int h = 0; h < dec.H; ++h)
+        chunked = chunked && dec.gamma[h] >= chunk_gamma_min(chunk_len(D));
+    const FwdPlan plan = chunked ? plan_fwd(B, H, N, D, causal ? 1 : 0, dt) : FwdPlan{};
     if (plan.bytes > 0 && (workspace == nullptr || workspace_bytes < plan.bytes))
         return LA_ERR_WORKSPACE;
     if ((s = bind_context()) != LA_OK) return s;
@@ -941,9 +960,9 @@ la_status forward_impl(const void* q, const void* k, const void* v, void* o, flo
         void* pk = phi_fused ? phi_k_out : nullptr;
         s = phi == LA_PHI_ELU1
                 ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N,
-                                              D, causal ? 1 : 0, plan, ws, st, G)
+                                              D, causal ? 1 : 0, plan, ws, st, G, dec)
                 : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads,
-                                                  N, D, causal ? 1 : 0, plan, ws, st, G);
+                                                  N, D, causal ? 1 : 0, plan, ws, st, G, dec);
     } else {
         s = dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D,
                             causal ? 1 : 0, st, G, &dec);

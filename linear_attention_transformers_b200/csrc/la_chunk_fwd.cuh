@@ -74,6 +74,8 @@ struct ChunkParams {
     // query head `head` reads k, v head head / kv_group, and the final state
     // (per key/value head) is written by the group's first query head
     int kv_group;
+    // decay factor per head (read by the DECAY kernels only; causal)
+    DecayArg dec;
 };
 
 
@@ -118,9 +120,14 @@ struct ChunkCfg {
 
 constexpr int kChunkThreads = 576;  // producer, MMA, 8 phi warps, P and O warpgroups
 
-template <int D, int C, int PHI, int MODE>
+// DECAY: the decayed recurrence, arranged as in chunk_fwd64_kernel (row
+// factors gamma^(t+1-m) on queries and gamma^(m-1-j) on keys; the state
+// accumulator rescaled in TMEM once per chunk; REDUCE decayed to the
+// segment's end).
+template <int D, int C, int PHI, int MODE, bool DECAY = false>
 __global__ void __launch_bounds__(kChunkThreads, 1)
 chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
+    static_assert(!DECAY || MODE != MODE_QUERY, "decay is causal");
     using namespace sm100;
     using Cfg = ChunkCfg<D, C>;
     constexpr int NS = Cfg::NSTAGE, NO = Cfg::NO;
@@ -159,6 +166,8 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                              ? prm.state_in + size_t(prm.in_per_head ? head : blockIdx.x) *
                                                   size_t(D * D + D)
                              : nullptr;
+    float lg = 0.f;  // log2(gamma) of this head
+    if constexpr (DECAY) lg = log2f(decay_of(prm.dec, head));
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -332,7 +341,16 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
             uint8_t* qt = smem + Cfg::q_slot(s) * Cfg::ATOM;
             uint8_t* kt = smem + Cfg::k_slot(s) * Cfg::ATOM;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
-            if (MODE == MODE_CAUSAL) {
+            if (DECAY && MODE == MODE_CAUSAL) {
+                const float m = 0.5f * float(nvalid);
+                if (u < 128)
+                    phi_tile_scaled<PHI, C, D, 128>(qt, u, nvalid, false, lg, 1.f, 1.f - m);
+                else
+                    phi_tile_scaled<PHI, C, D, 128>(kt, u - 128, nvalid, true, lg, -1.f, m - 1.f);
+            } else if (DECAY) {  // REDUCE: decayed to the segment's end
+                phi_tile_scaled<PHI, C, D, 256>(kt, u, nvalid, true, lg, -1.f,
+                                                float(tok1 - tok0 - 1 - c * C));
+            } else if (MODE == MODE_CAUSAL) {
                 if (u < 128)
                     phi_tile<PHI, C, D, 128>(qt, u, nvalid, false);
                 else
@@ -408,28 +426,32 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
             z16[1] = zf - __bfloat162float(__float2bfloat16_rn(zf));
             store_row_bf16<16>(sx, D, frow, D, z16);
         };
+        // decay: the initial state enters as gamma^(m_0) S_0
+        float s0 = 1.f;
+        if constexpr (DECAY) s0 = exp2f(lg * 0.5f * float(min(C, tok1 - tok0)));
         // ---- initial state: bf16 operand (+ TMEM accumulator in CAUSAL mode)
         if (MODE != MODE_REDUCE && frow >= 0) {
             for (int q = 0; q < D / 8; ++q) {
                 float v8[8];
 #pragma unroll
-                for (int t = 0; t < 8; ++t) v8[t] = st_in ? st_in[size_t(frow) * D + q * 8 + t] : 0.f;
+                for (int t = 0; t < 8; ++t)
+                    v8[t] = st_in ? s0 * st_in[size_t(frow) * D + q * 8 + t] : 0.f;
                 store_row_bf16<8>(sx, D, frow, q * 8, v8);
             }
-            put_z(st_in ? st_in[size_t(D) * D + frow] : 0.f);
+            put_z(st_in ? s0 * st_in[size_t(D) * D + frow] : 0.f);
         }
         if (MODE == MODE_CAUSAL && st_in) {
             for (int cc = 0; cc < D; cc += 16) {
                 float v16[16];
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    v16[t] = frow >= 0 ? st_in[size_t(frow) * D + cc + t] : 0.f;
+                    v16[t] = frow >= 0 ? s0 * st_in[size_t(frow) * D + cc + t] : 0.f;
                 tmem_st16(tmem + lane_base + Cfg::T_S + cc, v16);
             }
             float z16[16];
 #pragma unroll
             for (int t = 0; t < 16; ++t)
-                z16[t] = (t == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+                z16[t] = (t == 0 && frow >= 0) ? s0 * st_in[size_t(D) * D + frow] : 0.f;
             tmem_st16(tmem + lane_base + Cfg::T_Z, z16);
             tmem_wait_st();
         }
@@ -469,7 +491,43 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                     const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
                                              state_writer;
                     const size_t sidx = size_t(kv_head);
-                    if (!last || write_final) {
+                    if (DECAY && (!last || write_final)) {
+                        // accumulator gamma^(m-L) S -> gamma^(m') S for the
+                        // next chunk (operand and accumulator), S at the end
+                        const int L = min(C, tok1 - row0);
+                        const float m = 0.5f * float(L);
+                        const float f = last ? exp2f(lg * (float(L) - m))
+                                             : exp2f(lg * (float(L) - m +
+                                                           0.5f * float(min(C, tok1 - row0 - C))));
+#pragma unroll 1
+                        for (int v0 = 0; v0 < D; v0 += 16) {
+                            float sv[16];
+                            tmem_load<16>(tmem + lane_base + Cfg::T_S + v0, sv);
+#pragma unroll
+                            for (int t = 0; t < 16; ++t) sv[t] *= f;
+                            if (!last) tmem_st16(tmem + lane_base + Cfg::T_S + v0, sv);
+                            if (frow >= 0) {
+                                if (last)
+                                    for (int t = 0; t < 16; ++t)
+                                        prm.S_out[sidx * prm.stride_S + size_t(frow) * D + v0 + t] =
+                                            sv[t];
+                                else
+                                    store_row_bf16<16>(sx, D, frow, v0, sv);
+                            }
+                        }
+                        float zv[16];
+                        tmem_load<16>(tmem + lane_base + Cfg::T_Z, zv);
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) zv[t] *= f;
+                        if (!last) tmem_st16(tmem + lane_base + Cfg::T_Z, zv);
+                        if (frow >= 0) {
+                            if (!last)
+                                put_z(zv[0]);
+                            else if (prm.z_out)
+                                prm.z_out[sidx * prm.stride_z + frow] = zv[0];
+                        }
+                        tmem_wait_st();
+                    } else if (!last || write_final) {
 #pragma unroll 1
                         for (int v0 = 0; v0 < D; v0 += 16) {
                             float sv[16];

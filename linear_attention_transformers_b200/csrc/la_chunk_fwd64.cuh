@@ -55,9 +55,20 @@ struct Chunk64Cfg {
 // stage once the stores have read it.
 constexpr int kChunk64Threads = 608;
 
-template <int PHI, int MODE>
+// DECAY: the decayed recurrence S_i = gamma S_{i-1} + b_i v_i^T (CAUSAL and
+// REDUCE).  Within a chunk of L tokens, m = L/2, query row t carries
+// gamma^(t+1-m) and key row j gamma^(m-1-j) (phi_tile_scaled), so P and the
+// state products carry the decay weights; the state accumulator then holds
+// gamma^(m-L) S after the chunk, and the state epilogue rescales it in TMEM
+// to gamma^(m') S for the next chunk (m' of that chunk) before the next
+// accumulation, writing the same values as the next operand.  REDUCE scales
+// key row j of a segment of L_s tokens by gamma^(L_s-1-j) (the segment's
+// state at its end; factors <= 1).  The host takes this path only for
+// gamma >= 2^(-64/C), which keeps every scaled value below 2^64.
+template <int PHI, int MODE, bool DECAY = false>
 __global__ void __launch_bounds__(kChunk64Threads, 1)
 chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
+    static_assert(!DECAY || MODE != MODE_QUERY, "decay is causal");
     using namespace sm100;
     using Cfg = Chunk64Cfg;
     constexpr int C = Cfg::C, D = Cfg::D, NS = Cfg::NSTAGE, NO = Cfg::NO;
@@ -96,6 +107,8 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                              ? prm.state_in + size_t(prm.in_per_head ? head : blockIdx.x) *
                                                   size_t(D * D + D)
                              : nullptr;
+    float lg = 0.f;  // log2(gamma) of this head
+    if constexpr (DECAY) lg = log2f(decay_of(prm.dec, head));
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -259,7 +272,17 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
             uint8_t* st = smem + s * Cfg::STAGE;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
-            if (MODE == MODE_CAUSAL) {
+            if (DECAY && MODE == MODE_CAUSAL) {
+                const float m = 0.5f * float(nvalid);
+                if (u < 128)
+                    phi_tile_scaled<PHI, C, D, 128>(st, u, nvalid, false, lg, 1.f, 1.f - m);
+                else
+                    phi_tile_scaled<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true, lg,
+                                                    -1.f, m - 1.f);
+            } else if (DECAY) {  // REDUCE: decayed to the segment's end
+                phi_tile_scaled<PHI, C, D, 256>(st + Cfg::TILE, u, nvalid, true, lg, -1.f,
+                                                float(tok1 - tok0 - 1 - c * C));
+            } else if (MODE == MODE_CAUSAL) {
                 if (u < 128)
                     phi_tile<PHI, C, D, 128>(st, u, nvalid, false);
                 else
@@ -351,6 +374,10 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                 for (int t = 0; t < 32; ++t) z_dst[32 * half + t] = col[t];
             }
         };
+        // decay: the initial state enters as gamma^(m_0) S_0 (m_0: half the
+        // first chunk's tokens)
+        float s0 = 1.f;
+        if constexpr (DECAY) s0 = exp2f(lg * 0.5f * float(min(C, tok1 - tok0)));
         // initial / fixed state, transposed: column v of S (row 64: z)
         if (MODE != MODE_REDUCE && row <= D) {
             for (int half = 0; half < 2; ++half) {
@@ -358,7 +385,7 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
                     const int f = 32 * half + t;
-                    col[t] = st_in ? (row < D ? st_in[f * D + row] : st_in[D * D + f]) : 0.f;
+                    col[t] = st_in ? s0 * (row < D ? st_in[f * D + row] : st_in[D * D + f]) : 0.f;
                 }
                 put_state(row, half, col);
             }
@@ -370,7 +397,7 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int f = f0 + t;
-                    v16[t] = row < D ? st_in[f * D + row] : (row == D ? st_in[D * D + f] : 0.f);
+                    v16[t] = s0 * (row < D ? st_in[f * D + row] : (row == D ? st_in[D * D + f] : 0.f));
                 }
                 tmem_st16(tmem + lane_base + Cfg::T_S + f0, v16);
             }
@@ -402,7 +429,33 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                     const bool write_final = last && seg == prm.nseg - 1 && prm.S_out != nullptr &&
                                              state_writer;
                     const size_t sidx = size_t(kv_head);
-                    if (!last || write_final) {
+                    if (DECAY && (!last || write_final)) {
+                        // the accumulator holds gamma^(m-L) S: the next chunk
+                        // wants gamma^(m') S (operand and accumulator), the
+                        // final state S itself
+                        const int L = min(C, tok1 - row0);
+                        const float m = 0.5f * float(L);
+                        const float f = last ? exp2f(lg * (float(L) - m))
+                                             : exp2f(lg * (float(L) - m +
+                                                           0.5f * float(min(C, tok1 - row0 - C))));
+#pragma unroll 1
+                        for (int half = 0; half < 2; ++half) {
+                            float col[32];
+                            tmem_load<32>(tmem + lane_base + Cfg::T_S + 32 * half, col);
+#pragma unroll
+                            for (int t = 0; t < 32; ++t) col[t] *= f;
+                            if (last) {
+                                write_state(prm.S_out + sidx * prm.stride_S,
+                                            prm.z_out ? prm.z_out + sidx * prm.stride_z : nullptr,
+                                            half, col);
+                            } else {
+                                tmem_st16(tmem + lane_base + Cfg::T_S + 32 * half, col);
+                                tmem_st16(tmem + lane_base + Cfg::T_S + 32 * half + 16, col + 16);
+                                put_state(row, half, col);
+                            }
+                        }
+                        tmem_wait_st();
+                    } else if (!last || write_final) {
 #pragma unroll 1
                         for (int half = 0; half < 2; ++half) {
                             float col[32];

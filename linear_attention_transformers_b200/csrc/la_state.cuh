@@ -25,13 +25,19 @@ __device__ __forceinline__ void load_batch(const float* base, int p0, int step, 
         if (i < n) x[i] = base[size_t(p0 + i * step) * R];
 }
 
-// rec[h][p] <- sum_{p' < p} rec[h][p'] (exclusive prefix, in place).
+// rec[h][p] <- sum_{p' < p} rec[h][p'] (exclusive prefix, in place).  With
+// a decay factor per head (decayed recurrence; every segment before the
+// last holds seg_len tokens and its record is its state at its end) the
+// prefix is run_p = gamma^seg_len run_{p-1} + rec[p-1]; without one the
+// factor is 1 and the sum is the plain one, bit for bit.
 __global__ void __launch_bounds__(kStateThreads)
-state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head) {
+state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head,
+                            const DecayArg dec, int seg_len) {
     const size_t h = blockIdx.x / blocks_per_head;
     const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
     if (e >= R) return;
     float* base = rec + h * size_t(nseg) * R + e;
+    const float fac = dec.H > 0 ? powf(decay_of(dec, h), float(seg_len)) : 1.f;
     float run = 0.f;
     for (int p0 = 0; p0 < nseg; p0 += kStateBatch) {
         const int n = min(kStateBatch, nseg - p0);
@@ -41,7 +47,7 @@ state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks
         for (int i = 0; i < kStateBatch; ++i)
             if (i < n) {
                 base[size_t(p0 + i) * R] = run;
-                run += x[i];
+                run = fmaf(fac, run, x[i]);
             }
     }
 }

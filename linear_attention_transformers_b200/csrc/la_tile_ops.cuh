@@ -86,6 +86,43 @@ __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool 
         *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + i)) = x[i];
 }
 
+// phi_tile for the decayed recurrence: row r of the tile becomes
+// phi(x_r) * 2^(lg * (sgn * r + off)), evaluated in fp32 and rounded to bf16
+// once.  With lg = log2(gamma) the chunked kernels give query rows the
+// factor gamma^(r + 1 - m) and key rows gamma^(m - 1 - r), so that a query
+// row times a key row carries gamma^(i - j) (the decay weight between them),
+// with every factor within gamma^(+-C/2).  Rows >= nvalid are zero when
+// zero_tail.
+template <int PHI, int C, int D, int T>
+__device__ __forceinline__ void phi_tile_scaled(uint8_t* tile, int t, int nvalid, bool zero_tail,
+                                                float lg, float sgn, float off) {
+    using namespace sm100;
+    constexpr int CH = D / 8;
+    constexpr int PER = (C * CH) / T;
+    static_assert(PER >= 1 && (C * CH) % T == 0 && CH % PER == 0, "work split");
+    const int first = t * PER;
+    const int row = first / CH, q0 = first % CH;
+    uint4 x[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        x[i] = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q0 + i));
+    const bool zero = zero_tail && row >= nvalid;
+    const float sc = exp2f(lg * fmaf(sgn, float(row), off));
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float2 f = unpack_bf16(w[k]);
+            w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x) * sc, phi_fast<PHI>(f.y) * sc);
+        }
+        x[i] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + i)) = x[i];
+}
+
 // Sum of row `row` of a [C][D] bf16 row tile (fp32, fixed order).
 template <int C, int D>
 __device__ __forceinline__ float tile_row_sum(const uint8_t* tile, int row) {

@@ -104,3 +104,72 @@ def test_decay_rejects_bad_factors():
             api.la_forward_decay(q, k, v, bad)
     with pytest.raises(ValueError):
         api.la_forward_decay(q, k, v, [0.5])
+
+
+# ----------------------------------------------- tensor-core decayed forward
+# bf16 with D = 64 (128-token chunks) or D = 128 (64-token chunks) and every
+# gamma >= 2^(-64/C) runs the chunked tcgen05 kernels with chunk-local decay
+# factors; the profile shows which kernels ran.
+
+def _launched(fn):
+    api.la_profile_collect()
+    api.la_profile_enable(True)
+    try:
+        out = fn()
+        torch.cuda.synchronize()
+        return out, api.la_profile_collect()
+    finally:
+        api.la_profile_enable(False)
+
+
+CHUNK_GMIN = {64: 2.0 ** -0.5, 128: 0.5}
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("N", [1, 100, 129, 777, 1000])
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+def test_decay_forward_chunked(D, N, phi):
+    B, H = 2, 4
+    q, k, v = tensors(B, H, N, D, torch.bfloat16, seed=7 * N + D)
+    gm = np.array([CHUNK_GMIN[D], 0.9, 0.99, 1.0], dtype=np.float32)
+    g = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    (o, S, z), prof = _launched(lambda: api.la_forward_decay(q, k, v, gm, phi, return_state=True,
+                                                             g=g))
+    api.la_get_device_error()
+    assert "chunk_causal" in prof and "fwd_generic" not in prof, prof
+    o_ref, S_ref, z_ref = oracle.forward_decay(q, k, v, gm.astype(np.float64), PHIS[phi])
+    compare(o, o_ref, torch.bfloat16, "o")
+    check_state(S, z, S_ref, z_ref, torch.bfloat16)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_decay_forward_chunked_segments(D):
+    # few heads, long sequence: segment states (REDUCE decayed to each
+    # segment's end), the decayed exclusive scan, then the causal pass
+    B, H, N = 1, 2, 20000
+    q, k, v = tensors(B, H, N, D, torch.bfloat16, seed=D + 1)
+    gm = np.array([0.97, 0.9995], dtype=np.float32)
+    (o, S, z), prof = _launched(lambda: api.la_forward_decay(q, k, v, gm, return_state=True))
+    api.la_get_device_error()
+    assert "chunk_reduce" in prof and "state_scan" in prof and "chunk_causal" in prof, prof
+    o_ref, S_ref, z_ref = oracle.forward_decay(q, k, v, gm.astype(np.float64))
+    compare(o, o_ref, torch.bfloat16, "o")
+    check_state(S, z, S_ref, z_ref, torch.bfloat16)
+
+
+def test_decay_below_the_chunked_range_runs_token_sequential():
+    q, k, v = tensors(1, 2, 300, 64, torch.bfloat16, seed=9)
+    gm = np.array([0.6, 0.99], dtype=np.float32)  # 0.6 < 2^-0.5
+    o, prof = _launched(lambda: api.la_forward_decay(q, k, v, gm))
+    assert "fwd_generic" in prof and "chunk_causal" not in prof, prof
+    compare(o, oracle.forward_decay(q, k, v, gm.astype(np.float64))[0], torch.bfloat16, "o")
+
+
+def test_decay_chunked_matches_token_sequential_gamma_one():
+    # gamma = 1 through the decayed chunked kernels: the undecayed causal
+    # result within bf16 rounding (the same arithmetic with unit factors)
+    q, k, v = tensors(2, 2, 1000, 64, torch.bfloat16, seed=11)
+    o1 = api.la_forward_decay(q, k, v, [1.0, 1.0])
+    o0 = api.la_forward(q, k, v, True)
+    torch.cuda.synchronize()
+    compare(o1, o0.double().cpu().numpy(), torch.bfloat16, "gamma 1 vs plain")
