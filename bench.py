@@ -32,7 +32,8 @@ The printed JSON line also carries:
                 decode steps (B256 H32 D128, fp32 state in place), the same
                 with grouped-query attention (8 key/value heads) and the
                 1.4B-parameter LM layer shape forward + backward (B4 H16
-                N4096 D128) with both feature maps;
+                N4096 D128) with both feature maps, and the timed shape with
+                a decay factor per head (decayed recurrence);
   e2e           the headline metric with every step's inputs copied from
                 pinned host memory and its outputs (o, dq, dk, dv) read back
                 inside the timed region, consecutive steps pipelined over two
@@ -395,6 +396,29 @@ class TrainStep:
         self.backward()
 
 
+class DecayTrainStep(TrainStep):
+    """TrainStep of the decayed recurrence (one factor per head): the forward
+    keeps o and g, the backward takes them."""
+
+    def __init__(self, api, w, dev, stream, gamma):
+        super().__init__(api, w, dev, stream)
+        self.gamma = gamma
+        B, H, N, D = self.q.shape
+        need = max(api.la_workspace_size_decay(op, B, H, N, D, w.dtype)
+                   for op in (api.LA_OP_FORWARD, api.LA_OP_BACKWARD))
+        if need > self.ws.numel():
+            self.ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+    def forward(self, q=None, k=None, v=None, o=None):
+        self.api.la_forward_decay(self.q, self.k, self.v, self.gamma, self.w.phi, o=self.o,
+                                  workspace=self.ws, stream=self.stream, g=self.g)
+
+    def backward(self, q=None, k=None, v=None, dO=None, o=None, grads=None):
+        self.api.la_backward_decay(self.q, self.k, self.v, self.dO, self.gamma, self.w.phi,
+                                   dq=self.dq, dk=self.dk, dv=self.dv, workspace=self.ws,
+                                   stream=self.stream, o=self.o, g=self.g)
+
+
 def split_times(step, steps, stream):
     """Forward and backward milliseconds per step, from CUDA events recorded
     between the two calls on the launching stream (a separate, untimed-by-
@@ -412,10 +436,12 @@ def split_times(step, steps, stream):
     return f, b
 
 
-def graded_train(api, w, dev, stream, world, peaks, steps=20, warmup=5):
+def graded_train(api, w, dev, stream, world, peaks, steps=20, warmup=5, gamma=None):
     """A forward + backward workload at its full size: ms per step, tokens/s
-    and the roofline fractions of the step, the forward and the backward."""
-    step = TrainStep(api, w, dev, stream)
+    and the roofline fractions of the step, the forward and the backward.
+    gamma: per-head decay factors (the decayed recurrence)."""
+    step = TrainStep(api, w, dev, stream) if gamma is None else \
+        DecayTrainStep(api, w, dev, stream, gamma)
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -651,6 +677,8 @@ def run_ours(args, world, rank, local):
                 "causal_fwdbwd_b4h16n4096d128_relu_bf16"], dev, stream, world, peaks),
             "lm_layer_elu": graded_train(api, inputs.WORKLOADS[
                 "causal_fwdbwd_b4h16n4096d128_elu_bf16"], dev, stream, world, peaks),
+            "decay_train": graded_train(api, inputs.DECAY_TRAIN, dev, stream, world, peaks,
+                                        gamma=inputs.decay_factors(inputs.DECAY_TRAIN.H)),
         }
 
     cpu = None

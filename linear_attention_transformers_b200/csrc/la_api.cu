@@ -471,7 +471,8 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
                           const void* o_saved, const float* g_saved, const void* pq,
                           const void* pk, void* dq, void* dk, void* dv, int64_t heads,
                           int64_t N, int causal, const BwdPlan& p, char* ws, cudaStream_t st,
-                          int G, float* dk_part, float* dv_part) {
+                          int G, float* dk_part, float* dv_part,
+                          const la::DecayArg& dec = kNoDecay) {
     constexpr int C = D == 64 ? 128 : 64;
     const int64_t kv_heads = heads / G;
     // with grouped key/value heads the kernels store float32 partials per
@@ -491,6 +492,7 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     prm.kv_group = G;
     prm.dk_part = G > 1 ? dk_part : nullptr;
     prm.dv_part = G > 1 ? dv_part : nullptr;
+    prm.dec = dec;
     prm.N = int(N);
     // the forward's o and g: the caller's, or computed into the workspace
     // by la_backward before this runs
@@ -549,6 +551,19 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
             p1.rec_out = rrec;
         }
         if constexpr (D == 64) {
+            // decayed recurrence: the pipelined passes with chunk-local decay
+            // factors (the caller takes this path with one segment per head,
+            // no saved feature maps and no grouping)
+            if (dec.H > 0) {
+                if (p.seg.nseg != 1 || pin || G != 1) return LA_ERR_INVALID_ARG;
+                la_status s1 = launch_bwd_kernel(la::bwd_dq64_kernel<PHI, false, true>,
+                                                 la::Bwd1x64Cfg::SMEM, p1, heads, st, "bwd_dq",
+                                                 la::kBwd64Threads);
+                if (s1 != LA_OK) return s1;
+                return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false, false, true>,
+                                         la::Bwd2x64Cfg::SMEM, p2, heads, st, "bwd_dkdv",
+                                         la::kBwd64Threads);
+            }
             // one segment per head: the pipelined passes (pass 1 reads the
             // forward's phi(q) when given, and k itself: it centres phi(k))
             if (p.seg.nseg == 1) {
@@ -645,7 +660,7 @@ la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const v
                             const void* o_saved, const float* g_saved, const void* pq,
                             const void* pk, void* dq, void* dk, void* dv, int64_t heads,
                             int64_t N, int64_t D, int causal, const BwdPlan& p, char* ws,
-                            cudaStream_t st, int G) {
+                            cudaStream_t st, int G, const la::DecayArg& dec = kNoDecay) {
     // with grouped key/value heads each query head's dK, dV go to the
     // workspace first, in float32, and are summed per group after the passes
     const size_t part_bytes = round_up(size_t(heads) * size_t(N) * size_t(D) * 4, 256);
@@ -654,7 +669,9 @@ la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const v
     la_status s;
     if (D == 64)
         s = run_bwd_chunked<64, PHI>(q, k, v, dO, o_saved, g_saved, pq, pk, dq, dk, dv, heads,
-                                     N, causal, p, ws, st, G, dk_p, dv_p);
+                                     N, causal, p, ws, st, G, dk_p, dv_p, dec);
+    else if (dec.H > 0)  // the decayed backward runs chunked for D = 64 only
+        return LA_ERR_INVALID_ARG;
     else  // the D = 128 kernels evaluate the feature map themselves
         s = run_bwd_chunked<128, PHI>(q, k, v, dO, o_saved, g_saved, nullptr, nullptr, dq, dk,
                                       dv, heads, N, causal, p, ws, st, G, dk_p, dv_p);
@@ -1028,8 +1045,16 @@ la_status backward_impl(const void* q, const void* k, const void* v, const void*
     if ((phi_q == nullptr) != (phi_k == nullptr) || (phi_q && !o)) return LA_ERR_INVALID_ARG;
     if (phi_q && G != 1) return LA_ERR_UNSUPPORTED;
     if (phi_q && ((s = check_ptr(phi_q)) || (s = check_ptr(phi_k)))) return s;
-    // decayed calls run the token-sequential kernels
-    const BwdPlan bp = dec.H > 0 ? BwdPlan{} : plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt, G);
+    // decayed calls run the chunked passes for head size 64 when every factor
+    // is within their range and the plan keeps one segment per head, the
+    // token-sequential kernels otherwise
+    BwdPlan bp = plan_bwd_fast(B, H, N, D, causal ? 1 : 0, dt, G);
+    if (dec.H > 0) {
+        bool chunked = bp.fast && D == 64 && causal && G == 1 && bp.seg.nseg == 1;
+        for (int h = 0; h < dec.H; ++h)
+            chunked = chunked && dec.gamma[h] >= chunk_gamma_min(chunk_len(D));
+        if (!chunked) bp = BwdPlan{};
+    }
     const size_t need = bp.fast ? bp.bytes : plan_bwd(B, H, N, D, G).bytes;
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return LA_ERR_WORKSPACE;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1045,19 +1070,21 @@ la_status backward_impl(const void* q, const void* k, const void* v, const void*
             s = phi == LA_PHI_ELU1
                     ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o_ws, nullptr, nullptr, g_ws, nullptr,
                                                   nullptr, heads, N, D, causal ? 1 : 0, fp,
-                                                  wsp + bp.fwd_off, st, G)
+                                                  wsp + bp.fwd_off, st, G, dec)
                     : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o_ws, nullptr, nullptr, g_ws,
                                                       nullptr, nullptr, heads, N, D,
-                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st, G);
+                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st, G,
+                                                      dec);
             if (s != LA_OK) return s;
             o = o_ws;
             g = g_ws;
         }
         return phi == LA_PHI_ELU1
                    ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st, G)
+                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st, G, dec)
                    : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st, G);
+                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st, G,
+                                                     dec);
     }
     const BwdWorkspace w = plan_bwd(B, H, N, D, G);
     char* ws = static_cast<char*>(workspace);

@@ -57,6 +57,8 @@ struct BwdParams {
     // caller's sum over each group rounds to bf16 once
     float* dk_part;
     float* dv_part;
+    // decay factor per head (read by the DECAY kernels only; causal)
+    DecayArg dec;
 };
 
 template <int D, int C>
@@ -130,6 +132,16 @@ __device__ __forceinline__ float dphi_from_phi(float a) {
     if (PHI == PHI_ELU1) return fminf(a, 1.f);
     const float floor_val = __bfloat162float(__float2bfloat16_rn(1e-6f));
     return a > floor_val ? 1.f : 0.f;
+}
+
+// phi'(k) from the bf16 value b = bf16(phi(k) * beta) of a key row scaled
+// by the decay factor beta (the decayed passes): elu+1 takes min(b / beta, 1);
+// for relu+eps, k <= 0 left exactly bf16(1e-6 * beta) in the tile (the same
+// product, rounded the same way), so b above it means k > 0.
+template <int PHI>
+__device__ __forceinline__ float dphi_from_scaled_phi(float b, float beta, float binv) {
+    if (PHI == PHI_ELU1) return fminf(b * binv, 1.f);
+    return b > __bfloat162float(__float2bfloat16_rn(1e-6f * beta)) ? 1.f : 0.f;
 }
 
 // Load a state record into the bf16 operand tile [D][D] (row f) and return

@@ -63,7 +63,8 @@ constexpr int kBwd64Threads = 608;
 // the diagonal block for b == sp and unmasked for b > sp.  Block b is read
 // before columns 16b.. are written, and writes only reach columns of blocks
 // already read.
-__device__ __forceinline__ void mask_pack_upper(uint32_t reg, int sp, int jrow, const float* dgf) {
+__device__ __forceinline__ void mask_pack_upper(uint32_t reg, int sp, int jrow, const float* dgf,
+                                                float dscale = 1.f) {
     using namespace sm100;
 #pragma unroll 1
     for (int b = 0; b < 4; ++b) {
@@ -79,10 +80,10 @@ __device__ __forceinline__ void mask_pack_upper(uint32_t reg, int sp, int jrow, 
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const float4 d4 = reinterpret_cast<const float4*>(dgf + i0)[q];
-                    v[4 * q] += d4.x;
-                    v[4 * q + 1] += d4.y;
-                    v[4 * q + 2] += d4.z;
-                    v[4 * q + 3] += d4.w;
+                    v[4 * q] = fmaf(dscale, d4.x, v[4 * q]);
+                    v[4 * q + 1] = fmaf(dscale, d4.y, v[4 * q + 1]);
+                    v[4 * q + 2] = fmaf(dscale, d4.z, v[4 * q + 2]);
+                    v[4 * q + 3] = fmaf(dscale, d4.w, v[4 * q + 3]);
                 }
             }
             if (b == sp) {
@@ -138,9 +139,17 @@ __device__ __forceinline__ void mask_pack_lower(uint32_t reg, int sp, int irow, 
 // map is evaluated here).
 // PART: grouped key/value heads, dK and dV stored as float32 per-query-head
 // partials (prm.dk_part, dv_part) instead of the bf16 tiles.
-template <int PHI, bool PIN, bool PART = false>
+// DECAY: the decayed recurrence (one segment per head, phi evaluated here).
+// Within a chunk of L tokens, m = L/2, query rows a_i carry gamma^(i-m) and
+// key and value rows b_j, v_j carry beta_j = gamma^(m-j), so X1, X2 and the
+// products with dU, A carry gamma^(i-j) (the dg_i added to X2 takes beta_j
+// too); the suffix state accumulator (and r) hold gamma^(L-m) R of the
+// later tokens and are rescaled once per step; dK takes beta_j on r and
+// phi'(k) from b / beta_j.
+template <int PHI, bool PIN, bool PART = false, bool DECAY = false>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
+    static_assert(!(DECAY && PIN), "decay evaluates phi itself");
     using namespace sm100;
     using Cfg = Bwd2x64Cfg;
     constexpr int C = Cfg::C, D = Cfg::D, NS = Cfg::NSTAGE;
@@ -177,6 +186,8 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                      : nullptr;
     // chunk processed at step t (reverse token order)
     auto row_of = [&](int t) { return tok0 + (nchunks - 1 - t) * C; };
+    float lg = 0.f;  // log2(gamma) of this head
+    if constexpr (DECAY) lg = log2f(decay_of(prm.dec, head));
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -352,7 +363,15 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                 dgf[u] = d;
             }
             named_bar_sync(3, 256);  // rinv ready
-            if constexpr (!PIN) {
+            if constexpr (DECAY) {
+                const float m = 0.5f * float(nvalid);
+                if (u < 128)
+                    phi_tile_scaled<PHI, C, D, 128>(st, u, nvalid, true, lg, 1.f, -m);
+                else
+                    phi_tile_scaled<PHI, C, D, 128>(st + Cfg::TILE, u - 128, nvalid, true, lg,
+                                                    -1.f, m);
+                scale_tile_rows_exp2<C, D, 256>(st + 2 * Cfg::TILE, u, nvalid, lg, -1.f, m);
+            } else if constexpr (!PIN) {
                 if (u < 128)
                     phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
                 else
@@ -409,7 +428,13 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             if (PIN) continue;  // X2 is packed by feature-map warps 2-5
             if (!named_bar_all(1, 128, mbar_wait(x2_full, t & 1, abort_flag))) break;
             tc_fence_after();
-            mask_pack_upper(tmem + lane_base + Cfg::T_X2, sp, jrow, dgf);
+            if constexpr (DECAY) {
+                const float m = 0.5f * float(min(C, tok1 - row_of(t)));
+                mask_pack_upper(tmem + lane_base + Cfg::T_X2, sp, jrow, dgf,
+                                exp2f(lg * (m - float(jrow))));
+            } else {
+                mask_pack_upper(tmem + lane_base + Cfg::T_X2, sp, jrow, dgf);
+            }
             tc_fence_before();
             mbar_arrive(x2p_full);
         }
@@ -447,6 +472,13 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             const int s = t % NS;
             uint8_t* kt = smem + s * Cfg::STAGE + Cfg::TILE;   // B, then dK
             uint8_t* vt = smem + s * Cfg::STAGE + 2 * Cfg::TILE;  // dV
+            // decay: this row's beta_j (r term) and 1 / beta_j (phi' from b)
+            float beta = 1.f, binv = 1.f, m = 0.f;
+            if constexpr (DECAY) {
+                m = 0.5f * float(min(C, tok1 - row_of(t)));
+                beta = exp2f(lg * (m - float(jrow)));
+                binv = exp2f(lg * (float(jrow) - m));
+            }
             if (!named_bar_all(2, 128, mbar_wait(d_full, t & 1, abort_flag))) break;
             tc_fence_after();
 #pragma unroll 1
@@ -468,10 +500,20 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                     r16[4 * q + 3] = x.w;
                 }
                 float dk16[16];
+                if constexpr (DECAY) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    dk16[i] = (db16[i] + r16[i]) * dphi_from_phi<PHI>(b8a[i]);
-                    dk16[8 + i] = (db16[8 + i] + r16[8 + i]) * dphi_from_phi<PHI>(b8b[i]);
+                    for (int i = 0; i < 8; ++i) {
+                        dk16[i] = fmaf(beta, r16[i], db16[i]) *
+                                  dphi_from_scaled_phi<PHI>(b8a[i], beta, binv);
+                        dk16[8 + i] = fmaf(beta, r16[8 + i], db16[8 + i]) *
+                                      dphi_from_scaled_phi<PHI>(b8b[i], beta, binv);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        dk16[i] = (db16[i] + r16[i]) * dphi_from_phi<PHI>(b8a[i]);
+                        dk16[8 + i] = (db16[8 + i] + r16[8 + i]) * dphi_from_phi<PHI>(b8b[i]);
+                    }
                 }
                 if constexpr (PART) {
                     if (row_of(t) + jrow < prm.N) {
@@ -493,15 +535,30 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             // state after this chunk -> operands of the next (earlier) chunk
             if (!named_bar_all(2, 128, mbar_wait(r_full, t & 1, abort_flag))) break;
             tc_fence_after();
+            // decay: the accumulator holds gamma^(-m) R of this chunk's
+            // start; the next (earlier, full) chunk wants gamma^(C/2) R
+            const float fr = DECAY ? exp2f(lg * (0.5f * float(C) + m)) : 1.f;
 #pragma unroll 1
             for (int v0 = 0; v0 < D; v0 += 16) {
                 float rv[16];
                 tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
                 tmem_wait_ld();
+                if constexpr (DECAY) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) rv[i] *= fr;
+                    tmem_st16(tmem + lane_base + Cfg::T_R + v0, rv);
+                }
                 if (frow >= 0) store_row16_bf16(rp, D, frow, v0, rv);
             }
+            if constexpr (DECAY) tmem_wait_st();
             if (!named_bar_all(2, 128, mbar_wait(&rch_full[t & 1], (t >> 1) & 1, abort_flag))) break;
-            if (frow >= 0) rf[frow] += reinterpret_cast<const float*>(smem + Cfg::OFF_RCH)[(t & 3) * D + frow];
+            if constexpr (DECAY) {
+                if (frow >= 0)
+                    rf[frow] = fr * (rf[frow] + reinterpret_cast<const float*>(
+                                                     smem + Cfg::OFF_RCH)[(t & 3) * D + frow]);
+            } else {
+                if (frow >= 0) rf[frow] += reinterpret_cast<const float*>(smem + Cfg::OFF_RCH)[(t & 3) * D + frow];
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(rx_full);
@@ -573,9 +630,15 @@ struct Bwd1x64Cfg {
     static_assert(OFF_ONES % 1024 == 0 && OFF_SX % 1024 == 0, "swizzled tiles on 1 KB");
 };
 
-template <int PHI, bool PIN>
+// DECAY: the decayed recurrence (phi(q) evaluated here).  Within a chunk of
+// L tokens, m = L/2, dU rows and dg_i carry gamma^(i+1-m) and the centred
+// key rows gamma^(m-1-j), so W' B' carries gamma^(i-j); the state
+// accumulator holds gamma^(m-L) S' after the chunk and is rescaled in TMEM
+// to gamma^(m') S' (the next chunk's m') with the operand and z.
+template <int PHI, bool PIN, bool DECAY = false>
 __global__ void __launch_bounds__(kBwd64Threads, 1)
 bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
+    static_assert(!(DECAY && PIN), "decay evaluates phi itself");
     using namespace sm100;
     using Cfg = Bwd1x64Cfg;
     constexpr int C = Cfg::C, D = Cfg::D, NS = Cfg::NSTAGE;
@@ -605,6 +668,8 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
     const int tok1 = min(prm.N, tok0 + prm.seg_len);
     const int nchunks = (tok1 - tok0 + C - 1) / C;
     auto row_of = [&](int c) { return tok0 + c * C; };
+    float lg = 0.f;  // log2(gamma) of this head
+    if constexpr (DECAY) lg = log2f(decay_of(prm.dec, head));
 
     if (tid == 0) {
         for (int s = 0; s < NS; ++s) {
@@ -727,7 +792,12 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
             uint8_t* st = smem + s * Cfg::STAGE;
             // k -> phi(k) - c, the centred key features (from k even when the
             // forward's phi(k) is available: it is rounded once, from k)
-            phi_tile<PHI, C, D, 256, true>(st + Cfg::TILE, u, nvalid, true);
+            const float m = 0.5f * float(nvalid);
+            if constexpr (DECAY)
+                phi_tile_scaled<PHI, C, D, 256, true>(st + Cfg::TILE, u, nvalid, true, lg, -1.f,
+                                                      m - 1.f);
+            else
+                phi_tile<PHI, C, D, 256, true>(st + Cfg::TILE, u, nvalid, true);
             uint8_t* dot = st + 3 * Cfg::TILE;
             float dotp = 0.f;
 #pragma unroll
@@ -742,8 +812,11 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 }
             }
             dotp += __shfl_xor_sync(0xffffffffu, dotp, 1);
+            // decay: dU and dg of row r carry gamma^(r+1-m)
+            const float sr = DECAY ? exp2f(lg * (float(r) + 1.f - m)) : 1.f;
             const float ginv = 1.f / g;
             const float dg = valid ? -dotp * ginv : 0.f;
+            const float gs = ginv * sr;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 uint4* px = reinterpret_cast<uint4*>(dot + tile_chunk_off(C, r, 4 * part + j));
@@ -752,12 +825,12 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
                     const float2 f = unpack_bf16(w[t]);
-                    w[t] = valid ? pack_bf16(f.x * ginv, f.y * ginv) : 0u;
+                    w[t] = valid ? pack_bf16(f.x * gs, f.y * gs) : 0u;
                 }
                 *px = make_uint4(w[0], w[1], w[2], w[3]);
             }
             if (part == 0) {
-                reinterpret_cast<float*>(st + Cfg::OFF_DGF)[r] = dg;
+                reinterpret_cast<float*>(st + Cfg::OFF_DGF)[r] = dg * sr;
                 if (valid) prm.dgbuf[size_t(head) * prm.N + row0 + r] = dg;
             }
             fence_proxy_async_smem();
@@ -807,10 +880,20 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                 // state after this chunk -> operands of the next chunk
                 if (!named_bar_all(2, 128, mbar_wait(t_full, c & 1, abort_flag))) break;
                 tc_fence_after();
+                // decay: gamma^(m-C) S' (this full chunk) -> gamma^(m') S'
+                const float fs =
+                    DECAY ? exp2f(lg * (0.5f * float(C) + 0.5f * float(min(C, tok1 - row_of(c + 1)))))
+                          : 1.f;
 #pragma unroll 1
                 for (int h = 0; h < 2; ++h) {
                     float col[32];
                     tmem_load<32>(tmem + lane_base + Cfg::T_T + 32 * h, col);
+                    if constexpr (DECAY) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) col[i] *= fs;
+                        tmem_st16(tmem + lane_base + Cfg::T_T + 32 * h, col);
+                        tmem_st16(tmem + lane_base + Cfg::T_T + 32 * h + 16, col + 16);
+                    }
                     if (irow < D) {
                         store_row_bf16<32>(sxp, D, irow, 32 * h, col);
                     } else if (irow == D) {
@@ -818,6 +901,7 @@ bwd_dq64_kernel(const __grid_constant__ BwdParams prm) {
                         for (int i = 0; i < 32; ++i) zf[((c + 1) & 1) * D + 32 * h + i] = col[i];
                     }
                 }
+                if constexpr (DECAY) tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(sx_full);

@@ -438,20 +438,34 @@ chunk_fwd64_kernel(const __grid_constant__ ChunkParams prm) {
                         const float f = last ? exp2f(lg * (float(L) - m))
                                              : exp2f(lg * (float(L) - m +
                                                            0.5f * float(min(C, tok1 - row0 - C))));
+                        float* S_dst = prm.S_out ? prm.S_out + sidx * prm.stride_S : nullptr;
+                        float* z_dst = prm.z_out ? prm.z_out + sidx * prm.stride_z : nullptr;
 #pragma unroll 1
-                        for (int half = 0; half < 2; ++half) {
-                            float col[32];
-                            tmem_load<32>(tmem + lane_base + Cfg::T_S + 32 * half, col);
+                        for (int q4 = 0; q4 < 4; ++q4) {  // 16 columns at a time
+                            float col[16];
+                            tmem_load<16>(tmem + lane_base + Cfg::T_S + 16 * q4, col);
 #pragma unroll
-                            for (int t = 0; t < 32; ++t) col[t] *= f;
+                            for (int t = 0; t < 16; ++t) col[t] *= f;
                             if (last) {
-                                write_state(prm.S_out + sidx * prm.stride_S,
-                                            prm.z_out ? prm.z_out + sidx * prm.stride_z : nullptr,
-                                            half, col);
+                                if (row < D && S_dst) {
+                                    for (int t = 0; t < 16; ++t) S_dst[(16 * q4 + t) * D + row] = col[t];
+                                } else if (row == D && z_dst) {
+                                    for (int t = 0; t < 16; ++t) z_dst[16 * q4 + t] = col[t];
+                                }
                             } else {
-                                tmem_st16(tmem + lane_base + Cfg::T_S + 32 * half, col);
-                                tmem_st16(tmem + lane_base + Cfg::T_S + 32 * half + 16, col + 16);
-                                put_state(row, half, col);
+                                tmem_st16(tmem + lane_base + Cfg::T_S + 16 * q4, col);
+                                if (row < D) {
+                                    store_row_bf16<16>(sx, 80, row, 16 * q4, col);
+                                } else if (row == D) {
+                                    float hi[16], lo[16];
+#pragma unroll
+                                    for (int t = 0; t < 16; ++t) {
+                                        hi[t] = __bfloat162float(__float2bfloat16_rn(col[t]));
+                                        lo[t] = col[t] - hi[t];
+                                    }
+                                    store_row_bf16<16>(sx, 80, D, 16 * q4, hi);
+                                    store_row_bf16<16>(sx, 80, D + 1, 16 * q4, lo);
+                                }
                             }
                         }
                         tmem_wait_st();

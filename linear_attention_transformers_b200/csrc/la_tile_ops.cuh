@@ -93,9 +93,49 @@ __device__ __forceinline__ void phi_tile(uint8_t* tile, int t, int nvalid, bool 
 // row times a key row carries gamma^(i - j) (the decay weight between them),
 // with every factor within gamma^(+-C/2).  Rows >= nvalid are zero when
 // zero_tail.
-template <int PHI, int C, int D, int T>
+template <int PHI, int C, int D, int T, bool CENTER = false>
 __device__ __forceinline__ void phi_tile_scaled(uint8_t* tile, int t, int nvalid, bool zero_tail,
                                                 float lg, float sgn, float off) {
+    constexpr float kc = CENTER ? phi_center<PHI>() : 0.f;  // centred: (phi - c) * factor
+    using namespace sm100;
+    constexpr int CH = D / 8;
+    constexpr int PER = (C * CH) / T;
+    static_assert(PER >= 1 && (C * CH) % T == 0 && CH % PER == 0, "work split");
+    constexpr int GRP = PER > 4 ? 4 : PER;  // 16-byte chunks converted at a time
+    const int first = t * PER;
+    const int row = first / CH, q0 = first % CH;
+    const bool zero = zero_tail && row >= nvalid;
+    const float sc = exp2f(lg * fmaf(sgn, float(row), off));
+#pragma unroll
+    for (int g0 = 0; g0 < PER; g0 += GRP) {
+        uint4 x[GRP];
+#pragma unroll
+        for (int i = 0; i < GRP; ++i)
+            x[i] = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q0 + g0 + i));
+#pragma unroll
+        for (int i = 0; i < GRP; ++i) {
+            uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float2 f = unpack_bf16(w[k]);
+                w[k] = zero ? 0u
+                            : pack_bf16((phi_fast<PHI>(f.x) - kc) * sc,
+                                        (phi_fast<PHI>(f.y) - kc) * sc);
+            }
+            x[i] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < GRP; ++i)
+            *reinterpret_cast<uint4*>(tile + tile_chunk_off(C, row, q0 + g0 + i)) = x[i];
+    }
+}
+
+// Rows of a [C][D] bf16 row tile times 2^(lg * (sgn * r + off)) in place
+// (rows >= nvalid become zero): the decay factors of a tile the feature map
+// does not touch.  Same work split as phi_tile.
+template <int C, int D, int T>
+__device__ __forceinline__ void scale_tile_rows_exp2(uint8_t* tile, int t, int nvalid, float lg,
+                                                     float sgn, float off) {
     using namespace sm100;
     constexpr int CH = D / 8;
     constexpr int PER = (C * CH) / T;
@@ -106,15 +146,14 @@ __device__ __forceinline__ void phi_tile_scaled(uint8_t* tile, int t, int nvalid
 #pragma unroll
     for (int i = 0; i < PER; ++i)
         x[i] = *reinterpret_cast<const uint4*>(tile + tile_chunk_off(C, row, q0 + i));
-    const bool zero = zero_tail && row >= nvalid;
-    const float sc = exp2f(lg * fmaf(sgn, float(row), off));
+    const float sc = row < nvalid ? exp2f(lg * fmaf(sgn, float(row), off)) : 0.f;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         uint32_t w[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const float2 f = unpack_bf16(w[k]);
-            w[k] = zero ? 0u : pack_bf16(phi_fast<PHI>(f.x) * sc, phi_fast<PHI>(f.y) * sc);
+            w[k] = pack_bf16(f.x * sc, f.y * sc);
         }
         x[i] = make_uint4(w[0], w[1], w[2], w[3]);
     }

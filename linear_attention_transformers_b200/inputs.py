@@ -73,6 +73,18 @@ WORKLOADS = {
         PHI_ELU1, 4),
 }
 
+# decayed (gated) training step on the timed shape: one decay factor per
+# head, gamma_h = 1 - 2^-(5 + 7 h / (H - 1)) (0.969 ... 0.99976), the fixed
+# per-head decays of retention-style linear attention
+DECAY_TRAIN = Workload("decay_causal_fwdbwd_b8h16n8192d64_bf16", 8, 16, 8192, 64, torch.bfloat16,
+                       True, PHI_ELU1, 6, backward=True)
+
+
+def decay_factors(H: int) -> list:
+    """Per-head decay factors 1 - 2^-(5 + 7 h / (H - 1)), h = 0..H-1."""
+    return [1.0 - 2.0 ** -(5.0 + 7.0 * h / max(H - 1, 1)) for h in range(H)]
+
+
 # recurrent decode: batch 256, 32 heads of 128, fp32 state updated in place
 DECODE = dict(B=256, H=32, D=128, steps=1024, seed=4, dtype=torch.bfloat16, phi=PHI_ELU1)
 # the same decode with grouped-query attention: 8 key/value heads, each

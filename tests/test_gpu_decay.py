@@ -173,3 +173,49 @@ def test_decay_chunked_matches_token_sequential_gamma_one():
     o0 = api.la_forward(q, k, v, True)
     torch.cuda.synchronize()
     compare(o1, o0.double().cpu().numpy(), torch.bfloat16, "gamma 1 vs plain")
+
+
+# ---------------------------------------------- tensor-core decayed backward
+# bf16, D = 64, every gamma >= 2^(-0.5), one segment per head (fewer than 4
+# chunks, or enough heads to fill the GPU): the pipelined dQ and dK/dV
+# passes with chunk-local decay factors.
+
+@pytest.mark.parametrize("N", [1, 100, 129, 300, 384])
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+@pytest.mark.parametrize("saved", [False, True])
+def test_decay_backward_chunked(N, phi, saved):
+    B, H, D = 2, 4, 64
+    q, k, v, dO = tensors(B, H, N, D, torch.bfloat16, seed=5 * N + 1, dO=True)
+    gm = np.array([CHUNK_GMIN[D], 0.9, 0.99, 1.0], dtype=np.float32)
+
+    def run():
+        if saved:
+            g = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+            o = api.la_forward_decay(q, k, v, gm, phi, g=g)
+            return api.la_backward_decay(q, k, v, dO, gm, phi, o=o, g=g)
+        return api.la_backward_decay(q, k, v, dO, gm, phi)
+
+    (dq, dk, dv), prof = _launched(run)
+    api.la_get_device_error()
+    assert "bwd_dq" in prof and "bwd_dkdv" in prof and "bwd_generic" not in prof, prof
+    rq, rk, rv = oracle.backward_decay(q, k, v, dO, gm.astype(np.float64), PHIS[phi])
+    compare(dq, rq, torch.bfloat16, "dq")
+    compare(dk, rk, torch.bfloat16, "dk")
+    compare(dv, rv, torch.bfloat16, "dv")
+
+
+@pytest.mark.parametrize("phi", ["elu1", "relu_eps"])
+def test_decay_backward_chunked_many_heads(phi):
+    # 128 heads keep one segment per head at N = 1000 (8 chunks, ragged
+    # tail), with the retention-style factors of the decayed training
+    # workload (the chunked range's lower edge is covered at small N above)
+    B, H, N, D = 4, 32, 1000, 64
+    q, k, v, dO = tensors(B, H, N, D, torch.bfloat16, seed=77, dO=True)
+    gm = np.array(inputs.decay_factors(H), dtype=np.float32)
+    (dq, dk, dv), prof = _launched(lambda: api.la_backward_decay(q, k, v, dO, gm, phi))
+    api.la_get_device_error()
+    assert "bwd_dq" in prof and "bwd_generic" not in prof, prof
+    rq, rk, rv = oracle.backward_decay(q, k, v, dO, gm.astype(np.float64), PHIS[phi])
+    compare(dq, rq, torch.bfloat16, "dq")
+    compare(dk, rk, torch.bfloat16, "dk")
+    compare(dv, rv, torch.bfloat16, "dv")
