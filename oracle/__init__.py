@@ -23,6 +23,12 @@ Functions (all arrays [B, H, N, D] contiguous, D innermost):
   decode_step_decay(S, z, q, k, v, gamma, phi) -> o  (updates S, z in place)
       the decayed (gated) recurrence S_i = gamma S_{i-1} + b_i v_i^T, z_i =
       gamma z_{i-1} + b_i with one gamma in [0, 1] per head (gamma [H])
+  favor_features(x, omega)                 -> phi(x) [..., m]  (Performer)
+  favor_features_backward(x, omega, dphi)  -> dx
+      the positive random features of the Performer (FAVOR+), phi(x) =
+      m^-1/2 exp(-|x|^2/2) [exp(w_1.x), ..., exp(w_m.x)], omega [m, D] the
+      random directions; with phi = PHI_IDENTITY the functions above then
+      take phi(q), phi(k) as their q, k
 """
 from __future__ import annotations
 
@@ -35,6 +41,7 @@ import numpy as np
 
 PHI_ELU1 = 0
 PHI_RELU_EPS = 1
+PHI_IDENTITY = 2  # inputs are feature vectors already (Performer features)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "la_oracle.c")
@@ -206,6 +213,33 @@ def decode_step_decay(S: np.ndarray, z: np.ndarray, q, k, v, gamma, phi: int = P
     _load().oracle_decode_step_decay(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
                                      _ptr(o), B, H, D, int(phi))
     return o
+
+
+# ------------------------------------------------ Performer FAVOR+ features
+# "Efficient Transformers Survey", Low-Rank Approximations, Performer:
+# phi(x) = m^-1/2 exp(-|x|^2/2) [exp(w_1^T x), ..., exp(w_m^T x)], w_i drawn
+# from N(0, I_d) (passed in as omega [m, D]); phi(q)^T phi(k) is an unbiased
+# estimate of exp(q^T k) (Proposition "Performer Approximation Quality").
+# The 1/sqrt(d) of softmax attention is the caller's pre-normalisation of q
+# and k (x = q / d^(1/4)), as the page states.
+
+def favor_features(x, omega) -> np.ndarray:
+    """phi(x) for x [..., D] and omega [m, D]: float64 [..., m]."""
+    x = _f64(x)
+    w = _f64(omega)
+    m = w.shape[0]
+    proj = x @ w.T                                   # w_i^T x
+    half_sq = 0.5 * (x * x).sum(axis=-1, keepdims=True)
+    return np.exp(proj - half_sq) / np.sqrt(m)
+
+
+def favor_features_backward(x, omega, dphi) -> np.ndarray:
+    """dx of sum(dphi * phi(x)): d phi_i / dx = phi_i (w_i - x), so
+    dx = sum_i dphi_i phi_i w_i - x sum_i dphi_i phi_i."""
+    x = _f64(x)
+    w = _f64(omega)
+    g = _f64(dphi) * favor_features(x, w)            # dphi_i phi_i
+    return g @ w - x * g.sum(axis=-1, keepdims=True)
 
 
 # ---------------------------------------------------- grouped key/value heads

@@ -23,7 +23,9 @@
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *   - phi is elementwise with m = D; id 0 is elu(x)+1 (alpha = 1), id 1 is
- *     max(x,0) + 1e-6.  The pages leave phi generic.
+ *     max(x,0) + 1e-6.  The pages leave phi generic.  Id 2 is the identity:
+ *     the inputs are feature vectors already (positive random features of
+ *     the Performer, computed by the caller; phi' = 1).
  *   - causal sums include the diagonal (j <= i).
  *   - no epsilon is added to the denominator; both maps are > 0.
  *   - phi'(0) is taken from the x <= 0 branch (exp(0) = 1 for elu+1, 0 for
@@ -67,11 +69,14 @@
 
 #define ORACLE_PHI_ELU1 0
 #define ORACLE_PHI_RELU_EPS 1
+#define ORACLE_PHI_IDENTITY 2
 
 static double phi_of(double x, int phi)
 {
     if (phi == ORACLE_PHI_ELU1)
         return x > 0.0 ? x + 1.0 : exp(x);
+    if (phi == ORACLE_PHI_IDENTITY)
+        return x;
     return (x > 0.0 ? x : 0.0) + 1e-6;
 }
 
@@ -79,6 +84,8 @@ static double dphi_of(double x, int phi)
 {
     if (phi == ORACLE_PHI_ELU1)
         return x > 0.0 ? 1.0 : exp(x);
+    if (phi == ORACLE_PHI_IDENTITY)
+        return 1.0;
     return x > 0.0 ? 1.0 : 0.0;
 }
 

@@ -25,7 +25,13 @@ the wrong feature-map branch) fails at least one of them:
 - decayed (gated) recurrence: gamma = 1 is the causal oracle; recurrence ==
   decayed quadratic form; gamma = 0 returns v; identical keys give the
   bias-corrected exponential moving average of v; the final state is the
-  gamma^(N-1-j)-weighted sum; finite differences; decode continues it.
+  gamma^(N-1-j)-weighted sum; finite differences; decode continues it;
+- Performer FAVOR+ features: phi(q).phi(k) is an unbiased estimate of
+  exp(q.k) (a large Monte Carlo sample within 5 standard errors); x = 0 and
+  a zero direction give closed forms; the feature backward matches finite
+  differences; with many features the attention approaches softmax
+  attention; the identity map is the quadratic form of the given features
+  and its backward matches finite differences.
 """
 import numpy as np
 import pytest
@@ -423,3 +429,91 @@ def test_decay_rejects_out_of_range_factors():
         oracle.forward_decay(q, q, q, np.array([0.5, 1.5]))
     with pytest.raises(ValueError):
         oracle.forward_decay(q, q, q, np.array([0.5]))
+
+
+# ------------------------------------------------ Performer FAVOR+ features
+# "Efficient Transformers Survey", Low-Rank Approximations, Performer, and
+# Proposition "Performer Approximation Quality".
+
+def test_favor_features_are_an_unbiased_estimate_of_the_exp_kernel():
+    # E[phi(q)^T phi(k)] = exp(q^T k): the sample mean over m draws sits
+    # within a few standard errors of the closed form
+    g = np.random.default_rng(400)
+    D, m = 8, 200000
+    q, k = g.standard_normal(D) * 0.3, g.standard_normal(D) * 0.3
+    w = g.standard_normal((m, D))
+    pq, pk = oracle.favor_features(q, w), oracle.favor_features(k, w)
+    est = float(pq @ pk)
+    samples = m * pq * pk                      # the m terms whose mean is est
+    se = samples.std() / np.sqrt(m)
+    assert abs(est - np.exp(q @ k)) < 5 * se, (est, np.exp(q @ k), se)
+
+
+def test_favor_features_closed_forms():
+    g = np.random.default_rng(401)
+    w = g.standard_normal((16, 4))
+    # x = 0: every feature is m^-1/2
+    np.testing.assert_allclose(oracle.favor_features(np.zeros(4), w), np.full(16, 0.25),
+                               rtol=1e-15)
+    # a zero direction gives exp(-|x|^2/2) / sqrt(m); features are positive
+    x = g.standard_normal(4)
+    w0 = np.vstack([np.zeros(4), w])
+    f = oracle.favor_features(x, w0)
+    np.testing.assert_allclose(f[0], np.exp(-0.5 * x @ x) / np.sqrt(17), rtol=1e-14)
+    assert (f > 0).all()
+
+
+def test_favor_features_backward_matches_finite_differences():
+    g = np.random.default_rng(402)
+    x, w, dphi = g.standard_normal((3, 5)) * 0.5, g.standard_normal((7, 5)), g.standard_normal((3, 7))
+    got = oracle.favor_features_backward(x, w, dphi)
+    h = 1e-6
+    ref = np.zeros_like(x)
+    for i in range(x.shape[0]):
+        for j in range(x.shape[1]):
+            xp, xm = x.copy(), x.copy()
+            xp[i, j] += h
+            xm[i, j] -= h
+            ref[i, j] = ((oracle.favor_features(xp, w) - oracle.favor_features(xm, w)) * dphi).sum() / (2 * h)
+    np.testing.assert_allclose(got, ref, rtol=1e-6, atol=1e-9)
+
+
+def test_identity_map_is_the_quadratic_form_of_the_given_features():
+    g = np.random.default_rng(403)
+    a, b = np.exp(g.standard_normal((1, 2, 9, 4))), np.exp(g.standard_normal((1, 2, 9, 4)))
+    v = g.standard_normal((1, 2, 9, 4))
+    for causal in (True, False):
+        o, _, _ = oracle.forward(a, b, v, causal, oracle.PHI_IDENTITY)
+        w = np.einsum("bhid,bhjd->bhij", a, b)
+        if causal:
+            w = np.tril(w)
+        ref = np.einsum("bhij,bhje->bhie", w, v) / w.sum(-1, keepdims=True)
+        np.testing.assert_allclose(o, ref, rtol=1e-12)
+
+
+def test_performer_attention_approaches_softmax_attention():
+    # with many features, linear attention on phi(q), phi(k) reproduces
+    # softmax attention with weights exp(q_i^T k_j) (here x = q / d^(1/4)
+    # is already applied: the inputs are the pre-normalised q, k)
+    g = np.random.default_rng(404)
+    N, D, m = 12, 4, 100000
+    q, k, v = (g.standard_normal((1, 1, N, D)) * 0.4 for _ in range(3))
+    w = g.standard_normal((m, D))
+    pq, pk = oracle.favor_features(q, w), oracle.favor_features(k, w)
+    # the core with m-dimensional features: the identity map's quadratic form
+    wts = np.tril(np.einsum("bhim,bhjm->bhij", pq, pk))
+    o_perf = np.einsum("bhij,bhje->bhie", wts, v) / wts.sum(-1, keepdims=True)
+    sm = np.tril(np.exp(np.einsum("bhid,bhjd->bhij", q, k)))
+    o_soft = np.einsum("bhij,bhje->bhie", sm, v) / sm.sum(-1, keepdims=True)
+    assert np.abs(o_perf - o_soft).max() < 0.02 * np.abs(o_soft).max()
+
+
+def test_identity_map_backward_matches_finite_differences():
+    g = np.random.default_rng(405)
+    shape = (1, 1, 6, 3)
+    q, k = np.exp(g.standard_normal(shape) * 0.5), np.exp(g.standard_normal(shape) * 0.5)
+    v, dO = g.standard_normal(shape), g.standard_normal(shape)
+    got = oracle.backward(q, k, v, dO, True, oracle.PHI_IDENTITY)
+    ref = fd_grads(q, k, v, dO, True, oracle.PHI_IDENTITY)
+    for a, b in zip(got, ref):
+        np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-9)
