@@ -33,7 +33,8 @@
  *     returns a status; nothing crosses the ABI as an exception or abort.
  *   - phi is LA_PHI_ELU1: elu(x)+1 (= x+1 for x > 0, exp(x) otherwise) or
  *     LA_PHI_RELU_EPS: max(x, 0) + 1e-6.  Both are > 0, so no epsilon is
- *     added to the denominator.
+ *     added to the denominator.  LA_PHI_IDENTITY takes q and k as feature
+ *     vectors already (the caller keeps them positive).
  *   - Supported head sizes D: 16, 32, 64, 128.  N, B, H >= 0 (a zero size
  *     launches nothing and returns LA_OK; a requested final state is then
  *     zero-filled).  B*H*N*D must stay below 2^62, N below 2^31.
@@ -72,7 +73,10 @@ typedef enum la_status {
 
 typedef enum la_phi {
     LA_PHI_ELU1 = 0,      /* elu(x) + 1 */
-    LA_PHI_RELU_EPS = 1   /* max(x, 0) + 1e-6 */
+    LA_PHI_RELU_EPS = 1,  /* max(x, 0) + 1e-6 */
+    LA_PHI_IDENTITY = 2   /* q, k are feature vectors already (positive: e.g. the
+                             output of la_favor_features); phi' = 1, so the
+                             backward returns the features' gradients */
 } la_phi;
 
 typedef enum la_dtype {
@@ -260,6 +264,33 @@ LA_EXPORT la_status la_decode_step_decay(float *S, float *z, const void *q, cons
                                          const void *v, void *o, const float *gamma,
                                          int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
                                          la_stream_t stream);
+
+/*
+ * Performer positive random features (FAVOR+; "Efficient Transformers
+ * Survey", Low-Rank Approximations, Performer, and Proposition "Performer
+ * Approximation Quality"):
+ *     phi(x) = m^-1/2 exp(-|x|^2 / 2) [exp(w_1^T x), ..., exp(w_m^T x)],
+ * an unbiased estimate of the exponential kernel: E[phi(q)^T phi(k)] =
+ * exp(q^T k).  x: [B, H, N, D] bf16 rows (q or k, pre-normalised by the
+ * caller: x = q / D^(1/4) gives softmax attention's exp(q^T k / sqrt(D)));
+ * omega: [m, D] bf16, row i = w_i, drawn by the caller from N(0, I_D) (the
+ * random numbers are an input; one draw shared by every head); phi out:
+ * [B, H, N, m] bf16.  The features feed la_forward / la_backward with phi =
+ * LA_PHI_IDENTITY (q = phi(q), k = phi(k); values v of head size m).
+ * la_favor_features_backward returns dx [B, H, N, D] of sum(dphi * phi(x))
+ * given x, omega and dphi [B, H, N, m]: dx = sum_i dphi_i phi_i w_i -
+ * x sum_i dphi_i phi_i, with phi recomputed from x in float32 (the stored
+ * features are not read).  Supported: bf16 with m == D in {64, 128} (else
+ * LA_ERR_UNSUPPORTED); float32 accumulation, outputs rounded to bf16 once.
+ * No workspace.
+ */
+LA_EXPORT la_status la_favor_features(const void *x, const void *omega, void *phi, int64_t B,
+                                      int64_t H, int64_t N, int64_t D, int64_t m, la_dtype dt,
+                                      la_stream_t stream);
+LA_EXPORT la_status la_favor_features_backward(const void *x, const void *omega,
+                                               const void *dphi, void *dx, int64_t B, int64_t H,
+                                               int64_t N, int64_t D, int64_t m, la_dtype dt,
+                                               la_stream_t stream);
 
 /* Static English text for a status code (never NULL). */
 LA_EXPORT const char *la_status_string(la_status status);

@@ -14,6 +14,8 @@ raises ``RuntimeError``.
     la_forward_decay(q, k, v, gamma, phi="elu1", ...)        -> o [, S, z]  (causal)
     la_backward_decay(q, k, v, dO, gamma, phi="elu1", ...)   -> dq, dk, dv
     la_decode_step_decay(S, z, q, k, v, gamma, ...)          -> o   (S, z in place)
+    la_favor_features(x, omega)                              -> phi(x)  (Performer FAVOR+)
+    la_favor_features_backward(x, omega, dphi)               -> dx
     la_get_device_error(stream=None)                         -> raises on a device timeout
     LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
 
@@ -21,6 +23,9 @@ k and v may have fewer heads than q (grouped-query / multi-query attention:
 Hkv key/value heads shared by groups of H / Hkv query heads); the group size
 is read from their shapes.  The *_decay calls take one decay factor per head
 (gamma, H host values in [0, 1]): S_i = gamma S_{i-1} + phi(k_i) v_i^T.
+With phi="identity" q and k are taken as feature vectors already (for
+example la_favor_features(q, omega)), and the backward returns their
+gradients.
 """
 from __future__ import annotations
 
@@ -41,7 +46,7 @@ LA_F32 = 0
 LA_BF16 = 1
 LA_OP_FORWARD = 0
 LA_OP_BACKWARD = 1
-PHI = {"elu1": 0, "relu_eps": 1, 0: 0, 1: 1}
+PHI = {"elu1": 0, "relu_eps": 1, "identity": 2, 0: 0, 1: 1, 2: 2}
 DTYPE = {torch.float32: LA_F32, torch.bfloat16: LA_BF16}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -111,6 +116,11 @@ def load_library(path: str | None = None):
         lib.la_backward_decay.restype = ci
         lib.la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, vp, fp, i64, i64, i64, ci, ci, vp]
         lib.la_decode_step_decay.restype = ci
+        lib.la_favor_features.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, ci, vp]
+        lib.la_favor_features.restype = ci
+        lib.la_favor_features_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ci,
+                                                   vp]
+        lib.la_favor_features_backward.restype = ci
         lib.la_status_string.argtypes = [ci]
         lib.la_status_string.restype = ctypes.c_char_p
         lib.la_last_error.argtypes = []
@@ -161,7 +171,7 @@ def _ptr(t) -> int | None:
 
 def _phi(phi) -> int:
     if phi not in PHI:
-        raise ValueError(f"phi must be 'elu1' or 'relu_eps', got {phi!r}")
+        raise ValueError(f"phi must be 'elu1', 'relu_eps' or 'identity', got {phi!r}")
     return PHI[phi]
 
 
@@ -447,6 +457,50 @@ def la_decode_step_decay(S, z, q, k, v, gamma, phi="elu1", o=None, stream=None):
                                   D, DTYPE[q.dtype], _phi(phi), _stream_handle(stream))
     _check("la_decode_step_decay", st)
     return o
+
+
+# ------------------------------------------------ Performer FAVOR+ features
+def _check_omega(name, x, omega):
+    m = x.shape[-1]
+    if (omega.dtype != x.dtype or omega.device != x.device or omega.dim() != 2
+            or omega.shape[1] != x.shape[-1] or not omega.is_contiguous()):
+        raise ValueError(f"{name}: omega must be a contiguous [m, D] tensor like x")
+    return int(omega.shape[0]) if omega.dim() == 2 else m
+
+
+def la_favor_features(x, omega, out=None, stream=None):
+    """phi(x) = m^-1/2 exp(omega x - |x|^2/2) for x [B, H, N, D] (bf16) and
+    omega [m, D]: the Performer's positive random features [B, H, N, m]."""
+    lib = load_library()
+    _check_qkv("la_favor_features", x)
+    if x.dim() != 4:
+        raise ValueError("la_favor_features: x must be [B, H, N, D]")
+    m = _check_omega("la_favor_features", x, omega)
+    B, H, N, D = x.shape
+    out = torch.empty((B, H, N, m), dtype=x.dtype, device=x.device) if out is None else out
+    if tuple(out.shape) != (B, H, N, m) or out.dtype != x.dtype or not out.is_contiguous():
+        raise ValueError("la_favor_features: out must be contiguous [B, H, N, m] like x")
+    st = lib.la_favor_features(_ptr(x), _ptr(omega), _ptr(out), B, H, N, D, m, DTYPE[x.dtype],
+                               _stream_handle(stream))
+    _check("la_favor_features", st)
+    return out
+
+
+def la_favor_features_backward(x, omega, dphi, dx=None, stream=None):
+    """dx of sum(dphi * phi(x)) given x, omega and dphi (phi recomputed)."""
+    lib = load_library()
+    _check_qkv("la_favor_features_backward", x)
+    m = _check_omega("la_favor_features_backward", x, omega)
+    _check_qkv("la_favor_features_backward", dphi)
+    B, H, N, D = x.shape
+    if tuple(dphi.shape) != (B, H, N, m) or dphi.dtype != x.dtype:
+        raise ValueError("la_favor_features_backward: dphi must be [B, H, N, m] like x")
+    dx = torch.empty_like(x) if dx is None else dx
+    _check_qkv("la_favor_features_backward", x, dx)
+    st = lib.la_favor_features_backward(_ptr(x), _ptr(omega), _ptr(dphi), _ptr(dx), B, H, N, D, m,
+                                        DTYPE[x.dtype], _stream_handle(stream))
+    _check("la_favor_features_backward", st)
+    return dx
 
 
 def la_get_device_error(stream=None) -> None:

@@ -14,8 +14,10 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "la_chunk_bwd.cuh"
+#include "la_favor.cuh"
 #include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
@@ -52,7 +54,8 @@ la_status check_sizes(int64_t B, int64_t H, int64_t N, int64_t D) {
 
 la_status check_enums(la_dtype dt, la_phi phi) {
     if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
-    if (phi != LA_PHI_ELU1 && phi != LA_PHI_RELU_EPS) return LA_ERR_INVALID_ARG;
+    if (phi != LA_PHI_ELU1 && phi != LA_PHI_RELU_EPS && phi != LA_PHI_IDENTITY)
+        return LA_ERR_INVALID_ARG;
     return LA_OK;
 }
 
@@ -680,6 +683,35 @@ la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const v
     return launch_group_sum<__nv_bfloat16>(dv_p, dv, heads / G, N * D, G, st);
 }
 
+// ------------------------------------------------------------ FAVOR+ features
+template <int D, bool BWD>
+la_status launch_favor(const void* x, const void* omega, const void* dphi, void* out,
+                       int64_t heads, int64_t N, cudaStream_t st) {
+    using Cfg = la::FavorCfg<D, BWD>;
+    la::FavorParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_x, x, heads, N, D, Cfg::R) ||
+        !make_qkv_map(&prm.tm_w, omega, 1, D, D, D))
+        return LA_ERR_CUDA;
+    if (!BWD && !make_qkv_map(&prm.tm_phi, out, heads, N, D, Cfg::R)) return LA_ERR_CUDA;
+    if (BWD && (!make_qkv_map(&prm.tm_dphi, dphi, heads, N, D, Cfg::R) ||
+                !make_qkv_map(&prm.tm_dx, out, heads, N, D, Cfg::R)))
+        return LA_ERR_CUDA;
+    const int64_t tph = (N + Cfg::R - 1) / Cfg::R;
+    if (heads * tph >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
+    prm.tiles_per_head = int(tph);
+    prm.ntiles = int(heads * tph);
+    prm.log_scale = -0.5f * logf(float(D));
+    auto kern = la::favor_kernel<D, BWD>;
+    if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Cfg::SMEM))
+        return cuda_fail("cudaFuncSetAttribute", e);
+    const unsigned grid = unsigned(std::min<int64_t>(prm.ntiles, num_sms()));
+    la::LaunchScope scope(BWD ? "favor_bwd" : "favor_fwd", st);
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(prm);
+    return launch_status();
+}
+
 // ------------------------------------------------------------ generic path
 template <typename T, int PHI>
 la_status run_fwd_generic(const void* q, const void* k, const void* v, void* o, float* S_out,
@@ -768,15 +800,25 @@ la_status run_decode(float* S, float* z, const void* q, const void* k, const voi
     return launch_status();
 }
 
+// fn(std::integral_constant<int, PHI>) for the call's feature map
+template <typename Fn>
+la_status with_phi_map(la_phi phi, Fn&& fn) {
+    if (phi == LA_PHI_ELU1) return fn(std::integral_constant<int, PHI_ELU1>{});
+    if (phi == LA_PHI_RELU_EPS) return fn(std::integral_constant<int, PHI_RELU_EPS>{});
+    return fn(std::integral_constant<int, la::PHI_IDENTITY>{});
+}
+
 // dtype x phi dispatch helper
 template <template <typename, int> class F, typename... Args>
 la_status dispatch(la_dtype dt, la_phi phi, Args... args) {
     if (dt == LA_F32) {
-        return phi == LA_PHI_ELU1 ? F<float, PHI_ELU1>::run(args...)
-                                  : F<float, PHI_RELU_EPS>::run(args...);
+        return phi == LA_PHI_ELU1       ? F<float, PHI_ELU1>::run(args...)
+               : phi == LA_PHI_RELU_EPS ? F<float, PHI_RELU_EPS>::run(args...)
+                                        : F<float, la::PHI_IDENTITY>::run(args...);
     }
-    return phi == LA_PHI_ELU1 ? F<__nv_bfloat16, PHI_ELU1>::run(args...)
-                              : F<__nv_bfloat16, PHI_RELU_EPS>::run(args...);
+    return phi == LA_PHI_ELU1       ? F<__nv_bfloat16, PHI_ELU1>::run(args...)
+           : phi == LA_PHI_RELU_EPS ? F<__nv_bfloat16, PHI_RELU_EPS>::run(args...)
+                                    : F<__nv_bfloat16, la::PHI_IDENTITY>::run(args...);
 }
 
 template <typename T, int PHI>
@@ -975,11 +1017,11 @@ la_status forward_impl(const void* q, const void* k, const void* v, void* o, flo
         char* ws = static_cast<char*>(workspace);
         void* pq = phi_fused ? phi_q_out : nullptr;
         void* pk = phi_fused ? phi_k_out : nullptr;
-        s = phi == LA_PHI_ELU1
-                ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads, N,
-                                              D, causal ? 1 : 0, plan, ws, st, G, dec)
-                : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o, S_out, z_out, g_out, pq, pk, heads,
-                                                  N, D, causal ? 1 : 0, plan, ws, st, G, dec);
+        s = with_phi_map(phi, [&](auto P) {
+            return run_fwd_chunked_d<decltype(P)::value>(q, k, v, o, S_out, z_out, g_out, pq, pk,
+                                                         heads, N, D, causal ? 1 : 0, plan, ws,
+                                                         st, G, dec);
+        });
     } else {
         s = dispatch<FwdOp>(dt, phi, q, k, v, o, S_out, z_out, g_out, heads, N, D,
                             causal ? 1 : 0, st, G, &dec);
@@ -1067,24 +1109,20 @@ la_status backward_impl(const void* q, const void* k, const void* v, const void*
             const FwdPlan fp = plan_fwd(B, H, N, D, causal ? 1 : 0, dt);
             void* o_ws = wsp + bp.o_off;
             float* g_ws = reinterpret_cast<float*>(wsp + bp.g_off);
-            s = phi == LA_PHI_ELU1
-                    ? run_fwd_chunked_d<PHI_ELU1>(q, k, v, o_ws, nullptr, nullptr, g_ws, nullptr,
-                                                  nullptr, heads, N, D, causal ? 1 : 0, fp,
-                                                  wsp + bp.fwd_off, st, G, dec)
-                    : run_fwd_chunked_d<PHI_RELU_EPS>(q, k, v, o_ws, nullptr, nullptr, g_ws,
-                                                      nullptr, nullptr, heads, N, D,
-                                                      causal ? 1 : 0, fp, wsp + bp.fwd_off, st, G,
-                                                      dec);
+            s = with_phi_map(phi, [&](auto P) {
+                return run_fwd_chunked_d<decltype(P)::value>(
+                    q, k, v, o_ws, nullptr, nullptr, g_ws, nullptr, nullptr, heads, N, D,
+                    causal ? 1 : 0, fp, wsp + bp.fwd_off, st, G, dec);
+            });
             if (s != LA_OK) return s;
             o = o_ws;
             g = g_ws;
         }
-        return phi == LA_PHI_ELU1
-                   ? run_bwd_chunked_d<PHI_ELU1>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                 heads, N, D, causal ? 1 : 0, bp, wsp, st, G, dec)
-                   : run_bwd_chunked_d<PHI_RELU_EPS>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv,
-                                                     heads, N, D, causal ? 1 : 0, bp, wsp, st, G,
-                                                     dec);
+        return with_phi_map(phi, [&](auto P) {
+            return run_bwd_chunked_d<decltype(P)::value>(q, k, v, dO, o, g, phi_q, phi_k, dq, dk,
+                                                         dv, heads, N, D, causal ? 1 : 0, bp, wsp,
+                                                         st, G, dec);
+        });
     }
     const BwdWorkspace w = plan_bwd(B, H, N, D, G);
     char* ws = static_cast<char*>(workspace);
@@ -1191,6 +1229,47 @@ la_status la_decode_step(float* S, float* z, const void* q, const void* k, const
                          void* o, int64_t B, int64_t H, int64_t D, la_dtype dt, la_phi phi,
                          la_stream_t stream) {
     return la_decode_step_gqa(S, z, q, k, v, o, B, H, H, D, dt, phi, stream);
+}
+
+namespace {
+
+// FAVOR+ sizes: bf16, m = D in {64, 128}
+la_status check_favor(int64_t B, int64_t H, int64_t N, int64_t D, int64_t m, la_dtype dt) {
+    if (B < 0 || H < 0 || N < 0 || D <= 0 || m <= 0) return LA_ERR_INVALID_ARG;
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (dt != LA_BF16 || m != D || (D != 64 && D != 128)) return LA_ERR_UNSUPPORTED;
+    return check_sizes(B, H, N, D);
+}
+
+}  // namespace
+
+la_status la_favor_features(const void* x, const void* omega, void* phi, int64_t B, int64_t H,
+                            int64_t N, int64_t D, int64_t m, la_dtype dt, la_stream_t stream) {
+    la_status s;
+    if ((s = check_favor(B, H, N, D, m, dt)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(x)) || (s = check_ptr(omega)) || (s = check_ptr(phi))) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return D == 64 ? launch_favor<64, false>(x, omega, nullptr, phi, heads, N, st)
+                   : launch_favor<128, false>(x, omega, nullptr, phi, heads, N, st);
+}
+
+la_status la_favor_features_backward(const void* x, const void* omega, const void* dphi,
+                                     void* dx, int64_t B, int64_t H, int64_t N, int64_t D,
+                                     int64_t m, la_dtype dt, la_stream_t stream) {
+    la_status s;
+    if ((s = check_favor(B, H, N, D, m, dt)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(x)) || (s = check_ptr(omega)) || (s = check_ptr(dphi)) ||
+        (s = check_ptr(dx)))
+        return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    return D == 64 ? launch_favor<64, true>(x, omega, dphi, dx, heads, N, st)
+                   : launch_favor<128, true>(x, omega, dphi, dx, heads, N, st);
 }
 
 uint64_t la_launch_count(void) { return la::profiler().launches.load(); }

@@ -130,6 +130,7 @@ struct Bwd2Cfg {
 template <int PHI>
 __device__ __forceinline__ float dphi_from_phi(float a) {
     if (PHI == PHI_ELU1) return fminf(a, 1.f);
+    if (PHI == PHI_IDENTITY) return 1.f;
     const float floor_val = __bfloat162float(__float2bfloat16_rn(1e-6f));
     return a > floor_val ? 1.f : 0.f;
 }
@@ -141,6 +142,7 @@ __device__ __forceinline__ float dphi_from_phi(float a) {
 template <int PHI>
 __device__ __forceinline__ float dphi_from_scaled_phi(float b, float beta, float binv) {
     if (PHI == PHI_ELU1) return fminf(b * binv, 1.f);
+    if (PHI == PHI_IDENTITY) return 1.f;
     return b > __bfloat162float(__float2bfloat16_rn(1e-6f * beta)) ? 1.f : 0.f;
 }
 

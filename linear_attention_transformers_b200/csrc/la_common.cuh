@@ -8,7 +8,7 @@
 
 namespace la {
 
-enum : int { PHI_ELU1 = 0, PHI_RELU_EPS = 1 };
+enum : int { PHI_ELU1 = 0, PHI_RELU_EPS = 1, PHI_IDENTITY = 2 };
 
 // Error word for bounded waits (set by a kernel that gave up waiting).  The
 // library is one translation unit, so the definition lives here.
@@ -18,17 +18,21 @@ __device__ unsigned int g_device_error = 0;
 // phi is elementwise: elu(x)+1 (x+1 for x > 0, exp(x) otherwise) or
 // max(x,0)+1e-6.  The pages leave phi generic ("Efficient Transformers
 // Survey", Proposition "Linear Attention via Kernel Decomposition": any
-// phi: R^d -> R^m); m = D here.
+// phi: R^d -> R^m); m = D here.  PHI_IDENTITY: the inputs are feature
+// vectors already (the Performer's positive random features, computed by
+// la_favor_features), phi(x) = x and phi' = 1.
 
 // Accurate variant (libm expf) for the reference-quality kernels.
 template <int PHI>
 __device__ __forceinline__ float phi_exact(float x) {
     if (PHI == PHI_ELU1) return x > 0.f ? x + 1.f : expf(x);
+    if (PHI == PHI_IDENTITY) return x;
     return fmaxf(x, 0.f) + 1e-6f;
 }
 template <int PHI>
 __device__ __forceinline__ float dphi_exact(float x) {
     if (PHI == PHI_ELU1) return x > 0.f ? 1.f : expf(x);
+    if (PHI == PHI_IDENTITY) return 1.f;
     return x > 0.f ? 1.f : 0.f;
 }
 
@@ -48,11 +52,13 @@ __device__ __forceinline__ float exp_fast(float x) {
 template <int PHI>
 __device__ __forceinline__ float phi_fast(float x) {
     if (PHI == PHI_ELU1) return x > 0.f ? x + 1.f : exp_fast(x);
+    if (PHI == PHI_IDENTITY) return x;
     return fmaxf(x, 0.f) + 1e-6f;
 }
 template <int PHI>
 __device__ __forceinline__ float dphi_fast(float x) {
     if (PHI == PHI_ELU1) return x > 0.f ? 1.f : exp_fast(x);
+    if (PHI == PHI_IDENTITY) return 1.f;
     return x > 0.f ? 1.f : 0.f;
 }
 

@@ -150,6 +150,13 @@ def make_decode_gqa_inputs(B, H, Hkv, D, steps, seed, dtype=torch.bfloat16, devi
     return tuple(out)
 
 
+def make_favor_directions(m, D, seed, dtype=torch.bfloat16, device="cpu"):
+    """The Performer's random directions omega [m, D]: independent N(0, 1)
+    entries (generator seed + 2000), cast to ``dtype``."""
+    g = _gen(device, seed + 2000)
+    return torch.randn((m, D), generator=g, device=device, dtype=torch.float32).to(dtype)
+
+
 def make_decode_inputs(B, H, D, steps, seed, dtype=torch.bfloat16, device="cpu"):
     """q, k, v of shape [steps, B, H, D] for ``steps`` recurrent decode steps."""
     g = _gen(device, seed + 1000)

@@ -147,3 +147,27 @@ def test_decay_factors_are_validated_before_launch(lib):
         api.LA_ERR_INVALID_ARG
     assert lib.la_workspace_size_decay(api.LA_OP_BACKWARD, 2, 4, 1000, 64, api.LA_BF16) >= \
         lib.la_workspace_size(api.LA_OP_BACKWARD, 2, 4, 1000, 64, 1, api.LA_BF16)
+
+
+def test_favor_sizes_are_validated_before_launch(lib):
+    p = FAKE
+    # m != D, float32, D = 32: not offered
+    assert lib.la_favor_features(p, p, p, 1, 2, 8, 64, 128, api.LA_BF16, None) == \
+        api.LA_ERR_UNSUPPORTED
+    assert lib.la_favor_features(p, p, p, 1, 2, 8, 64, 64, api.LA_F32, None) == \
+        api.LA_ERR_UNSUPPORTED
+    assert lib.la_favor_features(p, p, p, 1, 2, 8, 32, 32, api.LA_BF16, None) == \
+        api.LA_ERR_UNSUPPORTED
+    assert lib.la_favor_features(p, p, p, -1, 2, 8, 64, 64, api.LA_BF16, None) == \
+        api.LA_ERR_INVALID_ARG
+    assert lib.la_favor_features(p, p, None, 1, 2, 8, 64, 64, api.LA_BF16, None) == \
+        api.LA_ERR_INVALID_ARG
+    assert lib.la_favor_features_backward(p, p, p, None, 1, 2, 8, 128, 128, api.LA_BF16,
+                                          None) == api.LA_ERR_INVALID_ARG
+    # nothing to do
+    assert lib.la_favor_features(p, p, p, 1, 2, 0, 64, 64, api.LA_BF16, None) == api.LA_OK
+    # the identity feature map is a valid enum
+    assert lib.la_forward(p, p, p, None, None, None, None, None, None, 1, 1, 8, 64, api.LA_BF16,
+                          1, 2, None, 0, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_forward(p, p, p, p, None, None, None, None, None, 1, 1, 8, 64, api.LA_BF16,
+                          1, 3, None, 0, None) == api.LA_ERR_INVALID_ARG
