@@ -292,6 +292,107 @@ LA_EXPORT la_status la_favor_features_backward(const void *x, const void *omega,
                                                int64_t N, int64_t D, int64_t m, la_dtype dt,
                                                la_stream_t stream);
 
+/*
+ * Sequence split across ranks (one process per GPU): the N tokens of every
+ * head are cut into consecutive shards, rank r holding shard r.  S and z are
+ * sums over tokens ("Efficient Transformers Survey", Proposition "Linear
+ * Attention via Kernel Decomposition", Statement; "Why It Matters": the
+ * state is carried along the sequence), so a rank's outputs need only one
+ * state record per head from the other ranks: the sum over the shards
+ * before it (causal) or over all shards (non-causal); the backward needs
+ * the same for the centred key features, and the sum of the query-side
+ * state over the shards after it (causal) or all shards.  The calls below
+ * are a rank's local steps; the caller moves the records between ranks
+ * (an all-gather of one record per head per rank, e.g. NCCL) and forms the
+ * incoming sums with la_state_range_sum.  Per rank and call order:
+ *
+ *   forward:  la_state_local(k, v, centred=0) -> rec;  all-gather rec;
+ *             la_state_range_sum(lo=0, hi=rank or P) -> in;
+ *             la_forward_sp(q, k, v, in) -> o, g.
+ *   backward: la_state_local(k, v, centred=1) -> rec;  all-gather;
+ *             la_state_range_sum(0, rank or P) -> in;
+ *             la_backward_sp_dq(..., o, g, in) -> dq, rec2;  all-gather rec2;
+ *             la_state_range_sum(rank+1 or 0, P) -> in2;
+ *             la_backward_sp_dkdv(..., g, in2) -> dk, dv.
+ *
+ * A state record is float32 [D*D + D]: S [D][D] (row = key feature) then z
+ * [D]; a record array is [B, H, D*D + D].  Tensors are this rank's shard,
+ * [B, H, N, D] with N its token count.  Tensor-core path only: bf16 with
+ * D = 64 or 128 (else LA_ERR_UNSUPPORTED), one key/value head per query
+ * head, no decay.  Workspace: la_workspace_size_sp(LA_OP_FORWARD, ...) for
+ * la_state_local and la_forward_sp, la_workspace_size_sp(LA_OP_BACKWARD,
+ * ...) (which also serves la_state_local) for the two backward calls.
+ */
+LA_EXPORT size_t la_workspace_size_sp(la_op op, int64_t B, int64_t H, int64_t N, int64_t D,
+                                      int causal, la_dtype dt);
+
+/*
+ * This shard's state record per head, written to state_out [B, H, D*D+D]:
+ * S = sum_j (phi(k_j) - c) v_j^T, z = sum_j (phi(k_j) - c), with c = 0, or
+ * with centred != 0 the constant the backward's dQ products subtract from
+ * the key features (1 for elu+1, 0 otherwise; la_backward's centred
+ * features).  N = 0 writes zeros.  Errors as la_forward.
+ */
+LA_EXPORT la_status la_state_local(const void *k, const void *v, float *state_out, int64_t B,
+                                   int64_t H, int64_t N, int64_t D, la_dtype dt, la_phi phi,
+                                   int centred, void *workspace, size_t workspace_bytes,
+                                   la_stream_t stream);
+
+/*
+ * out[h] = sum over p in [lo, hi) of states[p][h], added in increasing p
+ * (bitwise reproducible); states: [P, B, H, D*D+D] float32 (the records of
+ * ranks 0..P-1 in rank order, as an all-gather leaves them), out: [B, H,
+ * D*D+D].  lo == hi writes zeros (rank 0's causal prefix).  0 <= lo <= hi
+ * <= P, else LA_ERR_INVALID_ARG.  out must not alias states.
+ */
+LA_EXPORT la_status la_state_range_sum(const float *states, int64_t P, int64_t lo, int64_t hi,
+                                       float *out, int64_t B, int64_t H, int64_t D,
+                                       la_stream_t stream);
+
+/*
+ * la_forward on this shard starting from state_in [B, H, D*D+D]: causal,
+ * the sum of the states of the shards before (outputs then equal those of
+ * the whole sequence); non-causal, the sum over every shard (the local
+ * tokens' own state included).  o: [B, H, N, D]; g_out (nullable) float32
+ * [B, H, N] the denominators; state_out (nullable, causal only) receives
+ * state_in plus this shard's state, which is the next shard's state_in.
+ */
+LA_EXPORT la_status la_forward_sp(const void *q, const void *k, const void *v, void *o,
+                                  const float *state_in, float *state_out, float *g_out,
+                                  int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt,
+                                  int causal, la_phi phi, void *workspace,
+                                  size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Backward, first local step: dq of this shard, given the forward's o and g
+ * (required) and state_in, the centred record sum of la_state_local(...,
+ * centred=1) over the shards before (causal) or every shard (non-causal).
+ * state_out [B, H, D*D+D] receives this shard's query-side record, R =
+ * sum_i phi(q_i) du_i^T and r = sum_i phi(q_i) dg_i with du_i = dO_i / g_i
+ * and dg_i = -(dO_i . o_i) / g_i (the suffix state of the dK, dV products).
+ * The workspace keeps dg and the per-block records for la_backward_sp_dkdv:
+ * pass the same workspace, unchanged, to that call.
+ */
+LA_EXPORT la_status la_backward_sp_dq(const void *q, const void *k, const void *v,
+                                      const void *dO, const void *o, const float *g,
+                                      const float *state_in, void *dq, float *state_out,
+                                      int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt,
+                                      int causal, la_phi phi, void *workspace,
+                                      size_t workspace_bytes, la_stream_t stream);
+
+/*
+ * Backward, second local step: dk, dv of this shard, given g and state_in,
+ * the sum of la_backward_sp_dq's state_out over the shards after this one
+ * (causal) or every shard (non-causal), and the workspace la_backward_sp_dq
+ * filled.
+ */
+LA_EXPORT la_status la_backward_sp_dkdv(const void *q, const void *k, const void *v,
+                                        const void *dO, const float *g, const float *state_in,
+                                        void *dk, void *dv, int64_t B, int64_t H, int64_t N,
+                                        int64_t D, la_dtype dt, int causal, la_phi phi,
+                                        void *workspace, size_t workspace_bytes,
+                                        la_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 LA_EXPORT const char *la_status_string(la_status status);
 

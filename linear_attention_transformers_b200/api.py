@@ -16,6 +16,9 @@ raises ``RuntimeError``.
     la_decode_step_decay(S, z, q, k, v, gamma, ...)          -> o   (S, z in place)
     la_favor_features(x, omega)                              -> phi(x)  (Performer FAVOR+)
     la_favor_features_backward(x, omega, dphi)               -> dx
+    la_state_local / la_state_range_sum / la_forward_sp /
+    la_backward_sp_dq / la_backward_sp_dkdv                  (one rank's steps of a
+                                                              sequence split across ranks)
     la_get_device_error(stream=None)                         -> raises on a device timeout
     LinearAttention.apply(q, k, v, causal, phi)              -> o   (torch autograd)
 
@@ -121,6 +124,21 @@ def load_library(path: str | None = None):
         lib.la_favor_features_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ci,
                                                    vp]
         lib.la_favor_features_backward.restype = ci
+        lib.la_workspace_size_sp.argtypes = [ci, i64, i64, i64, i64, ci, ci]
+        lib.la_workspace_size_sp.restype = sz
+        lib.la_state_local.argtypes = [vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp, sz, vp]
+        lib.la_state_local.restype = ci
+        lib.la_state_range_sum.argtypes = [vp, i64, i64, i64, vp, i64, i64, i64, vp]
+        lib.la_state_range_sum.restype = ci
+        lib.la_forward_sp.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, ci, ci, ci,
+                                      vp, sz, vp]
+        lib.la_forward_sp.restype = ci
+        lib.la_backward_sp_dq.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                          ci, ci, ci, vp, sz, vp]
+        lib.la_backward_sp_dq.restype = ci
+        lib.la_backward_sp_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                            ci, ci, ci, vp, sz, vp]
+        lib.la_backward_sp_dkdv.restype = ci
         lib.la_status_string.argtypes = [ci]
         lib.la_status_string.restype = ctypes.c_char_p
         lib.la_last_error.argtypes = []
@@ -501,6 +519,136 @@ def la_favor_features_backward(x, omega, dphi, dx=None, stream=None):
                                         DTYPE[x.dtype], _stream_handle(stream))
     _check("la_favor_features_backward", st)
     return dx
+
+
+# ------------------------------------------------ sequence split across ranks
+def la_workspace_size_sp(op: int, B: int, H: int, N: int, D: int, causal: bool,
+                         dtype: torch.dtype) -> int:
+    return int(load_library().la_workspace_size_sp(int(op), B, H, N, D, int(bool(causal)),
+                                                   DTYPE[dtype]))
+
+
+def _workspace_sp(op, x, causal, workspace):
+    B, H, N, D = x.shape
+    need = la_workspace_size_sp(op, B, H, N, D, causal, x.dtype)
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < need:
+            raise ValueError(f"workspace smaller than the {need} bytes needed")
+        return workspace, workspace.numel() * workspace.element_size()
+    if need == 0:
+        return None, 0
+    workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    return workspace, need
+
+
+def _state_records(name, t, B, H, D, device, lead=()):
+    shape = (*lead, B, H, D * D + D)
+    if t.dtype != torch.float32 or tuple(t.shape) != shape or not t.is_contiguous() \
+            or t.device != device:
+        raise ValueError(f"{name}: state records must be contiguous float32 {shape}")
+
+
+def la_state_local(k, v, phi="elu1", centred=False, out=None, workspace=None, stream=None):
+    """This shard's state record per head, [B, H, D*D + D] float32: S (row =
+    key feature) then z, of phi(k) - c (c = 0, or the backward's centring
+    constant with ``centred``)."""
+    lib = load_library()
+    _check_qkv("la_state_local", k, v)
+    B, H, N, D = k.shape
+    out = torch.empty((B, H, D * D + D), dtype=torch.float32, device=k.device) \
+        if out is None else out
+    _state_records("la_state_local", out, B, H, D, k.device)
+    ws, ws_bytes = _workspace_sp(LA_OP_FORWARD, k, True, workspace)
+    st = lib.la_state_local(_ptr(k), _ptr(v), _ptr(out), B, H, N, D, DTYPE[k.dtype], _phi(phi),
+                            int(bool(centred)), _ptr(ws), ws_bytes, _stream_handle(stream))
+    _check("la_state_local", st)
+    return out
+
+
+def la_state_range_sum(states, lo: int, hi: int, out=None, stream=None):
+    """Sum of the records of ranks lo..hi-1 from gathered records [P, B, H, R]."""
+    lib = load_library()
+    if states.dim() != 4:
+        raise ValueError("la_state_range_sum: states must be [P, B, H, D*D + D]")
+    P, B, H, R = states.shape
+    D = int(round((-1 + (1 + 4 * R) ** 0.5) / 2))
+    _state_records("la_state_range_sum", states, B, H, D, states.device, (P,))
+    out = torch.empty((B, H, R), dtype=torch.float32, device=states.device) if out is None else out
+    _state_records("la_state_range_sum", out, B, H, D, states.device)
+    st = lib.la_state_range_sum(_ptr(states), P, int(lo), int(hi), _ptr(out), B, H, D,
+                                _stream_handle(stream))
+    _check("la_state_range_sum", st)
+    return out
+
+
+def la_forward_sp(q, k, v, state_in, causal: bool = True, phi="elu1", o=None, g=None,
+                  state_out=None, workspace=None, stream=None):
+    """la_forward on this rank's shard starting from ``state_in`` (the records
+    of the shards before it, causal; of every shard, non-causal)."""
+    lib = load_library()
+    _check_qkv("la_forward_sp", q, k, v)
+    B, H, N, D = q.shape
+    _state_records("la_forward_sp", state_in, B, H, D, q.device)
+    o = torch.empty_like(q) if o is None else o
+    _check_qkv("la_forward_sp", q, o)
+    if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
+                          or not g.is_contiguous()):
+        raise ValueError("la_forward_sp: g must be contiguous float32 [B, H, N]")
+    if state_out is not None:
+        _state_records("la_forward_sp", state_out, B, H, D, q.device)
+    ws, ws_bytes = _workspace_sp(LA_OP_FORWARD, q, causal, workspace)
+    st = lib.la_forward_sp(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(state_in), _ptr(state_out),
+                           _ptr(g), B, H, N, D, DTYPE[q.dtype], int(bool(causal)), _phi(phi),
+                           _ptr(ws), ws_bytes, _stream_handle(stream))
+    _check("la_forward_sp", st)
+    return o
+
+
+def la_backward_sp_dq(q, k, v, dO, o, g, state_in, causal: bool = True, phi="elu1", dq=None,
+                      state_out=None, workspace=None, stream=None):
+    """First local backward step: (dq, this shard's query-side record,
+    workspace); pass the workspace on to la_backward_sp_dkdv unchanged."""
+    lib = load_library()
+    _check_qkv("la_backward_sp_dq", q, k, v, dO, o)
+    B, H, N, D = q.shape
+    if g.dtype != torch.float32 or tuple(g.shape) != (B, H, N) or not g.is_contiguous():
+        raise ValueError("la_backward_sp_dq: g must be contiguous float32 [B, H, N]")
+    _state_records("la_backward_sp_dq", state_in, B, H, D, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    _check_qkv("la_backward_sp_dq", q, dq)
+    state_out = torch.empty((B, H, D * D + D), dtype=torch.float32, device=q.device) \
+        if state_out is None else state_out
+    _state_records("la_backward_sp_dq", state_out, B, H, D, q.device)
+    ws, ws_bytes = _workspace_sp(LA_OP_BACKWARD, q, causal, workspace)
+    st = lib.la_backward_sp_dq(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g),
+                               _ptr(state_in), _ptr(dq), _ptr(state_out), B, H, N, D,
+                               DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
+                               _stream_handle(stream))
+    _check("la_backward_sp_dq", st)
+    return dq, state_out, ws
+
+
+def la_backward_sp_dkdv(q, k, v, dO, g, state_in, workspace, causal: bool = True, phi="elu1",
+                        dk=None, dv=None, stream=None):
+    """Second local backward step: (dk, dv), with the workspace that
+    la_backward_sp_dq filled."""
+    lib = load_library()
+    _check_qkv("la_backward_sp_dkdv", q, k, v, dO)
+    B, H, N, D = q.shape
+    _state_records("la_backward_sp_dkdv", state_in, B, H, D, q.device)
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv("la_backward_sp_dkdv", k, dk, dv)
+    need = la_workspace_size_sp(LA_OP_BACKWARD, B, H, N, D, causal, q.dtype)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if ws_bytes < need:
+        raise ValueError("la_backward_sp_dkdv: pass the workspace la_backward_sp_dq filled")
+    st = lib.la_backward_sp_dkdv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(g), _ptr(state_in),
+                                 _ptr(dk), _ptr(dv), B, H, N, D, DTYPE[q.dtype],
+                                 int(bool(causal)), _phi(phi), _ptr(workspace), ws_bytes,
+                                 _stream_handle(stream))
+    _check("la_backward_sp_dkdv", st)
+    return dk, dv
 
 
 def la_get_device_error(stream=None) -> None:

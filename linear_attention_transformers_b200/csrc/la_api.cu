@@ -278,17 +278,18 @@ float chunk_gamma_min(int C) { return exp2f(-64.f / float(C)); }
 la_status launch_state_kernel(int which, float* rec, float* out, float* S, float* z,
                               int64_t heads, int nseg, int64_t D, cudaStream_t st,
                               int rec_step = 1, const la::DecayArg& dec = kNoDecay,
-                              int seg_len = 0) {
+                              int seg_len = 0, const float* init = nullptr) {
     const int R = int(D * D + D);
     const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
     const unsigned grid = unsigned(heads * bph);
     if (which == 0) {
         la::LaunchScope scope("state_scan", st);
         la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph,
-                                                                            dec, seg_len);
+                                                                            dec, seg_len, init);
     } else if (which == 3) {
         la::LaunchScope scope("state_rscan", st);
-        la::state_exclusive_rscan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph);
+        la::state_exclusive_rscan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph,
+                                                                             init);
     } else if (which == 1) {
         la::LaunchScope scope("state_sum", st);
         la::state_sum_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, out, nseg, R, bph);
@@ -1186,6 +1187,417 @@ la_status la_backward_noalloc(const void* q, const void* k, const void* v, const
     if ((s = static_scratch(&scratch)) != LA_OK) return s;
     return la_backward(q, k, v, dO, o, g, phi_q, phi_k, dq, dk, dv, B, H, N, D, dt, causal, phi,
                        scratch, size_t(LA_NOALLOC_MAX_BYTES), stream);
+}
+
+// ------------------------------------------------------------ sequence split across ranks
+// The tokens of every head split into consecutive shards, one per rank.
+// States are sums over tokens ("Efficient Transformers Survey", Proposition
+// "Linear Attention via Kernel Decomposition", Statement), so a rank's
+// causal outputs need only the sum of the states of the shards before it
+// (non-causal: of every shard), and the backward's suffix state of the
+// shards after it: one exchange of one record per head each way.
+}  // extern "C"
+
+namespace {
+
+// seg: the causal passes and the local reduce; qseg: the non-causal query
+// and gradient passes (one block each).  Backward workspace: dg [heads][N],
+// the centred prefix records of a split head (srec) and one (R, r) record
+// per pass-1 block (rrec), which the dK/dV call reads back.
+struct SpPlan {
+    bool fast = false;
+    int C = 0;
+    SegSplit seg, qseg;
+    size_t fwd_bytes = 0, dg_off = 0, srec_off = 0, rrec_off = 0, bwd_bytes = 0;
+};
+
+SpPlan plan_sp(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
+    SpPlan p;
+    if (!fast_path(dt, D) || N == 0 || B * H == 0) return p;
+    p.fast = true;
+    p.C = chunk_len(D);
+    const int64_t heads = B * H;
+    const int64_t nch = (N + p.C - 1) / p.C;
+    const int kNumSM = num_sms();
+    p.seg = split(N, p.C, pick_nseg(heads, nch));
+    const int64_t want = heads >= 2 * kNumSM ? 1 : (2 * kNumSM + heads - 1) / heads;
+    p.qseg = causal ? p.seg
+                    : split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
+    const size_t R4 = size_t(D * D + D) * sizeof(float);
+    p.fwd_bytes = p.seg.nseg > 1 ? round_up(size_t(heads) * p.seg.nseg * R4, 256) : 0;
+    size_t off = 0;
+    p.dg_off = off;
+    off += round_up(size_t(heads) * size_t(N) * sizeof(float), 256);
+    p.srec_off = off;
+    if (causal && p.seg.nseg > 1) off += round_up(size_t(heads) * p.seg.nseg * R4, 256);
+    p.rrec_off = off;
+    off += round_up(size_t(heads) * p.qseg.nseg * R4, 256);
+    p.bwd_bytes = std::max(off, p.fwd_bytes);
+    return p;
+}
+
+template <int D, int PHI>
+la_status run_state_local(const void* k, const void* v, float* out, int64_t heads, int64_t N,
+                          int centred, const SpPlan& p, char* ws, cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    const int64_t R = int64_t(D) * D + D;
+    la::ChunkParams r;
+    memset(&r, 0, sizeof(r));
+    if (!make_qkv_map(&r.tm_k, k, heads, N, D, C) || !make_qkv_map(&r.tm_v, v, heads, N, D, C))
+        return LA_ERR_CUDA;
+    r.N = int(N);
+    r.seg_len = p.seg.seg_len;
+    r.nseg = p.seg.nseg;
+    r.center = centred;
+    r.kv_group = 1;
+    float* dst = p.seg.nseg > 1 ? reinterpret_cast<float*>(ws) : out;
+    r.S_out = dst;
+    r.z_out = dst + D * D;
+    r.stride_S = r.stride_z = R;
+    la_status s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
+                                                           "chunk_reduce");
+    if (s != LA_OK || p.seg.nseg == 1) return s;
+    return launch_state_kernel(1, dst, out, nullptr, nullptr, heads, p.seg.nseg, D, st);
+}
+
+template <int D, int PHI>
+la_status run_fwd_sp(const void* q, const void* k, const void* v, void* o, const float* state_in,
+                     float* state_out, float* g_out, int64_t heads, int64_t N, int causal,
+                     const SpPlan& p, char* ws, cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    const int64_t R = int64_t(D) * D + D;
+    la::ChunkParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) || !make_qkv_map(&prm.tm_o, o, heads, N, D, C))
+        return LA_ERR_CUDA;
+    prm.N = int(N);
+    prm.g_out = g_out;
+    prm.kv_group = 1;
+    la_status s;
+    if (!causal) {
+        prm.seg_len = p.qseg.seg_len;
+        prm.nseg = p.qseg.nseg;
+        prm.state_in = state_in;
+        prm.in_per_head = 1;
+        return launch_chunk<D, C, PHI, la::MODE_QUERY>(prm, heads * p.qseg.nseg, st,
+                                                       "chunk_query");
+    }
+    prm.state_in = state_in;
+    prm.in_per_head = 1;
+    if (p.seg.nseg > 1) {
+        // segment starts: the incoming state plus the segments before
+        float* rec = reinterpret_cast<float*>(ws);
+        la::ChunkParams r = prm;
+        r.state_in = nullptr;
+        r.seg_len = p.seg.seg_len;
+        r.nseg = p.seg.nseg;
+        r.S_out = rec;
+        r.z_out = rec + D * D;
+        r.stride_S = r.stride_z = R;
+        r.g_out = nullptr;
+        if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
+                                                          "chunk_reduce")) != LA_OK)
+            return s;
+        if ((s = launch_state_kernel(0, rec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D, st,
+                                     1, kNoDecay, 0, state_in)) != LA_OK)
+            return s;
+        prm.state_in = rec;
+        prm.in_per_head = 0;
+    }
+    prm.seg_len = p.seg.seg_len;
+    prm.nseg = p.seg.nseg;
+    prm.S_out = state_out;
+    prm.z_out = state_out ? state_out + D * D : nullptr;
+    prm.stride_S = prm.stride_z = R;
+    return launch_chunk<D, C, PHI, la::MODE_CAUSAL>(prm, heads * p.seg.nseg, st, "chunk_causal");
+}
+
+template <int D, int PHI>
+la_status run_bwd_sp_dq(const void* q, const void* k, const void* v, const void* dO,
+                        const void* o, const float* g, const float* state_in, void* dq,
+                        float* state_out, int64_t heads, int64_t N, int causal, const SpPlan& p,
+                        char* ws, cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    constexpr int smem1 = la::Bwd1Cfg<D, C>::SMEM;
+    la::BwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_do, dO, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dq, dq, heads, N, D, C))
+        return LA_ERR_CUDA;
+    prm.kv_group = 1;
+    prm.N = int(N);
+    prm.gbuf = const_cast<float*>(g);
+    prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
+    prm.o_in = static_cast<const __nv_bfloat16*>(o);
+    float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
+    prm.rec_out = rrec;
+    prm.state_in = state_in;
+    prm.in_per_head = 1;
+    const SegSplit& sg = causal ? p.seg : p.qseg;
+    prm.seg_len = sg.seg_len;
+    prm.nseg = sg.nseg;
+    la_status s;
+    if (causal && p.seg.nseg > 1) {
+        // segment starts: the incoming centred state plus the centred
+        // states of the segments before (the dQ products' key features)
+        const int64_t R = int64_t(D) * D + D;
+        float* srec = reinterpret_cast<float*>(ws + p.srec_off);
+        la::ChunkParams red;
+        memset(&red, 0, sizeof(red));
+        red.tm_k = prm.tm_k;
+        red.tm_v = prm.tm_v;
+        red.N = int(N);
+        red.seg_len = p.seg.seg_len;
+        red.nseg = p.seg.nseg;
+        red.S_out = srec;
+        red.z_out = srec + D * D;
+        red.stride_S = red.stride_z = R;
+        red.center = 1;
+        red.kv_group = 1;
+        if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
+                                                          "chunk_reduce")) != LA_OK)
+            return s;
+        if ((s = launch_state_kernel(0, srec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D, st,
+                                     1, kNoDecay, 0, state_in)) != LA_OK)
+            return s;
+        prm.state_in = srec;
+        prm.in_per_head = 0;
+    }
+    s = causal ? launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, true, true>, smem1, prm,
+                                   heads * sg.nseg, st, "bwd_dq")
+               : launch_bwd_kernel(la::bwd_dq_kernel<D, C, PHI, false, true>, smem1, prm,
+                                   heads * sg.nseg, st, "bwd_dq");
+    if (s != LA_OK) return s;
+    // this rank's (R, r): the sum of its blocks' records (which stay in the
+    // workspace for the dK/dV call)
+    return launch_state_kernel(1, rrec, state_out, nullptr, nullptr, heads, sg.nseg, D, st);
+}
+
+template <int D, int PHI>
+la_status run_bwd_sp_dkdv(const void* q, const void* k, const void* v, const void* dO,
+                          const float* g, const float* state_in, void* dk, void* dv,
+                          int64_t heads, int64_t N, int causal, const SpPlan& p, char* ws,
+                          cudaStream_t st) {
+    constexpr int C = D == 64 ? 128 : 64;
+    constexpr int smem2 = la::Bwd2Cfg<D, C>::SMEM;
+    la::BwdParams prm;
+    memset(&prm, 0, sizeof(prm));
+    if (!make_qkv_map(&prm.tm_q, q, heads, N, D, C) || !make_qkv_map(&prm.tm_k, k, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_v, v, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_do, dO, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dk, dk, heads, N, D, C) ||
+        !make_qkv_map(&prm.tm_dv, dv, heads, N, D, C))
+        return LA_ERR_CUDA;
+    prm.kv_group = 1;
+    prm.N = int(N);
+    prm.gbuf = const_cast<float*>(g);
+    prm.dgbuf = reinterpret_cast<float*>(ws + p.dg_off);
+    if (!causal) {
+        prm.seg_len = p.qseg.seg_len;
+        prm.nseg = p.qseg.nseg;
+        prm.state_in = state_in;
+        prm.in_per_head = 1;
+        return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, false>, smem2, prm,
+                                 heads * p.qseg.nseg, st, "bwd_dkdv");
+    }
+    // block starts of the reverse walk: the incoming suffix state plus the
+    // records of the blocks after (left in the workspace by the dQ call)
+    float* rrec = reinterpret_cast<float*>(ws + p.rrec_off);
+    la_status s = launch_state_kernel(3, rrec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
+                                      st, 1, kNoDecay, 0, state_in);
+    if (s != LA_OK) return s;
+    prm.seg_len = p.seg.seg_len;
+    prm.nseg = p.seg.nseg;
+    prm.state_in = rrec;
+    prm.in_per_head = 0;
+    if constexpr (D == 64)
+        return launch_bwd_kernel(la::bwd_dkdv64_kernel<PHI, false>, la::Bwd2x64Cfg::SMEM, prm,
+                                 heads * p.seg.nseg, st, "bwd_dkdv", la::kBwd64Threads);
+    else
+        return launch_bwd_kernel(la::bwd_dkdv_kernel<D, C, PHI, true>, smem2, prm,
+                                 heads * p.seg.nseg, st, "bwd_dkdv");
+}
+
+// Shared checks of the sequence-parallel calls: the tensor-core path only
+// (bf16, D = 64 or 128, one key/value head per query head).
+la_status check_sp(int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, la_phi phi,
+                   const void* workspace) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if ((s = check_sizes(B, H, N, D)) != LA_OK) return s;
+    if (!fast_path(dt, D)) return LA_ERR_UNSUPPORTED;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+la_status check_ws(const void* workspace, size_t have, size_t need) {
+    if (need > 0 && (workspace == nullptr || have < need)) return LA_ERR_WORKSPACE;
+    return LA_OK;
+}
+
+template <typename Fn>
+la_status with_head_size(int64_t D, Fn&& fn) {
+    if (D == 64) return fn(std::integral_constant<int, 64>{});
+    return fn(std::integral_constant<int, 128>{});
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t la_workspace_size_sp(la_op op, int64_t B, int64_t H, int64_t N, int64_t D, int causal,
+                            la_dtype dt) {
+    if (check_sizes(B, H, N, D) != LA_OK || !fast_path(dt, D)) return 0;
+    const SpPlan p = plan_sp(B, H, N, D, causal ? 1 : 0, dt);
+    if (!p.fast) return 0;
+    if (op == LA_OP_FORWARD) return p.fwd_bytes;
+    if (op == LA_OP_BACKWARD) return p.bwd_bytes;
+    return 0;
+}
+
+la_status la_state_local(const void* k, const void* v, float* state_out, int64_t B, int64_t H,
+                         int64_t N, int64_t D, la_dtype dt, la_phi phi, int centred,
+                         void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    la_status s;
+    if ((s = check_sp(B, H, N, D, dt, phi, workspace)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if ((s = check_ptr(state_out)) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (cudaError_t e = cudaMemsetAsync(state_out, 0, size_t(heads * (D * D + D)) * 4, st))
+            return cuda_fail("cudaMemsetAsync", e);
+        return LA_OK;
+    }
+    if ((s = check_ptr(k)) || (s = check_ptr(v))) return s;
+    const SpPlan p = plan_sp(B, H, N, D, 1, dt);
+    if ((s = check_ws(workspace, workspace_bytes, p.fwd_bytes)) != LA_OK) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    char* ws = static_cast<char*>(workspace);
+    return with_phi_map(phi, [&](auto P) {
+        return with_head_size(D, [&](auto Dc) {
+            return run_state_local<decltype(Dc)::value, decltype(P)::value>(
+                k, v, state_out, heads, N, centred ? 1 : 0, p, ws, st);
+        });
+    });
+}
+
+la_status la_state_range_sum(const float* states, int64_t P, int64_t lo, int64_t hi,
+                             float* out, int64_t B, int64_t H, int64_t D, la_stream_t stream) {
+    la_status s;
+    if (B < 0 || H < 0 || D <= 0 || P < 0 || lo < 0 || hi < lo || hi > P)
+        return LA_ERR_INVALID_ARG;
+    if (!supported_d(D)) return LA_ERR_UNSUPPORTED;
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if (heads >= (int64_t(1) << 31) || P >= (int64_t(1) << 20)) return LA_ERR_UNSUPPORTED;
+    if ((s = check_ptr(out)) != LA_OK) return s;
+    if (hi > lo && (s = check_ptr(states)) != LA_OK) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int R = int(D * D + D);
+    const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
+    la::LaunchScope scope("state_range_sum", st);
+    la::state_range_sum_kernel<<<unsigned(heads * bph), la::kStateThreads, 0, st>>>(
+        states, out, int(lo), int(hi), heads, R, bph);
+    return launch_status();
+}
+
+la_status la_forward_sp(const void* q, const void* k, const void* v, void* o,
+                        const float* state_in, float* state_out, float* g_out, int64_t B,
+                        int64_t H, int64_t N, int64_t D, la_dtype dt, int causal, la_phi phi,
+                        void* workspace, size_t workspace_bytes, la_stream_t stream) {
+    la_status s;
+    if ((s = check_sp(B, H, N, D, dt, phi, workspace)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if ((s = check_ptr(state_in)) != LA_OK) return s;
+    if (state_out && !causal) return LA_ERR_INVALID_ARG;
+    if ((state_out && !aligned16(state_out)) || (g_out && !aligned16(g_out)))
+        return LA_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        // no tokens here: the state passes through unchanged
+        if (state_out) {
+            if (cudaError_t e = cudaMemcpyAsync(state_out, state_in,
+                                                size_t(heads * (D * D + D)) * 4,
+                                                cudaMemcpyDeviceToDevice, st))
+                return cuda_fail("cudaMemcpyAsync", e);
+        }
+        return LA_OK;
+    }
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
+        return s;
+    const SpPlan p = plan_sp(B, H, N, D, causal ? 1 : 0, dt);
+    if ((s = check_ws(workspace, workspace_bytes, p.fwd_bytes)) != LA_OK) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    char* ws = static_cast<char*>(workspace);
+    return with_phi_map(phi, [&](auto P) {
+        return with_head_size(D, [&](auto Dc) {
+            return run_fwd_sp<decltype(Dc)::value, decltype(P)::value>(
+                q, k, v, o, state_in, state_out, g_out, heads, N, causal ? 1 : 0, p, ws, st);
+        });
+    });
+}
+
+la_status la_backward_sp_dq(const void* q, const void* k, const void* v, const void* dO,
+                            const void* o, const float* g, const float* state_in, void* dq,
+                            float* state_out, int64_t B, int64_t H, int64_t N, int64_t D,
+                            la_dtype dt, int causal, la_phi phi, void* workspace,
+                            size_t workspace_bytes, la_stream_t stream) {
+    la_status s;
+    if ((s = check_sp(B, H, N, D, dt, phi, workspace)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0) return LA_OK;
+    if ((s = check_ptr(state_in)) || (s = check_ptr(state_out))) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (N == 0) {
+        if (cudaError_t e = cudaMemsetAsync(state_out, 0, size_t(heads * (D * D + D)) * 4, st))
+            return cuda_fail("cudaMemsetAsync", e);
+        return LA_OK;
+    }
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
+        (s = check_ptr(o)) || (s = check_ptr(g)) || (s = check_ptr(dq)))
+        return s;
+    const SpPlan p = plan_sp(B, H, N, D, causal ? 1 : 0, dt);
+    if ((s = check_ws(workspace, workspace_bytes, p.bwd_bytes)) != LA_OK) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    char* ws = static_cast<char*>(workspace);
+    return with_phi_map(phi, [&](auto P) {
+        return with_head_size(D, [&](auto Dc) {
+            return run_bwd_sp_dq<decltype(Dc)::value, decltype(P)::value>(
+                q, k, v, dO, o, g, state_in, dq, state_out, heads, N, causal ? 1 : 0, p, ws, st);
+        });
+    });
+}
+
+la_status la_backward_sp_dkdv(const void* q, const void* k, const void* v, const void* dO,
+                              const float* g, const float* state_in, void* dk, void* dv,
+                              int64_t B, int64_t H, int64_t N, int64_t D, la_dtype dt, int causal,
+                              la_phi phi, void* workspace, size_t workspace_bytes,
+                              la_stream_t stream) {
+    la_status s;
+    if ((s = check_sp(B, H, N, D, dt, phi, workspace)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(state_in)) != LA_OK) return s;
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
+        (s = check_ptr(g)) || (s = check_ptr(dk)) || (s = check_ptr(dv)))
+        return s;
+    const SpPlan p = plan_sp(B, H, N, D, causal ? 1 : 0, dt);
+    if ((s = check_ws(workspace, workspace_bytes, p.bwd_bytes)) != LA_OK) return s;
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* ws = static_cast<char*>(workspace);
+    return with_phi_map(phi, [&](auto P) {
+        return with_head_size(D, [&](auto Dc) {
+            return run_bwd_sp_dkdv<decltype(Dc)::value, decltype(P)::value>(
+                q, k, v, dO, g, state_in, dk, dv, heads, N, causal ? 1 : 0, p, ws, st);
+        });
+    });
 }
 
 namespace {

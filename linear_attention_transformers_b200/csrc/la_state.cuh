@@ -25,20 +25,22 @@ __device__ __forceinline__ void load_batch(const float* base, int p0, int step, 
         if (i < n) x[i] = base[size_t(p0 + i * step) * R];
 }
 
-// rec[h][p] <- sum_{p' < p} rec[h][p'] (exclusive prefix, in place).  With
-// a decay factor per head (decayed recurrence; every segment before the
-// last holds seg_len tokens and its record is its state at its end) the
-// prefix is run_p = gamma^seg_len run_{p-1} + rec[p-1]; without one the
-// factor is 1 and the sum is the plain one, bit for bit.
+// rec[h][p] <- init[h] + sum_{p' < p} rec[h][p'] (exclusive prefix, in
+// place; init is the state the head starts from, null = zero, e.g. the sum
+// of the states of the tokens other ranks hold before this rank's).  With a
+// decay factor per head (decayed recurrence; every segment before the last
+// holds seg_len tokens and its record is its state at its end) the prefix
+// is run_p = gamma^seg_len run_{p-1} + rec[p-1]; without one the factor is
+// 1 and the sum is the plain one, bit for bit.
 __global__ void __launch_bounds__(kStateThreads)
 state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head,
-                            const DecayArg dec, int seg_len) {
+                            const DecayArg dec, int seg_len, const float* __restrict__ init) {
     const size_t h = blockIdx.x / blocks_per_head;
     const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
     if (e >= R) return;
     float* base = rec + h * size_t(nseg) * R + e;
     const float fac = dec.H > 0 ? powf(decay_of(dec, h), float(seg_len)) : 1.f;
-    float run = 0.f;
+    float run = init ? init[h * size_t(R) + e] : 0.f;
     for (int p0 = 0; p0 < nseg; p0 += kStateBatch) {
         const int n = min(kStateBatch, nseg - p0);
         float x[kStateBatch];
@@ -52,14 +54,16 @@ state_exclusive_scan_kernel(float* __restrict__ rec, int nseg, int R, int blocks
     }
 }
 
-// rec[h][p] <- sum_{p' > p} rec[h][p'] (exclusive suffix, in place).
+// rec[h][p] <- init[h] + sum_{p' > p} rec[h][p'] (exclusive suffix, in
+// place; init null = zero).
 __global__ void __launch_bounds__(kStateThreads)
-state_exclusive_rscan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head) {
+state_exclusive_rscan_kernel(float* __restrict__ rec, int nseg, int R, int blocks_per_head,
+                             const float* __restrict__ init) {
     const size_t h = blockIdx.x / blocks_per_head;
     const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
     if (e >= R) return;
     float* base = rec + h * size_t(nseg) * R + e;
-    float run = 0.f;
+    float run = init ? init[h * size_t(R) + e] : 0.f;
     for (int p0 = nseg - 1; p0 >= 0; p0 -= kStateBatch) {
         const int n = min(kStateBatch, p0 + 1);
         float x[kStateBatch];
@@ -86,6 +90,34 @@ state_sum_kernel(const float* __restrict__ rec, float* __restrict__ out, int nse
         const int n = min(kStateBatch, nseg - p0);
         float x[kStateBatch];
         load_batch(base, p0, 1, n, R, x);
+#pragma unroll
+        for (int i = 0; i < kStateBatch; ++i)
+            if (i < n) run += x[i];
+    }
+    out[h * size_t(R) + e] = run;
+}
+
+// out[h] <- sum_{lo <= p < hi} recs[p][h] for records laid out [P][heads][R]
+// (one block of records per rank, in rank order, as an all-gather leaves
+// them), added in increasing p; lo >= hi gives zero.  The state a rank of a
+// sequence split across ranks starts from is the sum over the ranks before
+// it (causal) or over all ranks (non-causal); the suffix over the ranks
+// after it is the backward's.
+__global__ void __launch_bounds__(kStateThreads)
+state_range_sum_kernel(const float* __restrict__ recs, float* __restrict__ out, int lo, int hi,
+                       int64_t heads, int R, int blocks_per_head) {
+    const size_t h = blockIdx.x / blocks_per_head;
+    const int e = (blockIdx.x % blocks_per_head) * kStateThreads + threadIdx.x;
+    if (e >= R) return;
+    const size_t stride = size_t(heads) * size_t(R);
+    const float* base = recs + h * size_t(R) + e;
+    float run = 0.f;
+    for (int p0 = lo; p0 < hi; p0 += kStateBatch) {
+        const int n = min(kStateBatch, hi - p0);
+        float x[kStateBatch];
+#pragma unroll
+        for (int i = 0; i < kStateBatch; ++i)
+            if (i < n) x[i] = base[size_t(p0 + i) * stride];
 #pragma unroll
         for (int i = 0; i < kStateBatch; ++i)
             if (i < n) run += x[i];

@@ -116,3 +116,21 @@ def check_state(S, z, S_ref, z_ref, dtype):
         assert (err <= rel * scale + 1e-6).all(), \
             f"final {name}: max err {err.max():.3e} vs {rel:.1e} of scale {scale:.3e}"
         compare(got, ref, dtype, f"final {name}", elementwise=False)
+
+
+def relu_branch_as_kernel(ref, x):
+    """The oracle's dQ (x = q) or dK (x = k) for the relu+eps map with the
+    branch phi'(x) taken as the bf16 tensor-core kernels take it: from the
+    bf16 value phi(x) = bf16(max(x, 0) + 1e-6) they read, 1 where it exceeds
+    bf16(1e-6) and 0 otherwise.  The two readings differ only for
+    0 < x < ~4e-9 (where max(x, 0) + 1e-6 rounds to the x <= 0 value); there
+    the oracle's gradient entry (taken with phi' = 1) becomes 0.  Where
+    floating point decides a branch, both sides take it in the same (the
+    kernel's) precision; everything else stays the oracle's."""
+    xf = (x.detach().to("cpu") if isinstance(x, torch.Tensor) else torch.as_tensor(x)).float()
+    phi_b = (torch.clamp(xf, min=0.0) + 1e-6).to(torch.bfloat16).float()
+    floor = torch.tensor(1e-6, dtype=torch.float32).to(torch.bfloat16).float()
+    mask = ((xf > 0) & (phi_b <= floor)).numpy()
+    out = np.array(ref, dtype=np.float64, copy=True)
+    out[mask] = 0.0
+    return out

@@ -66,3 +66,13 @@ def test_ratios_of_planted_errors():
     assert rms == pytest.approx(2.0) and mx == pytest.approx(2.0)
     eps_rms, eps_max = NORM[torch.bfloat16]
     assert eps_rms < 0.1 and eps_max < 0.1  # a 10 % scale error is caught
+
+
+def test_relu_branch_as_kernel_changes_only_the_rounding_band():
+    # bf16 inputs: exactly the x > 0 whose max(x, 0) + 1e-6 rounds to
+    # bf16(1e-6) (here x below ~2e-9; 3e-9 already rounds up) take the
+    # kernel's phi' = 0; every other entry is kept
+    from parity_util import relu_branch_as_kernel
+    x = torch.tensor([1.2e-9, 3e-9, 0.0, -1e-9, -1.0, 6e-9, 1e-8, 1e-3]).to(torch.bfloat16)
+    out = relu_branch_as_kernel(np.arange(1.0, 9.0), x)
+    np.testing.assert_array_equal(out, [0.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0, 8.0])
