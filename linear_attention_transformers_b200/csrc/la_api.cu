@@ -220,11 +220,42 @@ SegSplit split(int64_t N, int C, int nseg) {
     return s;
 }
 
+// Reduce split for the starts of a causal pass cut into segments: only the
+// tokens before the last segment are summed (its own state is never a
+// start), each segment as `ratio` equal sub-segments (ratio dividing its
+// chunks) chosen so that the reduce blocks fill the SMs: the smallest
+// modelled makespan waves x (chunks per block + fill).
+struct StartSplit {
+    int ratio = 1, nsub = 0, sub_len = 0;
+};
+StartSplit start_split(int64_t heads, const SegSplit& seg, int C) {
+    StartSplit r;
+    if (seg.nseg <= 1) return r;
+    const int seg_chunks = seg.seg_len / C;
+    const int kNumSM = num_sms();
+    constexpr double kFill = 3.0;
+    double best = 0.0;
+    for (int q = 1; q <= std::min(seg_chunks, 16); ++q) {
+        if (seg_chunks % q) continue;
+        const int64_t blocks = heads * (seg.nseg - 1) * q;
+        const double cost =
+            double((blocks + kNumSM - 1) / kNumSM) * (double(seg_chunks / q) + kFill);
+        if (q == 1 || cost < best - 1e-9) {
+            best = cost;
+            r.ratio = q;
+        }
+    }
+    r.sub_len = seg.seg_len / r.ratio;
+    r.nsub = (seg.nseg - 1) * r.ratio;
+    return r;
+}
+
 struct FwdPlan {
     bool fast = false;
     int C = 0;
     SegSplit seg, qseg;
-    size_t rec_off = 0, tot_off = 0, bytes = 0;
+    StartSplit ss;  // causal, split heads: the reduce pass for the segment starts
+    size_t rec_off = 0, tot_off = 0, sub_off = 0, bytes = 0;
 };
 
 FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
@@ -238,8 +269,15 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
     p.seg = split(N, p.C, pick_nseg(heads, nch));
     const size_t R = size_t(D) * D + D;
     if (causal) {
+        // rec: the segment starts (or, decayed, the per-segment records
+        // scanned in place); sub: the start reduce's records
         p.rec_off = 0;
-        p.bytes = p.seg.nseg > 1 ? size_t(heads) * p.seg.nseg * R * sizeof(float) : 0;
+        p.bytes = 0;
+        if (p.seg.nseg > 1) {
+            p.ss = start_split(heads, p.seg, p.C);
+            p.sub_off = round_up(size_t(heads) * p.seg.nseg * R * sizeof(float), 256);
+            p.bytes = p.sub_off + size_t(heads) * p.ss.nsub * R * sizeof(float);
+        }
     } else {
         const int64_t want = heads >= 2 * kNumSM ? 1 : (2 * kNumSM + heads - 1) / heads;
         p.qseg = split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
@@ -282,22 +320,54 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
     const int R = int(D * D + D);
     const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
     const unsigned grid = unsigned(heads * bph);
+    // the sums and scans run over float4 columns (R is a multiple of 4)
+    const int R4 = R / 4;
+    const int bph4 = (R4 + la::kStateThreads - 1) / la::kStateThreads;
+    const unsigned grid4 = unsigned(heads * bph4);
     if (which == 0) {
         la::LaunchScope scope("state_scan", st);
-        la::state_exclusive_scan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph,
-                                                                            dec, seg_len, init);
+        la::state_exclusive_scan_kernel<<<grid4, la::kStateThreads, 0, st>>>(rec, nseg, R4, bph4,
+                                                                             dec, seg_len, init);
     } else if (which == 3) {
         la::LaunchScope scope("state_rscan", st);
-        la::state_exclusive_rscan_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, nseg, R, bph,
-                                                                             init);
+        la::state_exclusive_rscan_kernel<<<grid4, la::kStateThreads, 0, st>>>(rec, nseg, R4,
+                                                                              bph4, init);
     } else if (which == 1) {
         la::LaunchScope scope("state_sum", st);
-        la::state_sum_kernel<<<grid, la::kStateThreads, 0, st>>>(rec, out, nseg, R, bph);
+        la::state_sum_kernel<<<grid4, la::kStateThreads, 0, st>>>(rec, out, nseg, R4, bph4);
     } else {
         la::LaunchScope scope("state_unpack", st);
         la::state_unpack_kernel<<<grid, la::kStateThreads, 0, st>>>(out, S, z, int(D), bph,
                                                                      rec_step);
     }
+    return launch_status();
+}
+
+// Starts of the segments of a causal pass (no decay): the REDUCE pass of
+// `red` (its k, v maps, N, kv_group and centring) over the sub-segments of
+// the tokens before the last segment into `sub`, then starts[h][p] =
+// init[h] + the sub-segment records before segment p.
+template <int D, int C, int PHI>
+la_status run_segment_starts(const la::ChunkParams& red, int64_t heads, const SegSplit& seg,
+                             const StartSplit& ss, float* sub, float* starts, const float* init,
+                             cudaStream_t st) {
+    const int64_t R = int64_t(D) * D + D;
+    la::ChunkParams r = red;
+    r.state_in = nullptr;
+    r.g_out = nullptr;
+    r.store_phi = 0;
+    r.seg_len = ss.sub_len;
+    r.nseg = ss.nsub;
+    r.S_out = sub;
+    r.z_out = sub + D * D;
+    r.stride_S = r.stride_z = R;
+    la_status s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * ss.nsub, st, "chunk_reduce");
+    if (s != LA_OK) return s;
+    const int R4 = int(R / 4);
+    const int bph = (R4 + la::kStateThreads - 1) / la::kStateThreads;
+    la::LaunchScope scope("state_starts", st);
+    la::state_segment_starts_kernel<<<unsigned(heads * bph), la::kStateThreads, 0, st>>>(
+        sub, starts, seg.nseg, ss.ratio, R4, bph, init);
     return launch_status();
 }
 
@@ -323,21 +393,27 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
     float* rec = reinterpret_cast<float*>(ws + p.rec_off);
     la_status s;
     if (causal) {
-        if (p.seg.nseg > 1) {
+        if (p.seg.nseg > 1 && decay) {
+            // decayed: every segment's record, scanned with the decay factors
             la::ChunkParams r = prm;
             r.seg_len = p.seg.seg_len;
             r.nseg = p.seg.nseg;
             r.S_out = rec;
             r.z_out = rec + D * D;
             r.stride_S = r.stride_z = R;
-            if ((s = decay ? launch_chunk<D, C, PHI, la::MODE_REDUCE, true>(
-                                 r, heads * p.seg.nseg, st, "chunk_reduce")
-                           : launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
-                                                                     "chunk_reduce")) != LA_OK)
+            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE, true>(r, heads * p.seg.nseg, st,
+                                                                    "chunk_reduce")) != LA_OK)
                 return s;
             if ((s = launch_state_kernel(0, rec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
                                          st, 1, dec, p.seg.seg_len)) != LA_OK)
                 return s;
+        } else if (p.seg.nseg > 1) {
+            float* sub = reinterpret_cast<float*>(ws + p.sub_off);
+            if ((s = run_segment_starts<D, C, PHI>(prm, heads, p.seg, p.ss, sub, rec, nullptr,
+                                                   st)) != LA_OK)
+                return s;
+        }
+        if (p.seg.nseg > 1) {
             prm.state_in = rec;
             prm.in_per_head = 0;
         }
@@ -408,6 +484,9 @@ struct BwdPlan {
     size_t o_off = 0, fwd_off = 0;
     // grouped key/value heads (G > 1): dK, dV per query head, summed per group
     size_t part_off = 0;
+    // causal, split heads: the reduce pass for the dQ pass's segment starts
+    StartSplit ss;
+    size_t sub_off = 0;
     size_t bytes = 0;
 };
 
@@ -431,10 +510,13 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     if (causal) {
         p.qseg = p.seg;
         if (p.seg.nseg > 1) {
+            p.ss = start_split(heads, p.seg, p.C);
             p.srec_off = off;
             off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
             p.rrec_off = off;
             off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
+            p.sub_off = off;
+            off += round_up(size_t(heads) * p.ss.nsub * R * 4, 256);
         }
     } else {
         const int64_t want = heads >= 2 * kNumSM ? 1 : (2 * kNumSM + heads - 1) / heads;
@@ -545,11 +627,9 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
         p1.seg_len = p2.seg_len = p.seg.seg_len;
         p1.nseg = p2.nseg = p.seg.nseg;
         if (p.seg.nseg > 1) {
-            if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
-                                                             "chunk_reduce")) != LA_OK)
-                return s;
-            if ((s = launch_state_kernel(0, srec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D,
-                                         st)) != LA_OK)
+            float* sub = reinterpret_cast<float*>(ws + p.sub_off);
+            if ((s = run_segment_starts<D, C, PHI>(red, heads, p.seg, p.ss, sub, srec, nullptr,
+                                                   st)) != LA_OK)
                 return s;
             p1.state_in = srec;
             p1.rec_out = rrec;
@@ -1208,7 +1288,9 @@ struct SpPlan {
     bool fast = false;
     int C = 0;
     SegSplit seg, qseg;
-    size_t fwd_bytes = 0, dg_off = 0, srec_off = 0, rrec_off = 0, bwd_bytes = 0;
+    StartSplit ss;  // causal, split heads: the reduce pass for the segment starts
+    size_t fwd_sub_off = 0, fwd_bytes = 0;
+    size_t dg_off = 0, srec_off = 0, rrec_off = 0, sub_off = 0, bwd_bytes = 0;
 };
 
 SpPlan plan_sp(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype dt) {
@@ -1224,7 +1306,11 @@ SpPlan plan_sp(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype 
     p.qseg = causal ? p.seg
                     : split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
     const size_t R4 = size_t(D * D + D) * sizeof(float);
-    p.fwd_bytes = p.seg.nseg > 1 ? round_up(size_t(heads) * p.seg.nseg * R4, 256) : 0;
+    p.ss = start_split(heads, p.seg, p.C);
+    // forward: per-segment records (la_state_local) or starts, then the
+    // start reduce's sub-segment records
+    p.fwd_sub_off = p.seg.nseg > 1 ? round_up(size_t(heads) * p.seg.nseg * R4, 256) : 0;
+    p.fwd_bytes = p.fwd_sub_off + round_up(size_t(heads) * p.ss.nsub * R4, 256);
     size_t off = 0;
     p.dg_off = off;
     off += round_up(size_t(heads) * size_t(N) * sizeof(float), 256);
@@ -1232,6 +1318,8 @@ SpPlan plan_sp(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype 
     if (causal && p.seg.nseg > 1) off += round_up(size_t(heads) * p.seg.nseg * R4, 256);
     p.rrec_off = off;
     off += round_up(size_t(heads) * p.qseg.nseg * R4, 256);
+    p.sub_off = off;
+    if (causal) off += round_up(size_t(heads) * p.ss.nsub * R4, 256);
     p.bwd_bytes = std::max(off, p.fwd_bytes);
     return p;
 }
@@ -1287,22 +1375,12 @@ la_status run_fwd_sp(const void* q, const void* k, const void* v, void* o, const
     prm.in_per_head = 1;
     if (p.seg.nseg > 1) {
         // segment starts: the incoming state plus the segments before
-        float* rec = reinterpret_cast<float*>(ws);
-        la::ChunkParams r = prm;
-        r.state_in = nullptr;
-        r.seg_len = p.seg.seg_len;
-        r.nseg = p.seg.nseg;
-        r.S_out = rec;
-        r.z_out = rec + D * D;
-        r.stride_S = r.stride_z = R;
-        r.g_out = nullptr;
-        if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
-                                                          "chunk_reduce")) != LA_OK)
+        float* starts = reinterpret_cast<float*>(ws);
+        float* sub = reinterpret_cast<float*>(ws + p.fwd_sub_off);
+        if ((s = run_segment_starts<D, C, PHI>(prm, heads, p.seg, p.ss, sub, starts, state_in,
+                                               st)) != LA_OK)
             return s;
-        if ((s = launch_state_kernel(0, rec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D, st,
-                                     1, kNoDecay, 0, state_in)) != LA_OK)
-            return s;
-        prm.state_in = rec;
+        prm.state_in = starts;
         prm.in_per_head = 0;
     }
     prm.seg_len = p.seg.seg_len;
@@ -1343,25 +1421,17 @@ la_status run_bwd_sp_dq(const void* q, const void* k, const void* v, const void*
     if (causal && p.seg.nseg > 1) {
         // segment starts: the incoming centred state plus the centred
         // states of the segments before (the dQ products' key features)
-        const int64_t R = int64_t(D) * D + D;
         float* srec = reinterpret_cast<float*>(ws + p.srec_off);
+        float* sub = reinterpret_cast<float*>(ws + p.sub_off);
         la::ChunkParams red;
         memset(&red, 0, sizeof(red));
         red.tm_k = prm.tm_k;
         red.tm_v = prm.tm_v;
         red.N = int(N);
-        red.seg_len = p.seg.seg_len;
-        red.nseg = p.seg.nseg;
-        red.S_out = srec;
-        red.z_out = srec + D * D;
-        red.stride_S = red.stride_z = R;
         red.center = 1;
         red.kv_group = 1;
-        if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
-                                                          "chunk_reduce")) != LA_OK)
-            return s;
-        if ((s = launch_state_kernel(0, srec, nullptr, nullptr, nullptr, heads, p.seg.nseg, D, st,
-                                     1, kNoDecay, 0, state_in)) != LA_OK)
+        if ((s = run_segment_starts<D, C, PHI>(red, heads, p.seg, p.ss, sub, srec, state_in,
+                                               st)) != LA_OK)
             return s;
         prm.state_in = srec;
         prm.in_per_head = 0;
@@ -1498,11 +1568,11 @@ la_status la_state_range_sum(const float* states, int64_t P, int64_t lo, int64_t
     if (hi > lo && (s = check_ptr(states)) != LA_OK) return s;
     if ((s = bind_context()) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int R = int(D * D + D);
-    const int bph = (R + la::kStateThreads - 1) / la::kStateThreads;
+    const int R4 = int(D * D + D) / 4;  // float4 columns (R is a multiple of 4)
+    const int bph = (R4 + la::kStateThreads - 1) / la::kStateThreads;
     la::LaunchScope scope("state_range_sum", st);
     la::state_range_sum_kernel<<<unsigned(heads * bph), la::kStateThreads, 0, st>>>(
-        states, out, int(lo), int(hi), heads, R, bph);
+        states, out, int(lo), int(hi), heads, R4, bph);
     return launch_status();
 }
 
