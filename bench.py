@@ -132,7 +132,23 @@ def roofline_of(bytes_, flops, seconds, peaks, sustained=True):
 # from (`files`, under csrc/) hash to `sources`.  Captures run at a smaller
 # N (the profiling size rule); these kernels move each token's tiles once,
 # so traffic grows in proportion to tokens.
-MEASURED_TRAFFIC = {}
+_FWD64_SOURCES = ["la_chunk_fwd64.cuh", "la_chunk_fwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
+                  "la_common.cuh"]
+_BWD64_SOURCES = ["la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
+                  "la_common.cuh"]
+MEASURED_TRAFFIC = {
+    # one `ncu --set full` launch each at B8 H16 N4096 D64 (the timed
+    # workload at half its tokens)
+    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.389824e6 + 156.388096e6) / (8 * 16 * 4096),
+                     "files": _FWD64_SOURCES,
+                     "sources": "4428205c90e85ea659b2689738ef639eb8b0f0d693f025e685750113ac3f3f72"},
+    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.711104e6 + 52.814592e6) / (8 * 16 * 4096),
+               "files": _BWD64_SOURCES,
+               "sources": "3284c03f2cc26e248f2f0fc71dc80afb241386e8c7079cf32f7b44ff67780b89"},
+    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.682496e6 + 99.994880e6) / (8 * 16 * 4096),
+                 "files": _BWD64_SOURCES,
+                 "sources": "3284c03f2cc26e248f2f0fc71dc80afb241386e8c7079cf32f7b44ff67780b89"},
+}
 
 
 def kernel_sources_hash(files) -> str:
