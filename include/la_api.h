@@ -280,9 +280,10 @@ LA_EXPORT la_status la_decode_step_decay(float *S, float *z, const void *q, cons
  * la_favor_features_backward returns dx [B, H, N, D] of sum(dphi * phi(x))
  * given x, omega and dphi [B, H, N, m]: dx = sum_i dphi_i phi_i w_i -
  * x sum_i dphi_i phi_i, with phi recomputed from x in float32 (the stored
- * features are not read).  Supported: bf16 with m == D in {64, 128} (else
+ * features are not read).  Supported: bf16 with D and m each 64 or 128 (else
  * LA_ERR_UNSUPPORTED); float32 accumulation, outputs rounded to bf16 once.
- * No workspace.
+ * No workspace.  With m != D the features go to la_forward_mv /
+ * la_backward_mv (feature length m, head size D).
  */
 LA_EXPORT la_status la_favor_features(const void *x, const void *omega, void *phi, int64_t B,
                                       int64_t H, int64_t N, int64_t D, int64_t m, la_dtype dt,
@@ -291,6 +292,35 @@ LA_EXPORT la_status la_favor_features_backward(const void *x, const void *omega,
                                                const void *dphi, void *dx, int64_t B, int64_t H,
                                                int64_t N, int64_t D, int64_t m, la_dtype dt,
                                                la_stream_t stream);
+
+/*
+ * Attention whose feature vectors and values differ in length: q, k
+ * [B, H, N, Dk] (with LA_PHI_IDENTITY the features themselves, e.g. m = Dk
+ * Performer features from la_favor_features), v, o, dO, dv [B, H, N, Dv];
+ * S = sum_j phi(k_j) v_j^T is Dk x Dv ("Efficient Transformers Survey",
+ * Proposition "Linear Attention via Kernel Decomposition": phi maps R^d to
+ * R^m; Low-Rank Approximations, Performer).  Otherwise as la_forward /
+ * la_backward (g_out, saved o and g).  bf16, Dk and Dv each 64 or 128;
+ * Dk < Dv needs LA_PHI_IDENTITY (its widening zero features contribute
+ * nothing; a feature map would turn them into phi(0) != 0), else
+ * LA_ERR_UNSUPPORTED.  Implementation: the narrower side is widened with
+ * zero columns into the workspace (values: zero output columns; features:
+ * zero terms), the head-size max(Dk, Dv) kernels run, and the wider result
+ * is cut back; the copies cost 2 (forward) to 4 (backward) extra passes over
+ * one tensor of the wider size.  Dk == Dv is exactly la_forward /
+ * la_backward.  Workspace: la_workspace_size_mv.
+ */
+LA_EXPORT size_t la_workspace_size_mv(la_op op, int64_t B, int64_t H, int64_t N, int64_t Dk,
+                                      int64_t Dv, int causal, la_dtype dt);
+LA_EXPORT la_status la_forward_mv(const void *q, const void *k, const void *v, void *o,
+                                  float *g_out, int64_t B, int64_t H, int64_t N, int64_t Dk,
+                                  int64_t Dv, la_dtype dt, int causal, la_phi phi,
+                                  void *workspace, size_t workspace_bytes, la_stream_t stream);
+LA_EXPORT la_status la_backward_mv(const void *q, const void *k, const void *v, const void *dO,
+                                   const void *o, const float *g, void *dq, void *dk, void *dv,
+                                   int64_t B, int64_t H, int64_t N, int64_t Dk, int64_t Dv,
+                                   la_dtype dt, int causal, la_phi phi, void *workspace,
+                                   size_t workspace_bytes, la_stream_t stream);
 
 /*
  * Sequence split across ranks (one process per GPU): the N tokens of every

@@ -16,6 +16,7 @@ raises ``RuntimeError``.
     la_decode_step_decay(S, z, q, k, v, gamma, ...)          -> o   (S, z in place)
     la_favor_features(x, omega)                              -> phi(x)  (Performer FAVOR+)
     la_favor_features_backward(x, omega, dphi)               -> dx
+    la_forward_mv / la_backward_mv(q, k, v[, dO])            features of length m != D
     la_state_local / la_state_range_sum / la_forward_sp /
     la_backward_sp_dq / la_backward_sp_dkdv                  (one rank's steps of a
                                                               sequence split across ranks)
@@ -124,6 +125,14 @@ def load_library(path: str | None = None):
         lib.la_favor_features_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, ci,
                                                    vp]
         lib.la_favor_features_backward.restype = ci
+        lib.la_workspace_size_mv.argtypes = [ci, i64, i64, i64, i64, i64, ci, ci]
+        lib.la_workspace_size_mv.restype = sz
+        lib.la_forward_mv.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ci, ci, ci,
+                                      vp, sz, vp]
+        lib.la_forward_mv.restype = ci
+        lib.la_backward_mv.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                       i64, ci, ci, ci, vp, sz, vp]
+        lib.la_backward_mv.restype = ci
         lib.la_workspace_size_sp.argtypes = [ci, i64, i64, i64, i64, ci, ci]
         lib.la_workspace_size_sp.restype = sz
         lib.la_state_local.argtypes = [vp, vp, vp, i64, i64, i64, i64, ci, ci, ci, vp, sz, vp]
@@ -519,6 +528,78 @@ def la_favor_features_backward(x, omega, dphi, dx=None, stream=None):
                                         DTYPE[x.dtype], _stream_handle(stream))
     _check("la_favor_features_backward", st)
     return dx
+
+
+# ------------------------------------- feature length m != head size D
+def _check_mv(name, q, k, v, *vs):
+    _check_qkv(name, q, k)
+    _check_qkv(name, v, *vs)
+    if q.dim() != 4 or v.dim() != 4 or q.shape[:3] != v.shape[:3] or q.device != v.device \
+            or q.dtype != v.dtype:
+        raise ValueError(f"{name}: q, k [B, H, N, Dk] and v [B, H, N, Dv] of one device and dtype")
+
+
+def _workspace_mv(op, q, v, causal, workspace):
+    B, H, N, Dk = q.shape
+    need = int(load_library().la_workspace_size_mv(int(op), B, H, N, Dk, v.shape[-1],
+                                                   int(bool(causal)), DTYPE[q.dtype]))
+    if workspace is not None:
+        have = workspace.numel() * workspace.element_size()
+        if have < need:
+            raise ValueError(f"workspace smaller than the {need} bytes needed")
+        return workspace, have
+    if need == 0:
+        return None, 0
+    return torch.empty(need, dtype=torch.uint8, device=q.device), need
+
+
+def la_forward_mv(q, k, v, causal: bool = True, phi="identity", o=None, g=None, workspace=None,
+                  stream=None):
+    """o [B, H, N, Dv] of attention with features q, k [B, H, N, Dk] (e.g. m
+    Performer features) and values v [B, H, N, Dv]."""
+    lib = load_library()
+    _check_mv("la_forward_mv", q, k, v)
+    B, H, N, Dk = q.shape
+    Dv = v.shape[-1]
+    o = torch.empty_like(v) if o is None else o
+    _check_qkv("la_forward_mv", v, o)
+    if g is not None and (g.dtype != torch.float32 or tuple(g.shape) != (B, H, N)
+                          or not g.is_contiguous()):
+        raise ValueError("la_forward_mv: g must be contiguous float32 [B, H, N]")
+    ws, ws_bytes = _workspace_mv(LA_OP_FORWARD, q, v, causal, workspace)
+    st = lib.la_forward_mv(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(g), B, H, N, Dk, Dv,
+                           DTYPE[q.dtype], int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
+                           _stream_handle(stream))
+    _check("la_forward_mv", st)
+    return o
+
+
+def la_backward_mv(q, k, v, dO, causal: bool = True, phi="identity", o=None, g=None, dq=None,
+                   dk=None, dv=None, workspace=None, stream=None):
+    """dq, dk [B, H, N, Dk] and dv [B, H, N, Dv] of sum(dO * O) for
+    O = la_forward_mv(q, k, v, causal, phi); o, g optional as in la_backward."""
+    lib = load_library()
+    _check_mv("la_backward_mv", q, k, v, dO)
+    B, H, N, Dk = q.shape
+    Dv = v.shape[-1]
+    if (o is None) != (g is None):
+        raise ValueError("la_backward_mv: pass both o and g or neither")
+    if o is not None:
+        _check_qkv("la_backward_mv", v, o)
+        if g.dtype != torch.float32 or tuple(g.shape) != (B, H, N) or not g.is_contiguous():
+            raise ValueError("la_backward_mv: g must be contiguous float32 [B, H, N]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_qkv("la_backward_mv", q, dq, dk)
+    _check_qkv("la_backward_mv", v, dv)
+    ws, ws_bytes = _workspace_mv(LA_OP_BACKWARD, q, v, causal, workspace)
+    st = lib.la_backward_mv(_ptr(q), _ptr(k), _ptr(v), _ptr(dO), _ptr(o), _ptr(g), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, H, N, Dk, Dv, DTYPE[q.dtype],
+                            int(bool(causal)), _phi(phi), _ptr(ws), ws_bytes,
+                            _stream_handle(stream))
+    _check("la_backward_mv", st)
+    return dq, dk, dv
 
 
 # ------------------------------------------------ sequence split across ranks

@@ -18,6 +18,7 @@
 
 #include "la_chunk_bwd.cuh"
 #include "la_favor.cuh"
+#include "la_pad.cuh"
 #include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
@@ -765,25 +766,25 @@ la_status run_bwd_chunked_d(const void* q, const void* k, const void* v, const v
 }
 
 // ------------------------------------------------------------ FAVOR+ features
-template <int D, bool BWD>
+template <int D, int M, bool BWD>
 la_status launch_favor(const void* x, const void* omega, const void* dphi, void* out,
                        int64_t heads, int64_t N, cudaStream_t st) {
-    using Cfg = la::FavorCfg<D, BWD>;
+    using Cfg = la::FavorCfg<D, M, BWD>;
     la::FavorParams prm;
     memset(&prm, 0, sizeof(prm));
     if (!make_qkv_map(&prm.tm_x, x, heads, N, D, Cfg::R) ||
-        !make_qkv_map(&prm.tm_w, omega, 1, D, D, D))
+        !make_qkv_map(&prm.tm_w, omega, 1, M, D, M))
         return LA_ERR_CUDA;
-    if (!BWD && !make_qkv_map(&prm.tm_phi, out, heads, N, D, Cfg::R)) return LA_ERR_CUDA;
-    if (BWD && (!make_qkv_map(&prm.tm_dphi, dphi, heads, N, D, Cfg::R) ||
+    if (!BWD && !make_qkv_map(&prm.tm_phi, out, heads, N, M, Cfg::R)) return LA_ERR_CUDA;
+    if (BWD && (!make_qkv_map(&prm.tm_dphi, dphi, heads, N, M, Cfg::R) ||
                 !make_qkv_map(&prm.tm_dx, out, heads, N, D, Cfg::R)))
         return LA_ERR_CUDA;
     const int64_t tph = (N + Cfg::R - 1) / Cfg::R;
     if (heads * tph >= (int64_t(1) << 31)) return LA_ERR_UNSUPPORTED;
     prm.tiles_per_head = int(tph);
     prm.ntiles = int(heads * tph);
-    prm.log_scale = -0.5f * logf(float(D));
-    auto kern = la::favor_kernel<D, BWD>;
+    prm.log_scale = -0.5f * logf(float(M));
+    auto kern = la::favor_kernel<D, M, BWD>;
     if (cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              Cfg::SMEM))
         return cuda_fail("cudaFuncSetAttribute", e);
@@ -791,6 +792,51 @@ la_status launch_favor(const void* x, const void* omega, const void* dphi, void*
     la::LaunchScope scope(BWD ? "favor_bwd" : "favor_fwd", st);
     kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(prm);
     return launch_status();
+}
+
+// Head size D and m features, each 64 or 128.
+template <bool BWD>
+la_status launch_favor_dm(int64_t D, int64_t m, const void* x, const void* omega,
+                          const void* dphi, void* out, int64_t heads, int64_t N,
+                          cudaStream_t st) {
+    if (D == 64)
+        return m == 64 ? launch_favor<64, 64, BWD>(x, omega, dphi, out, heads, N, st)
+                       : launch_favor<64, 128, BWD>(x, omega, dphi, out, heads, N, st);
+    return m == 64 ? launch_favor<128, 64, BWD>(x, omega, dphi, out, heads, N, st)
+                   : launch_favor<128, 128, BWD>(x, omega, dphi, out, heads, N, st);
+}
+
+// Rows of `ws` bf16 elements -> rows of `wd` (zero-filled past ws, or cut).
+la_status copy_cols(const void* src, void* dst, int64_t rows, int64_t ws, int64_t wd,
+                    cudaStream_t st) {
+    const int64_t total = rows * (wd / 8);
+    if (total == 0) return LA_OK;
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, int64_t(num_sms()) * 16);
+    la::LaunchScope scope("copy_cols", st);
+    la::copy_cols_kernel<<<unsigned(blocks), 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                           static_cast<uint4*>(dst), rows,
+                                                           int(ws / 8), int(wd / 8));
+    return launch_status();
+}
+
+// Attention with m = Dk features and head size Dv != Dk: workspace layout.
+// D = max(Dk, Dv); the narrower side's tensors are widened to D (`npad`
+// tensors of heads x N x D bf16 each), then the inner call's own workspace.
+struct MvPlan {
+    int64_t D = 0;
+    int npad = 0;
+    size_t tile = 0, inner_off = 0, inner = 0, bytes = 0;
+};
+MvPlan plan_mv(la_op op, int64_t B, int64_t H, int64_t N, int64_t Dk, int64_t Dv, int causal) {
+    MvPlan p;
+    p.D = std::max(Dk, Dv);
+    const int64_t heads = B * H;
+    p.tile = round_up(size_t(heads) * size_t(N) * size_t(p.D) * 2, 256);
+    if (Dk != Dv) p.npad = op == LA_OP_FORWARD ? 2 : 4;  // (v, o) | (q, k); bwd: + dO, o, dv | dq, dk
+    p.inner_off = size_t(p.npad) * p.tile;
+    p.inner = la_workspace_size(op, B, H, N, p.D, causal, LA_BF16);
+    p.bytes = p.inner_off + p.inner;
+    return p;
 }
 
 // ------------------------------------------------------------ generic path
@@ -1670,6 +1716,118 @@ la_status la_backward_sp_dkdv(const void* q, const void* k, const void* v, const
     });
 }
 
+size_t la_workspace_size_mv(la_op op, int64_t B, int64_t H, int64_t N, int64_t Dk, int64_t Dv,
+                            int causal, la_dtype dt) {
+    if (dt != LA_BF16 || (Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128)) return 0;
+    if (check_sizes(B, H, N, std::max(Dk, Dv)) != LA_OK || B * H == 0 || N == 0) return 0;
+    if (op != LA_OP_FORWARD && op != LA_OP_BACKWARD) return 0;
+    return plan_mv(op, B, H, N, Dk, Dv, causal ? 1 : 0).bytes;
+}
+
+namespace {
+
+// Shared checks of la_forward_mv / la_backward_mv.
+la_status check_mv(int64_t B, int64_t H, int64_t N, int64_t Dk, int64_t Dv, la_dtype dt,
+                   la_phi phi) {
+    la_status s;
+    if ((s = check_enums(dt, phi)) != LA_OK) return s;
+    if (Dk <= 0 || Dv <= 0) return LA_ERR_INVALID_ARG;
+    if (dt != LA_BF16 || (Dk != 64 && Dk != 128) || (Dv != 64 && Dv != 128))
+        return LA_ERR_UNSUPPORTED;
+    // zero feature columns add nothing only when the features are given
+    if (Dk < Dv && phi != LA_PHI_IDENTITY) return LA_ERR_UNSUPPORTED;
+    return check_sizes(B, H, N, std::max(Dk, Dv));
+}
+
+}  // namespace
+
+la_status la_forward_mv(const void* q, const void* k, const void* v, void* o, float* g_out,
+                        int64_t B, int64_t H, int64_t N, int64_t Dk, int64_t Dv, la_dtype dt,
+                        int causal, la_phi phi, void* workspace, size_t workspace_bytes,
+                        la_stream_t stream) {
+    la_status s;
+    if ((s = check_mv(B, H, N, Dk, Dv, dt, phi)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(o)))
+        return s;
+    if ((g_out && !aligned16(g_out)) || (workspace && !aligned16(workspace)))
+        return LA_ERR_INVALID_ARG;
+    const MvPlan p = plan_mv(LA_OP_FORWARD, B, H, N, Dk, Dv, causal);
+    if (p.bytes > 0 && (workspace == nullptr || workspace_bytes < p.bytes))
+        return LA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    char* inner = p.inner > 0 ? ws + p.inner_off : nullptr;
+    if (Dk == Dv)
+        return la_forward(q, k, v, o, nullptr, nullptr, g_out, nullptr, nullptr, B, H, N, Dk, dt,
+                          causal, phi, inner, p.inner, stream);
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t rows = heads * N, D = p.D;
+    void* t0 = ws;
+    void* t1 = ws + p.tile;
+    if (Dv < Dk) {
+        // values widened with zero columns; the output's first Dv columns
+        if ((s = copy_cols(v, t0, rows, Dv, D, st)) != LA_OK) return s;
+        if ((s = la_forward(q, k, t0, t1, nullptr, nullptr, g_out, nullptr, nullptr, B, H, N, D,
+                            dt, causal, phi, inner, p.inner, stream)) != LA_OK)
+            return s;
+        return copy_cols(t1, o, rows, D, Dv, st);
+    }
+    // features widened with zero columns (identity map)
+    if ((s = copy_cols(q, t0, rows, Dk, D, st)) != LA_OK) return s;
+    if ((s = copy_cols(k, t1, rows, Dk, D, st)) != LA_OK) return s;
+    return la_forward(t0, t1, v, o, nullptr, nullptr, g_out, nullptr, nullptr, B, H, N, D, dt,
+                      causal, phi, inner, p.inner, stream);
+}
+
+la_status la_backward_mv(const void* q, const void* k, const void* v, const void* dO,
+                         const void* o, const float* g, void* dq, void* dk, void* dv, int64_t B,
+                         int64_t H, int64_t N, int64_t Dk, int64_t Dv, la_dtype dt, int causal,
+                         la_phi phi, void* workspace, size_t workspace_bytes,
+                         la_stream_t stream) {
+    la_status s;
+    if ((s = check_mv(B, H, N, Dk, Dv, dt, phi)) != LA_OK) return s;
+    const int64_t heads = B * H;
+    if (heads == 0 || N == 0) return LA_OK;
+    if ((s = check_ptr(q)) || (s = check_ptr(k)) || (s = check_ptr(v)) || (s = check_ptr(dO)) ||
+        (s = check_ptr(dq)) || (s = check_ptr(dk)) || (s = check_ptr(dv)))
+        return s;
+    if ((o == nullptr) != (g == nullptr)) return LA_ERR_INVALID_ARG;
+    if (o && ((s = check_ptr(o)) || (s = check_ptr(g)))) return s;
+    if (workspace && !aligned16(workspace)) return LA_ERR_INVALID_ARG;
+    const MvPlan p = plan_mv(LA_OP_BACKWARD, B, H, N, Dk, Dv, causal);
+    if (p.bytes > 0 && (workspace == nullptr || workspace_bytes < p.bytes))
+        return LA_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    char* inner = p.inner > 0 ? ws + p.inner_off : nullptr;
+    if (Dk == Dv)
+        return la_backward(q, k, v, dO, o, g, nullptr, nullptr, dq, dk, dv, B, H, N, Dk, dt,
+                           causal, phi, inner, p.inner, stream);
+    if ((s = bind_context()) != LA_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t rows = heads * N, D = p.D;
+    void* t[4] = {ws, ws + p.tile, ws + 2 * p.tile, ws + 3 * p.tile};
+    if (Dv < Dk) {
+        // v, dO (and o) widened; dV is the first Dv columns of the wide dV
+        if ((s = copy_cols(v, t[0], rows, Dv, D, st)) != LA_OK) return s;
+        if ((s = copy_cols(dO, t[1], rows, Dv, D, st)) != LA_OK) return s;
+        if (o && (s = copy_cols(o, t[2], rows, Dv, D, st)) != LA_OK) return s;
+        if ((s = la_backward(q, k, t[0], t[1], o ? t[2] : nullptr, g, nullptr, nullptr, dq, dk,
+                             t[3], B, H, N, D, dt, causal, phi, inner, p.inner, stream)) != LA_OK)
+            return s;
+        return copy_cols(t[3], dv, rows, D, Dv, st);
+    }
+    // features widened (identity map); dQ, dK are the first Dk columns
+    if ((s = copy_cols(q, t[0], rows, Dk, D, st)) != LA_OK) return s;
+    if ((s = copy_cols(k, t[1], rows, Dk, D, st)) != LA_OK) return s;
+    if ((s = la_backward(t[0], t[1], v, dO, o, g, nullptr, nullptr, t[2], t[3], dv, B, H, N, D,
+                         dt, causal, phi, inner, p.inner, stream)) != LA_OK)
+        return s;
+    if ((s = copy_cols(t[2], dq, rows, D, Dk, st)) != LA_OK) return s;
+    return copy_cols(t[3], dk, rows, D, Dk, st);
+}
+
 namespace {
 
 la_status decode_impl(float* S, float* z, const void* q, const void* k, const void* v, void* o,
@@ -1715,13 +1873,16 @@ la_status la_decode_step(float* S, float* z, const void* q, const void* k, const
 
 namespace {
 
-// FAVOR+ sizes: bf16, m = D in {64, 128}
+// FAVOR+ sizes: bf16, D and m each 64 or 128
 la_status check_favor(int64_t B, int64_t H, int64_t N, int64_t D, int64_t m, la_dtype dt) {
     if (B < 0 || H < 0 || N < 0 || D <= 0 || m <= 0) return LA_ERR_INVALID_ARG;
     if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
-    if (dt != LA_BF16 || m != D || (D != 64 && D != 128)) return LA_ERR_UNSUPPORTED;
-    return check_sizes(B, H, N, D);
+    if (dt != LA_BF16 || (D != 64 && D != 128) || (m != 64 && m != 128))
+        return LA_ERR_UNSUPPORTED;
+    la_status s = check_sizes(B, H, N, D);
+    return s != LA_OK ? s : check_sizes(B, H, N, m);
 }
+
 
 }  // namespace
 
@@ -1734,8 +1895,7 @@ la_status la_favor_features(const void* x, const void* omega, void* phi, int64_t
     if ((s = check_ptr(x)) || (s = check_ptr(omega)) || (s = check_ptr(phi))) return s;
     if ((s = bind_context()) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return D == 64 ? launch_favor<64, false>(x, omega, nullptr, phi, heads, N, st)
-                   : launch_favor<128, false>(x, omega, nullptr, phi, heads, N, st);
+    return launch_favor_dm<false>(D, m, x, omega, nullptr, phi, heads, N, st);
 }
 
 la_status la_favor_features_backward(const void* x, const void* omega, const void* dphi,
@@ -1750,8 +1910,7 @@ la_status la_favor_features_backward(const void* x, const void* omega, const voi
         return s;
     if ((s = bind_context()) != LA_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    return D == 64 ? launch_favor<64, true>(x, omega, dphi, dx, heads, N, st)
-                   : launch_favor<128, true>(x, omega, dphi, dx, heads, N, st);
+    return launch_favor_dm<true>(D, m, x, omega, dphi, dx, heads, N, st);
 }
 
 uint64_t la_launch_count(void) { return la::profiler().launches.load(); }

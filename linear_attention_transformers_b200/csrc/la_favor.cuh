@@ -19,13 +19,12 @@
 // phi in fp32 (no stored features are read, and none of their rounding
 // enters dx), G is formed in fp32 and split into two bf16 parts G_hi + G_lo
 // (each rounded once), and G_hi W + G_lo W accumulate in TMEM; the epilogue
-// subtracts x s.  The MMAs are nearly free: with m = D the kernels do 32
-// (D = 64) to 64 (D = 128) flops per byte moved, a tenth of the tensor
-// cores' balance point, so they run at the speed of HBM.  tcgen05 MMAs with
-// TMEM accumulators (two buffers), TMA-fed stages,
-// omega held in shared memory for the whole persistent kernel, one CTA per
-// SM looping over the 128-row tiles of every head.  m = D (64 or 128): the
-// attention kernels take features of the head size.
+// subtracts x s.  The MMAs are nearly free: the kernels do 2 D m / (D + m)
+// flops per byte moved (32 to 64), a tenth of the tensor cores' balance
+// point, so they run at the speed of HBM.  tcgen05 MMAs with TMEM
+// accumulators (two buffers), TMA-fed stages, omega held in shared memory
+// for the whole persistent kernel, one CTA per SM looping over the 128-row
+// tiles of every head.  D and m are each 64 or 128.
 #pragma once
 
 #include "la_chunk_bwd.cuh"
@@ -43,37 +42,40 @@ struct FavorParams {
     float log_scale;      // -ln(m) / 2
 };
 
-// Forward: per stage one x tile [128][D]; the output [128][m] is staged over
-// it once each row's |x|^2 is read.  Backward: per stage the x and dphi
-// tiles and one more [128][m] tile: G_hi is formed over dphi, G_lo in the
-// third tile, and dx is staged over the third tile once the MMAs have read
-// it.  TMEM (backward): per buffer b the product P (m columns) and the dx
+// Head size D, M = m features.  Forward: per stage one x tile [128][D] and
+// the output [128][M], staged over x when M <= D (once each row's |x|^2 is
+// read), else in its own tile.  Backward: per stage the x tile and two
+// [128][M] tiles: G_hi is formed over dphi, G_lo in the third tile; dx is
+// staged over x (each thread reads its row's x before it writes that row).
+// TMEM: per buffer b the product P (M columns) and, backward, the dx
 // accumulator (D columns).
-template <int D, bool BWD>
+template <int D, int M, bool BWD>
 struct FavorCfg {
     static constexpr int R = 128;
     static constexpr int NS = BWD ? 2 : 3;
-    static constexpr int TILE = R * D * 2;
-    static constexpr int STAGE = (BWD ? 3 : 1) * TILE;
-    static constexpr int OFF_W = NS * STAGE;            // omega [m][D] row tile (m = D)
-    static constexpr int OFF_S = OFF_W + D * D * 2;     // backward: row sums s [NS][R] float
+    static constexpr int XT = R * D * 2;                 // x / dx tile
+    static constexpr int PT = R * M * 2;                 // phi / dphi / G tile
+    static constexpr int OFF_OUT = (!BWD && M > D) ? XT : 0;  // forward output staging
+    static constexpr int STAGE = BWD ? XT + 2 * PT : XT + (M > D ? PT : 0);
+    static constexpr int OFF_W = NS * STAGE;            // omega [M][D] row tile
+    static constexpr int OFF_S = OFF_W + M * D * 2;     // backward: row sums s [NS][R] float
     static constexpr int OFF_BAR = OFF_S + (BWD ? NS * R * 4 : 0);
     static constexpr int NBAR = 4 * NS + 7;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
-    static constexpr int ACC = BWD ? 2 * D : D;  // TMEM columns per buffer
+    static constexpr int ACC = BWD ? M + D : M;  // TMEM columns per buffer
     static constexpr int T_COLS = 2 * ACC <= 128 ? 128 : (2 * ACC <= 256 ? 256 : 512);
     static constexpr int THREADS = BWD ? 320 : 192;
     static_assert(SMEM <= 227 * 1024, "shared memory budget");
     static_assert(2 * ACC <= 512, "TMEM budget");
 };
 
-template <int D, bool BWD>
-__global__ void __launch_bounds__(FavorCfg<D, BWD>::THREADS, 1)
+template <int D, int M, bool BWD>
+__global__ void __launch_bounds__(FavorCfg<D, M, BWD>::THREADS, 1)
 favor_kernel(const __grid_constant__ FavorParams prm) {
     using namespace sm100;
-    using Cfg = FavorCfg<D, BWD>;
-    constexpr int R = Cfg::R, NS = Cfg::NS, M = D;
+    using Cfg = FavorCfg<D, M, BWD>;
+    constexpr int R = Cfg::R, NS = Cfg::NS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -133,7 +135,7 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
 #pragma unroll
             for (int a = 0; a < D / 64; ++a)
                 tma_load_3d(smem + Cfg::OFF_W + a * M * 128, &prm.tm_w, w_full, a * 64, 0, 0);
-            constexpr uint32_t bytes = uint32_t((BWD ? 2 : 1) * Cfg::TILE);
+            constexpr uint32_t bytes = uint32_t(BWD ? Cfg::XT + Cfg::PT : Cfg::XT);
             int issued = 0;
             for (int i = 0; i < my_tiles; ++i) {
                 const int s = i % NS;
@@ -143,10 +145,12 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
                 uint8_t* st = smem + s * Cfg::STAGE;
                 mbar_arrive_expect_tx(&full[s], bytes);
 #pragma unroll
-                for (int a = 0; a < D / 64; ++a) {
+                for (int a = 0; a < D / 64; ++a)
                     tma_load_3d(st + a * R * 128, &prm.tm_x, &full[s], a * 64, row0, head);
-                    if (BWD)
-                        tma_load_3d(st + Cfg::TILE + a * R * 128, &prm.tm_dphi, &full[s], a * 64,
+                if (BWD) {
+#pragma unroll
+                    for (int a = 0; a < M / 64; ++a)
+                        tma_load_3d(st + Cfg::XT + a * R * 128, &prm.tm_dphi, &full[s], a * 64,
                                     row0, head);
                 }
                 issued = i + 1;
@@ -185,8 +189,8 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
                         break;
                     tc_fence_after();
                     const uint32_t accG = accP + uint32_t(M);
-                    const uint64_t gh = desc_k_base(st + Cfg::TILE);      // G_hi
-                    const uint64_t gl = desc_k_base(st + 2 * Cfg::TILE);  // G_lo
+                    const uint64_t gh = desc_k_base(st + Cfg::XT);            // G_hi
+                    const uint64_t gl = desc_k_base(st + Cfg::XT + Cfg::PT);  // G_lo
 #pragma unroll
                     for (int k = 0; k < M; k += 16)
                         umma_bf16(accG, gh + kstep_k(R, k), wm + kstep_mn(k), idG, k > 0);
@@ -212,8 +216,8 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
             if (!mbar_wait(&p_full[b], (i >> 1) & 1, abort_flag)) break;
             tc_fence_after();
             const uint8_t* xt = smem + s * Cfg::STAGE;
-            uint8_t* gt = smem + s * Cfg::STAGE + Cfg::TILE;       // dphi -> G_hi
-            uint8_t* lt = smem + s * Cfg::STAGE + 2 * Cfg::TILE;   // G_lo
+            uint8_t* gt = smem + s * Cfg::STAGE + Cfg::XT;             // dphi -> G_hi
+            uint8_t* lt = smem + s * Cfg::STAGE + Cfg::XT + Cfg::PT;   // G_lo
             float hsq = 0.f;
 #pragma unroll 4
             for (int q = 0; q < D / 8; ++q) {
@@ -269,7 +273,7 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
             tc_fence_after();
             uint8_t* xt = smem + s * Cfg::STAGE;
             const uint32_t acc = tmem + lane_base + uint32_t(b * Cfg::ACC) + (BWD ? uint32_t(M) : 0u);
-            uint8_t* ot = BWD ? xt + 2 * Cfg::TILE : xt;  // output staging
+            uint8_t* ot = xt + Cfg::OFF_OUT;  // output staging (dx: over x)
             if constexpr (BWD) {
                 // dx = G W - x s
                 const float sr = srow[s * R + r];
@@ -312,7 +316,7 @@ favor_kernel(const __grid_constant__ FavorParams prm) {
             named_bar_sync(1, 128);
             if (e == 0) {
 #pragma unroll
-                for (int a = 0; a < D / 64; ++a)
+                for (int a = 0; a < (BWD ? D : M) / 64; ++a)
                     tma_store_3d(BWD ? &prm.tm_dx : &prm.tm_phi, ot + a * R * 128, a * 64, row0,
                                  head);
                 bulk_commit();

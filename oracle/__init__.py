@@ -29,6 +29,10 @@ Functions (all arrays [B, H, N, D] contiguous, D innermost):
       m^-1/2 exp(-|x|^2/2) [exp(w_1.x), ..., exp(w_m.x)], omega [m, D] the
       random directions; with phi = PHI_IDENTITY the functions above then
       take phi(q), phi(k) as their q, k
+  forward_mv(q, k, v, causal, phi)         -> o [..., Dv]
+  backward_mv(q, k, v, dO, causal, phi)    -> dq, dk [..., Dk], dv [..., Dv]
+      features q, k of length Dk (e.g. m Performer features) and values of
+      length Dv: S is Dk x Dv
 """
 from __future__ import annotations
 
@@ -240,6 +244,46 @@ def favor_features_backward(x, omega, dphi) -> np.ndarray:
     w = _f64(omega)
     g = _f64(dphi) * favor_features(x, w)            # dphi_i phi_i
     return g @ w - x * g.sum(axis=-1, keepdims=True)
+
+
+# ------------------------------------------- feature length m != head size D
+# The Proposition "Linear Attention via Kernel Decomposition" takes phi:
+# R^d -> R^m, so S = sum_j phi(k_j) v_j^T is m x D ("Efficient Transformers
+# Survey"; with the Performer's m random features, Low-Rank Approximations,
+# Performer).  The functions above take one width for q, k and v; these
+# widen the narrower side with zero columns and cut the result back, which
+# is the same sums: a zero value column gives a zero output column (and dV
+# column), a zero feature column adds 0 to every a_i . b_j and to z (given
+# features, phi = PHI_IDENTITY, so the zero stays zero).
+
+def _widen(x, w: int) -> np.ndarray:
+    x = _f64(x)
+    out = np.zeros((*x.shape[:-1], w))
+    out[..., :x.shape[-1]] = x
+    return out
+
+
+def forward_mv(q, k, v, causal: bool, phi: int = PHI_IDENTITY) -> np.ndarray:
+    """o [B, H, N, Dv] for features q, k [B, H, N, Dk] and values v [..., Dv]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    dk, dv = q.shape[-1], v.shape[-1]
+    if dk < dv and phi != PHI_IDENTITY:
+        raise ValueError("zero feature columns need the identity map")
+    D = max(dk, dv)
+    o, _, _ = forward(_widen(q, D), _widen(k, D), _widen(v, D), causal, phi)
+    return np.ascontiguousarray(o[..., :dv])
+
+
+def backward_mv(q, k, v, dO, causal: bool, phi: int = PHI_IDENTITY):
+    """dq, dk [B, H, N, Dk] and dv [B, H, N, Dv] of sum(dO * O)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    dk_, dv_ = q.shape[-1], v.shape[-1]
+    if dk_ < dv_ and phi != PHI_IDENTITY:
+        raise ValueError("zero feature columns need the identity map")
+    D = max(dk_, dv_)
+    dq, dk, dv = backward(_widen(q, D), _widen(k, D), _widen(v, D), _widen(dO, D), causal, phi)
+    return (np.ascontiguousarray(dq[..., :dk_]), np.ascontiguousarray(dk[..., :dk_]),
+            np.ascontiguousarray(dv[..., :dv_]))
 
 
 # ---------------------------------------------------- grouped key/value heads

@@ -151,8 +151,10 @@ def test_decay_factors_are_validated_before_launch(lib):
 
 def test_favor_sizes_are_validated_before_launch(lib):
     p = FAKE
-    # m != D, float32, D = 32: not offered
-    assert lib.la_favor_features(p, p, p, 1, 2, 8, 64, 128, api.LA_BF16, None) == \
+    # m = 256 or 32, float32, D = 32: not offered
+    assert lib.la_favor_features(p, p, p, 1, 2, 8, 64, 256, api.LA_BF16, None) == \
+        api.LA_ERR_UNSUPPORTED
+    assert lib.la_favor_features(p, p, p, 1, 2, 8, 128, 32, api.LA_BF16, None) == \
         api.LA_ERR_UNSUPPORTED
     assert lib.la_favor_features(p, p, p, 1, 2, 8, 64, 64, api.LA_F32, None) == \
         api.LA_ERR_UNSUPPORTED
@@ -171,3 +173,26 @@ def test_favor_sizes_are_validated_before_launch(lib):
                           1, 2, None, 0, None) == api.LA_ERR_INVALID_ARG
     assert lib.la_forward(p, p, p, p, None, None, None, None, None, 1, 1, 8, 64, api.LA_BF16,
                           1, 3, None, 0, None) == api.LA_ERR_INVALID_ARG
+
+
+def test_mv_calls_reject_bad_arguments_before_launch(lib):
+    B, H, N = 1, 2, 100
+    bf, f32 = api.LA_BF16, api.LA_F32
+
+    def fwd(Dk=128, Dv=64, dt=bf, phi=0, ws=None, ws_bytes=0, q=FAKE):
+        return lib.la_forward_mv(q, FAKE, FAKE, FAKE, None, B, H, N, Dk, Dv, dt, 1, phi, ws,
+                                 ws_bytes, None)
+
+    need = lib.la_workspace_size_mv(api.LA_OP_FORWARD, B, H, N, 128, 64, 1, bf)
+    assert need >= 2 * B * H * N * 128 * 2  # widened v and o
+    assert fwd(ws=FAKE, ws_bytes=need, q=None) == api.LA_ERR_INVALID_ARG
+    assert fwd(Dk=96) == api.LA_ERR_UNSUPPORTED
+    assert fwd(dt=f32) == api.LA_ERR_UNSUPPORTED
+    assert fwd(Dk=64, Dv=128, phi=0) == api.LA_ERR_UNSUPPORTED      # zero features need identity
+    assert fwd(ws=FAKE, ws_bytes=need - 256) == api.LA_ERR_WORKSPACE
+    assert lib.la_workspace_size_mv(api.LA_OP_FORWARD, B, H, N, 128, 64, 1, f32) == 0
+    need_b = lib.la_workspace_size_mv(api.LA_OP_BACKWARD, B, H, N, 64, 128, 1, bf)
+    assert lib.la_backward_mv(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, B, H, N, 64,
+                              128, bf, 1, 2, FAKE, need_b, None) == api.LA_ERR_INVALID_ARG
+    assert lib.la_backward_mv(FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, B, H, N, 64,
+                              128, bf, 1, 2, FAKE, need_b - 256, None) == api.LA_ERR_WORKSPACE

@@ -517,3 +517,56 @@ def test_identity_map_backward_matches_finite_differences():
     ref = fd_grads(q, k, v, dO, True, oracle.PHI_IDENTITY)
     for a, b in zip(got, ref):
         np.testing.assert_allclose(a, b, rtol=1e-6, atol=1e-9)
+
+
+@pytest.mark.parametrize("dk,dv,phi", [(6, 3, PHI_ELU1), (6, 3, oracle.PHI_IDENTITY),
+                                       (3, 6, oracle.PHI_IDENTITY)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_mv_forward_is_the_quadratic_form_with_features_and_values_of_two_lengths(dk, dv, phi,
+                                                                                 causal):
+    # S = sum_j phi(k_j) v_j^T is dk x dv: the quadratic form of the
+    # Proposition with A [N, dk], B [N, dk] and V [N, dv], written directly
+    g = np.random.default_rng(406 + dk)
+    N = 11
+    if phi == oracle.PHI_IDENTITY:
+        q, k = np.exp(g.standard_normal((2, 1, N, dk)) * 0.5), np.exp(g.standard_normal((2, 1, N, dk)) * 0.5)
+        a, b = q, k
+    else:
+        q, k = g.standard_normal((2, 1, N, dk)), g.standard_normal((2, 1, N, dk))
+        a, b = oracle.phi_map(q, phi), oracle.phi_map(k, phi)
+    v = g.standard_normal((2, 1, N, dv))
+    w = np.einsum("bhid,bhjd->bhij", a, b)
+    if causal:
+        w = np.tril(w)
+    ref = np.einsum("bhij,bhje->bhie", w, v) / w.sum(-1, keepdims=True)
+    o = oracle.forward_mv(q, k, v, causal, phi)
+    assert o.shape == (2, 1, N, dv)
+    np.testing.assert_allclose(o, ref, rtol=1e-12)
+
+
+def test_mv_refuses_zero_features_under_a_feature_map():
+    x = np.ones((1, 1, 2, 3))
+    with pytest.raises(ValueError):
+        oracle.forward_mv(x, x, np.ones((1, 1, 2, 6)), True, PHI_ELU1)
+
+
+@pytest.mark.parametrize("dk,dv", [(5, 3), (3, 5)])
+def test_mv_backward_matches_finite_differences(dk, dv):
+    g = np.random.default_rng(407 + dk)
+    N, h = 7, 1e-6
+    q = np.exp(g.standard_normal((1, 1, N, dk)) * 0.5)
+    k = np.exp(g.standard_normal((1, 1, N, dk)) * 0.5)
+    v, dO = g.standard_normal((1, 1, N, dv)), g.standard_normal((1, 1, N, dv))
+    got = oracle.backward_mv(q, k, v, dO, True, oracle.PHI_IDENTITY)
+    loss = lambda qq, kk, vv: float((dO * oracle.forward_mv(qq, kk, vv, True)).sum())  # noqa: E731
+    for idx, x in enumerate((q, k, v)):
+        fd = np.zeros_like(x)
+        for pos in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[pos] += h
+            xm[pos] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[idx], args_m[idx] = xp, xm
+            fd[pos] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+        np.testing.assert_allclose(got[idx], fd, rtol=1e-6, atol=1e-9)
