@@ -130,6 +130,17 @@ decode_step_gqa_kernel(float* __restrict__ S, float* __restrict__ z,
     float4 s[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) s[r] = __ldcs(Sh + (rg + RG * r) * CG + cg);
+    // the queries of batch g0 (QB of them), loaded one batch ahead so that
+    // their latency hides behind the state loads and the previous batch
+    float xq[QB];
+    auto load_q = [&](int g0) {
+        if (tid < D) {
+#pragma unroll
+            for (int i = 0; i < QB; ++i)
+                xq[i] = g0 + i < G ? to_f32(q[(hk * G + g0 + i) * D + tid]) : 0.f;
+        }
+    };
+    load_q(0);
     if (tid < D) {
         const float xk = to_f32(k[hk * D + tid]);
         const float bf = kExact ? phi_exact<PHI>(xk) : phi_fast<PHI>(xk);
@@ -157,20 +168,19 @@ decode_step_gqa_kernel(float* __restrict__ S, float* __restrict__ z,
         const int nq = min(QB, G - g0);
         __syncthreads();  // a_s, part, den_s of the previous batch are consumed
         if (tid < D) {
-            for (int i = 0; i < nq; ++i) {
-                const float xq = to_f32(q[(hk * G + g0 + i) * D + tid]);
-                a_s[i][tid] = kExact ? phi_exact<PHI>(xq) : phi_fast<PHI>(xq);
-            }
+#pragma unroll
+            for (int i = 0; i < QB; ++i)
+                if (i < nq) a_s[i][tid] = kExact ? phi_exact<PHI>(xq[i]) : phi_fast<PHI>(xq[i]);
         }
+        if (g0 + QB < G) load_q(g0 + QB);
         __syncthreads();
-        if (tid < 32) {
-            // denominators phi(q) . z, one warp, fixed order
-            for (int i = 0; i < nq; ++i) {
-                float d = 0.f;
-                for (int f = tid; f < D; f += 32) d = fmaf(a_s[i][f], z_s[f], d);
-                d = warp_sum(d);
-                if (tid == 0) den_s[i] = d;
-            }
+        // denominators phi(q) . z, query i by warp i mod (warps), fixed order
+        for (int i = tid >> 5; i < nq; i += NT / 32) {
+            const int l = tid & 31;
+            float d = 0.f;
+            for (int f = l; f < D; f += 32) d = fmaf(a_s[i][f], z_s[f], d);
+            d = warp_sum(d);
+            if (l == 0) den_s[i] = d;
         }
         for (int i = 0; i < nq; ++i) {
             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
