@@ -698,42 +698,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             float tcoef = 0.f;
             if (kc != 0.f) {
                 float dot = 0.f, sa = 0.f;
+                // 32 columns per TMEM round trip (two loads, one wait)
 #pragma unroll 1
-                for (int f0 = 0; f0 < D; f0 += 16) {
-                    float av[16];
-                    tmem_ld16(tmem + lane_base + Cfg::T_O + f0, av);
-                    tmem_wait_ld();
+                for (int f0 = 0; f0 < D; f0 += 32) {
+                    float av[32];
+                    tmem_load<32>(tmem + lane_base + Cfg::T_O + f0, av);
                     if (irow >= 0) {
-                        float a8a[8], a8b[8];
-                        load_chunk8(qt, C, irow, f0 >> 3, a8a);
-                        load_chunk8(qt, C, irow, (f0 >> 3) + 1, a8b);
 #pragma unroll
-                        for (int t = 0; t < 8; ++t) {
-                            dot = fmaf(fmaf(dg, zf[f0 + t], av[t]), a8a[t], dot);
-                            dot = fmaf(fmaf(dg, zf[f0 + 8 + t], av[8 + t]), a8b[t], dot);
-                            sa += a8a[t] + a8b[t];
+                        for (int h = 0; h < 4; ++h) {
+                            float a8[8];
+                            load_chunk8(qt, C, irow, (f0 >> 3) + h, a8);
+#pragma unroll
+                            for (int t = 0; t < 8; ++t) {
+                                dot = fmaf(fmaf(dg, zf[f0 + 8 * h + t], av[8 * h + t]), a8[t], dot);
+                                sa += a8[t];
+                            }
                         }
                     }
                 }
                 tcoef = irow >= 0 ? -kc * dot / sa : 0.f;
             }
 #pragma unroll 1
-            for (int f0 = 0; f0 < D; f0 += 16) {
-                float av[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_O + f0, av);
-                tmem_wait_ld();
+            for (int f0 = 0; f0 < D; f0 += 32) {
+                float av[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_O + f0, av);
                 if (irow >= 0) {
-                    float a8a[8], a8b[8];
-                    load_chunk8(qt, C, irow, f0 >> 3, a8a);
-                    load_chunk8(qt, C, irow, (f0 >> 3) + 1, a8b);
-                    float dq16[16];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        dq16[t] = (fmaf(dg, zf[f0 + t], av[t]) + tcoef) * dphi_from_phi<PHI>(a8a[t]);
-                        dq16[8 + t] =
-                            (fmaf(dg, zf[f0 + 8 + t], av[8 + t]) + tcoef) * dphi_from_phi<PHI>(a8b[t]);
+                    for (int h = 0; h < 2; ++h) {
+                        float a8a[8], a8b[8];
+                        load_chunk8(qt, C, irow, (f0 >> 3) + 2 * h, a8a);
+                        load_chunk8(qt, C, irow, (f0 >> 3) + 2 * h + 1, a8b);
+                        float dq16[16];
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) {
+                            const int f = f0 + 16 * h + t;
+                            dq16[t] = (fmaf(dg, zf[f], av[16 * h + t]) + tcoef) *
+                                      dphi_from_phi<PHI>(a8a[t]);
+                            dq16[8 + t] = (fmaf(dg, zf[f + 8], av[16 * h + 8 + t]) + tcoef) *
+                                          dphi_from_phi<PHI>(a8b[t]);
+                        }
+                        store_row16_bf16(stg, C, irow, f0 + 16 * h, dq16);
                     }
-                    store_row16_bf16(stg, C, irow, f0, dq16);
                 }
             }
             fence_proxy_async_smem();
@@ -747,16 +752,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             }
             // ---- next state operand; segment (R, r) on the last chunk
             if (CAUSAL) {
-#pragma unroll 1
-                for (int v0 = 0; v0 < D; v0 += 16) {
-                    float sv[16];
-                    tmem_ld16(tmem + lane_base + Cfg::T_S + v0, sv);
-                    tmem_wait_ld();
-                    if (frow >= 0) store_row16_bf16(sprev, D, frow, v0, sv);
-                }
+                // z rides along with the first S columns' round trip
                 float zv[16];
                 tmem_ld16(tmem + lane_base + Cfg::T_Z, zv);
-                tmem_wait_ld();
+#pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 32) {
+                    float sv[32];
+                    tmem_load<32>(tmem + lane_base + Cfg::T_S + v0, sv);
+                    if (frow >= 0) {
+                        store_row16_bf16(sprev, D, frow, v0, sv);
+                        store_row16_bf16(sprev, D, frow, v0 + 16, sv + 16);
+                    }
+                }
                 if (frow >= 0) {
                     const __nv_bfloat16 zh = __float2bfloat16_rn(zv[0]);
                     zop_h[tile_off(16, 0, frow) / 2] = zh;
@@ -1062,22 +1069,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     if (e == 0) bulk_wait_read0();
                     named_bar_sync(1, 128);
                 }
+                // 32 columns of each product per TMEM round trip
 #pragma unroll 1
-                for (int i0 = 0; i0 < C; i0 += 16) {
-                    float pv[16], wv[16];
-                    tmem_ld16(tmem + lane_base + Cfg::T_1 + i0, pv);
-                    tmem_ld16(tmem + lane_base + Cfg::T_2 + i0, wv);
+                for (int i0 = 0; i0 < C; i0 += 32) {
+                    float pv[32], wv[32];
+                    sm100::tmem_ld16(tmem + lane_base + Cfg::T_1 + i0, pv);
+                    sm100::tmem_ld16(tmem + lane_base + Cfg::T_1 + i0 + 16, pv + 16);
+                    sm100::tmem_ld16(tmem + lane_base + Cfg::T_2 + i0, wv);
+                    sm100::tmem_ld16(tmem + lane_base + Cfg::T_2 + i0 + 16, wv + 16);
                     tmem_wait_ld();
                     if (jrow >= 0) {
-                        float a16[16], b16[16];
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) {
-                            const int i = i0 + k;
-                            a16[k] = i >= jrow ? pv[k] : 0.f;
-                            b16[k] = i >= jrow ? wv[k] + dgf[i] : 0.f;
+                        for (int h = 0; h < 2; ++h) {
+                            float a16[16], b16[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                const int i = i0 + 16 * h + k;
+                                a16[k] = i >= jrow ? pv[16 * h + k] : 0.f;
+                                b16[k] = i >= jrow ? wv[16 * h + k] + dgf[i] : 0.f;
+                            }
+                            store_row16_bf16(x1, C, jrow, i0 + 16 * h, a16);
+                            store_row16_bf16(x2, C, jrow, i0 + 16 * h, b16);
                         }
-                        store_row16_bf16(x1, C, jrow, i0, a16);
-                        store_row16_bf16(x2, C, jrow, i0, b16);
                     }
                 }
                 }
@@ -1131,16 +1144,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 bulk_commit();
             }
             if (CAUSAL) {
-#pragma unroll 1
-                for (int v0 = 0; v0 < D; v0 += 16) {
-                    float rv[16];
-                    tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
-                    tmem_wait_ld();
-                    if (frow >= 0) store_row16_bf16(rprev, D, frow, v0, rv);
-                }
+                // r rides along with the first R columns' round trip
                 float rz[16];
                 tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
-                tmem_wait_ld();
+#pragma unroll 1
+                for (int v0 = 0; v0 < D; v0 += 32) {
+                    float rv[32];
+                    tmem_load<32>(tmem + lane_base + Cfg::T_R + v0, rv);
+                    if (frow >= 0) {
+                        store_row16_bf16(rprev, D, frow, v0, rv);
+                        store_row16_bf16(rprev, D, frow, v0 + 16, rv + 16);
+                    }
+                }
                 if (frow >= 0) rf[frow] = rz[0] + rz[1];
             }
             fence_proxy_async_smem();
