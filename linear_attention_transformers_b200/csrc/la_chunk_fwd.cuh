@@ -528,20 +528,21 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                         }
                         tmem_wait_st();
                     } else if (!last || write_final) {
+                        // 32 state columns per TMEM round trip, z with the first
+                        float zv[16];
+                        sm100::tmem_ld16(tmem + lane_base + Cfg::T_Z, zv);
 #pragma unroll 1
-                        for (int v0 = 0; v0 < D; v0 += 16) {
-                            float sv[16];
-                            tmem_load<16>(tmem + lane_base + Cfg::T_S + v0, sv);
+                        for (int v0 = 0; v0 < D; v0 += 32) {
+                            float sv[32];
+                            tmem_load<32>(tmem + lane_base + Cfg::T_S + v0, sv);
                             if (frow >= 0) {
-                                store_row_bf16<16>(sx, D, frow, v0, sv);
+                                store_row_bf16<32>(sx, D, frow, v0, sv);
                                 if (write_final)
-                                    for (int t = 0; t < 16; ++t)
+                                    for (int t = 0; t < 32; ++t)
                                         prm.S_out[sidx * prm.stride_S + size_t(frow) * D + v0 + t] =
                                             sv[t];
                             }
                         }
-                        float zv[16];
-                        tmem_load<16>(tmem + lane_base + Cfg::T_Z, zv);
                         if (frow >= 0) {
                             put_z(zv[0]);
                             if (write_final && prm.z_out)
@@ -558,15 +559,19 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                 if (e == 0) bulk_wait_read0();
                 named_bar_sync(2, 128);
                 const uint32_t tO = tmem + lane_base + Cfg::T_O + bo * (D + 16);
-                float oz[16];
-                tmem_load<16>(tO + D, oz);
+                // the denominator columns ride along with the first 32
+                // numerator columns (one TMEM round trip for both)
+                float oz[16], ov[32];
+                sm100::tmem_ld16(tO + D, oz);
+                sm100::tmem_ld16(tO, ov);
+                sm100::tmem_ld16(tO + 16, ov + 16);
+                sm100::tmem_wait_ld();
                 const float inv = 1.f / (oz[0] + oz[1]);
                 if (prm.g_out && irow >= 0 && row0 + irow < tok1)
                     prm.g_out[size_t(head) * prm.N + row0 + irow] = oz[0] + oz[1];
 #pragma unroll 1
                 for (int v0 = 0; v0 < D; v0 += 32) {
-                    float ov[32];
-                    tmem_load<32>(tO + v0, ov);
+                    if (v0 > 0) tmem_load<32>(tO + v0, ov);
                     if (irow >= 0) {
 #pragma unroll
                         for (int t = 0; t < 32; ++t) ov[t] *= inv;
