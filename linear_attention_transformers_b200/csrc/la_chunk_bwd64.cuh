@@ -481,12 +481,23 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             }
             if (!named_bar_all(2, 128, mbar_wait(d_full, t & 1, abort_flag))) break;
             tc_fence_after();
+            // NB 16-column groups of dV and dB per TMEM round trip (one
+            // for the float32-partials variant, whose registers are tighter)
+            constexpr int NB = PART ? 1 : 2;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float dv16[16], db16[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_DV + c0, dv16);
-                tmem_ld16(tmem + lane_base + Cfg::T_DB + c0, db16);
+            for (int c2 = 0; c2 < D; c2 += 16 * NB) {
+                float dvx[16 * NB], dbx[16 * NB];
+#pragma unroll
+                for (int hh = 0; hh < NB; ++hh) {
+                    tmem_ld16(tmem + lane_base + Cfg::T_DV + c2 + 16 * hh, dvx + 16 * hh);
+                    tmem_ld16(tmem + lane_base + Cfg::T_DB + c2 + 16 * hh, dbx + 16 * hh);
+                }
                 tmem_wait_ld();
+#pragma unroll
+                for (int hh = 0; hh < NB; ++hh) {
+                const int c0 = c2 + 16 * hh;
+                float* dv16 = dvx + 16 * hh;
+                const float* db16 = dbx + 16 * hh;
                 float b8a[8], b8b[8];
                 load_chunk8(kt, C, jrow, c0 >> 3, b8a);
                 load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
@@ -526,6 +537,7 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
                     store_row16_bf16(vt, C, jrow, c0, dv16);
                     store_row16_bf16(kt, C, jrow, c0, dk16);
                 }
+                }
             }
             tc_fence_before();
             mbar_arrive(d_free);
@@ -539,16 +551,19 @@ bwd_dkdv64_kernel(const __grid_constant__ BwdParams prm) {
             // start; the next (earlier, full) chunk wants gamma^(C/2) R
             const float fr = DECAY ? exp2f(lg * (0.5f * float(C) + m)) : 1.f;
 #pragma unroll 1
-            for (int v0 = 0; v0 < D; v0 += 16) {
-                float rv[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_R + v0, rv);
-                tmem_wait_ld();
+            for (int v0 = 0; v0 < D; v0 += 32) {
+                float rv[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_R + v0, rv);
                 if constexpr (DECAY) {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) rv[i] *= fr;
+                    for (int i = 0; i < 32; ++i) rv[i] *= fr;
                     tmem_st16(tmem + lane_base + Cfg::T_R + v0, rv);
+                    tmem_st16(tmem + lane_base + Cfg::T_R + v0 + 16, rv + 16);
                 }
-                if (frow >= 0) store_row16_bf16(rp, D, frow, v0, rv);
+                if (frow >= 0) {
+                    store_row16_bf16(rp, D, frow, v0, rv);
+                    store_row16_bf16(rp, D, frow, v0 + 16, rv + 16);
+                }
             }
             if constexpr (DECAY) tmem_wait_st();
             if (!named_bar_all(2, 128, mbar_wait(&rch_full[t & 1], (t >> 1) & 1, abort_flag))) break;
