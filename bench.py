@@ -139,15 +139,15 @@ _BWD64_SOURCES = ["la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "
 MEASURED_TRAFFIC = {
     # one `ncu --set full` launch each at B8 H16 N4096 D64 (the timed
     # workload at half its tokens)
-    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.389824e6 + 156.388096e6) / (8 * 16 * 4096),
+    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.429760e6 + 156.376832e6) / (8 * 16 * 4096),
                      "files": _FWD64_SOURCES,
-                     "sources": "4428205c90e85ea659b2689738ef639eb8b0f0d693f025e685750113ac3f3f72"},
-    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.711104e6 + 52.814592e6) / (8 * 16 * 4096),
+                     "sources": "0f58f7cf746f364f634f86df1468f8d8ea5919d0f015d921d5650cbdbab58893"},
+    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.764864e6 + 53.445888e6) / (8 * 16 * 4096),
                "files": _BWD64_SOURCES,
-               "sources": "3284c03f2cc26e248f2f0fc71dc80afb241386e8c7079cf32f7b44ff67780b89"},
-    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.682496e6 + 99.994880e6) / (8 * 16 * 4096),
+               "sources": "a1579f5b5909c8a1adf65b4b6ea2271ddfa4fa1a55a7f5a9c2be109edabf8749"},
+    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.685056e6 + 100.026368e6) / (8 * 16 * 4096),
                  "files": _BWD64_SOURCES,
-                 "sources": "3284c03f2cc26e248f2f0fc71dc80afb241386e8c7079cf32f7b44ff67780b89"},
+                 "sources": "a1579f5b5909c8a1adf65b4b6ea2271ddfa4fa1a55a7f5a9c2be109edabf8749"},
 }
 
 
