@@ -165,3 +165,42 @@ def test_two_processes_over_gloo():
     rq, rk, rv = oracle.backward(q, k, v, dO, True, oracle.PHI_ELU1)
     for name, ref in (("o", o_ref), ("dq", rq), ("dk", rk), ("dv", rv)):
         compare(torch.cat([res[0][name], res[1][name]], dim=2), ref, torch.bfloat16, name)
+
+
+def _rank_autograd(rank, world, port, lens, outdir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, dO = inputs.make_tensors(1, 4, sum(lens), 128, torch.bfloat16, seed=23,
+                                          with_grad_out=True)
+        a = sum(lens[:rank])
+        qr, kr, vr = (t[:, :, a:a + lens[rank]].contiguous().cuda().requires_grad_(True)
+                      for t in (q, k, v))
+        dOr = dO[:, :, a:a + lens[rank]].contiguous().cuda()
+        o = seqpar.SequenceParallelLinearAttention.apply(qr, kr, vr, True, "relu_eps")
+        o.backward(dOr)
+        torch.cuda.synchronize()
+        api.la_get_device_error()
+        torch.save({n: t.detach().cpu() for n, t in (("o", o), ("dq", qr.grad), ("dk", kr.grad),
+                                                    ("dv", vr.grad))},
+                   os.path.join(outdir, f"r{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_autograd_wrapper_two_processes():
+    # torch autograd over the split sequence (head size 128, relu+eps)
+    lens = (700, 300)
+    with tempfile.TemporaryDirectory() as d:
+        mp.spawn(_rank_autograd, args=(2, _free_port(), lens, d), nprocs=2, join=True)
+        res = [torch.load(os.path.join(d, f"r{r}.pt")) for r in range(2)]
+    q, k, v, dO = inputs.make_tensors(1, 4, sum(lens), 128, torch.bfloat16, seed=23,
+                                      with_grad_out=True)
+    o_ref, _, _ = oracle.forward(q, k, v, True, oracle.PHI_RELU_EPS)
+    rq, rk, rv = oracle.backward(q, k, v, dO, True, oracle.PHI_RELU_EPS)
+    rq, rk = relu_branch_as_kernel(rq, q), relu_branch_as_kernel(rk, k)
+    for name, ref in (("o", o_ref), ("dq", rq), ("dk", rk), ("dv", rv)):
+        compare(torch.cat([res[0][name], res[1][name]], dim=2), ref, torch.bfloat16, name)
