@@ -128,3 +128,24 @@ def test_favor_rejects_unsupported_sizes():
     xf = torch.zeros(1, 1, 8, 64, dtype=torch.float32, device="cuda")
     with pytest.raises(api.LinearAttentionError):
         api.la_favor_features(xf, torch.zeros(64, 64, dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("N", [1, 64, 129])
+@pytest.mark.parametrize("dk,dv", [(128, 64), (64, 128)])
+def test_mv_short_sequences(N, dk, dv):
+    # identity-map attention with feature and value lengths of their own at
+    # one token, one chunk and a ragged tail
+    g = torch.Generator().manual_seed(N + dk)
+    pq = (torch.rand((2, 2, N, dk), generator=g) + 0.05).to(torch.bfloat16).cuda()
+    pk = (torch.rand((2, 2, N, dk), generator=g) + 0.05).to(torch.bfloat16).cuda()
+    v, _, _, dO = qkv(2, 2, N, dv, seed=N + dv, dO=True)
+    for causal in (True, False):
+        o = api.la_forward_mv(pq, pk, v, causal, "identity")
+        dpq, dpk, dvv = api.la_backward_mv(pq, pk, v, dO, causal, "identity")
+        torch.cuda.synchronize()
+        api.la_get_device_error()
+        compare(o, oracle.forward_mv(pq, pk, v, causal), torch.bfloat16, "o")
+        rq, rk, rv = oracle.backward_mv(pq, pk, v, dO, causal)
+        compare(dpq, rq, torch.bfloat16, "dq")
+        compare(dpk, rk, torch.bfloat16, "dk")
+        compare(dvv, rv, torch.bfloat16, "dv")

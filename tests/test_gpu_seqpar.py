@@ -204,3 +204,21 @@ def test_autograd_wrapper_two_processes():
     rq, rk = relu_branch_as_kernel(rq, q), relu_branch_as_kernel(rk, k)
     for name, ref in (("o", o_ref), ("dq", rq), ("dk", rk), ("dv", rv)):
         compare(torch.cat([res[0][name], res[1][name]], dim=2), ref, torch.bfloat16, name)
+
+
+@pytest.mark.parametrize("lens", [(1, 1, 1), (128, 1, 127, 0, 256), (64, 64), (5, 500, 3)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_sharded_edge_lengths(lens, D):
+    # one-token shards, shards on and off chunk boundaries, empty shards,
+    # five ranks, a single head
+    N = sum(lens)
+    q, k, v, dO = (t.cuda() for t in inputs.make_tensors(1, 1, N, D, torch.bfloat16,
+                                                         seed=3 * N + D, with_grad_out=True))
+    for causal in (True, False):
+        o, dq, dk, dv, _ = sharded(q, k, v, dO, lens, causal, "elu1")
+        o_ref, _, _ = oracle.forward(q, k, v, causal, oracle.PHI_ELU1)
+        rq, rk, rv = oracle.backward(q, k, v, dO, causal, oracle.PHI_ELU1)
+        compare(o, o_ref, torch.bfloat16, "o")
+        compare(dq, rq, torch.bfloat16, "dq")
+        compare(dk, rk, torch.bfloat16, "dk")
+        compare(dv, rv, torch.bfloat16, "dv")
