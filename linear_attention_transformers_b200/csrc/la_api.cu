@@ -19,6 +19,7 @@
 #include "la_chunk_bwd.cuh"
 #include "la_favor.cuh"
 #include "la_pad.cuh"
+#include "la_reduce.cuh"
 #include "la_chunk_bwd64.cuh"
 #include "la_chunk_fwd.cuh"
 #include "la_chunk_fwd64.cuh"
@@ -344,6 +345,24 @@ la_status launch_state_kernel(int which, float* rec, float* out, float* S, float
     return launch_status();
 }
 
+// The REDUCE pass (state record of each block's token range, no decay):
+// for head size 128 the compact reduce block (two per SM), otherwise the
+// chunked kernel's REDUCE mode.
+template <int D, int C, int PHI>
+la_status launch_reduce(const la::ChunkParams& r, int64_t grid, cudaStream_t st) {
+    if constexpr (D == 128) {
+        auto kern = la::reduce128_kernel<PHI>;
+        if (cudaError_t e = cudaFuncSetAttribute(
+                kern, cudaFuncAttributeMaxDynamicSharedMemorySize, la::Reduce128Cfg::SMEM))
+            return cuda_fail("cudaFuncSetAttribute", e);
+        la::LaunchScope scope("reduce128", st);
+        kern<<<unsigned(grid), la::kReduce128Threads, la::Reduce128Cfg::SMEM, st>>>(r);
+        return launch_status();
+    } else {
+        return launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, grid, st, "chunk_reduce");
+    }
+}
+
 // Starts of the segments of a causal pass (no decay): the REDUCE pass of
 // `red` (its k, v maps, N, kv_group and centring) over the sub-segments of
 // the tokens before the last segment into `sub`, then starts[h][p] =
@@ -362,7 +381,7 @@ la_status run_segment_starts(const la::ChunkParams& red, int64_t heads, const Se
     r.S_out = sub;
     r.z_out = sub + D * D;
     r.stride_S = r.stride_z = R;
-    la_status s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * ss.nsub, st, "chunk_reduce");
+    la_status s = launch_reduce<D, C, PHI>(r, heads * ss.nsub, st);
     if (s != LA_OK) return s;
     const int R4 = int(R / 4);
     const int bph = (R4 + la::kStateThreads - 1) / la::kStateThreads;
@@ -444,9 +463,7 @@ la_status run_fwd_chunked(const void* q, const void* k, const void* v, void* o, 
     r.S_out = rec;
     r.z_out = rec + D * D;
     r.stride_S = r.stride_z = R;
-    if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st, "chunk_reduce")) !=
-        LA_OK)
-        return s;
+    if ((s = launch_reduce<D, C, PHI>(r, heads * p.seg.nseg, st)) != LA_OK) return s;
     if ((s = launch_state_kernel(1, rec, tot, nullptr, nullptr, heads, p.seg.nseg, D, st)) != LA_OK)
         return s;
     // the state of each key/value head: the record of its group's first query head
@@ -701,9 +718,7 @@ la_status run_bwd_chunked(const void* q, const void* k, const void* v, const voi
     }
     float* stot = reinterpret_cast<float*>(ws + p.stot_off);
     float* rtot = reinterpret_cast<float*>(ws + p.rtot_off);
-    if ((s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(red, heads * p.seg.nseg, st,
-                                                     "chunk_reduce")) != LA_OK)
-        return s;
+    if ((s = launch_reduce<D, C, PHI>(red, heads * p.seg.nseg, st)) != LA_OK) return s;
     if ((s = launch_state_kernel(1, srec, stot, nullptr, nullptr, heads, p.seg.nseg, D, st)) !=
         LA_OK)
         return s;
@@ -1388,8 +1403,7 @@ la_status run_state_local(const void* k, const void* v, float* out, int64_t head
     r.S_out = dst;
     r.z_out = dst + D * D;
     r.stride_S = r.stride_z = R;
-    la_status s = launch_chunk<D, C, PHI, la::MODE_REDUCE>(r, heads * p.seg.nseg, st,
-                                                           "chunk_reduce");
+    la_status s = launch_reduce<D, C, PHI>(r, heads * p.seg.nseg, st);
     if (s != LA_OK || p.seg.nseg == 1) return s;
     return launch_state_kernel(1, dst, out, nullptr, nullptr, heads, p.seg.nseg, D, st);
 }
