@@ -78,7 +78,10 @@ struct Bwd1Cfg {
     static constexpr int OFF_DG = OFF_DU + C * D * 2;
     static constexpr int OFF_STG = OFF_DG + 16 * C * 2;
     static constexpr int OFF_ZF = OFF_STG + C * D * 2;
-    static constexpr int OFF_BAR = OFF_ZF + ((D * 4 + 15) / 16) * 16;
+    // z as float, two copies (chunk parity): with the state readout on its
+    // own warp group, chunk c's dQ reads one while chunk c's readout writes
+    // the other
+    static constexpr int OFF_BAR = OFF_ZF + 2 * (((D * 4 + 15) / 16) * 16);
     static constexpr int NBAR = 3 * NSTAGE + 9;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
@@ -203,11 +206,20 @@ constexpr int kBwdThreads = 448;  // producer, MMA, 8 phi warps, 4 epilogue warp
 
 // SAVED = the forward's O and g are given: no forward recompute; the
 // feature-map warps form dU = dO / g and dg = -(dO . O) / g directly.
+//
+// SPLIT (causal, saved, D = 128): the state readout (S -> the bf16 operand
+// of the next chunk, z, the segment's (R, r)) runs on the key half of the
+// feature-map warps (warps 6-9) while the epilogue warps form dQ, so the two
+// TMEM readouts of a chunk overlap instead of following each other; and the
+// MMA thread issues the next chunk's W = dU V^T as soon as its tiles are
+// ready (W has its own TMEM columns), so W is done when the epilogue comes
+// to mask it.
 template <int D, int C, int PHI, bool CAUSAL, bool SAVED>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd1Cfg<D, C>;
     constexpr int NS = Cfg::NSTAGE;
+    constexpr bool SPLIT = SAVED && CAUSAL && D == 128 && !Cfg::XT;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -252,7 +264,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         mbar_init(w_ready, 1);
         mbar_init(wt_ready, 128);
         mbar_init(da_ready, 1);
-        mbar_init(s_ready, 128);
+        mbar_init(s_ready, SPLIT ? 256 : 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -319,7 +331,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 const uint32_t duop = SAVED ? qs + 3 * Cfg::TILE : duop_g;
                 const uint32_t dgop = SAVED ? qs + Cfg::OFF_SDG : dgop_g;
                 if (!(ok = mbar_wait(&phi_done[s], (c / NS) & 1, abort_flag))) break;
-                if (!(ok = mbar_wait(s_ready, c & 1, abort_flag))) break;
+                // SPLIT: W needs only this chunk's tiles (its columns were
+                // last read by the previous chunk's mask); the state operand
+                // is waited for just before dU S^T
+                if (!SPLIT && !(ok = mbar_wait(s_ready, c & 1, abort_flag))) break;
                 tc_fence_after();
                 if (!SAVED) {
                     if (CAUSAL) {
@@ -359,6 +374,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                         umma_bf16(tP, desc_kmajor(duop, C, k), desc_kmajor(vs, C, k), idCC, k > 0);
                     umma_commit(w_ready);
                     if (!(ok = mbar_wait(wt_ready, c & 1, abort_flag))) break;
+                    if (SPLIT && !(ok = mbar_wait(s_ready, c & 1, abort_flag))) break;
                     tc_fence_after();
                     // dA = W' B
                     if (Cfg::XT) {
@@ -410,6 +426,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     dgt[tile_off(16, idx / C, idx % C) / 2] = __float2bfloat16_rn(0.f);
             }
         }
+        // SPLIT, warps 6-9 (one TMEM lane quarter each): after chunk c's
+        // products, S -> the bf16 operand of chunk c + 1 and z -> zf (the
+        // copy of the other parity)
+        auto readout_dq = [&](int c) -> bool {
+            if (!named_bar_all(2, 128, mbar_wait(da_ready, c & 1, abort_flag))) return false;
+            tc_fence_after();
+            const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+            const int frow = acc_row<D>(warp & 3, lane);
+            float zv[16];
+            tmem_ld16(tmem + lane_base + Cfg::T_Z, zv);
+#pragma unroll 1
+            for (int v0 = 0; v0 < D; v0 += 32) {
+                float sv[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_S + v0, sv);
+                store_row16_bf16(smem + Cfg::OFF_SPREV, D, frow, v0, sv);
+                store_row16_bf16(smem + Cfg::OFF_SPREV, D, frow, v0 + 16, sv + 16);
+            }
+            reinterpret_cast<float*>(smem + Cfg::OFF_ZF)[((c + 1) & 1) * D + frow] = zv[0];
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(s_ready);
+            return true;
+        };
+        // the readout warps' share of the initial state's arrival (the
+        // epilogue warps write the initial operand)
+        if (SPLIT && u >= 128) mbar_arrive(s_ready);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS;
             if (!mbar_wait(&full[s], (c / NS) & 1, abort_flag)) break;
@@ -474,6 +516,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             }
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
+            // SPLIT: the state readout of the previous chunk, after this
+            // chunk's feature map (which the next W waits for)
+            if (SPLIT && u >= 128 && c > 0 && !readout_dq(c - 1)) break;
+        }
+        if (SPLIT && u >= 128 && prm.rec_out && nchunks > 0 &&
+            named_bar_all(2, 128, mbar_wait(da_ready, (nchunks - 1) & 1, abort_flag))) {
+            // the segment's (R, r) after its last chunk
+            tc_fence_after();
+            const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+            const int frow = acc_row<D>(warp & 3, lane);
+            float* out = prm.rec_out + size_t(blockIdx.x) * (D * D + D);
+#pragma unroll 1
+            for (int v0 = 0; v0 < D; v0 += 32) {
+                float rv[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_R + v0, rv);
+                store16_f32(out + size_t(frow) * D + v0, rv);
+                store16_f32(out + size_t(frow) * D + v0 + 16, rv + 16);
+            }
+            float rz[16];
+            tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
+            tmem_wait_ld();
+            out[size_t(D) * D + frow] = rz[0] + rz[1];
         }
     } else {
         const int e = tid - 320;
@@ -694,6 +758,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             tc_fence_after();
             if (e == 0) bulk_wait_read0();
             named_bar_sync(1, 128);
+            const float* zfc = zf + (SPLIT ? (c & 1) * D : 0);  // z of the chunks before c
             constexpr float kc = phi_center<PHI>();
             float tcoef = 0.f;
             if (kc != 0.f) {
@@ -710,7 +775,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                             load_chunk8(qt, C, irow, (f0 >> 3) + h, a8);
 #pragma unroll
                             for (int t = 0; t < 8; ++t) {
-                                dot = fmaf(fmaf(dg, zf[f0 + 8 * h + t], av[8 * h + t]), a8[t], dot);
+                                dot = fmaf(fmaf(dg, zfc[f0 + 8 * h + t], av[8 * h + t]), a8[t], dot);
                                 sa += a8[t];
                             }
                         }
@@ -732,14 +797,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 #pragma unroll
                         for (int t = 0; t < 8; ++t) {
                             const int f = f0 + 16 * h + t;
-                            dq16[t] = (fmaf(dg, zf[f], av[16 * h + t]) + tcoef) *
+                            dq16[t] = (fmaf(dg, zfc[f], av[16 * h + t]) + tcoef) *
                                       dphi_from_phi<PHI>(a8a[t]);
-                            dq16[8 + t] = (fmaf(dg, zf[f + 8], av[16 * h + 8 + t]) + tcoef) *
+                            dq16[8 + t] = (fmaf(dg, zfc[f + 8], av[16 * h + 8 + t]) + tcoef) *
                                           dphi_from_phi<PHI>(a8b[t]);
                         }
                         store_row16_bf16(stg, C, irow, f0 + 16 * h, dq16);
                     }
                 }
+            }
+            if (SPLIT) {
+                // dA read: the next chunk's dA MMAs may overwrite it
+                tc_fence_before();
+                mbar_arrive(s_ready);
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every zf read done
@@ -750,6 +820,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     tma_store_3d(&prm.tm_dq, stg + a * C * 128, a * 64, row0, head);
                 bulk_commit();
             }
+            if (SPLIT) continue;  // the state readout runs on warps 6-9
             // ---- next state operand; segment (R, r) on the last chunk
             if (CAUSAL) {
                 // z rides along with the first S columns' round trip
@@ -803,11 +874,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
 // ======================================================================
 // PART: grouped key/value heads, dK and dV stored as float32 per-query-head
 // partials (prm.dk_part, dv_part) instead of the bf16 tiles.
+//
+// SPLIT (causal, D = 128): the suffix-state readout (R -> the bf16 operand
+// of the next, earlier chunk, r -> rf) runs on the key half of the
+// feature-map warps (warps 6-9) while the epilogue warps form dV and dK, so
+// the two TMEM readouts of a step overlap.
 template <int D, int C, int PHI, bool CAUSAL, bool PART = false>
 __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_constant__ BwdParams prm) {
     using namespace sm100;
     using Cfg = Bwd2Cfg<D, C>;
     constexpr int NS = Cfg::NSTAGE;
+    constexpr bool SPLIT = CAUSAL && D == 128 && !Cfg::XT;
+    static_assert(!SPLIT || 2 * D * 4 <= 1024, "two copies of r in the rf area");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -843,7 +921,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         mbar_init(x_ready, 1);
         mbar_init(xt_ready, 128);
         mbar_init(d_ready, 1);
-        mbar_init(r_ready, 128);
+        mbar_init(r_ready, SPLIT ? 256 : 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -968,6 +1046,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         }
         const float* gb = prm.gbuf + size_t(head) * prm.N;
         const float* dgb = prm.dgbuf + size_t(head) * prm.N;
+        // SPLIT, warps 6-9 (one TMEM lane quarter each): after step t's
+        // products, R -> the bf16 operand of step t + 1 and r -> rf (the
+        // copy of the other parity)
+        auto readout_dkdv = [&](int t) {
+            if (!named_bar_all(2, 128, mbar_wait(d_ready, t & 1, abort_flag))) return;
+            tc_fence_after();
+            const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
+            const int frow = acc_row<D>(warp & 3, lane);
+            float rz[16];
+            tmem_ld16(tmem + lane_base + Cfg::T_RZ, rz);
+#pragma unroll 1
+            for (int v0 = 0; v0 < D; v0 += 32) {
+                float rv[32];
+                tmem_load<32>(tmem + lane_base + Cfg::T_R + v0, rv);
+                store_row16_bf16(smem + Cfg::OFF_RPREV, D, frow, v0, rv);
+                store_row16_bf16(smem + Cfg::OFF_RPREV, D, frow, v0 + 16, rv + 16);
+            }
+            reinterpret_cast<float*>(smem + Cfg::OFF_RF)[((t + 1) & 1) * D + frow] = rz[0] + rz[1];
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(r_ready);
+        };
+        // the readout warps' share of the initial state's arrival
+        if (SPLIT && u >= 128) mbar_arrive(r_ready);
         for (int t = 0; t < nchunks; ++t) {
             const int s = t % NS;
             if (!mbar_wait(&full[s], (t / NS) & 1, abort_flag)) break;
@@ -994,6 +1096,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             scale_tile_rows<C, D, 256>(st + 3 * Cfg::TILE, u, nvalid, rinv);
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
+            // SPLIT: the suffix-state readout of the previous step, after
+            // this step's feature map (which this step's products wait for).
+            // A failed wait skips it but stays in the loop, so the
+            // 256-thread barrier above keeps its members.
+            if (SPLIT && u >= 128 && t > 0) readout_dkdv(t - 1);
         }
     } else {
         const int e = tid - 320;
@@ -1104,6 +1211,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 if (e == 0) bulk_wait_read0();
                 named_bar_sync(1, 128);
             }
+            const float* rfc = rf + (SPLIT ? (t & 1) * D : 0);  // r of the later chunks
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 16) {
                 float dv16[16], db16[16];
@@ -1117,8 +1225,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     float dk16[16];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
-                        dk16[k] = (db16[k] + rf[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
-                        dk16[8 + k] = (db16[8 + k] + rf[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
+                        dk16[k] = (db16[k] + rfc[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
+                        dk16[8 + k] = (db16[8 + k] + rfc[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
                     }
                     if constexpr (PART) {
                         if (row0 + jrow < prm.N) {
@@ -1132,6 +1240,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     }
                 }
             }
+            if (SPLIT) {
+                // dV, dB read: the next step's products may overwrite them
+                tc_fence_before();
+                mbar_arrive(r_ready);
+            }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every rf read done
             mbar_arrive(&empty[s]);
@@ -1143,6 +1256,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 }
                 bulk_commit();
             }
+            if (SPLIT) continue;  // the suffix-state readout runs on warps 6-9
             if (CAUSAL) {
                 // r rides along with the first R columns' round trip
                 float rz[16];
