@@ -82,7 +82,7 @@ struct Bwd1Cfg {
     // own warp group, chunk c's dQ reads one while chunk c's readout writes
     // the other
     static constexpr int OFF_BAR = OFF_ZF + 2 * (((D * 4 + 15) / 16) * 16);
-    static constexpr int NBAR = 3 * NSTAGE + 9;
+    static constexpr int NBAR = 3 * NSTAGE + 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int T_P = 0, T_O = C, T_OZ = C + D, T_S = C + D + 16, T_Z = C + 2 * D + 16;
@@ -111,7 +111,7 @@ struct Bwd2Cfg {
     static constexpr int OFF_STGV = STG_ALIAS ? OFF_X1 : OFF_X2 + C * C * 2;
     static constexpr int OFF_STGK = STG_ALIAS ? OFF_X2 : OFF_STGV + C * D * 2;
     static constexpr int OFF_BAR = STG_ALIAS ? OFF_X2 + C * C * 2 : OFF_STGK + C * D * 2;
-    static constexpr int NBAR = 3 * NSTAGE + 5;
+    static constexpr int NBAR = 3 * NSTAGE + 6;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     // X in TMEM (C = 128): X1, X2 are packed to bf16 in place over the low
@@ -237,6 +237,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     uint64_t* da_ready = p_ready + 6;    // commit: dA, state updates
     uint64_t* s_ready = p_ready + 7;     // 128: state operand for next chunk
     uint64_t* drain = p_ready + 8;
+    uint64_t* st_ready = p_ready + 9;    // commit (SPLIT): S, z, R, r updated
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -266,6 +267,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         mbar_init(da_ready, 1);
         mbar_init(s_ready, SPLIT ? 256 : 128);
         mbar_init(drain, 1);
+        mbar_init(st_ready, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -393,6 +395,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                 for (int k = 0; k < D; k += 16)
                     umma_bf16(tO, desc_kmajor(duop, C, k), desc_kmajor(sprev, D, k), idCD_k,
                               (CAUSAL || k > 0) ? 1u : 0u);
+                // SPLIT: dA is complete here; the epilogue starts on it while
+                // the state updates run
+                if (SPLIT) umma_commit(da_ready);
                 if (CAUSAL) {
                     // S += B^T V, z += B^T 1
 #pragma unroll
@@ -411,7 +416,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                         umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgop, 16, k), idD16, acc);
                     }
                 }
-                umma_commit(da_ready);
+                umma_commit(SPLIT ? st_ready : da_ready);
             }
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
@@ -430,7 +435,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         // products, S -> the bf16 operand of chunk c + 1 and z -> zf (the
         // copy of the other parity)
         auto readout_dq = [&](int c) -> bool {
-            if (!named_bar_all(2, 128, mbar_wait(da_ready, c & 1, abort_flag))) return false;
+            if (!named_bar_all(2, 128, mbar_wait(st_ready, c & 1, abort_flag))) return false;
             tc_fence_after();
             const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
             const int frow = acc_row<D>(warp & 3, lane);
@@ -521,7 +526,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             if (SPLIT && u >= 128 && c > 0 && !readout_dq(c - 1)) break;
         }
         if (SPLIT && u >= 128 && prm.rec_out && nchunks > 0 &&
-            named_bar_all(2, 128, mbar_wait(da_ready, (nchunks - 1) & 1, abort_flag))) {
+            named_bar_all(2, 128, mbar_wait(st_ready, (nchunks - 1) & 1, abort_flag))) {
             // the segment's (R, r) after its last chunk
             tc_fence_after();
             const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
@@ -813,6 +818,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every zf read done
+            // SPLIT: the state updates read the stage's tiles too
+            if (SPLIT) (void)mbar_wait(st_ready, c & 1, abort_flag);
             mbar_arrive(&empty[s]);  // this thread is done with the stage
             if (e == 0) {
 #pragma unroll
@@ -899,6 +906,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
     uint64_t* d_ready = x_ready + 2;    // commit: dV, dB, R
     uint64_t* r_ready = x_ready + 3;    // 128: R operand for the next (earlier) chunk
     uint64_t* drain = x_ready + 4;
+    uint64_t* r_done = x_ready + 5;     // commit (SPLIT): R, r updated
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -923,6 +931,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         mbar_init(d_ready, 1);
         mbar_init(r_ready, SPLIT ? 256 : 128);
         mbar_init(drain, 1);
+        mbar_init(r_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -1021,6 +1030,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                     umma_bf16(t4, desc_kmajor(vs, C, k), desc_kmajor(rprev, D, k), idCD_k,
                               (CAUSAL || k > 0) ? 1u : 0u);
                 }
+                // SPLIT: dV, dB are complete here; the epilogue starts on
+                // them while the suffix state updates
+                if (SPLIT) umma_commit(d_ready);
                 if (CAUSAL) {
 #pragma unroll
                     for (int k = 0; k < C; k += 16) {
@@ -1029,7 +1041,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                         umma_bf16(tRZ, desc_mnmajor(qs, C, k), desc_kmajor(dgs, 16, k), idD16, acc);
                     }
                 }
-                umma_commit(d_ready);
+                umma_commit(SPLIT ? r_done : d_ready);
             }
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
@@ -1050,7 +1062,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         // products, R -> the bf16 operand of step t + 1 and r -> rf (the
         // copy of the other parity)
         auto readout_dkdv = [&](int t) {
-            if (!named_bar_all(2, 128, mbar_wait(d_ready, t & 1, abort_flag))) return;
+            if (!named_bar_all(2, 128, mbar_wait(r_done, t & 1, abort_flag))) return;
             tc_fence_after();
             const uint32_t lane_base = uint32_t(32 * (warp & 3)) << 16;
             const int frow = acc_row<D>(warp & 3, lane);
@@ -1212,31 +1224,42 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
                 named_bar_sync(1, 128);
             }
             const float* rfc = rf + (SPLIT ? (t & 1) * D : 0);  // r of the later chunks
+            // SPLIT: 32 columns of dV and of dB per TMEM round trip
+            constexpr int NCOL = SPLIT ? 32 : 16;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float dv16[16], db16[16];
-                tmem_ld16(tmem + lane_base + Cfg::T_3 + c0, dv16);
-                tmem_ld16(tmem + lane_base + Cfg::T_4 + c0, db16);
-                tmem_wait_ld();
-                if (jrow >= 0) {
-                    float b8a[8], b8b[8];
-                    load_chunk8(kt, C, jrow, c0 >> 3, b8a);
-                    load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
-                    float dk16[16];
+            for (int c00 = 0; c00 < D; c00 += NCOL) {
+                float dvw[NCOL], dbw[NCOL];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        dk16[k] = (db16[k] + rfc[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
-                        dk16[8 + k] = (db16[8 + k] + rfc[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
-                    }
-                    if constexpr (PART) {
-                        if (row0 + jrow < prm.N) {
-                            const size_t off = (size_t(head) * prm.N + row0 + jrow) * D + c0;
-                            store16_f32(prm.dv_part + off, dv16);
-                            store16_f32(prm.dk_part + off, dk16);
+                for (int h = 0; h < NCOL / 16; ++h) {
+                    tmem_ld16(tmem + lane_base + Cfg::T_3 + c00 + 16 * h, dvw + 16 * h);
+                    tmem_ld16(tmem + lane_base + Cfg::T_4 + c00 + 16 * h, dbw + 16 * h);
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < NCOL / 16; ++h) {
+                    const int c0 = c00 + 16 * h;
+                    const float* dv16 = dvw + 16 * h;
+                    const float* db16 = dbw + 16 * h;
+                    if (jrow >= 0) {
+                        float b8a[8], b8b[8];
+                        load_chunk8(kt, C, jrow, c0 >> 3, b8a);
+                        load_chunk8(kt, C, jrow, (c0 >> 3) + 1, b8b);
+                        float dk16[16];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            dk16[k] = (db16[k] + rfc[c0 + k]) * dphi_from_phi<PHI>(b8a[k]);
+                            dk16[8 + k] = (db16[8 + k] + rfc[c0 + 8 + k]) * dphi_from_phi<PHI>(b8b[k]);
                         }
-                    } else {
-                        store_row16_bf16(stgv, C, jrow, c0, dv16);
-                        store_row16_bf16(stgk, C, jrow, c0, dk16);
+                        if constexpr (PART) {
+                            if (row0 + jrow < prm.N) {
+                                const size_t off = (size_t(head) * prm.N + row0 + jrow) * D + c0;
+                                store16_f32(prm.dv_part + off, dv16);
+                                store16_f32(prm.dk_part + off, dk16);
+                            }
+                        } else {
+                            store_row16_bf16(stgv, C, jrow, c0, dv16);
+                            store_row16_bf16(stgk, C, jrow, c0, dk16);
+                        }
                     }
                 }
             }
@@ -1247,6 +1270,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
             }
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every rf read done
+            // SPLIT: the suffix-state update reads the stage's tiles too
+            if (SPLIT) (void)mbar_wait(r_done, t & 1, abort_flag);
             mbar_arrive(&empty[s]);
             if (e == 0 && !PART) {
 #pragma unroll
