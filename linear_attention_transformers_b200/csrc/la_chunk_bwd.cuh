@@ -574,25 +574,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             zop_h[tile_off(16, r, cc) / 2] = __float2bfloat16_rn(0.f);
         }
         named_bar_sync(1, 128);
+        // one read of the record row feeds the operand and the accumulator
+        load_record_row<D>(st_in, frow, 1.f, sprev, tmem + lane_base + Cfg::T_S, CAUSAL && st_in);
+        const float z0 = (st_in && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
         if (frow >= 0) {
-            float z0;
-            load_state_row<D>(st_in, frow, sprev, &z0);
             const __nv_bfloat16 zh = __float2bfloat16_rn(z0);
             zop_h[tile_off(16, 0, frow) / 2] = zh;
             zop_h[tile_off(16, 1, frow) / 2] = __float2bfloat16_rn(z0 - __bfloat162float(zh));
             zf[frow] = z0;
         }
         if (CAUSAL && st_in) {
-            for (int cc = 0; cc < D; cc += 16) {
-                float v16[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    v16[t] = frow >= 0 ? st_in[size_t(frow) * D + cc + t] : 0.f;
-                tmem_st16(tmem + lane_base + Cfg::T_S + cc, v16);
-            }
             float z16[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) z16[t] = (t == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+            for (int t = 0; t < 16; ++t) z16[t] = t == 0 ? z0 : 0.f;
             tmem_st16(tmem + lane_base + Cfg::T_Z, z16);
             tmem_wait_st();
         }
@@ -1127,22 +1121,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dkdv_kernel(const __grid_c
         uint8_t* stgv = smem + Cfg::OFF_STGV;
         uint8_t* stgk = smem + Cfg::OFF_STGK;
 
-        if (frow >= 0) {
-            float r0;
-            load_state_row<D>(st_in, frow, rprev, &r0);
-            rf[frow] = r0;
-        }
+        // one read of the record row feeds the operand and the accumulator
+        load_record_row<D>(st_in, frow, 1.f, rprev, tmem + lane_base + Cfg::T_R, CAUSAL && st_in);
+        const float r0 = (st_in && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+        if (frow >= 0) rf[frow] = r0;
         if (CAUSAL && st_in) {
-            for (int cc = 0; cc < D; cc += 16) {
-                float v16[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    v16[t] = frow >= 0 ? st_in[size_t(frow) * D + cc + t] : 0.f;
-                tmem_st16(tmem + lane_base + Cfg::T_R + cc, v16);
-            }
             float z16[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) z16[t] = (t == 0 && frow >= 0) ? st_in[size_t(D) * D + frow] : 0.f;
+            for (int t = 0; t < 16; ++t) z16[t] = t == 0 ? r0 : 0.f;
             tmem_st16(tmem + lane_base + Cfg::T_RZ, z16);
             tmem_wait_st();
         }

@@ -430,30 +430,19 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
         float s0 = 1.f;
         if constexpr (DECAY) s0 = exp2f(lg * 0.5f * float(min(C, tok1 - tok0)));
         // ---- initial state: bf16 operand (+ TMEM accumulator in CAUSAL mode)
-        if (MODE != MODE_REDUCE && frow >= 0) {
-            for (int q = 0; q < D / 8; ++q) {
-                float v8[8];
+        if (MODE != MODE_REDUCE) {
+            // one read of the record row feeds the operand and the accumulator
+            const bool to_tmem = MODE == MODE_CAUSAL && st_in != nullptr;
+            load_record_row<D>(st_in, frow, s0, sx, tmem + lane_base + Cfg::T_S, to_tmem);
+            const float z0 = (st_in && frow >= 0) ? s0 * st_in[size_t(D) * D + frow] : 0.f;
+            if (frow >= 0) put_z(z0);
+            if (to_tmem) {
+                float z16[16];
 #pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    v8[t] = st_in ? s0 * st_in[size_t(frow) * D + q * 8 + t] : 0.f;
-                store_row_bf16<8>(sx, D, frow, q * 8, v8);
+                for (int t = 0; t < 16; ++t) z16[t] = t == 0 ? z0 : 0.f;
+                tmem_st16(tmem + lane_base + Cfg::T_Z, z16);
+                tmem_wait_st();
             }
-            put_z(st_in ? s0 * st_in[size_t(D) * D + frow] : 0.f);
-        }
-        if (MODE == MODE_CAUSAL && st_in) {
-            for (int cc = 0; cc < D; cc += 16) {
-                float v16[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    v16[t] = frow >= 0 ? s0 * st_in[size_t(frow) * D + cc + t] : 0.f;
-                tmem_st16(tmem + lane_base + Cfg::T_S + cc, v16);
-            }
-            float z16[16];
-#pragma unroll
-            for (int t = 0; t < 16; ++t)
-                z16[t] = (t == 0 && frow >= 0) ? s0 * st_in[size_t(D) * D + frow] : 0.f;
-            tmem_st16(tmem + lane_base + Cfg::T_Z, z16);
-            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();

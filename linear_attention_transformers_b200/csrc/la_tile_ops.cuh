@@ -225,6 +225,37 @@ __device__ __forceinline__ void store_row_bf16(uint8_t* tile, int rows, int row,
     }
 }
 
+// Row `row` of a float32 state record (rec + row * D, 16-byte aligned; null
+// or row < 0 = zeros), times `scale`, into row `row` of the bf16 operand tile
+// (rows = D) and, when `to_tmem`, into the TMEM columns from `tm` of this
+// thread's lane as float32 (warp-collective then: every lane calls it).  One
+// read of the row, 32 columns (eight 16-byte loads in flight) per round trip.
+template <int D>
+__device__ __forceinline__ void load_record_row(const float* rec, int row, float scale,
+                                                uint8_t* tile, uint32_t tm, bool to_tmem) {
+    constexpr int W = D < 32 ? D : 32;
+    const bool valid = rec != nullptr && row >= 0;
+    const float4* src = reinterpret_cast<const float4*>(rec + (valid ? size_t(row) * D : 0));
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += W) {
+        float v[W];
+#pragma unroll
+        for (int j = 0; j < W / 4; ++j) {
+            const float4 x = valid ? __ldg(src + c0 / 4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[4 * j] = x.x * scale;
+            v[4 * j + 1] = x.y * scale;
+            v[4 * j + 2] = x.z * scale;
+            v[4 * j + 3] = x.w * scale;
+        }
+        if (row >= 0) store_row_bf16<W>(tile, D, row, c0, v);
+        if (to_tmem) {
+#pragma unroll
+            for (int h = 0; h < W / 16; ++h) sm100::tmem_st16(tm + c0 + 16 * h, v + 16 * h);
+        }
+    }
+    if (to_tmem) sm100::tmem_wait_st();
+}
+
 // Load NV consecutive TMEM columns of this thread's lane (NV multiple of 16).
 template <int NV>
 __device__ __forceinline__ void tmem_load(uint32_t taddr, float* v) {
