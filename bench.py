@@ -137,17 +137,17 @@ _FWD64_SOURCES = ["la_chunk_fwd64.cuh", "la_chunk_fwd.cuh", "la_tile_ops.cuh", "
 _BWD64_SOURCES = ["la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "la_sm100.cuh",
                   "la_common.cuh"]
 MEASURED_TRAFFIC = {
-    # one `ncu --set full` launch each at B8 H16 N4096 D64 (the timed
-    # workload at half its tokens)
-    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.429760e6 + 156.376832e6) / (8 * 16 * 4096),
+    # one ncu launch each (the fourth of each kernel; DRAM byte counters) at
+    # B8 H16 N4096 D64, the timed workload at half its tokens
+    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.394688e6 + 158.814976e6) / (8 * 16 * 4096),
                      "files": _FWD64_SOURCES,
-                     "sources": "0f58f7cf746f364f634f86df1468f8d8ea5919d0f015d921d5650cbdbab58893"},
-    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.764864e6 + 53.445888e6) / (8 * 16 * 4096),
+                     "sources": "8bcebbcf1ed37f1201997187a0234b234545cea7b36d51bc13516deaf81a4591"},
+    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.693952e6 + 49.244160e6) / (8 * 16 * 4096),
                "files": _BWD64_SOURCES,
-               "sources": "a1579f5b5909c8a1adf65b4b6ea2271ddfa4fa1a55a7f5a9c2be109edabf8749"},
-    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.685056e6 + 100.026368e6) / (8 * 16 * 4096),
+               "sources": "65fd8f4e35fd287a2431db12a5bd9e93399486b61cdf35775e41dbeaea4dda3d"},
+    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.684544e6 + 96.190720e6) / (8 * 16 * 4096),
                  "files": _BWD64_SOURCES,
-                 "sources": "a1579f5b5909c8a1adf65b4b6ea2271ddfa4fa1a55a7f5a9c2be109edabf8749"},
+                 "sources": "65fd8f4e35fd287a2431db12a5bd9e93399486b61cdf35775e41dbeaea4dda3d"},
 }
 
 

@@ -526,10 +526,16 @@ chunk_fwd_kernel(const __grid_constant__ ChunkParams prm) {
                             tmem_load<32>(tmem + lane_base + Cfg::T_S + v0, sv);
                             if (frow >= 0) {
                                 store_row_bf16<32>(sx, D, frow, v0, sv);
-                                if (write_final)
-                                    for (int t = 0; t < 32; ++t)
-                                        prm.S_out[sidx * prm.stride_S + size_t(frow) * D + v0 + t] =
-                                            sv[t];
+                                if (write_final) {
+                                    // S_out, its head stride and D * 4 are
+                                    // multiples of 16 bytes
+                                    float4* dst = reinterpret_cast<float4*>(
+                                        prm.S_out + sidx * prm.stride_S + size_t(frow) * D + v0);
+#pragma unroll
+                                    for (int t = 0; t < 8; ++t)
+                                        dst[t] = make_float4(sv[4 * t], sv[4 * t + 1],
+                                                             sv[4 * t + 2], sv[4 * t + 3]);
+                                }
                             }
                         }
                         if (frow >= 0) {
