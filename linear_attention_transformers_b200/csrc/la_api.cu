@@ -226,15 +226,16 @@ SegSplit split(int64_t N, int C, int nseg) {
 // tokens before the last segment are summed (its own state is never a
 // start), each segment as `ratio` equal sub-segments (ratio dividing its
 // chunks) chosen so that the reduce blocks fill the SMs: the smallest
-// modelled makespan waves x (chunks per block + fill).
+// modelled makespan waves x (chunks per block + fill).  A wave holds two
+// blocks per SM at head size 128 (the compact reduce block), one otherwise.
 struct StartSplit {
     int ratio = 1, nsub = 0, sub_len = 0;
 };
-StartSplit start_split(int64_t heads, const SegSplit& seg, int C) {
+StartSplit start_split(int64_t heads, const SegSplit& seg, int C, int64_t D) {
     StartSplit r;
     if (seg.nseg <= 1) return r;
     const int seg_chunks = seg.seg_len / C;
-    const int kNumSM = num_sms();
+    const int kNumSM = num_sms() * (D == 128 ? 2 : 1);
     constexpr double kFill = 3.0;
     double best = 0.0;
     for (int q = 1; q <= std::min(seg_chunks, 16); ++q) {
@@ -276,7 +277,7 @@ FwdPlan plan_fwd(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtyp
         p.rec_off = 0;
         p.bytes = 0;
         if (p.seg.nseg > 1) {
-            p.ss = start_split(heads, p.seg, p.C);
+            p.ss = start_split(heads, p.seg, p.C, D);
             p.sub_off = round_up(size_t(heads) * p.seg.nseg * R * sizeof(float), 256);
             p.bytes = p.sub_off + size_t(heads) * p.ss.nsub * R * sizeof(float);
         }
@@ -528,7 +529,7 @@ BwdPlan plan_bwd_fast(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la
     if (causal) {
         p.qseg = p.seg;
         if (p.seg.nseg > 1) {
-            p.ss = start_split(heads, p.seg, p.C);
+            p.ss = start_split(heads, p.seg, p.C, D);
             p.srec_off = off;
             off += round_up(size_t(heads) * p.seg.nseg * R * 4, 256);
             p.rrec_off = off;
@@ -1367,7 +1368,7 @@ SpPlan plan_sp(int64_t B, int64_t H, int64_t N, int64_t D, int causal, la_dtype 
     p.qseg = causal ? p.seg
                     : split(N, p.C, int(std::max<int64_t>(1, std::min<int64_t>(want, nch))));
     const size_t R4 = size_t(D * D + D) * sizeof(float);
-    p.ss = start_split(heads, p.seg, p.C);
+    p.ss = start_split(heads, p.seg, p.C, D);
     // forward: per-segment records (la_state_local) or starts, then the
     // start reduce's sub-segment records
     p.fwd_sub_off = p.seg.nseg > 1 ? round_up(size_t(heads) * p.seg.nseg * R4, 256) : 0;
