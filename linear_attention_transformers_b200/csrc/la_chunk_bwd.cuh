@@ -82,7 +82,7 @@ struct Bwd1Cfg {
     // own warp group, chunk c's dQ reads one while chunk c's readout writes
     // the other
     static constexpr int OFF_BAR = OFF_ZF + 2 * (((D * 4 + 15) / 16) * 16);
-    static constexpr int NBAR = 3 * NSTAGE + 10;
+    static constexpr int NBAR = 6 * NSTAGE + 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 16 + 1024;
     static constexpr int T_P = 0, T_O = C, T_OZ = C + D, T_S = C + D + 16, T_Z = C + 2 * D + 16;
@@ -238,6 +238,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
     uint64_t* s_ready = p_ready + 7;     // 128: state operand for next chunk
     uint64_t* drain = p_ready + 8;
     uint64_t* st_ready = p_ready + 9;    // commit (SPLIT): S, z, R, r updated
+    // SPLIT: the stage's q tile has barriers of its own (k, v, dO are
+    // released by the products' commit, q by the epilogue once dQ is formed)
+    uint64_t* fullq = p_ready + 10;       // TMA landed (q)
+    uint64_t* phiq_done = fullq + NS;     // 128: phi(q) applied
+    uint64_t* emptyq = fullq + 2 * NS;    // 128: epilogue done with q
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Cfg::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Cfg::OFF_MISC + 4);
 
@@ -256,7 +261,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&phi_done[s], 256);
-            mbar_init(&empty[s], 128);
+            mbar_init(&empty[s], SPLIT ? 1 : 128);
+            mbar_init(&fullq[s], 1);
+            mbar_init(&phiq_done[s], 128);
+            mbar_init(&emptyq[s], 128);
         }
         mbar_init(p_ready, 1);
         mbar_init(pt_ready, 128);
@@ -286,16 +294,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             tma_prefetch_desc(&prm.tm_k);
             tma_prefetch_desc(&prm.tm_v);
             tma_prefetch_desc(&prm.tm_do);
-            int issued = 0;
+            int issued = 0, issued_q = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS;
                 if (c >= NS && !mbar_wait(&empty[s], ((c / NS) - 1) & 1, abort_flag)) break;
                 uint8_t* st = smem + s * Cfg::STAGE;
-                mbar_arrive_expect_tx(&full[s], 4 * Cfg::TILE);
+                mbar_arrive_expect_tx(&full[s], (SPLIT ? 3 : 4) * Cfg::TILE);
                 const int row = tok0 + c * C;
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a) {
-                    tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
+                    if (!SPLIT)
+                        tma_load_3d(st + a * C * 128, &prm.tm_q, &full[s], a * 64, row, head);
                     tma_load_3d(st + Cfg::TILE + a * C * 128, &prm.tm_k, &full[s], a * 64, row,
                                 kv_head);
                     tma_load_3d(st + 2 * Cfg::TILE + a * C * 128, &prm.tm_v, &full[s], a * 64, row,
@@ -304,9 +313,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                                 head);
                 }
                 issued = c + 1;
+                if (SPLIT) {
+                    // q of chunk c, once the epilogue is done with chunk c - NS
+                    if (c >= NS && !mbar_wait(&emptyq[s], ((c / NS) - 1) & 1, abort_flag)) break;
+                    mbar_arrive_expect_tx(&fullq[s], Cfg::TILE);
+#pragma unroll
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_3d(st + a * C * 128, &prm.tm_q, &fullq[s], a * 64, row, head);
+                    issued_q = c + 1;
+                }
             }
             for (int c = max(0, issued - NS); c < issued; ++c)
                 mbar_wait_drain(&full[c % NS], (c / NS) & 1);
+            for (int c = max(0, issued_q - NS); c < issued_q; ++c)
+                mbar_wait_drain(&fullq[c % NS], (c / NS) & 1);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -408,7 +428,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     }
                 }
                 if (rec) {
-                    // R += A^T dU, r += A^T [dg_hi; dg_lo]
+                    // R += A^T dU, r += A^T [dg_hi; dg_lo] (SPLIT: phi(q) comes
+                    // on its own barrier)
+                    if (SPLIT && !(ok = mbar_wait(&phiq_done[s], (c / NS) & 1, abort_flag))) break;
+                    if (SPLIT) tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < C; k += 16) {
                         const uint32_t acc = (c > 0 || k > 0) ? 1u : 0u;
@@ -417,6 +440,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
                     }
                 }
                 umma_commit(SPLIT ? st_ready : da_ready);
+                // SPLIT: k, v, dU and the DG operand are read by now
+                if (SPLIT) umma_commit(&empty[s]);
             }
             umma_commit(drain);
             mbar_wait_drain(drain, 0);
@@ -463,10 +488,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             uint8_t* st = smem + s * Cfg::STAGE;
             const int nvalid = min(C, tok1 - (tok0 + c * C));
             // q -> phi(q); k -> phi(k) - c (the centred key features: see
-            // the epilogue's all-ones correction)
-            if (u < 128)
-                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
-            else
+            // the epilogue's all-ones correction).  SPLIT: q comes later, on
+            // its own barrier
+            if (u < 128) {
+                if (!SPLIT) phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+            } else
                 phi_tile<PHI, C, D, 128, true>(st + Cfg::TILE, u - 128, nvalid, true);
             if (SAVED) {
                 // dU = dO / g in place, dg = -(dO . O) / g; 256 / C threads per row
@@ -521,6 +547,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             }
             fence_proxy_async_smem();
             mbar_arrive(&phi_done[s]);
+            if (SPLIT && u < 128) {
+                // phi(q) of chunk c (read by R += A^T dU and the epilogue)
+                if (!mbar_wait(&fullq[s], (c / NS) & 1, abort_flag)) break;
+                phi_tile<PHI, C, D, 128>(st, u, nvalid, true);
+                fence_proxy_async_smem();
+                mbar_arrive(&phiq_done[s]);
+            }
             // SPLIT: the state readout of the previous chunk, after this
             // chunk's feature map (which the next W waits for)
             if (SPLIT && u >= 128 && c > 0 && !readout_dq(c - 1)) break;
@@ -753,7 +786,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             // centred key features phi(k) - c, which differ from the true dA
             // only along the all-ones vector; that component is restored from
             // <dA_i, a_i> = 0 (t = -(T . a_i) / (1 . a_i)).
-            if (!named_bar_all(1, 128, mbar_wait(da_ready, c & 1, abort_flag))) break;
+            {
+                // SPLIT: phi(q) of the chunk has its own barrier
+                const bool ok = mbar_wait(da_ready, c & 1, abort_flag) &&
+                                (!SPLIT || mbar_wait(&phiq_done[s], (c / NS) & 1, abort_flag));
+                if (!named_bar_all(1, 128, ok)) break;
+            }
             tc_fence_after();
             if (e == 0) bulk_wait_read0();
             named_bar_sync(1, 128);
@@ -813,8 +851,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) bwd_dq_kernel(const __grid_con
             fence_proxy_async_smem();
             named_bar_sync(1, 128);  // staging complete; every zf read done
             // SPLIT: the state updates read the stage's tiles too
-            if (SPLIT) (void)mbar_wait(st_ready, c & 1, abort_flag);
-            mbar_arrive(&empty[s]);  // this thread is done with the stage
+            if (SPLIT) {
+                // R += A^T dU reads q too; k, v, dO go back with the
+                // products' own commit
+                (void)mbar_wait(st_ready, c & 1, abort_flag);
+                mbar_arrive(&emptyq[s]);
+            } else {
+                mbar_arrive(&empty[s]);  // this thread is done with the stage
+            }
             if (e == 0) {
 #pragma unroll
                 for (int a = 0; a < D / 64; ++a)
