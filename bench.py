@@ -139,15 +139,15 @@ _BWD64_SOURCES = ["la_chunk_bwd64.cuh", "la_chunk_bwd.cuh", "la_tile_ops.cuh", "
 MEASURED_TRAFFIC = {
     # one ncu launch each (the fourth of each kernel; DRAM byte counters) at
     # B8 H16 N4096 D64, the timed workload at half its tokens
-    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.394688e6 + 158.814976e6) / (8 * 16 * 4096),
+    "chunk_causal": {"D": 64, "bytes_per_token_head": (201.394944e6 + 155.971072e6) / (8 * 16 * 4096),
                      "files": _FWD64_SOURCES,
                      "sources": "8bcebbcf1ed37f1201997187a0234b234545cea7b36d51bc13516deaf81a4591"},
-    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.693952e6 + 49.244160e6) / (8 * 16 * 4096),
+    "bwd_dq": {"D": 64, "bytes_per_token_head": (337.735168e6 + 49.178368e6) / (8 * 16 * 4096),
                "files": _BWD64_SOURCES,
-               "sources": "65fd8f4e35fd287a2431db12a5bd9e93399486b61cdf35775e41dbeaea4dda3d"},
-    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.684544e6 + 96.190720e6) / (8 * 16 * 4096),
+               "sources": "cf3a81aef51868101c532774411a259712c05b9e423fc79c5ecc8ecef1c6d207"},
+    "bwd_dkdv": {"D": 64, "bytes_per_token_head": (272.699392e6 + 96.399872e6) / (8 * 16 * 4096),
                  "files": _BWD64_SOURCES,
-                 "sources": "65fd8f4e35fd287a2431db12a5bd9e93399486b61cdf35775e41dbeaea4dda3d"},
+                 "sources": "cf3a81aef51868101c532774411a259712c05b9e423fc79c5ecc8ecef1c6d207"},
 }
 
 
